@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE SwiGLU layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload NAME] [--instances M]
+
+A step is one whole layer call (router, top-k, buckets, every active routed
+and shared expert, weighted combine) over one batch of seeded synthetic
+input.  The default workload is the Mixtral-8x7B-shaped decode layer
+(T=8, d=4096, E=8, k=2, F=14336, bf16), whose 2.8 GB of expert weights are
+far larger than the 126 MB L2, so every step streams its weights from HBM.
+Workloads whose weights fit in L2 rotate through M distinct layer instances
+(--instances) so that each step reads cold weights.
+
+Rank 0 prints one JSON line.  With N > 1 (torchrun, one process per GPU)
+every rank runs an independent replica (the layer forward has no exchange
+step: replicas only); the time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle instead (rank 0 only), one token
+of the same workload per step, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_43_b200 import synth  # noqa: E402
+
+METRIC = "MoE layer tokens/s; achieved HBM GB/s (T≤8) or TFLOPS (T=4096) vs peak"
+DEFAULT_WORKLOAD = "mixtral_T8_d4096_E8k2_F14336"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+REF_BUDGET_S = 150.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return (float(j["hbm_gbs"]), float(j["bf16_tflops"]),
+                float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), "measured")
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def _profile_traffic(kernel: str, workload: str, src_sha: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for ln in f:
+            if ":" in ln and not ln.startswith("#"):
+                k, v = ln.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256") != src_sha:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def _kernel_src_sha(files):
+    import hashlib
+    h = hashlib.sha256()
+    for fn in files:
+        with open(os.path.join(ROOT, "mixture_experts_layer_43_b200", "csrc", fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+class ClockSampler:
+    """nvidia-smi samples of the SM clock and throttle reasons while running."""
+
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str, period_ms: int = 100):
+        self.uuid = uuid
+        self.period_ms = period_ms
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.period_ms), "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for ln in f:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 9:
+                    continue
+                if self.uuid and parts[0] != self.uuid:
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        try:
+            sm = [float(r[1]) for r in rows]
+            mx = max(float(r[2]) for r in rows)
+        except ValueError:
+            return None
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _active_bytes(sh, counts, n_shared):
+    """Algorithmic bytes of one experts launch: every distinct active routed
+    expert and every shared expert read once, x read, out written."""
+    act = int(np.count_nonzero(counts))
+    per = synth.weight_bytes_per_expert(sh)
+    shared = n_shared * synth.weight_bytes_per_expert(sh, sh.Fs) if n_shared else 0
+    return act * per + shared + sh.T * sh.d * 2 + sh.T * sh.d * 4, act
+
+
+def _cpu_baseline(inp, sh, budget_s=12.0, max_s=30.0):
+    import oracle
+    n_threads = oracle.max_threads()
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        oracle.forward(inp, tokens=[done % sh.T])
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or el >= max_s:
+            break
+    return {"value": done / el, "unit": "tokens/s", "cores": n_threads, "kind": "oracle",
+            "sample": (f"{done} tokens of the {sh.name} batch, one fp64 oracle call per "
+                       f"token (routing + every selected and shared expert), {el:.1f} s")}
+
+
+def run_reference(args, sh):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    import oracle
+    inp = synth.make_inputs(sh, seed=args.seed)
+    n_threads = oracle.max_threads()
+    for i in range(args.warmup):
+        oracle.forward(inp, tokens=[i % sh.T])
+    t0 = time.perf_counter()
+    steps = 0
+    while steps < args.steps:
+        oracle.forward(inp, tokens=[steps % sh.T])
+        steps += 1
+        if time.perf_counter() - t0 > REF_BUDGET_S:
+            break
+    el = time.perf_counter() - t0
+    val = steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+        "n_gpus": ws, "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": sh.name, "shape": synth.describe(sh),
+                   "sample_per_step": "one token of the batch"},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": n_threads, "kind": "oracle",
+                         "sample": f"{steps} steps of one token each, fp64 oracle"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_b200(args, sh):
+    import torch
+    from mixture_experts_layer_43_b200 import binding as B
+    from mixture_experts_layer_43_b200 import device as D
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
+
+    # layer instances: enough distinct weights that every step reads cold HBM
+    per_inst = synth.weight_bytes_per_expert(sh) * sh.E + (
+        synth.weight_bytes_per_expert(sh, sh.Fs) * sh.S if sh.S else 0)
+    n_inst = args.instances or max(1, min(32, -(-4 * L2_BYTES // per_inst)))
+    insts = []
+    base = synth.make_inputs(sh, seed=args.seed)
+    layers = [D.DeviceLayer(base, device=str(dev))]
+    for i in range(1, n_inst):
+        inp_i = synth.make_inputs(sh, seed=args.seed + 1000 * i)
+        layers.append(D.DeviceLayer(inp_i, device=str(dev)))
+        del inp_i
+    T = sh.T
+    x = D.upload_x(base.x, dev)
+    out = torch.empty((T, sh.d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    st = stream.cuda_stream
+    plan = B.moe_plan_create(layers[0].config(T))
+    routing = D.Routing(T, sh.k, sh.E, dev)
+
+    def step(i, ev_a=None, ev_b=None):
+        L = layers[i % n_inst]
+        B.moe_route(plan, L.weights, x.data_ptr(), T, out.data_ptr(), st)
+        if ev_a is not None:
+            ev_a.record(stream)
+        B.moe_experts(plan, L.weights, x.data_ptr(), T, out.data_ptr(), st)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+        # algorithmic bytes: from each instance's own routing on this x
+        act_bytes = []
+        acts = []
+        for i in range(n_inst):
+            B.moe_forward(plan, layers[i].weights, x.data_ptr(), T, out.data_ptr(),
+                          routing.struct, st)
+            stream.synchronize()
+            b, a = _active_bytes(sh, routing.counts.cpu().numpy(), layers[i].n_shared)
+            act_bytes.append(b)
+            acts.append(a)
+        status = B.moe_get_device_status(plan)
+        if status != B.MOE_OK:
+            raise RuntimeError("device status after warm-up: " + B.moe_status_string(status))
+
+        K = args.steps
+        ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if uuid and not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(uuid) as clk:
+            t_start.record(stream)
+            for i in range(K):
+                step(i, ev_a[i], ev_b[i])
+            t_end.record(stream)
+            torch.cuda.synchronize(dev)
+        if ws > 1:
+            torch.distributed.barrier()
+        clocks = clk.summary()
+        total_ms = t_start.elapsed_time(t_end)
+        kern_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+        launches = 2 * K
+
+        # e2e: pinned host x in, pinned host out back, every step
+        x_host = torch.from_numpy(base.x.view(np.int16)).pin_memory()
+        out_host = torch.empty((T, sh.d), dtype=torch.float32).pin_memory()
+        e_start = torch.cuda.Event(enable_timing=True)
+        e_end = torch.cuda.Event(enable_timing=True)
+        K2 = max(1, K // 4)
+        torch.cuda.synchronize(dev)
+        e_start.record(stream)
+        for i in range(K2):
+            x.copy_(x_host, non_blocking=True)
+            B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, out.data_ptr(),
+                          None, st)
+            out_host.copy_(out, non_blocking=True)
+        e_end.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e_start.elapsed_time(e_end)
+
+    t_max = total_ms
+    e2e_max = e2e_ms
+    if ws > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([total_ms, e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max, e2e_max = float(tt[0]), float(tt[1])
+    B.moe_plan_destroy(plan)
+
+    tokens_per_s = ws * T * K / (t_max / 1e3)
+    kern_avg_s = float(np.mean(kern_ms)) / 1e3
+    alg_bytes = float(np.mean([act_bytes[i % n_inst] for i in range(K)]))
+    achieved = alg_bytes / kern_avg_s / 1e9
+    src_sha = _kernel_src_sha(["decode.cu", "moe_internal.cuh"])
+    traffic = _profile_traffic("decode_experts_kernel", sh.name, src_sha)
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": ws,
+        "steps": K, "warmup": args.warmup, "ms_per_step": t_max / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if sh.wfmt == synth.WFMT_BF16 else "q4_0/bf16",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x; no trained weights)",
+        "config": {"workload": sh.name, "shape": synth.describe(sh), "T": T,
+                   "instances": n_inst,
+                   "l2": ("inputs larger than L2: each step streams "
+                          f"{alg_bytes / 1e9:.2f} GB of distinct expert weights; "
+                          f"{n_inst} layer instance(s) rotated"),
+                   "active_experts_per_step": float(np.mean(acts)),
+                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "kernel": "decode_experts_kernel",
+                     "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "kernel_ms_avg": kern_avg_s * 1e3,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)"},
+        "e2e": {"value": ws * T * K2 / (e2e_max / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": T * sh.d * 2, "d2h_bytes_per_step": T * sh.d * 4},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if ws == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = _cpu_baseline(base, sh)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=("b200", "reference"), default="b200")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--instances", type=int, default=0)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    sh = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, sh)
+    return run_b200(args, sh)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

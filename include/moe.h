@@ -1,0 +1,192 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: the forward pass of a Mixture-of-Experts
+ * SwiGLU FFN layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer, per token t ("Fused MoE Triton kernel: 5 launches instead of
+ * 24" page, list of fused steps: top-k routing weights, dispatch of tokens to
+ * the chosen experts, parallel expert compute, weighted aggregation; "CUDA:
+ * fuse shared experts into MMVQ" page, section on shared experts: always
+ * active, added to every token):
+ *
+ *   l_e   = x_t . Wr[e] (+ b_e)                     router logits, fp32 FMA
+ *   p     = softmax(l) over all E experts
+ *   K     = the top_k experts with the largest l_e (ties: lower index)
+ *   w_j   = p_j / sum_{K} p                         renormalised weights
+ *   out_t = sum_{j in K} w_j FFN_j(x_t) + sum_s FFN_s(x_t)
+ *   FFN(x) = Wd (SiLU(Wg x) * (Wu x)),  SiLU(z) = z / (1 + e^-z)
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers, owned by the caller, aligned to
+ *    16 bytes (TMA requires 16-byte aligned bases and row pitches).  The
+ *    library never copies or frees them.  Weights stay in place.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Compute entry points only enqueue work: they neither allocate nor
+ *    synchronise, so they may be captured in a CUDA graph.
+ *  - Every entry point returns a moe_status_t; nothing is thrown or aborted
+ *    across the ABI.  Host-side argument checks run before any launch, so an
+ *    invalid call enqueues nothing.
+ *  - Matrices are row-major with the reduction dimension contiguous
+ *    ("[out][in]"):  x [T][d] bf16;  router_w [E][d] fp32;  router_b [E] fp32;
+ *    routed gate/up [E][F][d], down [E][d][F];  shared gate/up [S][Fs][d],
+ *    down [S][d][Fs];  out [T][d] fp32.
+ *  - bf16 values are raw IEEE bfloat16 bit patterns (uint16).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or shape */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid request outside what this build runs */
+    MOE_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+    MOE_ERR_OOM = 4,           /* plan workspace allocation failed */
+    MOE_ERR_DEVICE_FLAG = 5,   /* a kernel flagged an inconsistent state */
+    MOE_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out */
+} moe_status_t;
+
+/* Weight formats.
+ * MOE_WFMT_BF16: every expert matrix is bf16 in the layouts above.
+ * MOE_WFMT_Q4_0: blocks of 32 consecutive weights along the reduction dim,
+ *   each an fp16 scale d and 32 codes q in 0..15, weight = d * (q - 8)
+ *   (the 35B-A3B Q4_0 workload; the "MoE on RTX 5090 reaches 41% of
+ *   bandwidth" page names Q4_0, measurement-setup paragraph; the MMVQ page
+ *   asks that quantised weights be read once and never expanded, section
+ *   "what MMVQ is").  The kernels read the packed form written by
+ *   moe_q4_0_pack, not the canonical 18-byte blocks. */
+typedef enum moe_wfmt {
+    MOE_WFMT_BF16 = 0,
+    MOE_WFMT_Q4_0 = 1
+} moe_wfmt_t;
+
+/* Execution regime.  AUTO picks DECODE for T <= MOE_DECODE_MAX_T and
+ * PREFILL otherwise.  DECODE streams every active expert's weights once in a
+ * single persistent launch (CUDA cores + mma.sync, fused combine).  PREFILL
+ * runs the grouped GEMMs on tcgen05 tensor cores (bf16 only). */
+typedef enum moe_regime {
+    MOE_REGIME_AUTO = 0,
+    MOE_REGIME_DECODE = 1,
+    MOE_REGIME_PREFILL = 2
+} moe_regime_t;
+
+#define MOE_DECODE_MAX_T 8
+
+typedef struct moe_config {
+    int32_t t_max;        /* largest T any forward call will pass */
+    int32_t d_model;      /* d; multiple of 64 */
+    int32_t d_ff;         /* F, routed expert hidden size; multiple of 32 */
+    int32_t n_experts;    /* E >= 1 routed experts (<= 1024) */
+    int32_t top_k;        /* 1 <= k <= min(E, 16) */
+    int32_t n_shared;     /* S >= 0 shared experts (<= 8) */
+    int32_t d_ff_shared;  /* Fs, hidden size of each shared expert (0 if S=0) */
+    int32_t wfmt;         /* moe_wfmt_t */
+    int32_t regime;       /* moe_regime_t */
+    int32_t device;       /* CUDA device ordinal the plan lives on */
+} moe_config_t;
+
+/* One stack of expert matrices.  bf16: `data` is the bf16 stack, `scales`
+ * must be NULL.  Q4_0: `data` = packed codes, `scales` = packed fp16 scales
+ * (both from moe_q4_0_pack). */
+typedef struct moe_matrix {
+    const void* data;
+    const void* scales;
+} moe_matrix_t;
+
+typedef struct moe_weights {
+    const float* router_w;       /* [E][d] fp32 */
+    const float* router_b;       /* [E] fp32, or NULL for no bias */
+    moe_matrix_t gate, up, down; /* routed experts, E stacked */
+    moe_matrix_t shared_gate, shared_up, shared_down; /* S stacked; ignored if S=0 */
+} moe_weights_t;
+
+/* Optional copies of the routing tables of the last call (device pointers,
+ * each may be NULL).  ids/weights are [T][k] with each token's experts in
+ * descending logit order, ties to the lower index; counts [E]; offsets
+ * [E+1] exclusive prefix sums of counts; slot_pair [T*k]: slot s (ordered by
+ * expert, then ascending token) holds the pair index t*k + j. */
+typedef struct moe_routing {
+    int32_t* ids;
+    float* weights;
+    int32_t* counts;
+    int32_t* offsets;
+    int32_t* slot_pair;
+} moe_routing_t;
+
+typedef struct moe_plan_s* moe_plan_t;
+
+/* Validate `cfg`, select the device, size and allocate the plan workspace
+ * for cfg->t_max tokens and resolve the driver's tensor-map encoder.  On
+ * success *out receives the plan; on failure *out is NULL and nothing is
+ * left allocated.  Allocates device memory (the only call that does, apart
+ * from none).  Errors: INVALID_ARG (shape limits above), UNSUPPORTED
+ * (PREFILL regime with Q4_0, or a device that is not sm_100), CUDA, OOM. */
+moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out);
+
+/* Free the plan's workspace.  The caller must make sure no work enqueued
+ * with the plan is still running.  NULL is ignored. */
+void moe_plan_destroy(moe_plan_t plan);
+
+/* The whole layer: route, bucket, experts, weighted combine.
+ * x [T][d] bf16, out [T][d] fp32 (overwritten), 0 <= T <= t_max.
+ * `routing` may be NULL; when given, the routing tables are copied to it
+ * (device-to-device, on `stream`).  T = 0 enqueues nothing.
+ * Launches: 2 kernels in the decode regime (router+buckets, experts), 5 in
+ * the prefill regime (router, buckets+gather, gate/up GEMM, down GEMM with
+ * fused combine, plus a zero-fill of `out`). */
+moe_status_t moe_forward(moe_plan_t plan, const moe_weights_t* w,
+                         const void* x, int32_t T, float* out,
+                         moe_routing_t* routing, void* stream);
+
+/* The two halves of moe_forward, for callers that time them separately.
+ * moe_route: router, top-k, buckets and work list into the plan's
+ * workspace; also zero-fills `out`.  moe_experts: expert FFNs and the
+ * weighted combine into `out`, reading the workspace moe_route wrote with
+ * the same T.  moe_forward == moe_route then moe_experts. */
+moe_status_t moe_route(moe_plan_t plan, const moe_weights_t* w,
+                       const void* x, int32_t T, float* out, void* stream);
+moe_status_t moe_experts(moe_plan_t plan, const moe_weights_t* w,
+                         const void* x, int32_t T, float* out, void* stream);
+
+/* Copy the routing tables of the last moe_route/moe_forward (T tokens) from
+ * the workspace to `routing` (device pointers; NULL members skipped). */
+moe_status_t moe_routing_get(moe_plan_t plan, int32_t T, moe_routing_t* routing,
+                             void* stream);
+
+/* Number of kernels the last moe_forward/moe_route/moe_experts call enqueued. */
+int32_t moe_last_launch_count(moe_plan_t plan);
+
+/* Read and clear the sticky device error word (synchronises `plan`'s device).
+ * OK, DEVICE_FLAG (a kernel saw an out-of-range id or count) or TIMEOUT (a
+ * bounded wait gave up). */
+moe_status_t moe_get_device_status(moe_plan_t plan);
+
+/* Bytes of the packed Q4_0 form of n_mats matrices of [rows][k] weights.
+ * k must be a multiple of 32.  Returns INVALID_ARG otherwise. */
+moe_status_t moe_q4_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
+                                   size_t* code_bytes, size_t* scale_bytes);
+
+/* Repack canonical Q4_0 blocks ([n_mats][rows][k/32] blocks of 18 bytes: a
+ * little-endian fp16 scale, then 16 bytes whose byte j holds code j in the
+ * low nibble and code j+16 in the high nibble) into the kernel layout:
+ *   codes  [n_mats][k/32][rows][16 bytes], the 32 codes of each block
+ *          permuted so one 32-bit word feeds one tensor-core fragment;
+ *   scales [n_mats][k/32][rows] fp16.
+ * Same 4.5 bits per weight.  All pointers are device pointers; `blocks`
+ * needs no alignment, `codes`/`scales` 16 bytes.  Enqueued on `stream`. */
+moe_status_t moe_q4_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
+                           int64_t k, void* codes, void* scales, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

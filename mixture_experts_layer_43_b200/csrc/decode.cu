@@ -1,0 +1,641 @@
+// decode.cu -- decode-regime kernels (T <= MOE_DECODE_MAX_T tokens per call).
+//
+// Two launches per layer call:
+//  1. decode_route_kernel: router logits (fp32 FMA), softmax + top-k with
+//     renormalised weights, per-expert buckets (counts, exclusive offsets,
+//     stable slot order), the expert work list, and the zero-fill of `out`.
+//     ("Fused MoE Triton kernel: 5 launches instead of 24" page, fused steps
+//     one and two; its launch table's routing and dispatch rows.)
+//  2. decode_experts_kernel: ONE persistent launch over every active routed
+//     expert and every shared expert ("CUDA: fuse shared experts into MMVQ"
+//     page: shared experts go through the same pass as the routed ones).
+//     Each work unit is (expert, slice of FS hidden rows): it streams the
+//     slice's gate/up rows, forms h = SiLU(gate) * up for the expert's
+//     tokens, streams the matching columns of the down matrix and adds
+//     w * (Wd h) into `out` (the weighted aggregation, fused).  Weights move
+//     HBM -> shared memory by TMA through a ring of stages fed by one
+//     producer warp, so every SM keeps tens of KB in flight ("MoE on RTX 5090
+//     reaches 41% of bandwidth" page: small reads per kernel cap bandwidth;
+//     the fix it predicts is more bytes per launch).  The contraction over
+//     the <= 8 tokens of an expert runs on mma.sync (bf16 in, fp32
+//     accumulate); Q4_0 codes are dequantised in registers and never written
+//     back ("MMVQ" page: read quantised weights once, never expand them).
+#include <float.h>
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+// ============================================================== router ===
+constexpr int kRouteThreads = 256;
+constexpr int kRouteWarps = kRouteThreads / 32;
+
+__global__ void __launch_bounds__(kRouteThreads) decode_route_kernel(const RouteArgs a) {
+    __shared__ float s_part[kRouteWarps][kDecodeTok];
+    __shared__ float s_log[kDecodeTok][kMaxExperts];
+    __shared__ int s_cnt[kMaxExperts];
+    __shared__ int s_ids[kDecodeTok * kMaxTopK];
+    __shared__ float s_w[kDecodeTok * kMaxTopK];
+    __shared__ float s_sel[kDecodeTok][kMaxTopK];
+    __shared__ int s_wsum[kRouteWarps];
+    __shared__ uint32_t s_ticket;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int T = a.T, d = a.d, E = a.E, k = a.k;
+
+    // ---- zero-fill out [T][d] (the expert kernel accumulates into it)
+    {
+        const int n4 = (T * d) >> 2;
+        float4* o = reinterpret_cast<float4*>(a.out);
+        for (int i = blockIdx.x * kRouteThreads + tid; i < n4; i += gridDim.x * kRouteThreads)
+            o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    // ---- logits: CTA owns experts_per_cta experts, each split over wpe warps
+    const int epc = a.experts_per_cta;
+    const int wpe = kRouteWarps / epc;
+    const int le = warp / wpe, part = warp % wpe;
+    const int e = blockIdx.x * epc + le;
+    float acc[kDecodeTok];
+#pragma unroll
+    for (int t = 0; t < kDecodeTok; ++t) acc[t] = 0.f;
+    if (e < E) {
+        const int chunk = d / wpe;
+        const int i_end = (part + 1) * chunk;
+        const float* wrow = a.wr + static_cast<size_t>(e) * d;
+        for (int i = part * chunk + lane * 4; i < i_end; i += 128) {
+            const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + i));
+#pragma unroll
+            for (int t = 0; t < kDecodeTok; ++t) {
+                if (t < T) {
+                    const uint2 xv = __ldg(reinterpret_cast<const uint2*>(
+                        a.x + static_cast<size_t>(t) * d + i));
+                    acc[t] = fmaf(__uint_as_float(xv.x << 16), wv.x, acc[t]);
+                    acc[t] = fmaf(__uint_as_float(xv.x & 0xffff0000u), wv.y, acc[t]);
+                    acc[t] = fmaf(__uint_as_float(xv.y << 16), wv.z, acc[t]);
+                    acc[t] = fmaf(__uint_as_float(xv.y & 0xffff0000u), wv.w, acc[t]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kDecodeTok; ++t) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < kDecodeTok; ++t) s_part[warp][t] = acc[t];
+    }
+    __syncthreads();
+    if (tid < epc * T) {
+        const int le2 = tid / T, t = tid % T;
+        const int e2 = blockIdx.x * epc + le2;
+        if (e2 < E) {
+            float s = 0.f;
+            for (int p = 0; p < wpe; ++p) s += s_part[le2 * wpe + p][t];   // fixed order
+            if (a.br) s += a.br[e2];
+            a.ws.logits[t * E + e2] = s;
+        }
+    }
+
+    // ---- the last CTA to finish does top-k, buckets and the work list
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_ticket = atomicAdd(a.ws.ticket, 1u);
+    __syncthreads();
+    if (s_ticket != gridDim.x - 1) return;
+    __threadfence();
+
+    for (int i = tid; i < T * E; i += kRouteThreads) {
+        float v = __ldcg(a.ws.logits + i);
+        if (isnan(v)) v = -INFINITY;               // NaN never wins a slot
+        s_log[i / E][i % E] = v;
+    }
+    __syncthreads();
+
+    // top-k per token: warp t; a taken expert is marked NaN
+    if (warp < T) {
+        const int t = warp;
+        for (int j = 0; j < k; ++j) {
+            float bv = -INFINITY;
+            int be = INT_MAX;
+            for (int x = lane; x < E; x += 32) {
+                const float v = s_log[t][x];
+                if (!isnan(v) && (v > bv || (v == bv && x < be))) { bv = v; be = x; }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+            }
+            if (lane == 0) {
+                if (be >= E) { atomicOr(a.ws.err, kErrBadId); be = 0; }
+                s_ids[t * k + j] = be;
+                s_sel[t][j] = bv;
+                s_log[t][be] = NAN;
+            }
+            __syncwarp();
+        }
+        // renormalised softmax over the selected logits == softmax over all E
+        // experts restricted to the top-k and renormalised
+        if (lane < k) {
+            const float m = s_sel[t][0];
+            float den = 0.f;
+            for (int j = 0; j < k; ++j) den += expf(s_sel[t][j] - m);
+            float wj = expf(s_sel[t][lane] - m) / den;
+            if (!(m > -INFINITY)) wj = 1.f / k;
+            s_w[t * k + lane] = wj;
+        }
+    }
+    __syncthreads();
+
+    // buckets: counts per expert, then one block scan of (count, active) pairs
+    const int P = T * k;
+    for (int x = tid; x < E; x += kRouteThreads) {
+        int c = 0;
+        for (int p = 0; p < P; ++p) c += (s_ids[p] == x);
+        s_cnt[x] = c;
+    }
+    __syncthreads();
+    constexpr int kPer = kMaxExperts / kRouteThreads;   // experts per thread (4)
+    int loc[kPer];
+    int run = 0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int x = tid * kPer + q;
+        const int c = (x < E) ? s_cnt[x] : 0;
+        loc[q] = run;
+        run += (c << 16) | (c > 0 ? 1 : 0);
+    }
+    int incl = run;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int base = incl - run;
+    for (int w2 = 0; w2 < warp; ++w2) base += s_wsum[w2];
+    int total = 0;
+    for (int w2 = 0; w2 < kRouteWarps; ++w2) total += s_wsum[w2];
+    const int n_routed = total & 0xffff;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+        const int x = tid * kPer + q;
+        if (x < E) {
+            const int ex = base + loc[q];
+            const int off = ex >> 16, act = ex & 0xffff;
+            const int c = s_cnt[x];
+            a.ws.counts[x] = c;
+            a.ws.offsets[x] = off;
+            if (c > 0) {
+                if (c > kDecodeTok) atomicOr(a.ws.err, kErrTooManyTok);
+                a.ws.items[act] = WorkItem{x, off, c, 0};
+            }
+            s_cnt[x] = off;   // reuse as offsets
+        }
+    }
+    if (tid == 0) {
+        a.ws.offsets[E] = total >> 16;
+        a.ws.n_items[0] = n_routed;
+        a.ws.n_items[1] = a.S;
+    }
+    if (tid < a.S) a.ws.items[n_routed + tid] = WorkItem{E + tid, -1, T, 0};
+    __syncthreads();
+    // stable slots: rank of pair p among earlier pairs with the same expert
+    for (int p = tid; p < P; p += kRouteThreads) {
+        const int x = s_ids[p];
+        int rank = 0;
+        for (int q = 0; q < p; ++q) rank += (s_ids[q] == x);
+        const int slot = s_cnt[x] + rank;
+        a.ws.slot_pair[slot] = p;
+        a.ws.slot_token[slot] = p / k;
+        a.ws.slot_w[slot] = s_w[p];
+        a.ws.ids[p] = x;
+        a.ws.wts[p] = s_w[p];
+    }
+    if (tid == 0) *a.ws.ticket = 0u;   // ready for the next call
+}
+
+cudaError_t launch_decode_route(const RouteArgs& a, cudaStream_t stream) {
+    const int grid = (a.E + a.experts_per_cta - 1) / a.experts_per_cta;
+    decode_route_kernel<<<grid, kRouteThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+// ============================================================ experts ===
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kDecodeThreads = kConsumers + 32;   // + one producer warp
+
+template <int FS, bool Q4>
+struct DecodeCfg {
+    static constexpr int RG = FS / 16;            // 16-row groups in a slice
+    static constexpr int ROLES = 2 * RG;          // (matrix, row group) pairs of phase A
+    static constexpr int KSPLIT = kConsumerWarps / ROLES;
+    static_assert(KSPLIT >= 1 && ROLES * KSPLIT == kConsumerWarps, "warp roles");
+    static_assert(!Q4 || FS >= 32, "Q4_0 slices hold whole blocks");
+    // bf16: phase A stage = gate+up [FS rows][KT cols]; phase B = down [RJ rows][FS cols]
+    // Q4_0: phase A stage = gate+up [KB block cols][FS rows]; phase B = [NB][RJ rows]
+    static constexpr int STAGE = Q4 ? 2 * 512 * 18 : 32768;
+    static constexpr int KT = 8192 / FS;          // bf16 phase A k columns
+    static constexpr int KB = 512 / FS;           // Q4_0 phase A block columns
+    static constexpr int NB = FS / 32;            // Q4_0 block columns in a slice
+    static constexpr int RJ = Q4 ? 32768 / FS : 16384 / FS;   // phase B rows per stage
+    static constexpr int HS = FS + 8;             // h row stride (bf16 elements)
+};
+
+struct alignas(16) DecodeSmemTail {
+    int tok[kDecodeTok];
+    float w[kDecodeTok];
+    int abort_flag;
+    int pad[3];
+};
+
+__device__ __forceinline__ uint32_t q4_pair(uint32_t w, int s) {
+    // ((w >> s) & 0x000F000F) puts two codes in the low mantissa bits of two
+    // bf16 values 128 + q; subtracting 136 leaves q - 8 exactly.
+    uint32_t v = ((w >> s) & 0x000F000Fu) | 0x43004300u;
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&v);
+    b = __hsub2(b, __floats2bfloat162_rn(136.f, 136.f));
+    return *reinterpret_cast<uint32_t*>(&b);
+}
+
+template <int FS, bool Q4>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
+    using C = DecodeCfg<FS, Q4>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int ns = a.n_stages;
+    uint8_t* ring = smem;
+    uint8_t* xs = ring + static_cast<size_t>(ns) * C::STAGE;
+    float* gu = reinterpret_cast<float*>(xs + kDecodeTok * a.xs_stride);  // [KSPLIT][2][FS][8]
+    __nv_bfloat16* hhi = reinterpret_cast<__nv_bfloat16*>(gu + C::KSPLIT * 2 * FS * kDecodeTok);
+    __nv_bfloat16* hlo = hhi + kDecodeTok * C::HS;
+    DecodeSmemTail* tail = reinterpret_cast<DecodeSmemTail*>(hlo + kDecodeTok * C::HS);
+    uint64_t* full = reinterpret_cast<uint64_t*>(tail + 1);
+    uint64_t* empty = full + ns;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int d = a.d, E = a.E;
+    if (tid == 0) {
+        for (int s = 0; s < ns; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kConsumerWarps);
+        }
+        tail->abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int n_routed = a.n_items[0], n_shared = a.n_items[1];
+    const int sl_r = a.F / FS, sl_s = a.S ? a.Fs / FS : 0;
+    const int n_units = n_routed * sl_r + n_shared * sl_s;
+    const int nA = Q4 ? (d / 32 + C::KB - 1) / C::KB : (d + C::KT - 1) / C::KT;
+    const int nB = (d + C::RJ - 1) / C::RJ;
+    volatile int* abort_flag = &tail->abort_flag;
+
+    // unit -> (item index, slice)
+    auto unit_item = [&](int u, int& ii, int& sl) {
+        if (u < n_routed * sl_r) { ii = u / sl_r; sl = u % sl_r; }
+        else { const int v = u - n_routed * sl_r; ii = n_routed + v / sl_s; sl = v % sl_s; }
+    };
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&a.tm_gate); prefetch_tensormap(&a.tm_up);
+            prefetch_tensormap(&a.tm_down);
+            if (a.S) { prefetch_tensormap(&a.tm_sgate); prefetch_tensormap(&a.tm_sup);
+                       prefetch_tensormap(&a.tm_sdown); }
+            const uint64_t pol = l2_policy_evict_first();
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+                int ii, sl;
+                unit_item(u, ii, sl);
+                const WorkItem item = a.items[ii];
+                const bool shared = item.expert >= E;
+                const int ex = shared ? item.expert - E : item.expert;
+                const int Fh = shared ? a.Fs : a.F;
+                const int f0 = sl * FS;
+                const CUtensorMap* mg = shared ? &a.tm_sgate : &a.tm_gate;
+                const CUtensorMap* mu = shared ? &a.tm_sup : &a.tm_up;
+                const CUtensorMap* md = shared ? &a.tm_sdown : &a.tm_down;
+                const CUtensorMap* mgs = shared ? &a.tm_sgate_sc : &a.tm_gate_sc;
+                const CUtensorMap* mus = shared ? &a.tm_sup_sc : &a.tm_up_sc;
+                const CUtensorMap* mds = shared ? &a.tm_sdown_sc : &a.tm_down_sc;
+                for (int st = 0; st < nA + nB && ok; ++st, ++it) {
+                    const int slot = it % ns;
+                    if (it >= static_cast<uint32_t>(ns)) {
+                        if (*abort_flag || !mbar_wait_bounded(&empty[slot], ((it / ns) - 1) & 1)) {
+                            atomicOr(a.err, kErrTimeout); *abort_flag = 1; ok = false; break;
+                        }
+                    }
+                    uint8_t* dst = ring + static_cast<size_t>(slot) * C::STAGE;
+                    if (st < nA) {
+                        if constexpr (!Q4) {
+                            const int k0 = st * C::KT;
+                            const int nbox = min(C::KT, d - k0) / 64;
+                            mbar_arrive_expect_tx(&full[slot], 2 * nbox * FS * 128);
+                            const int row = ex * Fh + f0;
+                            for (int b = 0; b < nbox; ++b) {
+                                tma_load_2d(dst + b * FS * 128, mg, &full[slot], k0 + 64 * b, row, pol);
+                                tma_load_2d(dst + FS * C::KT * 2 + b * FS * 128, mu, &full[slot],
+                                            k0 + 64 * b, row, pol);
+                            }
+                        } else {
+                            const int kb0 = st * C::KB;
+                            const int c2 = ex * (d / 32) + kb0;
+                            mbar_arrive_expect_tx(&full[slot], 2 * C::KB * FS * 18);
+                            uint8_t* g = dst;
+                            uint8_t* u2 = dst + C::KB * FS * 18;
+                            tma_load_3d(g, mg, &full[slot], 0, f0, c2, pol);
+                            tma_load_2d(g + C::KB * FS * 16, mgs, &full[slot], f0, c2, pol);
+                            tma_load_3d(u2, mu, &full[slot], 0, f0, c2, pol);
+                            tma_load_2d(u2 + C::KB * FS * 16, mus, &full[slot], f0, c2, pol);
+                        }
+                    } else {
+                        const int j0 = (st - nA) * C::RJ;
+                        const int nbox = min(C::RJ, d - j0) / 128;
+                        if constexpr (!Q4) {
+                            mbar_arrive_expect_tx(&full[slot], nbox * 128 * FS * 2);
+                            for (int b = 0; b < nbox; ++b)
+                                tma_load_2d(dst + b * 128 * FS * 2, md, &full[slot], f0,
+                                            ex * d + j0 + 128 * b, pol);
+                        } else {
+                            const int c2 = ex * (Fh / 32) + f0 / 32;
+                            mbar_arrive_expect_tx(&full[slot], nbox * C::NB * 128 * 18);
+                            for (int b = 0; b < nbox; ++b) {
+                                uint8_t* bd = dst + b * (C::NB * 128 * 18);
+                                tma_load_3d(bd, md, &full[slot], 0, j0 + 128 * b, c2, pol);
+                                tma_load_2d(bd + C::NB * 128 * 16, mds, &full[slot],
+                                            j0 + 128 * b, c2, pol);
+                            }
+                        }
+                    }
+                }
+            }
+            // drain: every issued stage must land before the CTA may exit
+            const uint32_t first = it > static_cast<uint32_t>(ns) ? it - ns : 0;
+            for (uint32_t q = first; q < it; ++q)
+                if (!mbar_wait_bounded(&full[q % ns], (q / ns) & 1)) {
+                    atomicOr(a.err, kErrTimeout);
+                    break;
+                }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int g = lane >> 2, tig = lane & 3;
+    const int role = warp % C::ROLES, ks = warp / C::ROLES;
+    const int mat = role / C::RG, rg = role % C::RG;
+    const uint32_t xs_u = smem_u32(xs);
+    uint32_t it = 0;
+    int prev_item = -1;
+
+    auto wait_full = [&](int slot, uint32_t parity) -> bool {
+        if (*abort_flag) return false;
+        if (mbar_wait_bounded(&full[slot], parity)) return true;
+        atomicOr(a.err, kErrTimeout);
+        *abort_flag = 1;
+        return false;
+    };
+
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+        int ii, sl;
+        unit_item(u, ii, sl);
+        const WorkItem item = a.items[ii];
+        const bool shared = item.expert >= E;
+        const int ntok = min(item.count, kDecodeTok);
+
+        if (ii != prev_item) {
+            named_bar_sync(1, kConsumers);
+            if (tid < kDecodeTok) {
+                int t = 0;
+                float w = 0.f;
+                if (tid < ntok) {
+                    if (shared) { t = tid; w = 1.f; }
+                    else { t = a.slot_token[item.slot_begin + tid]; w = a.slot_w[item.slot_begin + tid]; }
+                }
+                tail->tok[tid] = t;
+                tail->w[tid] = w;
+            }
+            named_bar_sync(1, kConsumers);
+            const int cpr = d / 8;                       // 16-byte chunks per row
+            for (int idx = tid; idx < kDecodeTok * cpr; idx += kConsumers) {
+                const int t = idx / cpr, c = idx % cpr;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (t < ntok)
+                    v = __ldg(reinterpret_cast<const uint4*>(
+                        a.x + static_cast<size_t>(tail->tok[t]) * d + c * 8));
+                *reinterpret_cast<uint4*>(xs + t * a.xs_stride + c * 16) = v;
+            }
+            named_bar_sync(1, kConsumers);
+            prev_item = ii;
+        }
+
+        // ------------------------------------------- phase A: gate and up
+        float cacc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int st = 0; st < nA; ++st, ++it) {
+            const int slot = it % ns;
+            const bool ok = wait_full(slot, (it / ns) & 1);
+            const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
+            if (ok) {
+                if constexpr (!Q4) {
+                    const int k0 = st * C::KT;
+                    const int kmax = min(C::KT, d - k0) / 16;
+                    const uint32_t tile = smem_u32(stage) + mat * (FS * C::KT * 2);
+                    const int m = lane >> 3, r = lane & 7;
+                    const uint32_t arow = rg * 16 + ((m & 1) << 3) + r;
+#pragma unroll 4
+                    for (int kk = ks; kk < kmax; kk += C::KSPLIT) {
+                        uint32_t a0, a1, a2, a3, b0, b1;
+                        ldsm_x4(tile + (kk >> 2) * (FS * 128) +
+                                    swz_offset(arow, (kk & 3) * 2 + (m >> 1), 128),
+                                a0, a1, a2, a3);
+                        ldsm_x2(xs_u + (lane & 7) * a.xs_stride +
+                                    (k0 + kk * 16 + ((lane >> 3) & 1) * 8) * 2,
+                                b0, b1);
+                        mma_bf16_16816(cacc, a0, a1, a2, a3, b0, b1);
+                    }
+                } else {
+                    const int kb0 = st * C::KB;
+                    const int nkb = min(C::KB, d / 32 - kb0);
+                    const uint8_t* mb = stage + mat * (C::KB * FS * 18);
+                    const uint32_t* codes = reinterpret_cast<const uint32_t*>(mb);
+                    const __half* scl = reinterpret_cast<const __half*>(mb + C::KB * FS * 16);
+                    const int r0 = rg * 16 + g;
+#pragma unroll 2
+                    for (int bb = ks; bb < nkb; bb += C::KSPLIT) {
+                        const uint32_t w0 = codes[(bb * FS + r0) * 4 + tig];
+                        const uint32_t w8 = codes[(bb * FS + r0 + 8) * 4 + tig];
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4(xs_u + (lane & 7) * a.xs_stride +
+                                    ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2,
+                                b0, b1, b2, b3);
+                        float cb[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_bf16_16816(cb, q4_pair(w0, 0), q4_pair(w8, 0), q4_pair(w0, 4),
+                                       q4_pair(w8, 4), b0, b1);
+                        mma_bf16_16816(cb, q4_pair(w0, 8), q4_pair(w8, 8), q4_pair(w0, 12),
+                                       q4_pair(w8, 12), b2, b3);
+                        const float s0 = __half2float(scl[bb * FS + r0]);
+                        const float s8 = __half2float(scl[bb * FS + r0 + 8]);
+                        cacc[0] = fmaf(s0, cb[0], cacc[0]);
+                        cacc[1] = fmaf(s0, cb[1], cacc[1]);
+                        cacc[2] = fmaf(s8, cb[2], cacc[2]);
+                        cacc[3] = fmaf(s8, cb[3], cacc[3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        }
+        {
+            float* gq = gu + ((ks * 2 + mat) * FS) * kDecodeTok;
+            const int r = rg * 16 + g;
+            gq[r * kDecodeTok + 2 * tig] = cacc[0];
+            gq[r * kDecodeTok + 2 * tig + 1] = cacc[1];
+            gq[(r + 8) * kDecodeTok + 2 * tig] = cacc[2];
+            gq[(r + 8) * kDecodeTok + 2 * tig + 1] = cacc[3];
+        }
+        named_bar_sync(1, kConsumers);
+        // h = SiLU(gate) * up, kept as a bf16 pair hi + lo (|h - hi - lo| <= 2^-16 |h|)
+        for (int idx = tid; idx < FS * kDecodeTok; idx += kConsumers) {
+            const int f = idx / kDecodeTok, t = idx % kDecodeTok;
+            float gv = 0.f, uv = 0.f;
+#pragma unroll
+            for (int q = 0; q < C::KSPLIT; ++q) {
+                gv += gu[((q * 2 + 0) * FS + f) * kDecodeTok + t];
+                uv += gu[((q * 2 + 1) * FS + f) * kDecodeTok + t];
+            }
+            const float h = gv / (1.f + expf(-gv)) * uv;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+            hhi[t * C::HS + f] = hi;
+            hlo[t * C::HS + f] = __float2bfloat16_rn(h - __bfloat162float(hi));
+        }
+        named_bar_sync(1, kConsumers);
+        uint32_t bh[C::RG][2], bl[C::RG][2];
+#pragma unroll
+        for (int kk = 0; kk < C::RG; ++kk) {
+            const uint32_t off = ((lane & 7) * C::HS + kk * 16 + ((lane >> 3) & 1) * 8) * 2;
+            ldsm_x2(smem_u32(hhi) + off, bh[kk][0], bh[kk][1]);
+            ldsm_x2(smem_u32(hlo) + off, bl[kk][0], bl[kk][1]);
+        }
+        const int t0 = 2 * tig, t1 = t0 + 1;
+        const int tok0 = tail->tok[t0], tok1 = tail->tok[t1];
+        const float w0 = tail->w[t0], w1 = tail->w[t1];
+        const bool v0 = t0 < ntok, v1 = t1 < ntok;
+
+        // --------------------------------------- phase B: down + combine
+        for (int st = 0; st < nB; ++st, ++it) {
+            const int slot = it % ns;
+            const bool ok = wait_full(slot, (it / ns) & 1);
+            const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
+            const int j0 = st * C::RJ;
+            const int rows = min(C::RJ, d - j0);
+            if (ok) {
+                for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
+                    float c[4] = {0.f, 0.f, 0.f, 0.f};
+                    if constexpr (!Q4) {
+                        const uint32_t tile = smem_u32(stage);
+                        const int m = lane >> 3, r = lane & 7;
+                        const uint32_t arow = rgb * 16 + ((m & 1) << 3) + r;
+#pragma unroll
+                        for (int kk = 0; kk < C::RG; ++kk) {
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4(tile + swz_offset(arow, kk * 2 + (m >> 1), FS * 2), a0, a1, a2, a3);
+                            mma_bf16_16816(c, a0, a1, a2, a3, bh[kk][0], bh[kk][1]);
+                            mma_bf16_16816(c, a0, a1, a2, a3, bl[kk][0], bl[kk][1]);
+                        }
+                    } else {
+                        const uint8_t* bbase = stage + (rgb >> 3) * (C::NB * 128 * 18);
+                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);
+                        const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * 128 * 16);
+                        const int rib = (rgb & 7) * 16 + g;
+#pragma unroll
+                        for (int bb = 0; bb < C::NB; ++bb) {
+                            const uint32_t w0c = codes[(bb * 128 + rib) * 4 + tig];
+                            const uint32_t w8c = codes[(bb * 128 + rib + 8) * 4 + tig];
+                            const uint32_t p0 = q4_pair(w0c, 0), q0 = q4_pair(w8c, 0);
+                            const uint32_t p1 = q4_pair(w0c, 4), q1 = q4_pair(w8c, 4);
+                            const uint32_t p2 = q4_pair(w0c, 8), q2 = q4_pair(w8c, 8);
+                            const uint32_t p3 = q4_pair(w0c, 12), q3 = q4_pair(w8c, 12);
+                            float cb[4] = {0.f, 0.f, 0.f, 0.f};
+                            mma_bf16_16816(cb, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1]);
+                            mma_bf16_16816(cb, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                            mma_bf16_16816(cb, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
+                            mma_bf16_16816(cb, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                            const float s0 = __half2float(scl[bb * 128 + rib]);
+                            const float s8 = __half2float(scl[bb * 128 + rib + 8]);
+                            c[0] = fmaf(s0, cb[0], c[0]);
+                            c[1] = fmaf(s0, cb[1], c[1]);
+                            c[2] = fmaf(s8, cb[2], c[2]);
+                            c[3] = fmaf(s8, cb[3], c[3]);
+                        }
+                    }
+                    const int j = j0 + rgb * 16 + g;
+                    if (v0) {
+                        red_add_f32(a.out + static_cast<size_t>(tok0) * d + j, w0 * c[0]);
+                        red_add_f32(a.out + static_cast<size_t>(tok0) * d + j + 8, w0 * c[2]);
+                    }
+                    if (v1) {
+                        red_add_f32(a.out + static_cast<size_t>(tok1) * d + j, w1 * c[1]);
+                        red_add_f32(a.out + static_cast<size_t>(tok1) * d + j + 8, w1 * c[3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        }
+    }
+}
+
+int decode_stage_bytes(int fs, bool q4) {
+    if (q4) return 2 * 512 * 18;
+    (void)fs;
+    return 32768;
+}
+
+size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages) {
+    const int ksplit = kConsumerWarps / (2 * (fs / 16));
+    size_t b = 1024;                                            // alignment slack
+    b += static_cast<size_t>(n_stages) * decode_stage_bytes(fs, q4);
+    b += static_cast<size_t>(kDecodeTok) * (d * 2 + 16);       // staged x
+    b += static_cast<size_t>(ksplit) * 2 * fs * kDecodeTok * 4;  // gate/up results
+    b += 2ull * kDecodeTok * (fs + 8) * 2;                      // h hi/lo
+    b += sizeof(DecodeSmemTail);
+    b += 2ull * n_stages * 8;                                   // barriers
+    return b;
+}
+
+template <int FS, bool Q4>
+static cudaError_t launch_one(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
+    auto* k = decode_experts_kernel<FS, Q4>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    k<<<grid, kDecodeThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, bool q4, int grid, size_t smem,
+                                  cudaStream_t stream) {
+    if (q4) {
+        if (fs == 64) return launch_one<64, true>(a, grid, smem, stream);
+        if (fs == 32) return launch_one<32, true>(a, grid, smem, stream);
+    } else {
+        if (fs == 64) return launch_one<64, false>(a, grid, smem, stream);
+        if (fs == 32) return launch_one<32, false>(a, grid, smem, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

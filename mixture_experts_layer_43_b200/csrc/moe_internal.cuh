@@ -1,0 +1,240 @@
+// moe_internal.cuh -- internal declarations and device helpers shared by the
+// kernels of libmoe_b200.so (sm_100a only).  Inline PTX for the mbarrier,
+// TMA (cp.async.bulk.tensor), ldmatrix, mma.sync and reduction instructions.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ----------------------------------------------------------------- limits
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 16;
+constexpr int kMaxShared = 8;
+constexpr int kDecodeTok = 8;        // mma N: tokens per expert pass (>= MOE_DECODE_MAX_T)
+static_assert(MOE_DECODE_MAX_T <= kDecodeTok, "decode pass holds every token");
+
+// Device error word bits (sticky until moe_get_device_status reads them).
+constexpr uint32_t kErrBadId = 1u;        // an expert id or count out of range
+constexpr uint32_t kErrTimeout = 2u;      // a bounded wait ran out
+constexpr uint32_t kErrTooManyTok = 4u;   // an expert got more tokens than a pass holds
+
+// Bounded waits give up after this long (a healthy wait lasts microseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Work item of the decode regime: one expert and the tokens routed to it.
+struct WorkItem {
+    int32_t expert;      // 0..E-1 routed, E+s shared expert s
+    int32_t slot_begin;  // first slot in the bucket order (routed) or -1 (shared: tokens 0..T-1)
+    int32_t count;       // tokens in this item (<= kDecodeTok)
+    int32_t pad;
+};
+
+// Plan workspace (device pointers), sized for t_max at plan creation.
+struct Workspace {
+    float* logits;         // [t_max][E] fp32
+    int32_t* ids;          // [t_max][k]
+    float* wts;            // [t_max][k]
+    int32_t* counts;       // [E]
+    int32_t* offsets;      // [E+1]
+    int32_t* slot_pair;    // [t_max*k]
+    int32_t* slot_token;   // [t_max*k]
+    float* slot_w;         // [t_max*k]
+    WorkItem* items;       // [E + S]
+    int32_t* n_items;      // [2]: routed items, shared items
+    uint32_t* ticket;      // last-CTA ticket of the decode router
+    uint32_t* err;         // sticky device error word
+    // prefill
+    uint16_t* x_perm;      // [t_max*k][d] bf16 rows gathered per slot
+    uint16_t* h_routed;    // [t_max*k][F] bf16
+    uint16_t* h_shared;    // [t_max][S*Fs] bf16
+    int32_t* tiles;        // prefill tile schedule
+    int32_t* n_tiles;      // [4]
+};
+
+// ---------------------------------------------------------- launch args
+struct RouteArgs {
+    const uint16_t* x;     // [T][d] bf16
+    const float* wr;       // [E][d]
+    const float* br;       // [E] or nullptr
+    float* out;            // [T][d] zero-filled here
+    Workspace ws;
+    int T, d, E, k, S;
+    int experts_per_cta;   // 1, 2, 4 or 8
+};
+
+struct DecodeArgs {
+    // bf16: 2D maps over the weight stacks.  Q4_0: 3D maps over the codes.
+    CUtensorMap tm_gate, tm_up, tm_down;
+    CUtensorMap tm_sgate, tm_sup, tm_sdown;
+    // Q4_0 only: 2D maps over the scales.
+    CUtensorMap tm_gate_sc, tm_up_sc, tm_down_sc;
+    CUtensorMap tm_sgate_sc, tm_sup_sc, tm_sdown_sc;
+    const uint16_t* x;          // [T][d] bf16
+    float* out;                 // [T][d] fp32, accumulated into
+    const WorkItem* items;
+    const int32_t* n_items;
+    const int32_t* slot_token;
+    const float* slot_w;
+    uint32_t* err;
+    int T, d, F, Fs, E, S;
+    int n_stages;               // ring depth
+    int xs_stride;              // bytes per token row of the staged x
+    int kt;                     // phase A: k columns (bf16) / block columns (Q4_0) per stage
+    int rj;                     // phase B: output rows per stage
+};
+
+// Host launchers (decode.cu, q4_pack.cu).
+cudaError_t launch_decode_route(const RouteArgs& a, cudaStream_t stream);
+cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, bool q4, int grid,
+                                  size_t smem, cudaStream_t stream);
+size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages);
+int decode_stage_bytes(int fs, bool q4);
+cudaError_t launch_q4_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint16_t* scales, cudaStream_t stream);
+
+// --------------------------------------------------------- device helpers
+#ifdef __CUDACC__
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait until the phase with the given parity has completed, for at most
+// kWaitLimitNs.  Returns false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    }
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// TMA tiled loads (no multicast), completing on an mbarrier of this CTA.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4}], [%2], %5;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+          "r"(c0), "r"(c1), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t c0, int32_t c1, int32_t c2, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5}], [%2], %6;"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)),
+          "r"(c0), "r"(c1), "r"(c2), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ldmatrix: four / two 8x8 b16 matrices; row addresses from lanes 0-31 / 0-15.
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                        uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                 : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+// c += A(16x16 bf16, row-major) * B(16x8 bf16, col-major), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+// Named barrier among `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
+// `row_bytes` (128, 64 or 32) long and that TMA wrote with the swizzle mode of
+// the same width: the chunk index is XORed with address bits 7.. of the row
+// (128B: row % 8; 64B: (row / 2) % 4; 32B: (row / 4) % 2).  The tile base
+// must be aligned to the swizzle span.
+__device__ __forceinline__ uint32_t swz_offset(uint32_t row, uint32_t chunk, uint32_t row_bytes) {
+    uint32_t x;
+    if (row_bytes == 128) x = chunk ^ (row & 7);
+    else if (row_bytes == 64) x = chunk ^ ((row >> 1) & 3);
+    else x = chunk ^ ((row >> 2) & 1);
+    return row * row_bytes + x * 16;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+#endif  // __CUDACC__
+
+}  // namespace moe

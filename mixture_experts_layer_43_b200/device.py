@@ -1,0 +1,101 @@
+"""Device-memory plumbing around the C ABI: upload a layer's tensors with
+PyTorch (device memory and streams only), repack Q4_0 through the library's
+own moe_q4_0_pack kernel, and fill the moe_weights_t / moe_config_t structs.
+No arithmetic of the layer happens here."""
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+from . import synth
+
+
+def _dev(a: np.ndarray, device) -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a).to(device, non_blocking=False)
+
+
+class DeviceLayer:
+    """One layer instance resident in HBM, ready for moe_forward."""
+
+    def __init__(self, inp: synth.MoEInputs, device: str = "cuda:0",
+                 stream: Optional[torch.cuda.Stream] = None):
+        sh = inp.shape
+        self.shape = sh
+        self.device = torch.device(device)
+        self.q4 = sh.wfmt == synth.WFMT_Q4_0
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self.router_w = _dev(inp.router_w.astype(np.float32), self.device)
+        self.router_b = None if inp.router_b is None else _dev(inp.router_b.astype(np.float32),
+                                                               self.device)
+        self._keep = []
+
+        def mat(arr, n_mats, rows, k):
+            if arr is None:
+                return B.moe_matrix_t(None, None)
+            if not self.q4:
+                t = _dev(arr, self.device)
+                self._keep.append(t)
+                return B.moe_matrix_t(t.data_ptr(), None)
+            canon = _dev(arr.reshape(-1), self.device)
+            cb, sb = B.moe_q4_0_packed_bytes(n_mats, rows, k)
+            codes = torch.empty(cb, dtype=torch.uint8, device=self.device)
+            scales = torch.empty(sb // 2, dtype=torch.int16, device=self.device)
+            B.moe_q4_0_pack(canon.data_ptr(), n_mats, rows, k, codes.data_ptr(),
+                            scales.data_ptr(), st.cuda_stream)
+            st.synchronize()
+            del canon
+            self._keep += [codes, scales]
+            return B.moe_matrix_t(codes.data_ptr(), scales.data_ptr())
+
+        E, F, d, S, Fs = sh.E, sh.F, sh.d, sh.S, sh.Fs
+        w = B.moe_weights_t()
+        w.router_w = self.router_w.data_ptr()
+        w.router_b = self.router_b.data_ptr() if self.router_b is not None else None
+        w.gate = mat(inp.gate, E, F, d)
+        w.up = mat(inp.up, E, F, d)
+        w.down = mat(inp.down, E, d, F)
+        has_shared = S > 0 and inp.shared_gate is not None
+        if has_shared:
+            w.shared_gate = mat(inp.shared_gate, S, Fs, d)
+            w.shared_up = mat(inp.shared_up, S, Fs, d)
+            w.shared_down = mat(inp.shared_down, S, d, Fs)
+        self.weights = w
+        self.n_shared = S if has_shared else 0
+
+    def config(self, t_max: int, regime: int = B.MOE_REGIME_AUTO) -> B.moe_config_t:
+        sh = self.shape
+        return B.moe_config_t(t_max, sh.d, sh.F, sh.E, sh.k, self.n_shared,
+                              sh.Fs if self.n_shared else 0, sh.wfmt, regime,
+                              self.device.index or 0)
+
+    def weight_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in self._keep)
+
+
+def upload_x(x_bits: np.ndarray, device) -> torch.Tensor:
+    return _dev(x_bits, torch.device(device))
+
+
+class Routing:
+    """Device buffers for the routing tables moe_forward can copy out."""
+
+    def __init__(self, T: int, k: int, E: int, device):
+        dev = torch.device(device)
+        self.ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.slot_pair = torch.empty(T * k, dtype=torch.int32, device=dev)
+        self.struct = B.moe_routing_t(self.ids.data_ptr(), self.weights.data_ptr(),
+                                      self.counts.data_ptr(), self.offsets.data_ptr(),
+                                      self.slot_pair.data_ptr())
+
+    def numpy(self):
+        return (self.ids.cpu().numpy(), self.weights.cpu().numpy(), self.counts.cpu().numpy(),
+                self.offsets.cpu().numpy(), self.slot_pair.cpu().numpy())

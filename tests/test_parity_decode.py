@@ -1,0 +1,128 @@
+"""GPU parity of the decode regime (T <= 8): the C-ABI call against the fp64
+oracle on seeded inputs, at the full sizes of the decode workloads and at
+small shapes that cover ragged tails, k = E, E = 1, several shared experts
+and T = 0."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_43_b200 import binding as B
+from mixture_experts_layer_43_b200 import device as D
+from mixture_experts_layer_43_b200 import synth
+
+from gpu_util import compare, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+W = synth.WORKLOADS
+SMALL = [
+    # ragged: d = 3 x 128 (partial stages), F = 3 slices of 32, Fs != F
+    synth.MoEShape("ragged_bf16", T=3, d=384, E=5, k=3, F=96, S=1, Fs=64),
+    synth.MoEShape("ragged_q4", T=3, d=384, E=5, k=3, F=96, S=1, Fs=64, wfmt=synth.WFMT_Q4_0),
+    synth.MoEShape("k_eq_E", T=2, d=256, E=4, k=4, F=64),
+    synth.MoEShape("one_expert", T=5, d=128, E=1, k=1, F=32),
+    synth.MoEShape("two_shared", T=6, d=256, E=16, k=2, F=64, S=2, Fs=96),
+    synth.MoEShape("two_shared_q4", T=7, d=256, E=16, k=2, F=64, S=2, Fs=96,
+                   wfmt=synth.WFMT_Q4_0),
+    synth.MoEShape("multi_unit", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512),
+    synth.MoEShape("multi_unit_q4", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512,
+                   wfmt=synth.WFMT_Q4_0),
+    synth.MoEShape("biased", T=8, d=512, E=64, k=6, F=128, S=2, Fs=128, zipf_bias=1.1),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _check(sh, seed=0, T=None):
+    inp = synth.make_inputs(sh, seed=seed)
+    layer = D.DeviceLayer(inp)
+    T = sh.T if T is None else T
+    out, routing, launches = run_gpu(layer, inp.x, T)
+    assert launches == 2
+    sub = synth.MoEInputs(sh, inp.x[:T], inp.router_w, inp.router_b, inp.gate, inp.up,
+                          inp.down, inp.shared_gate, inp.shared_up, inp.shared_down)
+    res = oracle.forward(sub)
+    return compare(sub, out, routing, res)
+
+
+@pytest.mark.parametrize("name", ["tiny_T4_d256_E8k2_F512", "a3b_T1_d2048_E256k8_F512_S1",
+                                  "a3b_q4_T1_d2048_E256k8_F512_S1",
+                                  "a3b_q4_T8_d2048_E256k8_F512_S1"])
+def test_decode_workloads_full_size(name):
+    err = _check(W[name])
+    print(f"{name}: rel L2 {err:.3e}")
+
+
+def test_decode_mixtral_full_size():
+    err = _check(W["mixtral_T8_d4096_E8k2_F14336"])
+    print(f"mixtral: rel L2 {err:.3e}")
+
+
+@pytest.mark.parametrize("sh", SMALL, ids=[s.name for s in SMALL])
+def test_decode_small_shapes(sh):
+    _check(sh, seed=1)
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 8])
+def test_decode_every_T(T):
+    _check(synth.MoEShape("tsweep", T=8, d=512, E=32, k=4, F=256, S=1, Fs=256), seed=2, T=T)
+
+
+def test_decode_T0_enqueues_nothing():
+    sh = synth.MoEShape("t0", T=1, d=256, E=4, k=2, F=64)
+    inp = synth.make_inputs(sh)
+    layer = D.DeviceLayer(inp)
+    plan = B.moe_plan_create(layer.config(4))
+    try:
+        out = torch.full((1, sh.d), 7.0, device="cuda")
+        x = D.upload_x(inp.x, "cuda")
+        B.moe_forward(plan, layer.weights, x.data_ptr(), 0, out.data_ptr())
+        assert B.moe_last_launch_count(plan) == 0
+        torch.cuda.synchronize()
+        assert torch.all(out == 7.0)
+    finally:
+        B.moe_plan_destroy(plan)
+
+
+def test_decode_repeatable():
+    """Routing is bitwise repeatable; the output differs at most by the order
+    of the fp32 atomic additions of the combine."""
+    sh = synth.MoEShape("rep", T=8, d=1024, E=32, k=4, F=512, S=1, Fs=512)
+    inp = synth.make_inputs(sh, seed=4)
+    layer = D.DeviceLayer(inp)
+    plan = B.moe_plan_create(layer.config(8))
+    try:
+        o1, r1, _ = run_gpu(layer, inp.x, 8, plan=plan)
+        o2, r2, _ = run_gpu(layer, inp.x, 8, plan=plan)
+    finally:
+        B.moe_plan_destroy(plan)
+    for a, b in zip(r1, r2):
+        assert np.array_equal(a, b)
+    assert np.max(np.abs(o1 - o2)) <= 1e-5 * np.max(np.abs(o1))
+
+
+def test_decode_invalid_call_enqueues_nothing():
+    sh = synth.MoEShape("bad", T=2, d=256, E=4, k=2, F=64)
+    inp = synth.make_inputs(sh)
+    layer = D.DeviceLayer(inp)
+    plan = B.moe_plan_create(layer.config(2))
+    try:
+        x = D.upload_x(inp.x, "cuda")
+        out = torch.zeros((2, sh.d), device="cuda")
+        with pytest.raises(B.MoeError) as e:
+            B.moe_forward(plan, layer.weights, x.data_ptr(), 3, out.data_ptr())   # T > t_max
+        assert e.value.status == B.MOE_ERR_INVALID_ARG
+        with pytest.raises(B.MoeError):
+            B.moe_forward(plan, layer.weights, x.data_ptr() + 2, 2, out.data_ptr())  # misaligned
+        w = B.moe_weights_t()
+        w.router_w = layer.weights.router_w
+        with pytest.raises(B.MoeError):
+            B.moe_forward(plan, w, x.data_ptr(), 2, out.data_ptr())          # missing weights
+        assert B.moe_get_device_status(plan) == B.MOE_OK
+    finally:
+        B.moe_plan_destroy(plan)
