@@ -229,17 +229,19 @@ def run_b200(args, sh):
                                 device_id=dev)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
 
-    # layer instances: enough distinct weights that every step reads cold HBM
-    per_inst = synth.weight_bytes_per_expert(sh) * sh.E + (
-        synth.weight_bytes_per_expert(sh, sh.Fs) * sh.S if sh.S else 0)
-    n_inst = args.instances or max(1, min(32, -(-4 * L2_BYTES // per_inst)))
-    insts = []
+    # layer instances: distinct device copies, enough of them that the
+    # weights one step reads are cold in L2 (>= 4x L2 over the rotation)
     base = synth.make_inputs(sh, seed=args.seed)
     layers = [D.DeviceLayer(base, device=str(dev))]
-    for i in range(1, n_inst):
-        inp_i = synth.make_inputs(sh, seed=args.seed + 1000 * i)
-        layers.append(D.DeviceLayer(inp_i, device=str(dev)))
-        del inp_i
+    E_act = sh.E * (1.0 - (1.0 - sh.k / sh.E) ** sh.T)
+    active_est = (E_act * synth.weight_bytes_per_expert(sh) + sh.S * (
+        synth.weight_bytes_per_expert(sh, sh.Fs) if sh.S else 0) + sh.E * sh.d * 4)
+    per_inst = layers[0].weight_bytes() + sh.E * sh.d * 4
+    n_inst = args.instances or int(min(128, max(1, -(-4 * L2_BYTES // int(active_est)))))
+    n_inst = max(1, min(n_inst, int(60e9 // per_inst)))
+    for _ in range(1, n_inst):
+        layers.append(layers[0].clone())
+    torch.cuda.synchronize(dev)
     T = sh.T
     x = D.upload_x(base.x, dev)
     out = torch.empty((T, sh.d), dtype=torch.float32, device=dev)

@@ -68,6 +68,25 @@ class DeviceLayer:
         self.weights = w
         self.n_shared = S if has_shared else 0
 
+    def clone(self) -> "DeviceLayer":
+        """Same values at new device addresses (a distinct instance for
+        timing with cold caches)."""
+        c = DeviceLayer.__new__(DeviceLayer)
+        c.shape, c.device, c.q4, c.n_shared = self.shape, self.device, self.q4, self.n_shared
+        c.router_w = self.router_w.clone()
+        c.router_b = None if self.router_b is None else self.router_b.clone()
+        c._keep = [t.clone() for t in self._keep]
+        remap = {t.data_ptr(): n.data_ptr() for t, n in zip(self._keep, c._keep)}
+        w = B.moe_weights_t()
+        w.router_w = c.router_w.data_ptr()
+        w.router_b = c.router_b.data_ptr() if c.router_b is not None else None
+        for name in ("gate", "up", "down", "shared_gate", "shared_up", "shared_down"):
+            m = getattr(self.weights, name)
+            setattr(w, name, B.moe_matrix_t(remap.get(m.data) if m.data else None,
+                                            remap.get(m.scales) if m.scales else None))
+        c.weights = w
+        return c
+
     def config(self, t_max: int, regime: int = B.MOE_REGIME_AUTO) -> B.moe_config_t:
         sh = self.shape
         return B.moe_config_t(t_max, sh.d, sh.F, sh.E, sh.k, self.n_shared,

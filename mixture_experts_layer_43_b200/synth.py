@@ -73,6 +73,10 @@ WORKLOADS = {
     "a3b_q4_T8_d2048_E256k8_F512_S1": MoEShape(
         "a3b_q4_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512,
         S=1, Fs=512, wfmt=WFMT_Q4_0),
+    # A smaller case of the Mixtral-shaped decode kernel (same T, d, E, k;
+    # F cut to 2048 so the whole layer is 0.4 GB) for detailed profiling.
+    "mixtral_small_T8_d4096_E8k2_F2048": MoEShape(
+        "mixtral_small_T8_d4096_E8k2_F2048", T=8, d=4096, E=8, k=2, F=2048),
     "deepseek_T4096_d2048_E64k6_F1408_S2": MoEShape(
         "deepseek_T4096_d2048_E64k6_F1408_S2", T=4096, d=2048, E=64, k=6,
         F=1408, S=2, Fs=1408, zipf_bias=1.1),
