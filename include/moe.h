@@ -153,6 +153,31 @@ moe_status_t moe_route(moe_plan_t plan, const moe_weights_t* w,
 moe_status_t moe_experts(moe_plan_t plan, const moe_weights_t* w,
                          const void* x, int32_t T, float* out, void* stream);
 
+/* moe_route_noalloc: moe_route for callers that cannot allocate device
+ * memory (no plan needed).  The source pages have no counterpart to this
+ * entry point; it exists for host programs that may not call cudaMalloc
+ * while they serve a batch -- engines that forbid allocations on their hot
+ * path, plugin interfaces whose enqueue step may only launch work, code that
+ * runs while the allocator is locked.
+ * It runs the decode-regime router kernel with its scratch (fp32 logits,
+ * ticket, work list, slot maps, error word) in a 64 KiB file-scope device
+ * array of the library instead of a plan workspace; it calls no cudaMalloc,
+ * cudaFree or other allocating routine.  Each GPU that loads the library
+ * holds that array until the process exits.
+ * Inputs: cfg (d_model, n_experts, top_k, n_shared as for moe_plan_create;
+ * t_max, d_ff, wfmt, regime and device are ignored), w->router_w/router_b,
+ * x [T][d] bf16.  Outputs: out [T][d] zero-filled, and every member of
+ * `routing` (all five required) filled as moe_routing_get would.
+ * 0 <= T <= MOE_DECODE_MAX_T; a larger T returns MOE_ERR_INVALID_ARG (the
+ * scratch array holds at most that many tokens).  Runs on the current
+ * device.  The first call on a device resolves the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call on a device shares the one array, so calls whose work overlaps
+ * on the GPU race: serialise them. */
+moe_status_t moe_route_noalloc(const moe_config_t* cfg, const moe_weights_t* w,
+                               const void* x, int32_t T, float* out,
+                               moe_routing_t* routing, void* stream);
+
 /* Copy the routing tables of the last moe_route/moe_forward (T tokens) from
  * the workspace to `routing` (device pointers; NULL members skipped). */
 moe_status_t moe_routing_get(moe_plan_t plan, int32_t T, moe_routing_t* routing,

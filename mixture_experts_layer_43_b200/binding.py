@@ -88,6 +88,9 @@ def lib() -> ctypes.CDLL:
     for name in ("moe_route", "moe_experts"):
         getattr(L, name).argtypes = [P, ctypes.POINTER(moe_weights_t), P, I32, P, P]
         getattr(L, name).restype = S
+    L.moe_route_noalloc.argtypes = [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t),
+                                    P, I32, P, ctypes.POINTER(moe_routing_t), P]
+    L.moe_route_noalloc.restype = S
     L.moe_routing_get.argtypes = [P, I32, ctypes.POINTER(moe_routing_t), P]
     L.moe_routing_get.restype = S
     L.moe_last_launch_count.argtypes = [P]
@@ -142,6 +145,13 @@ def moe_route(plan: int, w: moe_weights_t, x: int, T: int, out: int, stream: int
 
 def moe_experts(plan: int, w: moe_weights_t, x: int, T: int, out: int, stream: int = 0) -> None:
     _check(lib().moe_experts(plan, ctypes.byref(w), x, T, out, stream), "moe_experts")
+
+
+def moe_route_noalloc(cfg: moe_config_t, w: moe_weights_t, x: int, T: int, out: int,
+                      routing: moe_routing_t, stream: int = 0) -> None:
+    """moe_route without a plan: scratch in the library's static device array."""
+    _check(lib().moe_route_noalloc(ctypes.byref(cfg), ctypes.byref(w), x, T, out,
+                                   ctypes.byref(routing), stream), "moe_route_noalloc")
 
 
 def moe_routing_get(plan: int, T: int, routing: moe_routing_t, stream: int = 0) -> None:
