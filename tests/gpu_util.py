@@ -7,7 +7,11 @@ Acceptance (the contract of the layer):
     that fp32 and fp64 may order differently);
   * counts, offsets and the slot order bit-exact against the oracle's
     bucketing of the GPU's own ids (they are a pure function of the ids);
-  * routing weights within 1e-6 absolute;
+  * routing weights within relative 16*sqrt(d)*2^-24: the GPU sums the d
+    products of a logit in fp32, whose rounding error grows like sqrt(d)*2^-24
+    times the partial sums (|partial sums| <~ 1 here), and a renormalised
+    weight's relative error is the difference of two such logit errors; the
+    factor 16 is the margin (observed <= 4.2e-6 at d = 2048, bound 4.3e-5);
   * out within relative L2 2e-3 (bf16 weights) or 5e-3 (Q4_0 weights),
     over all tokens whose ids matched.
 """
@@ -23,7 +27,12 @@ from mixture_experts_layer_43_b200 import synth
 
 TOL = {synth.WFMT_BF16: 2e-3, synth.WFMT_Q4_0: 5e-3}
 GAP_REL = 1e-5
-W_ABS = 1e-6
+W_ABS = 1e-7
+
+
+def w_rtol(d: int) -> float:
+    """Relative tolerance of the renormalised routing weights (see above)."""
+    return 16.0 * np.sqrt(d) * 2.0 ** -24
 
 
 def run_gpu(layer: D.DeviceLayer, x_bits: np.ndarray, T: int, regime=B.MOE_REGIME_AUTO,
@@ -76,7 +85,7 @@ def compare(inp: synth.MoEInputs, gpu_out, routing, oracle_res, tokens=None, tol
         f"expert ids differ on non-tied tokens {np.where(~ok_ids & ~waived)[0].tolist()}")
     for t in range(len(tok)):                     # ids valid and distinct everywhere
         assert len(set(g_ids[t].tolist())) == sh.k and g_ids[t].min() >= 0 and g_ids[t].max() < sh.E
-    np.testing.assert_allclose(g_w[ok_ids], o_w[ok_ids], rtol=0, atol=W_ABS)
+    np.testing.assert_allclose(g_w[ok_ids], o_w[ok_ids], rtol=w_rtol(sh.d), atol=W_ABS)
     # buckets are a pure function of the ids: compare with the oracle's
     if tokens is None:
         c, o, sp = oracle.buckets(ids.astype(np.int32), sh.E)
