@@ -22,11 +22,17 @@ struct moe_plan_s {
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     int route_epc = 1;
     int last_launches = 0;
-    // tensor maps of the last weights seen by the decode regime
-    bool maps_valid = false;
-    moe_weights_t maps_w{};
-    int maps_fs = 0;
-    DecodeArgs dargs{};
+    // tensor maps of the weights seen by the decode regime (small cache, so a
+    // caller that rotates several layers' weights does not re-encode them)
+    static constexpr int kMapCache = 64;
+    struct MapEntry {
+        bool valid = false;
+        int fs = 0;
+        moe_weights_t w{};
+        DecodeArgs args{};
+    };
+    MapEntry maps[kMapCache];
+    int maps_next = 0;
     // prefill regime state (tensor maps of the last weights/x)
     PrefillState* pf = nullptr;
 };
@@ -175,10 +181,14 @@ int pick_fs(const moe_plan_s* p, int T) {
     return best;
 }
 
-moe_status_t build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
-    if (p->maps_valid && p->maps_fs == fs && same_weights(p->maps_w, *w)) return MOE_OK;
+DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
+    for (auto& e : p->maps)
+        if (e.valid && e.fs == fs && same_weights(e.w, *w)) return &e.args;
+    auto& ent = p->maps[p->maps_next];
+    p->maps_next = (p->maps_next + 1) % moe_plan_s::kMapCache;
+    ent.valid = false;
     const moe_config_t& c = p->cfg;
-    DecodeArgs& a = p->dargs;
+    DecodeArgs& a = ent.args;
     memset(&a, 0, sizeof(a));
     const int64_t E = c.n_experts, d = c.d_model, F = c.d_ff, S = c.n_shared, Fs = c.d_ff_shared;
     bool ok = true;
@@ -208,14 +218,11 @@ moe_status_t build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
             ok &= map_q4_scales(p, &a.tm_sdown_sc, w->shared_down.scales, S, d, Fs, 128, nb);
         }
     }
-    if (!ok) {
-        p->maps_valid = false;
-        return MOE_ERR_INVALID_ARG;
-    }
-    p->maps_valid = true;
-    p->maps_w = *w;
-    p->maps_fs = fs;
-    return MOE_OK;
+    if (!ok) return nullptr;
+    ent.valid = true;
+    ent.w = *w;
+    ent.fs = fs;
+    return &a;
 }
 
 moe_status_t route_decode(moe_plan_s* p, const moe_weights_t* w, const void* x, int T, float* out,
@@ -240,9 +247,9 @@ moe_status_t experts_decode(moe_plan_s* p, const moe_weights_t* w, const void* x
     const moe_config_t& c = p->cfg;
     const bool q4 = c.wfmt == MOE_WFMT_Q4_0;
     const int fs = pick_fs(p, T);
-    moe_status_t s = build_decode_maps(p, w, fs);
-    if (s) return s;
-    DecodeArgs& a = p->dargs;
+    DecodeArgs* ap = build_decode_maps(p, w, fs);
+    if (!ap) return MOE_ERR_INVALID_ARG;
+    DecodeArgs& a = *ap;
     a.x = static_cast<const uint16_t*>(x);
     a.out = out;
     a.items = p->ws.items;
@@ -339,8 +346,9 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     // workspace: one allocation, carved into 256-byte aligned pieces
     const int64_t T = cfg->t_max, E = cfg->n_experts, k = cfg->top_k, d = cfg->d_model;
     const int64_t S = cfg->n_shared, Fs = cfg->d_ff_shared, F = cfg->d_ff;
-    const bool prefill = cfg->regime != MOE_REGIME_DECODE && cfg->wfmt == MOE_WFMT_BF16 &&
-                         cfg->t_max > MOE_DECODE_MAX_T;
+    const bool prefill = cfg->wfmt == MOE_WFMT_BF16 &&
+                         (cfg->regime == MOE_REGIME_PREFILL ||
+                          (cfg->regime == MOE_REGIME_AUTO && cfg->t_max > MOE_DECODE_MAX_T));
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 255) & ~size_t(255); return o; };
     const size_t o_logits = take(T * E * 4), o_ids = take(T * k * 4), o_wts = take(T * k * 4);
@@ -353,7 +361,7 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
         o_xp = take(T * k * d * 2);
         o_hr = take(T * k * F * 2);
         o_hs = take(T * S * Fs * 2);
-        o_tiles = take(prefill_tile_capacity(cfg) * sizeof(int32_t) * 4);
+        o_tiles = take(prefill_tile_capacity(cfg) * sizeof(int32_t));
         o_nt = take(64);
     }
     p->ws_bytes = off;

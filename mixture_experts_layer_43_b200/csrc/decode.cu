@@ -401,12 +401,15 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
     uint32_t it = 0;
     int prev_item = -1;
 
+    // warp-uniform: the ldmatrix / mma.sync that follow are warp-collective
     auto wait_full = [&](int slot, uint32_t parity) -> bool {
-        if (*abort_flag) return false;
-        if (mbar_wait_bounded(&full[slot], parity)) return true;
-        atomicOr(a.err, kErrTimeout);
-        *abort_flag = 1;
-        return false;
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], parity));
+        if (!ok && lane == 0) {
+            atomicOr(a.err, kErrTimeout);
+            *abort_flag = 1;
+        }
+        return ok;
     };
 
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
@@ -619,9 +622,18 @@ size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages) {
 template <int FS, bool Q4>
 static cudaError_t launch_one(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
     auto* k = decode_experts_kernel<FS, Q4>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    // the dynamic shared memory limit is raised once per device (and again
+    // only if a later launch needs more)
+    static int set_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || set_bytes[dev] < static_cast<int>(smem)) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) set_bytes[dev] = static_cast<int>(smem);
+    }
     k<<<grid, kDecodeThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
