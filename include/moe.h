@@ -65,10 +65,12 @@ typedef enum moe_wfmt {
     MOE_WFMT_Q4_0 = 1
 } moe_wfmt_t;
 
-/* Execution regime.  AUTO picks DECODE for T <= MOE_DECODE_MAX_T and
- * PREFILL otherwise.  DECODE streams every active expert's weights once in a
- * single persistent launch (CUDA cores + mma.sync, fused combine).  PREFILL
- * runs the grouped GEMMs on tcgen05 tensor cores (bf16 only). */
+/* Execution regime.  AUTO picks DECODE for T <= MOE_DECODE_MAX_T (and for
+ * every T with Q4_0 weights, up to MOE_DECODE_MAX_T) and PREFILL otherwise.
+ * DECODE streams every active expert's weights once, through a TMA ring,
+ * with the <= 8 tokens of an expert as the N side of mma.sync and the
+ * weighted combine fused.  PREFILL runs grouped GEMMs on tcgen05 tensor
+ * cores with accumulators in tensor memory (bf16 only). */
 typedef enum moe_regime {
     MOE_REGIME_AUTO = 0,
     MOE_REGIME_DECODE = 1,
@@ -79,12 +81,14 @@ typedef enum moe_regime {
 
 typedef struct moe_config {
     int32_t t_max;        /* largest T any forward call will pass */
-    int32_t d_model;      /* d; multiple of 64 */
-    int32_t d_ff;         /* F, routed expert hidden size; multiple of 32 */
+    int32_t d_model;      /* d; multiple of 128 */
+    int32_t d_ff;         /* F, routed expert hidden size; multiple of 32
+                             (of 64 for the prefill regime) */
     int32_t n_experts;    /* E >= 1 routed experts (<= 1024) */
     int32_t top_k;        /* 1 <= k <= min(E, 16) */
     int32_t n_shared;     /* S >= 0 shared experts (<= 8) */
-    int32_t d_ff_shared;  /* Fs, hidden size of each shared expert (0 if S=0) */
+    int32_t d_ff_shared;  /* Fs, hidden size of each shared expert (0 if S=0);
+                             same multiples as d_ff */
     int32_t wfmt;         /* moe_wfmt_t */
     int32_t regime;       /* moe_regime_t */
     int32_t device;       /* CUDA device ordinal the plan lives on */
@@ -123,9 +127,9 @@ typedef struct moe_plan_s* moe_plan_t;
 /* Validate `cfg`, select the device, size and allocate the plan workspace
  * for cfg->t_max tokens and resolve the driver's tensor-map encoder.  On
  * success *out receives the plan; on failure *out is NULL and nothing is
- * left allocated.  Allocates device memory (the only call that does, apart
- * from none).  Errors: INVALID_ARG (shape limits above), UNSUPPORTED
- * (PREFILL regime with Q4_0, or a device that is not sm_100), CUDA, OOM. */
+ * left allocated.  This is the only entry point that allocates device
+ * memory.  Errors: INVALID_ARG (shape limits above), UNSUPPORTED (PREFILL
+ * regime with Q4_0, or a device that is not sm_100), CUDA, OOM. */
 moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out);
 
 /* Free the plan's workspace.  The caller must make sure no work enqueued
@@ -136,18 +140,23 @@ void moe_plan_destroy(moe_plan_t plan);
  * x [T][d] bf16, out [T][d] fp32 (overwritten), 0 <= T <= t_max.
  * `routing` may be NULL; when given, the routing tables are copied to it
  * (device-to-device, on `stream`).  T = 0 enqueues nothing.
- * Launches: 2 kernels in the decode regime (router+buckets, experts), 5 in
- * the prefill regime (router, buckets+gather, gate/up GEMM, down GEMM with
- * fused combine, plus a zero-fill of `out`). */
+ * Launches: decode regime -- 1 cooperative kernel (router, top-k, buckets,
+ * every routed and shared expert, weighted combine; a grid barrier separates
+ * routing from the experts); if the device cannot co-schedule that grid, the
+ * two-launch path of moe_route + moe_experts.  Prefill regime -- 4 kernels
+ * (router, bucket scatter + row gather, gate/up GEMM, down GEMM with the
+ * weighted combine).  Work enqueued with one plan must not overlap on the
+ * GPU with other work of the same plan (they share the workspace). */
 moe_status_t moe_forward(moe_plan_t plan, const moe_weights_t* w,
                          const void* x, int32_t T, float* out,
                          moe_routing_t* routing, void* stream);
 
-/* The two halves of moe_forward, for callers that time them separately.
- * moe_route: router, top-k, buckets and work list into the plan's
- * workspace; also zero-fills `out`.  moe_experts: expert FFNs and the
- * weighted combine into `out`, reading the workspace moe_route wrote with
- * the same T.  moe_forward == moe_route then moe_experts. */
+/* The same layer as moe_forward in two steps, for callers that time or
+ * schedule them separately.  moe_route: router, top-k, buckets and work
+ * list into the plan's workspace; also zero-fills `out` (decode: 1 kernel;
+ * prefill: 2, including the gather of x rows per expert).  moe_experts:
+ * expert FFNs and the weighted combine into `out`, reading what moe_route
+ * wrote with the same T (decode: 1 kernel; prefill: 2 GEMM kernels). */
 moe_status_t moe_route(moe_plan_t plan, const moe_weights_t* w,
                        const void* x, int32_t T, float* out, void* stream);
 moe_status_t moe_experts(moe_plan_t plan, const moe_weights_t* w,

@@ -21,6 +21,7 @@ struct moe_plan_s {
     size_t ws_bytes = 0;
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
     int route_epc = 1;
+    bool coop = false;          // cooperative launches available (fused decode kernel)
     int last_launches = 0;
     // tensor maps of the weights seen by the decode regime (small cache, so a
     // caller that rotates several layers' weights does not re-encode them)
@@ -242,8 +243,9 @@ moe_status_t route_decode(moe_plan_s* p, const moe_weights_t* w, const void* x, 
     return cuda_status(launch_decode_route(r, st));
 }
 
-moe_status_t experts_decode(moe_plan_s* p, const moe_weights_t* w, const void* x, int T, float* out,
-                            cudaStream_t st) {
+// Fill the per-call fields of the decode arguments; returns the smem bytes.
+moe_status_t decode_args(moe_plan_s* p, const moe_weights_t* w, const void* x, int T, float* out,
+                         bool fused, DecodeArgs** out_args, int* out_fs, size_t* out_smem) {
     const moe_config_t& c = p->cfg;
     const bool q4 = c.wfmt == MOE_WFMT_Q4_0;
     const int fs = pick_fs(p, T);
@@ -264,14 +266,47 @@ moe_status_t experts_decode(moe_plan_s* p, const moe_weights_t* w, const void* x
     a.E = c.n_experts;
     a.S = c.n_shared;
     a.xs_stride = c.d_model * 2 + 16;
-    const size_t fixed = decode_smem_bytes(fs, q4, c.d_model, 0);
+    a.wr = w->router_w;
+    a.br = w->router_b;
+    a.k = c.top_k;
+    a.ws = p->ws;
+    a.gbar = p->ws.gbar;
+    const size_t extra = fused ? decode_fused_extra_smem() : 0;
+    const size_t fixed = decode_smem_bytes(fs, q4, c.d_model, 0) + extra;
     const int stage = decode_stage_bytes(fs, q4);
     int ns = static_cast<int>((p->smem_optin - fixed) / (stage + 16));
     if (ns > 8) ns = 8;
     if (ns < 2) return MOE_ERR_UNSUPPORTED;
+    // the fused kernel keeps the T x E logits in the ring during routing
+    if (fused && static_cast<size_t>(ns) * stage < static_cast<size_t>(T) * c.n_experts * 4)
+        return MOE_ERR_UNSUPPORTED;
     a.n_stages = ns;
-    const size_t smem = decode_smem_bytes(fs, q4, c.d_model, ns);
-    return cuda_status(launch_decode_experts(a, fs, q4, p->num_sms, smem, st));
+    *out_args = ap;
+    *out_fs = fs;
+    *out_smem = decode_smem_bytes(fs, q4, c.d_model, ns) + extra;
+    return MOE_OK;
+}
+
+moe_status_t experts_decode(moe_plan_s* p, const moe_weights_t* w, const void* x, int T, float* out,
+                            cudaStream_t st) {
+    DecodeArgs* a = nullptr;
+    int fs = 0;
+    size_t smem = 0;
+    moe_status_t s = decode_args(p, w, x, T, out, false, &a, &fs, &smem);
+    if (s) return s;
+    return cuda_status(launch_decode_experts(*a, fs, p->cfg.wfmt == MOE_WFMT_Q4_0, p->num_sms,
+                                             smem, st));
+}
+
+moe_status_t forward_decode_fused(moe_plan_s* p, const moe_weights_t* w, const void* x, int T,
+                                  float* out, cudaStream_t st) {
+    DecodeArgs* a = nullptr;
+    int fs = 0;
+    size_t smem = 0;
+    moe_status_t s = decode_args(p, w, x, T, out, true, &a, &fs, &smem);
+    if (s) return s;
+    return cuda_status(launch_decode_fused(*a, fs, p->cfg.wfmt == MOE_WFMT_Q4_0, p->num_sms, smem,
+                                           st));
 }
 
 moe_status_t copy_routing(moe_plan_s* p, int T, moe_routing_t* r, cudaStream_t st) {
@@ -342,6 +377,10 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     int epc = 1;
     while (epc < 8 && (cfg->n_experts + epc - 1) / epc > sms) epc *= 2;
     p->route_epc = epc;
+    int coop = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, cfg->device) != cudaSuccess)
+        coop = 0;
+    p->coop = coop != 0;
 
     // workspace: one allocation, carved into 256-byte aligned pieces
     const int64_t T = cfg->t_max, E = cfg->n_experts, k = cfg->top_k, d = cfg->d_model;
@@ -355,7 +394,7 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     const size_t o_counts = take(E * 4), o_offsets = take((E + 1) * 4);
     const size_t o_sp = take(T * k * 4), o_st = take(T * k * 4), o_sw = take(T * k * 4);
     const size_t o_items = take((E + S) * sizeof(WorkItem)), o_nitems = take(16);
-    const size_t o_ticket = take(16), o_err = take(16);
+    const size_t o_ticket = take(16), o_err = take(16), o_gbar = take(16);
     size_t o_xp = 0, o_hr = 0, o_hs = 0, o_tiles = 0, o_nt = 0;
     if (prefill) {
         o_xp = take(T * k * d * 2);
@@ -384,6 +423,7 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     w.n_items = reinterpret_cast<int32_t*>(b + o_nitems);
     w.ticket = reinterpret_cast<uint32_t*>(b + o_ticket);
     w.err = reinterpret_cast<uint32_t*>(b + o_err);
+    w.gbar = reinterpret_cast<uint32_t*>(b + o_gbar);
     if (prefill) {
         w.x_perm = reinterpret_cast<uint16_t*>(b + o_xp);
         w.h_routed = reinterpret_cast<uint16_t*>(b + o_hr);
@@ -458,15 +498,31 @@ moe_status_t moe_experts(moe_plan_t p, const moe_weights_t* w, const void* x, in
 
 moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const void* x, int32_t T, float* out,
                          moe_routing_t* routing, void* stream) {
-    moe_status_t s = moe_route(p, w, x, T, out, stream);
+    moe_status_t s = check_call(p, w, x, T, out);
+    if (s) return s;
+    p->last_launches = 0;
+    if (T == 0) return MOE_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (use_decode(p, T) && p->coop) {
+        DeviceGuard dg(p->cfg.device);
+        s = forward_decode_fused(p, w, x, T, out, st);
+        if (s == MOE_OK) {
+            p->last_launches = 1;
+            if (routing) s = copy_routing(p, T, routing, st);
+            return s;
+        }
+        if (s != MOE_ERR_UNSUPPORTED) return s;
+        // fall through to the two-launch path (same kernels, separate router)
+    }
+    s = moe_route(p, w, x, T, out, stream);
     if (s) return s;
     const int l1 = p->last_launches;
     s = moe_experts(p, w, x, T, out, stream);
     if (s) return s;
     p->last_launches += l1;
-    if (routing && T > 0) {
+    if (routing) {
         DeviceGuard dg(p->cfg.device);
-        s = copy_routing(p, T, routing, static_cast<cudaStream_t>(stream));
+        s = copy_routing(p, T, routing, st);
     }
     return s;
 }

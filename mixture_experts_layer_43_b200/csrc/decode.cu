@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kRouteThreads) decode_route_kernel(const Route
         const int chunk = d / wpe;
         const int i_end = (part + 1) * chunk;
         const float* wrow = a.wr + static_cast<size_t>(e) * d;
+        // unrolled so that several router rows' loads are in flight at once
+#pragma unroll 4
         for (int i = part * chunk + lane * 4; i < i_end; i += 128) {
             const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + i));
 #pragma unroll
@@ -115,30 +117,11 @@ __global__ void __launch_bounds__(kRouteThreads) decode_route_kernel(const Route
     }
     __syncthreads();
 
-    // top-k per token: warp t; a taken expert is marked NaN
+    // top-k per token: warp t (register-resident logits, see warp_topk)
     if (warp < T) {
         const int t = warp;
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int be = INT_MAX;
-            for (int x = lane; x < E; x += 32) {
-                const float v = s_log[t][x];
-                if (!isnan(v) && (v > bv || (v == bv && x < be))) { bv = v; be = x; }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-            }
-            if (lane == 0) {
-                if (be >= E) { atomicOr(a.ws.err, kErrBadId); be = 0; }
-                s_ids[t * k + j] = be;
-                s_sel[t][j] = bv;
-                s_log[t][be] = NAN;
-            }
-            __syncwarp();
-        }
+        warp_topk_any(s_log[t], E, k, &s_ids[t * k], s_sel[t], a.ws.err);
+        __syncwarp();
         // renormalised softmax over the selected logits == softmax over all E
         // experts restricted to the top-k and renormalised
         if (lane < k) {
@@ -265,48 +248,78 @@ __device__ __forceinline__ uint32_t q4_pair(uint32_t w, int s) {
     return *reinterpret_cast<uint32_t*>(&b);
 }
 
+// Work list the experts pipeline reads: generic pointers, so the same code
+// serves the two-launch path (global memory, written by the router kernel)
+// and the fused kernel (shared memory, computed by every CTA itself).
+struct WorkView {
+    int n_routed, n_shared;
+    const WorkItem* items;        // routed items (ascending expert), then shared items
+    const int32_t* slot_token;    // slot -> token
+    const float* slot_w;          // slot -> routing weight
+};
+
+// Shared-memory carve-up of the experts pipeline.
+struct DecodeSmem {
+    uint8_t* ring;
+    uint8_t* xs;
+    float* gu;
+    __nv_bfloat16* hhi;
+    __nv_bfloat16* hlo;
+    DecodeSmemTail* tail;
+    uint64_t* full;
+    uint64_t* empty;
+};
+
 template <int FS, bool Q4>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
-decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
+__device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const DecodeArgs& a) {
     using C = DecodeCfg<FS, Q4>;
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    DecodeSmem sm;
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    sm.ring = smem;
+    sm.xs = sm.ring + static_cast<size_t>(a.n_stages) * C::STAGE;
+    sm.gu = reinterpret_cast<float*>(sm.xs + kDecodeTok * a.xs_stride);   // [KSPLIT][2][FS][8]
+    sm.hhi = reinterpret_cast<__nv_bfloat16*>(sm.gu + C::KSPLIT * 2 * FS * kDecodeTok);
+    sm.hlo = sm.hhi + kDecodeTok * C::HS;
+    sm.tail = reinterpret_cast<DecodeSmemTail*>(sm.hlo + kDecodeTok * C::HS);
+    sm.full = reinterpret_cast<uint64_t*>(sm.tail + 1);
+    sm.empty = sm.full + a.n_stages;
+    return sm;
+}
+
+// The expert stage: work units are (expert, slice of FS hidden rows), shared
+// experts' units first, then the routed experts' in ascending expert order;
+// CTA b takes units b, b + gridDim.x, ...  Warp 8 (lane 0) is the TMA
+// producer, warps 0-7 consume.  Barriers must be initialised by the caller.
+template <int FS, bool Q4>
+__device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const DecodeSmem& sm,
+                                                 const WorkView& wv) {
+    using C = DecodeCfg<FS, Q4>;
     const int ns = a.n_stages;
-    uint8_t* ring = smem;
-    uint8_t* xs = ring + static_cast<size_t>(ns) * C::STAGE;
-    float* gu = reinterpret_cast<float*>(xs + kDecodeTok * a.xs_stride);  // [KSPLIT][2][FS][8]
-    __nv_bfloat16* hhi = reinterpret_cast<__nv_bfloat16*>(gu + C::KSPLIT * 2 * FS * kDecodeTok);
-    __nv_bfloat16* hlo = hhi + kDecodeTok * C::HS;
-    DecodeSmemTail* tail = reinterpret_cast<DecodeSmemTail*>(hlo + kDecodeTok * C::HS);
-    uint64_t* full = reinterpret_cast<uint64_t*>(tail + 1);
-    uint64_t* empty = full + ns;
+    uint8_t* ring = sm.ring;
+    uint8_t* xs = sm.xs;
+    float* gu = sm.gu;
+    __nv_bfloat16* hhi = sm.hhi;
+    __nv_bfloat16* hlo = sm.hlo;
+    DecodeSmemTail* tail = sm.tail;
+    uint64_t* full = sm.full;
+    uint64_t* empty = sm.empty;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int d = a.d, E = a.E;
-    if (tid == 0) {
-        for (int s = 0; s < ns; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kConsumerWarps);
-        }
-        tail->abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    const int n_routed = a.n_items[0], n_shared = a.n_items[1];
+    const int n_routed = wv.n_routed, n_shared = wv.n_shared;
     const int sl_r = a.F / FS, sl_s = a.S ? a.Fs / FS : 0;
-    const int n_units = n_routed * sl_r + n_shared * sl_s;
+    const int n_su = n_shared * sl_s;
+    const int n_units = n_su + n_routed * sl_r;
     const int nA = Q4 ? (d / 32 + C::KB - 1) / C::KB : (d + C::KT - 1) / C::KT;
     const int nB = (d + C::RJ - 1) / C::RJ;
     volatile int* abort_flag = &tail->abort_flag;
 
-    // unit -> (item index, slice)
+    // unit -> (item index, slice): shared units first
     auto unit_item = [&](int u, int& ii, int& sl) {
-        if (u < n_routed * sl_r) { ii = u / sl_r; sl = u % sl_r; }
-        else { const int v = u - n_routed * sl_r; ii = n_routed + v / sl_s; sl = v % sl_s; }
+        if (u < n_su) { ii = n_routed + u / sl_s; sl = u % sl_s; }
+        else { const int v = u - n_su; ii = v / sl_r; sl = v % sl_r; }
     };
-
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
@@ -320,7 +333,7 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
                 int ii, sl;
                 unit_item(u, ii, sl);
-                const WorkItem item = a.items[ii];
+                const WorkItem item = wv.items[ii];
                 const bool shared = item.expert >= E;
                 const int ex = shared ? item.expert - E : item.expert;
                 const int Fh = shared ? a.Fs : a.F;
@@ -415,7 +428,7 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
         int ii, sl;
         unit_item(u, ii, sl);
-        const WorkItem item = a.items[ii];
+        const WorkItem item = wv.items[ii];
         const bool shared = item.expert >= E;
         const int ntok = min(item.count, kDecodeTok);
 
@@ -426,7 +439,7 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
                 float w = 0.f;
                 if (tid < ntok) {
                     if (shared) { t = tid; w = 1.f; }
-                    else { t = a.slot_token[item.slot_begin + tid]; w = a.slot_w[item.slot_begin + tid]; }
+                    else { t = wv.slot_token[item.slot_begin + tid]; w = wv.slot_w[item.slot_begin + tid]; }
                 }
                 tail->tok[tid] = t;
                 tail->w[tid] = w;
@@ -601,6 +614,238 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
     }
 }
 
+
+template <int FS, bool Q4>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const DecodeSmem sm = decode_smem<FS, Q4>(smem_raw, a);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < a.n_stages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], kConsumerWarps);
+        }
+        sm.tail->abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const WorkView wv{a.n_items[0], a.n_items[1], a.items, a.slot_token, a.slot_w};
+    experts_pipeline<FS, Q4>(a, sm, wv);
+}
+
+// ====================================================== fused decode ===
+// One cooperative launch for the whole layer (T <= 8):
+//   R  every CTA computes the router logits of experts b, b+G, ... (fp32 FMA,
+//      each dot product split over 8 warps and summed in a fixed order) and
+//      zero-fills its share of `out`;
+//   -  grid barrier (arrival counter + generation word, bounded wait);
+//   T  every CTA reads all T x E logits and computes the same top-k,
+//      renormalised weights, stable slots and work list in its own shared
+//      memory (no second barrier); CTA 0 also writes the routing tables;
+//   X  the experts pipeline, reading the work list from shared memory.
+// Compared with the two-launch path this removes the launch gap between
+// router and experts and the router kernel's last-CTA tail.
+constexpr int kFusedMaxPairs = kDecodeTok * kMaxTopK;   // 128
+constexpr int kFusedMaxItems = kFusedMaxPairs + kMaxShared;
+
+struct alignas(16) FusedRouteSmem {
+    WorkItem items[kFusedMaxItems];
+    int ids[kFusedMaxPairs];
+    float w[kFusedMaxPairs];
+    int slot_token[kFusedMaxPairs];
+    float slot_w[kFusedMaxPairs];
+    int lt[kFusedMaxPairs];
+    int cnt[kFusedMaxPairs];
+    int first[kFusedMaxPairs];
+    float sel[kDecodeTok][kMaxTopK];
+    int n_routed;
+    int pad[3];
+};
+
+size_t decode_fused_extra_smem() { return sizeof(FusedRouteSmem); }
+
+// Grid-wide barrier of a cooperative launch; thread 0 of each CTA calls it.
+__device__ __forceinline__ bool grid_barrier(uint32_t* gbar, uint32_t nblocks) {
+    volatile uint32_t* gen_p = gbar + 1;
+    const uint32_t gen = *gen_p;
+    __threadfence();
+    const uint32_t arrived = atomicAdd(gbar, 1u);
+    if (arrived == nblocks - 1) {
+        *gbar = 0u;                  // ready for the next launch
+        __threadfence();
+        atomicAdd(gbar + 1, 1u);
+        return true;
+    }
+    const uint64_t t0 = globaltimer_ns();
+    while (*gen_p == gen) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+        __nanosleep(64);
+    }
+    __threadfence();
+    return true;
+}
+
+template <int FS, bool Q4>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
+    using C = DecodeCfg<FS, Q4>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const DecodeSmem sm = decode_smem<FS, Q4>(smem_raw, a);
+    FusedRouteSmem* rs = reinterpret_cast<FusedRouteSmem*>(sm.empty + a.n_stages);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int T = a.T, d = a.d, E = a.E, k = a.k, S = a.S;
+    const int G = gridDim.x, b = blockIdx.x;
+    if (tid == 0) {
+        for (int s = 0; s < a.n_stages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], kConsumerWarps);
+        }
+        sm.tail->abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    // ---- R: logits of this CTA's experts; zero-fill of out
+    if (warp < kConsumerWarps) {
+        {
+            float4* o = reinterpret_cast<float4*>(a.out);
+            const int n4 = (T * d) >> 2;
+            for (int i = b * kConsumers + tid; i < n4; i += G * kConsumers)
+                o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float* part = reinterpret_cast<float*>(sm.ring);          // [n_loc][8 chunks][8 tok]
+        const int n_loc = (E - b + G - 1) / G;
+        const int chunk = d / kConsumerWarps;
+        for (int item = warp; item < n_loc * kConsumerWarps; item += kConsumerWarps) {
+            const int loc = item / kConsumerWarps, ch = item % kConsumerWarps;
+            const int e = b + loc * G;
+            float acc[kDecodeTok];
+#pragma unroll
+            for (int t = 0; t < kDecodeTok; ++t) acc[t] = 0.f;
+            const float* wrow = a.wr + static_cast<size_t>(e) * d;
+#pragma unroll 4
+            for (int i = ch * chunk + lane * 4; i < (ch + 1) * chunk; i += 128) {
+                const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + i));
+#pragma unroll
+                for (int t = 0; t < kDecodeTok; ++t) {
+                    if (t < T) {
+                        const uint2 xv = __ldg(reinterpret_cast<const uint2*>(
+                            a.x + static_cast<size_t>(t) * d + i));
+                        acc[t] = fmaf(__uint_as_float(xv.x << 16), wv.x, acc[t]);
+                        acc[t] = fmaf(__uint_as_float(xv.x & 0xffff0000u), wv.y, acc[t]);
+                        acc[t] = fmaf(__uint_as_float(xv.y << 16), wv.z, acc[t]);
+                        acc[t] = fmaf(__uint_as_float(xv.y & 0xffff0000u), wv.w, acc[t]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < kDecodeTok; ++t) {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+                    acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int t = 0; t < kDecodeTok; ++t) part[(loc * kConsumerWarps + ch) * kDecodeTok + t] = acc[t];
+            }
+        }
+        named_bar_sync(1, kConsumers);
+        for (int i = tid; i < n_loc * T; i += kConsumers) {
+            const int loc = i / T, t = i % T;
+            const int e = b + loc * G;
+            float v = 0.f;
+            for (int ch = 0; ch < kConsumerWarps; ++ch) v += part[(loc * kConsumerWarps + ch) * kDecodeTok + t];
+            if (a.br) v += a.br[e];
+            a.ws.logits[t * E + e] = v;
+        }
+    }
+    __syncthreads();
+    if (tid == 0 && !grid_barrier(a.gbar, G)) {
+        atomicOr(a.err, kErrTimeout);
+        sm.tail->abort_flag = 1;
+    }
+    __syncthreads();
+
+    // ---- T: routing, computed redundantly by every CTA
+    const int P = T * k;
+    if (warp < kConsumerWarps) {
+        float* lg = reinterpret_cast<float*>(sm.ring);            // [T][E]
+        for (int i = tid; i < T * E; i += kConsumers) {
+            float v = __ldcg(a.ws.logits + i);
+            if (isnan(v)) v = -INFINITY;
+            lg[i] = v;
+        }
+        named_bar_sync(1, kConsumers);
+        if (warp < T) {
+            const int t = warp;
+            warp_topk_any(lg + t * E, E, k, &rs->ids[t * k], rs->sel[t], a.err);
+            __syncwarp();
+            if (lane < k) {
+                const float m = rs->sel[t][0];
+                float den = 0.f;
+                for (int j = 0; j < k; ++j) den += expf(rs->sel[t][j] - m);
+                float wj = expf(rs->sel[t][lane] - m) / den;
+                if (!(m > -INFINITY)) wj = 1.f / k;
+                rs->w[t * k + lane] = wj;
+            }
+        }
+        named_bar_sync(1, kConsumers);
+        // stable slots: pairs with a smaller expert id come first, ties by pair index
+        for (int p = tid; p < P; p += kConsumers) {
+            const int e = rs->ids[p];
+            int lt = 0, before = 0, cnt = 0;
+            for (int q = 0; q < P; ++q) {
+                const int eq = rs->ids[q];
+                lt += eq < e;
+                cnt += eq == e;
+                before += (eq == e) & (q < p);
+            }
+            const int slot = lt + before;
+            rs->slot_token[slot] = p / k;
+            rs->slot_w[slot] = rs->w[p];
+            rs->lt[p] = lt;
+            rs->cnt[p] = cnt;
+            rs->first[p] = before == 0;
+            if (b == 0) {
+                a.ws.slot_pair[slot] = p;
+                a.ws.slot_token[slot] = p / k;
+                a.ws.slot_w[slot] = rs->w[p];
+                a.ws.ids[p] = e;
+                a.ws.wts[p] = rs->w[p];
+            }
+        }
+        named_bar_sync(1, kConsumers);
+        for (int p = tid; p < P; p += kConsumers) {
+            if (!rs->first[p]) continue;
+            const int e = rs->ids[p];
+            int idx = 0;
+            for (int q = 0; q < P; ++q) idx += rs->first[q] & (rs->ids[q] < e);
+            rs->items[idx] = WorkItem{e, rs->lt[p], rs->cnt[p], 0};
+        }
+        if (tid == 0) {
+            int n = 0;
+            for (int q = 0; q < P; ++q) n += rs->first[q];
+            rs->n_routed = n;
+            for (int s2 = 0; s2 < S; ++s2) rs->items[n + s2] = WorkItem{E + s2, -1, T, 0};
+        }
+        if (b == 0) {
+            for (int x = tid; x <= E; x += kConsumers) {
+                int lt = 0, cnt = 0;
+                for (int q = 0; q < P; ++q) {
+                    lt += rs->ids[q] < x;
+                    cnt += rs->ids[q] == x;
+                }
+                a.ws.offsets[x] = lt;
+                if (x < E) a.ws.counts[x] = cnt;
+            }
+        }
+    }
+    __syncthreads();
+    const WorkView wv{rs->n_routed, S, rs->items, rs->slot_token, rs->slot_w};
+    experts_pipeline<FS, Q4>(a, sm, wv);
+    (void)sizeof(C);
+}
+
 int decode_stage_bytes(int fs, bool q4) {
     if (q4) return 2 * 512 * 18;
     (void)fs;
@@ -636,6 +881,45 @@ static cudaError_t launch_one(const DecodeArgs& a, int grid, size_t smem, cudaSt
     }
     k<<<grid, kDecodeThreads, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <int FS, bool Q4>
+static cudaError_t launch_fused_one(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
+    auto* k = decode_fused_kernel<FS, Q4>;
+    static int set_bytes[64] = {0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || set_bytes[dev] < static_cast<int>(smem)) {
+        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) set_bytes[dev] = static_cast<int>(smem);
+    }
+    // cooperative: every CTA is resident at once, which the grid barrier needs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, a);
+}
+
+cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, bool q4, int grid, size_t smem,
+                                cudaStream_t stream) {
+    if (q4) {
+        if (fs == 64) return launch_fused_one<64, true>(a, grid, smem, stream);
+        if (fs == 32) return launch_fused_one<32, true>(a, grid, smem, stream);
+    } else {
+        if (fs == 64) return launch_fused_one<64, false>(a, grid, smem, stream);
+        if (fs == 32) return launch_fused_one<32, false>(a, grid, smem, stream);
+    }
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, bool q4, int grid, size_t smem,

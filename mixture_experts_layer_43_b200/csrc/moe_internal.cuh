@@ -9,7 +9,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/moe.h"
+#include "moe.h"
 
 namespace moe {
 
@@ -50,6 +50,7 @@ struct Workspace {
     int32_t* n_items;      // [2]: routed items, shared items
     uint32_t* ticket;      // last-CTA ticket of the decode router
     uint32_t* err;         // sticky device error word
+    uint32_t* gbar;        // grid barrier of the fused decode kernel: arrivals, generation
     // prefill
     uint16_t* x_perm;      // [t_max*k][d] bf16 rows gathered per slot
     uint16_t* h_routed;    // [t_max*k][F] bf16
@@ -88,6 +89,12 @@ struct DecodeArgs {
     int xs_stride;              // bytes per token row of the staged x
     int kt;                     // phase A: k columns (bf16) / block columns (Q4_0) per stage
     int rj;                     // phase B: output rows per stage
+    // fused single-launch path only: router inputs, routing tables, grid barrier
+    const float* wr;            // [E][d]
+    const float* br;            // [E] or nullptr
+    int k;
+    Workspace ws;
+    uint32_t* gbar;             // [0] arrivals, [1] generation
 };
 
 // Host launchers (decode.cu, q4_pack.cu).
@@ -95,6 +102,9 @@ cudaError_t launch_decode_route(const RouteArgs& a, cudaStream_t stream);
 cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, bool q4, int grid,
                                   size_t smem, cudaStream_t stream);
 size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages);
+cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, bool q4, int grid, size_t smem,
+                                cudaStream_t stream);
+size_t decode_fused_extra_smem();
 int decode_stage_bytes(int fs, bool q4);
 cudaError_t launch_q4_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
                              uint8_t* codes, uint16_t* scales, cudaStream_t stream);
@@ -311,6 +321,64 @@ __device__ __forceinline__ void tmem_ld_wait() {
 __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};"
                  ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
+}
+
+// --------------------------------------------------------- warp top-k
+// Top-k of one token's E logits (shared memory, E <= 32 * PER) by one warp.
+// Each lane keeps logits lane, lane+32, ... in registers; a bitmask marks the
+// ones already taken, so a round is a register scan plus one shuffle argmax.
+// Order: descending logit, equal logits -> lower expert index; NaN counts as
+// -inf.  Lane 0 writes ids[j] and the selected logits sel[j].
+template <int PER>
+__device__ __forceinline__ void warp_topk(const float* row, int E, int k, int* ids, float* sel,
+                                          uint32_t* err) {
+    const int lane = threadIdx.x & 31;
+    float v[PER];
+    uint32_t taken = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int x = lane + 32 * i;
+        float t = -INFINITY;
+        if (x < E) {
+            t = row[x];
+            if (isnan(t)) t = -INFINITY;
+        } else {
+            taken |= 1u << i;
+        }
+        v[i] = t;
+    }
+    for (int j = 0; j < k; ++j) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int x = lane + 32 * i;
+            if (!((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && x < bi))) { bv = v[i]; bi = x; }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if (bi >= E) {                 // cannot happen for k <= E; keep ids in range
+            if (lane == 0) atomicOr(err, kErrBadId);
+            bi = 0;
+        } else if ((bi & 31) == lane) {
+            taken |= 1u << (bi >> 5);
+        }
+        if (lane == 0) { ids[j] = bi; sel[j] = bv; }
+    }
+}
+
+// warp_topk with PER chosen from E at run time.
+__device__ __forceinline__ void warp_topk_any(const float* row, int E, int k, int* ids, float* sel,
+                                              uint32_t* err) {
+    if (E <= 32) warp_topk<1>(row, E, k, ids, sel, err);
+    else if (E <= 64) warp_topk<2>(row, E, k, ids, sel, err);
+    else if (E <= 128) warp_topk<4>(row, E, k, ids, sel, err);
+    else if (E <= 256) warp_topk<8>(row, E, k, ids, sel, err);
+    else warp_topk<32>(row, E, k, ids, sel, err);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -3,14 +3,14 @@
 // Four launches per layer call:
 //  1. prefill_router_kernel: router logits for 32 tokens per CTA with fp32
 //     FMAs, top-k with renormalised weights, the CTA's per-expert histogram,
-//     and the zero-fill of its rows of `out`.  The last CTA (ticket) turns
-//     the histograms into per-chunk bucket bases, the per-expert counts and
-//     exclusive offsets, and the tile tables of the two GEMMs.
+//     and the zero-fill of its rows of `out`.
 //     ("Fused MoE Triton kernel: 5 launches instead of 24" page, fused steps
 //     one and two.)
-//  2. prefill_scatter_kernel: stable slot of every (token, choice) pair
-//     (ascending token inside each expert) and the gather of x rows into
-//     expert-contiguous X_perm.
+//  2. prefill_scatter_kernel: every CTA reduces the histograms to its chunk's
+//     bucket base per expert (counts, exclusive offsets), gives each
+//     (token, choice) pair its stable slot (ascending token inside each
+//     expert) and gathers x rows into expert-contiguous X_perm; CTA 0 also
+//     writes counts, offsets and the tile tables of the two GEMMs.
 //  3. prefill_gemm_kernel<kGateUp>: grouped GEMM H = SiLU(X_perm Wg^T) *
 //     (X_perm Wu^T) over every expert's rows, plus the shared experts over
 //     all tokens, on tcgen05 tensor cores (fused step three).
@@ -36,7 +36,7 @@ namespace moe {
 
 constexpr int kChunkTok = 32;        // tokens per router / scatter CTA
 constexpr int kRouterThreads = 256;
-constexpr int kRouterKC = 32;        // d columns per router k-step
+constexpr int kRouterKC = 128;       // d columns per router k-chunk (double-buffered)
 constexpr int kRouterEC = 64;        // experts per router pass
 
 struct PrefillRouteArgs {
@@ -45,21 +45,35 @@ struct PrefillRouteArgs {
     const float* br;
     float* out;
     Workspace ws;
-    int32_t* hist;      // [n_chunks][E] counts, then bucket bases (in place)
+    int32_t* hist;      // [n_chunks][E] per-chunk expert counts
     int T, d, E, k, S, F, Fs;
 };
 
+size_t router_smem_bytes(int E) {
+    return static_cast<size_t>(kChunkTok) * E * 4 +                      // logits
+           2ull * kRouterKC * (kChunkTok + kRouterEC) * 4 +               // x, w chunks x2
+           (kChunkTok * kMaxTopK + E) * 4 +                               // ids, histogram
+           static_cast<size_t>(kChunkTok) * kMaxTopK * 4;                 // selected logits
+}
+
 // ============================================================ router ===
+// Logits of 32 tokens x 64 experts per pass with fp32 FMAs.  128-column
+// chunks of x (bf16 -> fp32) and of the router matrix are double-buffered in
+// shared memory (stored transposed, k-major), and the next chunk's global
+// loads are in flight while the current chunk is multiplied.  Each thread
+// owns 4 tokens x 4 experts (16 FMAs per two 128-bit shared loads, so the
+// FMA pipe rather than shared-memory bandwidth bounds the loop); the two
+// 128-thread halves of the CTA take the two 64-column halves of each chunk
+// and their partial sums are added in a fixed order at the end.
 __global__ void __launch_bounds__(kRouterThreads)
 prefill_router_kernel(const PrefillRouteArgs a) {
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     const int E = a.E, d = a.d, k = a.k, T = a.T;
     float* s_log = reinterpret_cast<float*>(sm_raw);                   // [32][E]
-    float* s_x = s_log + kChunkTok * E;                                 // [KC][32]
-    float* s_w = s_x + kRouterKC * kChunkTok;                           // [KC][64]
-    int* s_ids = reinterpret_cast<int*>(s_w + kRouterKC * kRouterEC);   // [32*k]
+    float* s_x = s_log + kChunkTok * E;                                 // [2][KC][32]
+    float* s_w = s_x + 2 * kRouterKC * kChunkTok;                       // [2][KC][64]
+    int* s_ids = reinterpret_cast<int*>(s_w + 2 * kRouterKC * kRouterEC); // [32*k]
     int* s_hist = s_ids + kChunkTok * kMaxTopK;                         // [E]
-    __shared__ uint32_t s_ticket;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int t0 = blockIdx.x * kChunkTok;
@@ -73,107 +87,122 @@ prefill_router_kernel(const PrefillRouteArgs a) {
     }
     for (int e = tid; e < E; e += kRouterThreads) s_hist[e] = 0;
 
-    // logits[32 tokens][E]: thread (ty, tx) owns tokens 2ty..2ty+1, experts 4tx..4tx+3
-    const int ty = tid >> 4, tx = tid & 15;
+    // loader roles: x -- token xt = tid % 32, 16 columns at xk = (tid / 32) * 16;
+    // w -- expert we = tid % 64, 32 columns at wk = (tid / 64) * 32
+    const int xt = tid & 31, xk = (tid >> 5) * 16;
+    const int we = tid & 63, wk = (tid >> 6) * 32;
+    // compute roles: k half kh, tokens 4*tt.., experts 4*te..
+    const int kh = tid >> 7, tt = (tid >> 4) & 7, te = tid & 15;
+    const int nkc = d / kRouterKC;
     for (int e0 = 0; e0 < E; e0 += kRouterEC) {
         const int ne = min(kRouterEC, E - e0);
-        float acc[2][4] = {};
-        for (int kc = 0; kc < d; kc += kRouterKC) {
-            __syncthreads();
-            {   // x chunk: 32 tokens x 32 columns, thread loads 4 bf16
-                const int t = tid >> 3, c = (tid & 7) * 4;
-                float v[4] = {0.f, 0.f, 0.f, 0.f};
-                if (t < nt) {
-                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(
-                        a.x + static_cast<size_t>(t0 + t) * d + kc + c));
-                    v[0] = __uint_as_float(u.x << 16);
-                    v[1] = __uint_as_float(u.x & 0xffff0000u);
-                    v[2] = __uint_as_float(u.y << 16);
-                    v[3] = __uint_as_float(u.y & 0xffff0000u);
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) s_x[(c + q) * kChunkTok + t] = v[q];
+        uint4 xr[2];
+        float4 wr4[8];
+        auto gload = [&](int kc) {
+            const int kb = kc * kRouterKC;
+            if (xt < nt) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    a.x + static_cast<size_t>(t0 + xt) * d + kb + xk);
+                xr[0] = __ldg(src);
+                xr[1] = __ldg(src + 1);
+            } else {
+                xr[0] = xr[1] = make_uint4(0u, 0u, 0u, 0u);
             }
-            {   // router chunk: 64 experts x 32 columns, thread loads 8 floats
-                const int e = tid >> 2, c = (tid & 3) * 8;
-                float4 w0 = make_float4(0.f, 0.f, 0.f, 0.f), w1 = w0;
-                if (e < ne) {
-                    const float* src = a.wr + static_cast<size_t>(e0 + e) * d + kc + c;
-                    w0 = __ldg(reinterpret_cast<const float4*>(src));
-                    w1 = __ldg(reinterpret_cast<const float4*>(src + 4));
-                }
-                const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            if (we < ne) {
+                const float4* src = reinterpret_cast<const float4*>(
+                    a.wr + static_cast<size_t>(e0 + we) * d + kb + wk);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) s_w[(c + q) * kRouterEC + e] = wv[q];
+                for (int q = 0; q < 8; ++q) wr4[q] = __ldg(src + q);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) wr4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            __syncthreads();
+        };
+        auto sstore = [&](int buf) {
+            float* xs = s_x + buf * kRouterKC * kChunkTok;
+            float* ws = s_w + buf * kRouterKC * kRouterEC;
+            const uint32_t xu[8] = {xr[0].x, xr[0].y, xr[0].z, xr[0].w,
+                                    xr[1].x, xr[1].y, xr[1].z, xr[1].w};
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                xs[(xk + 2 * q) * kChunkTok + xt] = __uint_as_float(xu[q] << 16);
+                xs[(xk + 2 * q + 1) * kChunkTok + xt] = __uint_as_float(xu[q] & 0xffff0000u);
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                ws[(wk + 4 * q + 0) * kRouterEC + we] = wr4[q].x;
+                ws[(wk + 4 * q + 1) * kRouterEC + we] = wr4[q].y;
+                ws[(wk + 4 * q + 2) * kRouterEC + we] = wr4[q].z;
+                ws[(wk + 4 * q + 3) * kRouterEC + we] = wr4[q].w;
+            }
+        };
+        float acc[4][4] = {};
+        __syncthreads();
+        gload(0);
+        sstore(0);
+        __syncthreads();
+        for (int kc = 0; kc < nkc; ++kc) {
+            const int buf = kc & 1;
+            if (kc + 1 < nkc) gload(kc + 1);           // in flight during the FMAs
+            const float* xs = s_x + buf * kRouterKC * kChunkTok + kh * (kRouterKC / 2) * kChunkTok;
+            const float* ws = s_w + buf * kRouterKC * kRouterEC + kh * (kRouterKC / 2) * kRouterEC;
 #pragma unroll 8
-            for (int kk = 0; kk < kRouterKC; ++kk) {
-                const float2 xv = *reinterpret_cast<const float2*>(&s_x[kk * kChunkTok + 2 * ty]);
-                const float4 wv = *reinterpret_cast<const float4*>(&s_w[kk * kRouterEC + 4 * tx]);
-                acc[0][0] = fmaf(xv.x, wv.x, acc[0][0]);
-                acc[0][1] = fmaf(xv.x, wv.y, acc[0][1]);
-                acc[0][2] = fmaf(xv.x, wv.z, acc[0][2]);
-                acc[0][3] = fmaf(xv.x, wv.w, acc[0][3]);
-                acc[1][0] = fmaf(xv.y, wv.x, acc[1][0]);
-                acc[1][1] = fmaf(xv.y, wv.y, acc[1][1]);
-                acc[1][2] = fmaf(xv.y, wv.z, acc[1][2]);
-                acc[1][3] = fmaf(xv.y, wv.w, acc[1][3]);
+            for (int kk = 0; kk < kRouterKC / 2; ++kk) {
+                const float4 xv = *reinterpret_cast<const float4*>(&xs[kk * kChunkTok + 4 * tt]);
+                const float4 wv = *reinterpret_cast<const float4*>(&ws[kk * kRouterEC + 4 * te]);
+                const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
+                const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], wa[j], acc[i][j]);
             }
+            if (kc + 1 < nkc) sstore(buf ^ 1);
+            __syncthreads();
         }
+        // the upper half hands its partial sums to the lower half (in s_w,
+        // free after the last chunk), which adds them in a fixed order
+        float* red = s_w;                                  // [128 threads][16]
+        if (kh == 1) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int e = 4 * tx + j;
-                if (e < ne) {
-                    float v = acc[i][j];
-                    if (a.br) v += a.br[e0 + e];
-                    if (isnan(v)) v = -INFINITY;
-                    s_log[(2 * ty + i) * E + e0 + e] = v;
+                for (int j = 0; j < 4; ++j) red[(i * 4 + j) * 128 + (tid - 128)] = acc[i][j];
+        }
+        __syncthreads();
+        if (kh == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int e = 4 * te + j;
+                    if (e < ne) {
+                        float v = acc[i][j] + red[(i * 4 + j) * 128 + tid];
+                        if (a.br) v += a.br[e0 + e];
+                        if (isnan(v)) v = -INFINITY;
+                        s_log[(4 * tt + i) * E + e0 + e] = v;
+                    }
                 }
-            }
-    }
-    __syncthreads();
-
-    // top-k per token (warp per token); taken experts are marked NaN
-    for (int t = warp; t < nt; t += kRouterThreads / 32) {
-        float* lg = s_log + t * E;
-        float sel0 = 0.f, selv[kMaxTopK];
-        int seli[kMaxTopK];
-        for (int j = 0; j < k; ++j) {
-            float bv = -INFINITY;
-            int be = INT_MAX;
-            for (int x = lane; x < E; x += 32) {
-                const float v = lg[x];
-                if (!isnan(v) && (v > bv || (v == bv && x < be))) { bv = v; be = x; }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-            }
-            if (be >= E) { be = 0; if (lane == 0) atomicOr(a.ws.err, kErrBadId); }
-            selv[j] = bv;
-            seli[j] = be;
-            __syncwarp();
-            if (lane == 0) lg[be] = NAN;
-            __syncwarp();
         }
-        sel0 = selv[0];
-        float den = 0.f;
-        for (int j = 0; j < k; ++j) den += expf(selv[j] - sel0);
+        __syncthreads();
+    }
+
+    // top-k per token (warp per token, register-resident logits)
+    for (int t = warp; t < nt; t += kRouterThreads / 32) {
+        int* ids = s_ids + t * k;
+        float* sel = reinterpret_cast<float*>(s_hist + E) + t * kMaxTopK;   // [32][16] scratch
+        warp_topk_any(s_log + t * E, E, k, ids, sel, a.ws.err);
+        __syncwarp();
         if (lane < k) {
-            float wj = 0.f;
-            for (int j = 0; j < k; ++j) if (j == lane) wj = expf(selv[j] - sel0) / den;
-            if (!(sel0 > -INFINITY)) wj = 1.f / k;
-            int ij = 0;
-            for (int j = 0; j < k; ++j) if (j == lane) ij = seli[j];
+            const float m = sel[0];
+            float den = 0.f;
+            for (int j = 0; j < k; ++j) den += expf(sel[j] - m);
+            float wj = expf(sel[lane] - m) / den;
+            if (!(m > -INFINITY)) wj = 1.f / k;
+            const int ij = ids[lane];
             const size_t p = static_cast<size_t>(t0 + t) * k + lane;
             a.ws.ids[p] = ij;
             a.ws.wts[p] = wj;
-            s_ids[t * k + lane] = ij;
             atomicAdd(&s_hist[ij], 1);
         }
     }
@@ -181,87 +210,101 @@ prefill_router_kernel(const PrefillRouteArgs a) {
     for (int e = tid; e < E; e += kRouterThreads)
         a.hist[static_cast<size_t>(blockIdx.x) * E + e] = s_hist[e];
 
-    // ---- last CTA: bucket bases, counts, offsets, tile tables
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_ticket = atomicAdd(a.ws.ticket, 1u);
-    __syncthreads();
-    if (s_ticket != gridDim.x - 1) return;
-    __threadfence();
-
-    const int nch = gridDim.x;
-    // per expert: totals and, in place, the prefix over earlier chunks
-    for (int e = tid; e < E; e += kRouterThreads) {
-        int run = 0;
-        for (int c = 0; c < nch; ++c) {
-            int* h = a.hist + static_cast<size_t>(c) * E + e;
-            const int v = __ldcg(h);
-            *h = run;
-            run += v;
-        }
-        s_hist[e] = run;        // count of expert e
-    }
-    __syncthreads();
-    // exclusive scan over experts of (count, gemm1 tiles, gemm2 tiles)
-    const int nt1 = (a.F + 127) / 128, nt2 = (d + 255) / 256;
-    // scratch reuse: s_ids holds 512 ints, s_x 1024, s_w 2048; E <= 256 here
-    int* s_off = s_ids;
-    int* s_tb1 = reinterpret_cast<int*>(s_x);
-    int* s_tb2 = reinterpret_cast<int*>(s_w);
-    if (tid == 0) {
-        int o = 0, b1 = 0, b2 = 0;
-        for (int e = 0; e < E; ++e) {
-            const int c = s_hist[e];
-            const int mt = (c + 127) / 128;
-            s_off[e] = o; s_tb1[e] = b1; s_tb2[e] = b2;
-            o += c; b1 += mt * nt1; b2 += mt * nt2;
-        }
-        s_off[E] = o; s_tb1[E] = b1; s_tb2[E] = b2;
-    }
-    __syncthreads();
-    for (int e = tid; e <= E; e += kRouterThreads) {
-        a.ws.offsets[e] = s_off[e];
-        a.ws.tiles[e] = s_tb1[e];
-        a.ws.tiles[E + 1 + e] = s_tb2[e];
-        if (e < E) a.ws.counts[e] = s_hist[e];
-    }
-    // chunk bases += expert offset
-    for (int i = tid; i < nch * E; i += kRouterThreads) a.hist[i] += s_off[i % E];
-    if (tid == 0) {
-        const int mts = (T + 127) / 128;
-        const int nts1 = a.S * ((a.Fs + 127) / 128);
-        a.ws.n_tiles[0] = s_tb1[E] + (a.S ? mts * nts1 : 0);
-        a.ws.n_tiles[1] = s_tb2[E] + (a.S ? mts * nt2 : 0);
-        a.ws.n_tiles[2] = s_tb1[E];
-        a.ws.n_tiles[3] = s_tb2[E];
-        if (s_off[E] != T * k) atomicOr(a.ws.err, kErrBadId);
-        *a.ws.ticket = 0u;
-    }
 }
 
 // ============================================================ scatter ===
 struct ScatterArgs {
     const uint16_t* x;
     Workspace ws;
-    const int32_t* hist;   // bucket bases per chunk
-    int T, d, E, k;
+    const int32_t* hist;   // [n_chunks][E] per-chunk expert counts
+    int T, d, E, k, S, F, Fs;
 };
 
-__global__ void __launch_bounds__(256) prefill_scatter_kernel(const ScatterArgs a) {
+constexpr int kScatterThreads = 256;
+
+__global__ void __launch_bounds__(kScatterThreads) prefill_scatter_kernel(const ScatterArgs a) {
     __shared__ int s_ids[kChunkTok * kMaxTopK];
     __shared__ int s_slot[kChunkTok * kMaxTopK];
+    __shared__ int s_tot[256], s_pre[256], s_off[257], s_wsum[kScatterThreads / 32];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = blockIdx.x * kChunkTok;
-    const int nt = min(kChunkTok, a.T - t0);
-    const int k = a.k, np = nt * k;
+    const int E = a.E, k = a.k, c0 = blockIdx.x, nch = gridDim.x;
+    const int t0 = c0 * kChunkTok;
+    const int nt = min(kChunkTok, a.T - t0), np = nt * k;
     const size_t p0 = static_cast<size_t>(t0) * k;
-    for (int i = tid; i < np; i += 256) s_ids[i] = a.ws.ids[p0 + i];
+
+    // per expert: total count and count in the chunks before this one;
+    // nseg threads per expert split the chunk range (E <= 256)
+    for (int e = tid; e < E; e += kScatterThreads) { s_tot[e] = 0; s_pre[e] = 0; }
+    for (int i = tid; i < np; i += kScatterThreads) s_ids[i] = a.ws.ids[p0 + i];
     __syncthreads();
-    for (int i = tid; i < np; i += 256) {
+    {
+        const int nseg = max(1, kScatterThreads / E);
+        const int e = tid % E, seg = tid / E;
+        if (seg < nseg && tid < nseg * E) {
+            const int per = (nch + nseg - 1) / nseg;
+            const int c_lo = seg * per, c_hi = min(nch, c_lo + per);
+            int tot = 0, pre = 0;
+#pragma unroll 8
+            for (int c = c_lo; c < c_hi; ++c) {
+                const int v = __ldg(a.hist + static_cast<size_t>(c) * E + e);
+                tot += v;
+                pre += (c < c0) ? v : 0;
+            }
+            atomicAdd(&s_tot[e], tot);
+            atomicAdd(&s_pre[e], pre);
+        }
+    }
+    __syncthreads();
+    // exclusive scan of the totals over experts (one expert per thread)
+    {
+        const int v = tid < E ? s_tot[tid] : 0;
+        int incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += u;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < warp; ++w) base += s_wsum[w];
+        if (tid < E) s_off[tid] = base + incl - v;
+        if (tid == kScatterThreads - 1) s_off[E] = base + incl;
+    }
+    __syncthreads();
+    if (c0 == 0) {
+        // counts, offsets and the GEMM tile tables (tile starts per expert)
+        const int nt1 = (a.F + 127) / 128, nt2 = (a.d + 255) / 256;
+        if (tid == 0) {
+            int b1 = 0, b2 = 0;
+            for (int e = 0; e < E; ++e) {
+                const int mt = (s_tot[e] + 127) / 128;
+                a.ws.tiles[e] = b1;
+                a.ws.tiles[E + 1 + e] = b2;
+                b1 += mt * nt1;
+                b2 += mt * nt2;
+            }
+            a.ws.tiles[E] = b1;
+            a.ws.tiles[2 * E + 1] = b2;
+            const int mts = (a.T + 127) / 128;
+            const int nts1 = a.S * ((a.Fs + 127) / 128);
+            a.ws.n_tiles[0] = b1 + (a.S ? mts * nts1 : 0);
+            a.ws.n_tiles[1] = b2 + (a.S ? mts * nt2 : 0);
+            a.ws.n_tiles[2] = b1;
+            a.ws.n_tiles[3] = b2;
+            if (s_off[E] != a.T * k) atomicOr(a.ws.err, kErrBadId);
+        }
+        for (int e = tid; e <= E; e += kScatterThreads) {
+            a.ws.offsets[e] = s_off[e];
+            if (e < E) a.ws.counts[e] = s_tot[e];
+        }
+    }
+    // stable slots: rank among the chunk's earlier pairs with the same expert
+    for (int i = tid; i < np; i += kScatterThreads) {
         const int e = s_ids[i];
         int rank = 0;
         for (int j = 0; j < i; ++j) rank += (s_ids[j] == e);
-        const int slot = a.hist[static_cast<size_t>(blockIdx.x) * a.E + e] + rank;
+        const int slot = s_off[e] + s_pre[e] + rank;
         s_slot[i] = slot;
         a.ws.slot_pair[slot] = static_cast<int>(p0) + i;
         a.ws.slot_token[slot] = t0 + i / k;
@@ -270,7 +313,7 @@ __global__ void __launch_bounds__(256) prefill_scatter_kernel(const ScatterArgs 
     __syncthreads();
     // gather x rows into X_perm (one warp per pair, 16 bytes per lane)
     const int cpr = a.d / 8;
-    for (int i = warp; i < np; i += 8) {
+    for (int i = warp; i < np; i += kScatterThreads / 32) {
         const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + i / k) * a.d);
         uint4* dst = reinterpret_cast<uint4*>(a.ws.x_perm + static_cast<size_t>(s_slot[i]) * a.d);
         for (int c = lane; c < cpr; c += 32) dst[c] = __ldg(src + c);
@@ -284,6 +327,7 @@ constexpr int kStageB = kBN * kBK * 2;             // 32 KB
 constexpr int kStageBytes = kStageA + kStageB;     // 48 KB
 constexpr int kGemmThreads = 192;                  // producer, MMA, 4 epilogue warps
 constexpr int kGateUp = 1, kDown = 2;
+constexpr int kEpiStage = 4 * 32 * 32 * 4;          // down epilogue staging, 4 KB per warp
 
 struct GemmArgs {
     CUtensorMap tmA_r, tmA_s;       // A: X_perm / x (gate-up), H_r / H_s (down)
@@ -375,7 +419,8 @@ prefill_gemm_kernel(const __grid_constant__ GemmArgs a) {
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
-    uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes);
+    float* stage_out = reinterpret_cast<float*>(ring + kStages * kStageBytes);   // 4 x [32][32]
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStages * kStageBytes + kEpiStage);
     uint64_t* empty = full + kStages;
     uint64_t* tfull = empty + kStages;
     uint64_t* tempty = tfull + 2;
@@ -518,26 +563,44 @@ prefill_gemm_kernel(const __grid_constant__ GemmArgs a) {
                     }
                 }
             } else {
+                // weighted combine: each thread scales its row, a warp stages its
+                // 32 rows x 32 columns (16-byte chunks XOR-swizzled by row, so
+                // both the row-wise writes and the column-wise reads are free of
+                // bank conflicts), then every reduction instruction adds whole
+                // 128-byte row segments (4 rows per instruction)
                 int tok = 0;
-                float w = 1.f;
+                float w = 0.f;
                 if (row_ok) {
-                    if (g.shared) tok = g.row0 + r;
+                    if (g.shared) { tok = g.row0 + r; w = 1.f; }
                     else { tok = a.slot_token[g.row0 + r]; w = a.slot_w[g.row0 + r]; }
                 }
-                float* orow = a.out + static_cast<size_t>(tok) * a.d + g.n0;
+                float* stg = stage_out + (warp - 2) * (32 * 32);
+                const int cc = lane & 7;
 #pragma unroll 1
                 for (int c = 0; c < kBN / 32; ++c) {
                     uint32_t yv[32];
                     tmem_ld32(taddr + 32 * c, yv);
                     tmem_ld_wait();
-                    if (row_ok && g.n0 + 32 * c < a.d) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            red_add_v4_f32(orow + 32 * c + 4 * i, w * __uint_as_float(yv[4 * i]),
-                                           w * __uint_as_float(yv[4 * i + 1]),
-                                           w * __uint_as_float(yv[4 * i + 2]),
-                                           w * __uint_as_float(yv[4 * i + 3]));
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(stg + lane * 32 + ((j ^ (lane & 7)) * 4)) =
+                            make_float4(w * __uint_as_float(yv[4 * j]), w * __uint_as_float(yv[4 * j + 1]),
+                                        w * __uint_as_float(yv[4 * j + 2]), w * __uint_as_float(yv[4 * j + 3]));
+                    __syncwarp();
+                    if (g.n0 + 32 * c < a.d) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int rr = 4 * i + (lane >> 3);
+                            const int tok_r = __shfl_sync(0xffffffffu, tok, rr);
+                            const bool ok_r = __shfl_sync(0xffffffffu, row_ok ? 1 : 0, rr) != 0;
+                            const float4 v =
+                                *reinterpret_cast<const float4*>(stg + rr * 32 + ((cc ^ (rr & 7)) * 4));
+                            if (ok_r)
+                                red_add_v4_f32(a.out + static_cast<size_t>(tok_r) * a.d + g.n0 + 32 * c + 4 * cc,
+                                               v.x, v.y, v.z, v.w);
+                        }
                     }
+                    __syncwarp();
                 }
             }
             tc_fence_before();
@@ -552,8 +615,8 @@ prefill_gemm_kernel(const __grid_constant__ GemmArgs a) {
 }
 
 size_t gemm_smem_bytes(int E) {
-    return 1024 + static_cast<size_t>(kStages) * kStageBytes + (2 * kStages + 4) * 8 + 16 +
-           static_cast<size_t>(E + 2) * 4;
+    return 1024 + static_cast<size_t>(kStages) * kStageBytes + kEpiStage + (2 * kStages + 4) * 8 +
+           16 + static_cast<size_t>(E + 2) * 4;
 }
 
 // ================================================================= host ===
@@ -624,8 +687,7 @@ moe_status_t prefill_route(PrefillState* st, const moe_config_t& c, const Worksp
     r.T = T; r.d = c.d_model; r.E = c.n_experts; r.k = c.top_k; r.S = c.n_shared;
     r.F = c.d_ff; r.Fs = c.n_shared ? c.d_ff_shared : 0;
     const int nch = (T + kChunkTok - 1) / kChunkTok;
-    const size_t smem = (kChunkTok * c.n_experts + kRouterKC * kChunkTok + kRouterKC * kRouterEC) * 4 +
-                        (kChunkTok * kMaxTopK + c.n_experts) * 4;
+    const size_t smem = router_smem_bytes(c.n_experts);
     static int set_smem = 0;
     if (static_cast<int>(smem) > set_smem) {
         if (cudaFuncSetAttribute(prefill_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -637,8 +699,8 @@ moe_status_t prefill_route(PrefillState* st, const moe_config_t& c, const Worksp
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     ScatterArgs sa{};
     sa.x = x; sa.ws = ws; sa.hist = st->hist; sa.T = T; sa.d = c.d_model; sa.E = c.n_experts;
-    sa.k = c.top_k;
-    prefill_scatter_kernel<<<nch, 256, 0, stream>>>(sa);
+    sa.k = c.top_k; sa.S = c.n_shared; sa.F = c.d_ff; sa.Fs = c.n_shared ? c.d_ff_shared : 0;
+    prefill_scatter_kernel<<<nch, kScatterThreads, 0, stream>>>(sa);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     *launches = 2;
     return MOE_OK;

@@ -61,6 +61,27 @@ def run_gpu(layer: D.DeviceLayer, x_bits: np.ndarray, T: int, regime=B.MOE_REGIM
             B.moe_plan_destroy(plan)
 
 
+def run_gpu_split(layer: D.DeviceLayer, x_bits: np.ndarray, T: int, regime=B.MOE_REGIME_AUTO):
+    """The same layer through moe_route + moe_experts (the two-launch path)."""
+    sh = layer.shape
+    plan = B.moe_plan_create(layer.config(max(T, 1), regime))
+    try:
+        x = D.upload_x(x_bits[:T], layer.device)
+        out = torch.full((T, sh.d), float("nan"), dtype=torch.float32, device=layer.device)
+        r = D.Routing(T, sh.k, sh.E, layer.device)
+        st = torch.cuda.current_stream(layer.device).cuda_stream
+        B.moe_route(plan, layer.weights, x.data_ptr(), T, out.data_ptr(), st)
+        n1 = B.moe_last_launch_count(plan)
+        B.moe_experts(plan, layer.weights, x.data_ptr(), T, out.data_ptr(), st)
+        n2 = B.moe_last_launch_count(plan)
+        B.moe_routing_get(plan, T, r.struct, st)
+        torch.cuda.synchronize(layer.device)
+        assert B.moe_get_device_status(plan) == B.MOE_OK
+        return out.cpu().numpy().astype(np.float64), r.numpy(), n1 + n2
+    finally:
+        B.moe_plan_destroy(plan)
+
+
 def waived_tokens(logits: np.ndarray, k: int) -> np.ndarray:
     """Tokens whose k-th / (k+1)-th oracle logits nearly tie."""
     T, E = logits.shape

@@ -11,7 +11,7 @@ from mixture_experts_layer_43_b200 import binding as B
 from mixture_experts_layer_43_b200 import device as D
 from mixture_experts_layer_43_b200 import synth
 
-from gpu_util import compare, run_gpu
+from gpu_util import compare, run_gpu, run_gpu_split
 
 pytestmark = pytest.mark.gpu
 
@@ -38,12 +38,18 @@ def _gpu():
         pytest.skip("needs a CUDA device")
 
 
-def _check(sh, seed=0, T=None):
+def _check(sh, seed=0, T=None, split=False):
+    """split=False: moe_forward (the single fused cooperative launch);
+    split=True: moe_route + moe_experts (router kernel, then experts kernel)."""
     inp = synth.make_inputs(sh, seed=seed)
     layer = D.DeviceLayer(inp)
     T = sh.T if T is None else T
-    out, routing, launches = run_gpu(layer, inp.x, T)
-    assert launches == 2
+    if split:
+        out, routing, launches = run_gpu_split(layer, inp.x, T)
+        assert launches == 2
+    else:
+        out, routing, launches = run_gpu(layer, inp.x, T)
+        assert launches == 1
     sub = synth.MoEInputs(sh, inp.x[:T], inp.router_w, inp.router_b, inp.gate, inp.up,
                           inp.down, inp.shared_gate, inp.shared_up, inp.shared_down)
     res = oracle.forward(sub)
@@ -66,6 +72,12 @@ def test_decode_mixtral_full_size():
 @pytest.mark.parametrize("sh", SMALL, ids=[s.name for s in SMALL])
 def test_decode_small_shapes(sh):
     _check(sh, seed=1)
+
+
+@pytest.mark.parametrize("sh", SMALL[:6] + [W["a3b_q4_T8_d2048_E256k8_F512_S1"]],
+                         ids=[s.name for s in SMALL[:6]] + ["a3b_q4_T8"])
+def test_decode_two_launch_path(sh):
+    _check(sh, seed=5, split=True)
 
 
 @pytest.mark.parametrize("T", [1, 2, 5, 8])
