@@ -148,6 +148,24 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+def reduce_max_over_ranks(values, device=None):
+    """Each value's maximum over all ranks: a multi-GPU job is as slow as its
+    slowest replica.  Identity without an initialised process group."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tokens_per_s(world_size: int, tokens_per_step: int, steps: int, t_max_ms: float) -> float:
+    """Whole-job throughput of `world_size` replicas that each ran `steps`
+    layer calls of `tokens_per_step` tokens in at most `t_max_ms`."""
+    return world_size * tokens_per_step * steps / (t_max_ms / 1e3)
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -368,17 +386,15 @@ def run_b200(args, sh):
         torch.cuda.synchronize(dev)
         e2e_ms = e_start.elapsed_time(e_end)
 
-    t_max = total_ms
-    e2e_max = e2e_ms
-    if ws > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([total_ms, e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max, e2e_max = float(tt[0]), float(tt[1])
+    t_max, e2e_max = reduce_max_over_ranks([total_ms, e2e_ms], device=dev)
     B.moe_plan_destroy(plan)
 
-    tokens_per_s = ws * T * K / (t_max / 1e3)
-    kern_avg_s = float(np.mean(kern_ms)) / 1e3
+    tokens_per_s = job_tokens_per_s(ws, T, K, t_max)
+    kern_evt_s = float(np.mean(kern_ms)) / 1e3
+    # A decode step is exactly one launch (the fused kernel), so its duration
+    # is the graph step time (event nodes around such short kernels add
+    # their own overhead); prefill: event nodes around the two GEMM launches.
+    kern_avg_s = kern_evt_s if prefill else min(kern_evt_s, total_ms / K / 1e3)
     alg_bytes = float(np.mean([act_bytes[i % n_inst] for i in range(K)]))
     alg_flops = float(np.mean([act_flops[i % n_inst] for i in range(K)]))
     if prefill:
@@ -405,6 +421,7 @@ def run_b200(args, sh):
                 "traffic": _profile_traffic("decode_fused_kernel", sh.name, src_sha),
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "kernel_ms_avg": kern_avg_s * 1e3,
+                "kernel_ms_event_nodes": kern_evt_s * 1e3,
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs, copy)"}
         l2 = ("inputs larger than L2: each step streams "
               f"{alg_bytes / 1e9:.3f} GB of distinct expert weights; "
@@ -425,7 +442,7 @@ def run_b200(args, sh):
                    "active_experts_per_step": float(np.mean(acts)),
                    "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
         "roofline": roof,
-        "e2e": {"value": ws * T * K2 / (e2e_max / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(ws, T, K2, e2e_max), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * sh.d * 2, "d2h_bytes_per_step": T * sh.d * 4},
         "gpu_launches": launches,
         "clocks": clocks,
@@ -441,6 +458,66 @@ def run_b200(args, sh):
     return 0
 
 
+def run_sweep(args):
+    """Achieved HBM bandwidth of the fused decode kernel against the bytes
+    one launch reads (the pages' bandwidth-vs-bytes-per-kernel measurement,
+    cold data): a T=8, d=4096, E=8, k=2 layer with F from 32 to 14336, each
+    point timed on a rotation of layer copies larger than 4x L2.  Prints one
+    JSON line per point."""
+    import torch
+    from mixture_experts_layer_43_b200 import binding as B
+    from mixture_experts_layer_43_b200 import device as D
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    hbm_gbs = _peaks()[0]
+    stream = torch.cuda.Stream(device=dev)
+    st = stream.cuda_stream
+    for F in (32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 14336):
+        sh = synth.MoEShape(f"sweep_F{F}", T=8, d=4096, E=8, k=2, F=F)
+        base, xb = D.random_bf16_layer(sh, seed=args.seed, device=str(dev))
+        x = D.upload_x(xb, dev)
+        out = torch.empty((sh.T, sh.d), dtype=torch.float32, device=dev)
+        plan = B.moe_plan_create(base.config(sh.T))
+        routing = D.Routing(sh.T, sh.k, sh.E, dev)
+        with torch.cuda.stream(stream):
+            B.moe_forward(plan, base.weights, x.data_ptr(), sh.T, out.data_ptr(), routing.struct, st)
+        stream.synchronize()
+        act, n_act = _active_bytes(sh, routing.counts.cpu().numpy(), 0)
+        act += sh.E * sh.d * 4
+        n_inst = int(min(256, max(1, -(-4 * L2_BYTES // act))))
+        n_inst = max(1, min(n_inst, int(40e9 // (base.weight_bytes() + 1))))
+        layers = [base] + [base.clone() for _ in range(n_inst - 1)]
+        S = n_inst * max(1, -(-64 // n_inst))
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), sh.T, out.data_ptr(), None, st)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(S):
+                    B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), sh.T,
+                                  out.data_ptr(), None, st)
+            g.replay()
+            stream.synchronize()
+            R = max(3, min(200, -(-args.steps // S)))
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(R):
+                g.replay()
+            b.record(stream)
+            stream.synchronize()
+        us = a.elapsed_time(b) * 1e3 / (R * S)
+        gbs = act / (us * 1e-6) / 1e9
+        print(json.dumps({"sweep": "bytes_per_launch", "F": F, "bytes_per_launch": act,
+                          "active_experts": n_act, "us_per_launch": us, "achieved_gbs": gbs,
+                          "frac_of_peak": gbs / hbm_gbs, "instances": n_inst}), flush=True)
+        del g
+        B.moe_plan_destroy(plan)
+        del layers, base
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -452,9 +529,13 @@ def main(argv=None):
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep-bytes", action="store_true",
+                    help="bandwidth vs bytes per launch of the decode kernel, one JSON line per point")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.sweep_bytes:
+        return run_sweep(args)
     sh = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, sh)

@@ -211,7 +211,7 @@ cudaError_t launch_decode_route(const RouteArgs& a, cudaStream_t stream) {
 }
 
 // ============================================================ experts ===
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumers + 32;   // + one producer warp
 
@@ -288,9 +288,10 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
 }
 
 // The expert stage: work units are (expert, slice of FS hidden rows), shared
-// experts' units first, then the routed experts' in ascending expert order;
-// CTA b takes units b, b + gridDim.x, ...  Warp 8 (lane 0) is the TMA
-// producer, warps 0-7 consume.  Barriers must be initialised by the caller.
+// experts' units first, then the routed experts' in ascending expert order
+// (assignment to CTAs: see experts_pipeline).  The last warp (lane 0) is the
+// TMA producer, the others consume.  Barriers must be initialised by the
+// caller.
 template <int FS, bool Q4>
 __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const DecodeSmem& sm,
                                                  const WorkView& wv) {
@@ -315,6 +316,18 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
     const int nB = (d + C::RJ - 1) / C::RJ;
     volatile int* abort_flag = &tail->abort_flag;
 
+    // Unit assignment.  When an expert has at least as many slices as there
+    // are CTAs, CTA b takes units b, b+G, ...: the CTAs stream neighbouring
+    // slices of one expert together and each keeps its x rows staged across
+    // units.  Otherwise CTA b takes the contiguous range [b*U/G, (b+1)*U/G),
+    // so that its consecutive units still share an expert.
+    const bool interleave = sl_r >= static_cast<int>(gridDim.x);
+    const int u_begin = interleave ? static_cast<int>(blockIdx.x)
+        : static_cast<int>((static_cast<long long>(blockIdx.x) * n_units) / gridDim.x);
+    const int u_end = interleave ? n_units
+        : static_cast<int>((static_cast<long long>(blockIdx.x + 1) * n_units) / gridDim.x);
+    const int u_step = interleave ? static_cast<int>(gridDim.x) : 1;
+
     // unit -> (item index, slice): shared units first
     auto unit_item = [&](int u, int& ii, int& sl) {
         if (u < n_su) { ii = n_routed + u / sl_s; sl = u % sl_s; }
@@ -330,7 +343,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             const uint64_t pol = l2_policy_evict_first();
             uint32_t it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            for (int u = u_begin; u < u_end && ok; u += u_step) {
                 int ii, sl;
                 unit_item(u, ii, sl);
                 const WorkItem item = wv.items[ii];
@@ -425,7 +438,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
         return ok;
     };
 
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+    for (int u = u_begin; u < u_end; u += u_step) {
         int ii, sl;
         unit_item(u, ii, sl);
         const WorkItem item = wv.items[ii];

@@ -36,8 +36,9 @@ namespace moe {
 
 constexpr int kChunkTok = 32;        // tokens per router / scatter CTA
 constexpr int kRouterThreads = 256;
-constexpr int kRouterKC = 128;       // d columns per router k-chunk (double-buffered)
+constexpr int kRouterKC = 64;        // d columns per router k-chunk (double-buffered)
 constexpr int kRouterEC = 64;        // experts per router pass
+constexpr int kRouterPitch = kRouterKC + 8;   // bf16 elements per smem row (conflict-free ldmatrix)
 
 struct PrefillRouteArgs {
     const uint16_t* x;
@@ -49,30 +50,34 @@ struct PrefillRouteArgs {
     int T, d, E, k, S, F, Fs;
 };
 
+constexpr int kRouterXTile = kChunkTok * kRouterPitch;          // bf16 elements
+constexpr int kRouterWTile = kRouterEC * kRouterPitch;          // bf16 elements, one part
+
 size_t router_smem_bytes(int E) {
     return static_cast<size_t>(kChunkTok) * E * 4 +                      // logits
-           2ull * kRouterKC * (kChunkTok + kRouterEC) * 4 +               // x, w chunks x2
+           2ull * (kRouterXTile + 3 * kRouterWTile) * 2 +                 // x, 3 w parts, x2
            (kChunkTok * kMaxTopK + E) * 4 +                               // ids, histogram
            static_cast<size_t>(kChunkTok) * kMaxTopK * 4;                 // selected logits
 }
 
 // ============================================================ router ===
-// Logits of 32 tokens x 64 experts per pass with fp32 FMAs.  128-column
-// chunks of x (bf16 -> fp32) and of the router matrix are double-buffered in
-// shared memory (stored transposed, k-major), and the next chunk's global
-// loads are in flight while the current chunk is multiplied.  Each thread
-// owns 4 tokens x 4 experts (16 FMAs per two 128-bit shared loads, so the
-// FMA pipe rather than shared-memory bandwidth bounds the loop); the two
-// 128-thread halves of the CTA take the two 64-column halves of each chunk
-// and their partial sums are added in a fixed order at the end.
+// Logits of 32 tokens x 64 experts per pass on the tensor cores, exactly as
+// accurate as fp32 arithmetic on the products: each fp32 router weight w is
+// split into three bf16 parts hi + mid + lo that sum to w exactly (each part
+// holds the next 8 significant bits), so every x*part product (bf16 x) is
+// exact in fp32 and mma.sync accumulates the three partial logits in fp32.
+// (TF32 would instead round w to 10 bits.)  64-column chunks of x and of
+// the split router matrix are double-buffered in shared memory; the next
+// chunk's global loads are in flight while the current one is multiplied.
+// Warp w handles tokens 16*(w/4).. and experts 16*(w%4)..  of the pass.
 __global__ void __launch_bounds__(kRouterThreads)
 prefill_router_kernel(const PrefillRouteArgs a) {
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     const int E = a.E, d = a.d, k = a.k, T = a.T;
     float* s_log = reinterpret_cast<float*>(sm_raw);                   // [32][E]
-    float* s_x = s_log + kChunkTok * E;                                 // [2][KC][32]
-    float* s_w = s_x + 2 * kRouterKC * kChunkTok;                       // [2][KC][64]
-    int* s_ids = reinterpret_cast<int*>(s_w + 2 * kRouterKC * kRouterEC); // [32*k]
+    __nv_bfloat16* s_x = reinterpret_cast<__nv_bfloat16*>(s_log + kChunkTok * E);   // [2][32][pitch]
+    __nv_bfloat16* s_w = s_x + 2 * kRouterXTile;                        // [2][3][64][pitch]
+    int* s_ids = reinterpret_cast<int*>(s_w + 2 * 3 * kRouterWTile);    // [32*k]
     int* s_hist = s_ids + kChunkTok * kMaxTopK;                         // [E]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -87,103 +92,107 @@ prefill_router_kernel(const PrefillRouteArgs a) {
     }
     for (int e = tid; e < E; e += kRouterThreads) s_hist[e] = 0;
 
-    // loader roles: x -- token xt = tid % 32, 16 columns at xk = (tid / 32) * 16;
-    // w -- expert we = tid % 64, 32 columns at wk = (tid / 64) * 32
-    const int xt = tid & 31, xk = (tid >> 5) * 16;
-    const int we = tid & 63, wk = (tid >> 6) * 32;
-    // compute roles: k half kh, tokens 4*tt.., experts 4*te..
-    const int kh = tid >> 7, tt = (tid >> 4) & 7, te = tid & 15;
+    // loader roles: x -- token tid/8, 8 columns at (tid%8)*8; w -- expert
+    // tid/4, 16 columns at (tid%4)*16
+    const int xt = tid >> 3, xk = (tid & 7) * 8;
+    const int we = tid >> 2, wk = (tid & 3) * 16;
+    const int tg = warp >> 2, eq = warp & 3;
+    const int g = lane >> 2, tig = lane & 3;
     const int nkc = d / kRouterKC;
     for (int e0 = 0; e0 < E; e0 += kRouterEC) {
         const int ne = min(kRouterEC, E - e0);
-        uint4 xr[2];
-        float4 wr4[8];
+        uint4 xr;
+        float4 wr4[4];
         auto gload = [&](int kc) {
             const int kb = kc * kRouterKC;
-            if (xt < nt) {
-                const uint4* src = reinterpret_cast<const uint4*>(
-                    a.x + static_cast<size_t>(t0 + xt) * d + kb + xk);
-                xr[0] = __ldg(src);
-                xr[1] = __ldg(src + 1);
-            } else {
-                xr[0] = xr[1] = make_uint4(0u, 0u, 0u, 0u);
-            }
+            xr = make_uint4(0u, 0u, 0u, 0u);
+            if (xt < nt)
+                xr = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + xt) * d + kb + xk));
             if (we < ne) {
                 const float4* src = reinterpret_cast<const float4*>(
                     a.wr + static_cast<size_t>(e0 + we) * d + kb + wk);
 #pragma unroll
-                for (int q = 0; q < 8; ++q) wr4[q] = __ldg(src + q);
+                for (int q = 0; q < 4; ++q) wr4[q] = __ldg(src + q);
             } else {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) wr4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int q = 0; q < 4; ++q) wr4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
             }
         };
         auto sstore = [&](int buf) {
-            float* xs = s_x + buf * kRouterKC * kChunkTok;
-            float* ws = s_w + buf * kRouterKC * kRouterEC;
-            const uint32_t xu[8] = {xr[0].x, xr[0].y, xr[0].z, xr[0].w,
-                                    xr[1].x, xr[1].y, xr[1].z, xr[1].w};
+            *reinterpret_cast<uint4*>(s_x + buf * kRouterXTile + xt * kRouterPitch + xk) = xr;
+            const float wf[16] = {wr4[0].x, wr4[0].y, wr4[0].z, wr4[0].w, wr4[1].x, wr4[1].y,
+                                  wr4[1].z, wr4[1].w, wr4[2].x, wr4[2].y, wr4[2].z, wr4[2].w,
+                                  wr4[3].x, wr4[3].y, wr4[3].z, wr4[3].w};
+            uint32_t hi[8], mid[8], lo[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                xs[(xk + 2 * q) * kChunkTok + xt] = __uint_as_float(xu[q] << 16);
-                xs[(xk + 2 * q + 1) * kChunkTok + xt] = __uint_as_float(xu[q] & 0xffff0000u);
+                float p0 = wf[2 * q], p1 = wf[2 * q + 1];
+                const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                p0 -= __low2float(h);                 // exact: fp32 minus its bf16 rounding
+                p1 -= __high2float(h);
+                const __nv_bfloat162 m = __floats2bfloat162_rn(p0, p1);
+                p0 -= __low2float(m);
+                p1 -= __high2float(m);
+                const __nv_bfloat162 l = __floats2bfloat162_rn(p0, p1);   // exact: <= 8 bits left
+                hi[q] = *reinterpret_cast<const uint32_t*>(&h);
+                mid[q] = *reinterpret_cast<const uint32_t*>(&m);
+                lo[q] = *reinterpret_cast<const uint32_t*>(&l);
             }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                ws[(wk + 4 * q + 0) * kRouterEC + we] = wr4[q].x;
-                ws[(wk + 4 * q + 1) * kRouterEC + we] = wr4[q].y;
-                ws[(wk + 4 * q + 2) * kRouterEC + we] = wr4[q].z;
-                ws[(wk + 4 * q + 3) * kRouterEC + we] = wr4[q].w;
-            }
+            __nv_bfloat16* wb = s_w + buf * 3 * kRouterWTile + we * kRouterPitch + wk;
+            uint4* d0 = reinterpret_cast<uint4*>(wb);
+            uint4* d1 = reinterpret_cast<uint4*>(wb + kRouterWTile);
+            uint4* d2 = reinterpret_cast<uint4*>(wb + 2 * kRouterWTile);
+            d0[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);   d0[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            d1[0] = make_uint4(mid[0], mid[1], mid[2], mid[3]); d1[1] = make_uint4(mid[4], mid[5], mid[6], mid[7]);
+            d2[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);   d2[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
         };
-        float acc[4][4] = {};
+        float acc[2][4] = {};
         __syncthreads();
         gload(0);
         sstore(0);
         __syncthreads();
         for (int kc = 0; kc < nkc; ++kc) {
             const int buf = kc & 1;
-            if (kc + 1 < nkc) gload(kc + 1);           // in flight during the FMAs
-            const float* xs = s_x + buf * kRouterKC * kChunkTok + kh * (kRouterKC / 2) * kChunkTok;
-            const float* ws = s_w + buf * kRouterKC * kRouterEC + kh * (kRouterKC / 2) * kRouterEC;
-#pragma unroll 8
-            for (int kk = 0; kk < kRouterKC / 2; ++kk) {
-                const float4 xv = *reinterpret_cast<const float4*>(&xs[kk * kChunkTok + 4 * tt]);
-                const float4 wv = *reinterpret_cast<const float4*>(&ws[kk * kRouterEC + 4 * te]);
-                const float xa[4] = {xv.x, xv.y, xv.z, xv.w};
-                const float wa[4] = {wv.x, wv.y, wv.z, wv.w};
+            if (kc + 1 < nkc) gload(kc + 1);           // in flight during the MMAs
+            const uint32_t xs = smem_u32(s_x + buf * kRouterXTile);
+            const uint32_t ws = smem_u32(s_w + buf * 3 * kRouterWTile);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+            for (int kk = 0; kk < kRouterKC / 16; ++kk) {
+                uint32_t a0, a1, a2, a3;
+                {
+                    const int m = lane >> 3, r = lane & 7;
+                    const int row = tg * 16 + ((m & 1) << 3) + r;
+                    ldsm_x4(xs + (row * kRouterPitch + kk * 16 + (m >> 1) * 8) * 2, a0, a1, a2, a3);
+                }
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(xa[i], wa[j], acc[i][j]);
+                for (int n8 = 0; n8 < 2; ++n8) {
+                    const int erow = eq * 16 + n8 * 8 + (lane & 7);
+                    const uint32_t boff = (erow * kRouterPitch + kk * 16 + ((lane >> 3) & 1) * 8) * 2;
+#pragma unroll
+                    for (int part = 0; part < 3; ++part) {
+                        uint32_t b0, b1;
+                        ldsm_x2(ws + part * kRouterWTile * 2 + boff, b0, b1);
+                        mma_bf16_16816(acc[n8], a0, a1, a2, a3, b0, b1);
+                    }
+                }
             }
             if (kc + 1 < nkc) sstore(buf ^ 1);
             __syncthreads();
         }
-        // the upper half hands its partial sums to the lower half (in s_w,
-        // free after the last chunk), which adds them in a fixed order
-        float* red = s_w;                                  // [128 threads][16]
-        if (kh == 1) {
+        // C fragment: rows (tokens) g, g+8; columns (experts) 2tig, 2tig+1
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
+        for (int n8 = 0; n8 < 2; ++n8)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) red[(i * 4 + j) * 128 + (tid - 128)] = acc[i][j];
-        }
-        __syncthreads();
-        if (kh == 0) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int e = 4 * te + j;
-                    if (e < ne) {
-                        float v = acc[i][j] + red[(i * 4 + j) * 128 + tid];
-                        if (a.br) v += a.br[e0 + e];
-                        if (isnan(v)) v = -INFINITY;
-                        s_log[(4 * tt + i) * E + e0 + e] = v;
-                    }
+            for (int q = 0; q < 4; ++q) {
+                const int t = tg * 16 + g + (q >> 1) * 8;
+                const int e = eq * 16 + n8 * 8 + 2 * tig + (q & 1);
+                if (e < ne) {
+                    float v = acc[n8][q];
+                    if (a.br) v += a.br[e0 + e];
+                    if (isnan(v)) v = -INFINITY;
+                    s_log[t * E + e0 + e] = v;
                 }
-        }
+            }
         __syncthreads();
     }
 

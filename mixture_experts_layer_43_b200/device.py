@@ -97,6 +97,44 @@ class DeviceLayer:
         return sum(t.numel() * t.element_size() for t in self._keep)
 
 
+def random_bf16_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") -> DeviceLayer:
+    """A bf16 layer whose router and x come from synth (same routing as
+    make_inputs with this seed) and whose expert weights are drawn on the
+    device from a seeded N(0, w_std) generator -- for timing sweeps where the
+    weight values do not matter and host generation would dominate."""
+    assert shape.wfmt == synth.WFMT_BF16
+    inp = synth.make_inputs(shape, seed=seed, x_only=True)
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+
+    def mats(n, rows, cols):
+        t = torch.randn((n, rows, cols), generator=gen, device=dev, dtype=torch.float32)
+        return (t * shape.w_std).to(torch.bfloat16).view(torch.int16)
+
+    L = DeviceLayer.__new__(DeviceLayer)
+    L.shape, L.device, L.q4 = shape, dev, False
+    L.router_w = _dev(inp.router_w.astype(np.float32), dev)
+    L.router_b = None if inp.router_b is None else _dev(inp.router_b.astype(np.float32), dev)
+    E, F, d, S, Fs = shape.E, shape.F, shape.d, shape.S, shape.Fs
+    L._keep = [mats(E, F, d), mats(E, F, d), mats(E, d, F)]
+    w = B.moe_weights_t()
+    w.router_w = L.router_w.data_ptr()
+    w.router_b = L.router_b.data_ptr() if L.router_b is not None else None
+    w.gate = B.moe_matrix_t(L._keep[0].data_ptr(), None)
+    w.up = B.moe_matrix_t(L._keep[1].data_ptr(), None)
+    w.down = B.moe_matrix_t(L._keep[2].data_ptr(), None)
+    L.n_shared = 0
+    if S:
+        L._keep += [mats(S, Fs, d), mats(S, Fs, d), mats(S, d, Fs)]
+        w.shared_gate = B.moe_matrix_t(L._keep[3].data_ptr(), None)
+        w.shared_up = B.moe_matrix_t(L._keep[4].data_ptr(), None)
+        w.shared_down = B.moe_matrix_t(L._keep[5].data_ptr(), None)
+        L.n_shared = S
+    L.weights = w
+    return L, inp.x
+
+
 def upload_x(x_bits: np.ndarray, device) -> torch.Tensor:
     return _dev(x_bits, torch.device(device))
 
