@@ -197,8 +197,20 @@ int32_t moe_last_launch_count(moe_plan_t plan);
 
 /* Read and clear the sticky device error word (synchronises `plan`'s device).
  * OK, DEVICE_FLAG (a kernel saw an out-of-range id or count) or TIMEOUT (a
- * bounded wait gave up). */
+ * bounded wait -- of a pipeline stage or the fused kernel's grid barrier --
+ * gave up, after at most 2 s; the kernel then skipped its remaining work, so
+ * that call's `out` is incomplete; the plan's barrier state is reset). */
 moe_status_t moe_get_device_status(moe_plan_t plan);
+
+/* Failure-path check (the pages have no counterpart): make the next fused
+ * decode launch of `plan` unable to pass its grid barrier, by writing an
+ * arrival count no launch can complete into the plan's barrier word (an
+ * async memset on `stream`).  That launch waits the bounded 2 s, skips its
+ * expert work, and exits; moe_get_device_status then returns
+ * MOE_ERR_TIMEOUT and resets the barrier, after which the plan works
+ * normally again.  Nothing hangs and nothing faults.  UNSUPPORTED if the
+ * device cannot run the fused (cooperative) launch. */
+moe_status_t moe_debug_stall_barrier(moe_plan_t plan, void* stream);
 
 /* Bytes of the packed Q4_0 form of n_mats matrices of [rows][k] weights.
  * k must be a multiple of 32.  Returns INVALID_ARG otherwise. */

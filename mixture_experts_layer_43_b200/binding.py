@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
     L.moe_last_launch_count.restype = I32
     L.moe_get_device_status.argtypes = [P]
     L.moe_get_device_status.restype = S
+    L.moe_debug_stall_barrier.argtypes = [P, P]
+    L.moe_debug_stall_barrier.restype = S
     L.moe_q4_0_packed_bytes.argtypes = [I64, I64, I64, ctypes.POINTER(ctypes.c_size_t),
                                         ctypes.POINTER(ctypes.c_size_t)]
     L.moe_q4_0_packed_bytes.restype = S
@@ -165,6 +167,10 @@ def moe_last_launch_count(plan: int) -> int:
 def moe_get_device_status(plan: int) -> int:
     """Raw status of the sticky device error word (not raised)."""
     return lib().moe_get_device_status(plan)
+
+
+def moe_debug_stall_barrier(plan: int, stream: int = 0) -> None:
+    _check(lib().moe_debug_stall_barrier(plan, stream), "moe_debug_stall_barrier")
 
 
 def moe_q4_0_packed_bytes(n_mats: int, rows: int, k: int):

@@ -543,9 +543,21 @@ moe_status_t moe_get_device_status(moe_plan_t p) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaMemcpy(&v, p->ws.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
     if (v && cudaMemset(p->ws.err, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
-    if (v & kErrTimeout) return MOE_ERR_TIMEOUT;
+    if (v & kErrTimeout) {
+        // a launch gave up waiting: leave the grid barrier words clean for the next one
+        if (cudaMemset(p->ws.gbar, 0, 16) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_ERR_TIMEOUT;
+    }
     if (v) return MOE_ERR_DEVICE_FLAG;
     return MOE_OK;
+}
+
+moe_status_t moe_debug_stall_barrier(moe_plan_t p, void* stream) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (!p->coop) return MOE_ERR_UNSUPPORTED;
+    DeviceGuard dg(p->cfg.device);
+    // an arrival count no launch can complete (each arrival adds 1)
+    return cuda_status(cudaMemsetAsync(p->ws.gbar, 0x40, 4, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_q4_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k, size_t* code_bytes,
