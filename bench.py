@@ -518,6 +518,59 @@ def run_sweep(args):
     return 0
 
 
+def run_sweep_t(args):
+    """Decode vs prefill regime on the 35B-A3B-shaped bf16 layer (d=2048,
+    E=256, k=8, F=512, 1 shared expert) for T = 1..8 (both regimes run
+    there) and the prefill regime for T = 16..256: time per layer call and
+    tokens/s, one JSON line per (regime, T), timed on rotated layer copies."""
+    import torch
+    from mixture_experts_layer_43_b200 import binding as B
+    from mixture_experts_layer_43_b200 import device as D
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    st = stream.cuda_stream
+    t_max = 256
+    sh = synth.MoEShape("a3b_sweep_T", T=t_max, d=2048, E=256, k=8, F=512, S=1, Fs=512)
+    base, xb = D.random_bf16_layer(sh, seed=args.seed, device=str(dev))
+    n_inst = 24
+    layers = [base] + [base.clone() for _ in range(n_inst - 1)]
+    x = D.upload_x(xb, dev)
+    out = torch.empty((t_max, sh.d), dtype=torch.float32, device=dev)
+    plans = {r: B.moe_plan_create(base.config(t_max if r == B.MOE_REGIME_PREFILL else 8, r))
+             for r in (B.MOE_REGIME_DECODE, B.MOE_REGIME_PREFILL)}
+    points = [(B.MOE_REGIME_DECODE, T) for T in range(1, 9)] + \
+             [(B.MOE_REGIME_PREFILL, T) for T in (1, 2, 4, 8, 16, 32, 64, 128, 256)]
+    for regime, T in points:
+        plan = plans[regime]
+        S = n_inst * 2
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, out.data_ptr(), None, st)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(S):
+                    B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, out.data_ptr(),
+                                  None, st)
+            g.replay()
+            stream.synchronize()
+            R = 20
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(R):
+                g.replay()
+            b.record(stream)
+            stream.synchronize()
+        us = a.elapsed_time(b) * 1e3 / (R * S)
+        print(json.dumps({"sweep": "tokens_per_call", "regime": "decode" if regime == 1 else "prefill",
+                          "T": T, "us_per_call": us, "tokens_per_s": T / (us * 1e-6)}), flush=True)
+        del g
+    for p in plans.values():
+        B.moe_plan_destroy(p)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -531,11 +584,15 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--sweep-bytes", action="store_true",
                     help="bandwidth vs bytes per launch of the decode kernel, one JSON line per point")
+    ap.add_argument("--sweep-t", action="store_true",
+                    help="decode vs prefill regime over tokens per call, one JSON line per point")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.sweep_bytes:
         return run_sweep(args)
+    if args.sweep_t:
+        return run_sweep_t(args)
     sh = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, sh)

@@ -510,17 +510,19 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         ldsm_x4(xs_u + (lane & 7) * a.xs_stride +
                                     ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2,
                                 b0, b1, b2, b3);
-                        float cb[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_bf16_16816(cb, q4_pair(w0, 0), q4_pair(w8, 0), q4_pair(w0, 4),
+                        // the block's two 16-wide halves go to independent
+                        // accumulators (no mma -> mma dependency inside a block)
+                        float cb0[4] = {0.f, 0.f, 0.f, 0.f}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_bf16_16816(cb0, q4_pair(w0, 0), q4_pair(w8, 0), q4_pair(w0, 4),
                                        q4_pair(w8, 4), b0, b1);
-                        mma_bf16_16816(cb, q4_pair(w0, 8), q4_pair(w8, 8), q4_pair(w0, 12),
+                        mma_bf16_16816(cb1, q4_pair(w0, 8), q4_pair(w8, 8), q4_pair(w0, 12),
                                        q4_pair(w8, 12), b2, b3);
                         const float s0 = __half2float(scl[bb * FS + r0]);
                         const float s8 = __half2float(scl[bb * FS + r0 + 8]);
-                        cacc[0] = fmaf(s0, cb[0], cacc[0]);
-                        cacc[1] = fmaf(s0, cb[1], cacc[1]);
-                        cacc[2] = fmaf(s8, cb[2], cacc[2]);
-                        cacc[3] = fmaf(s8, cb[3], cacc[3]);
+                        cacc[0] = fmaf(s0, cb0[0] + cb1[0], cacc[0]);
+                        cacc[1] = fmaf(s0, cb0[1] + cb1[1], cacc[1]);
+                        cacc[2] = fmaf(s8, cb0[2] + cb1[2], cacc[2]);
+                        cacc[3] = fmaf(s8, cb0[3] + cb1[3], cacc[3]);
                     }
                 }
             }
@@ -597,17 +599,18 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                             const uint32_t p1 = q4_pair(w0c, 4), q1 = q4_pair(w8c, 4);
                             const uint32_t p2 = q4_pair(w0c, 8), q2 = q4_pair(w8c, 8);
                             const uint32_t p3 = q4_pair(w0c, 12), q3 = q4_pair(w8c, 12);
-                            float cb[4] = {0.f, 0.f, 0.f, 0.f};
-                            mma_bf16_16816(cb, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1]);
-                            mma_bf16_16816(cb, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
-                            mma_bf16_16816(cb, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
-                            mma_bf16_16816(cb, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                            // two independent accumulator chains (halves of the block)
+                            float cb0[4] = {0.f, 0.f, 0.f, 0.f}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+                            mma_bf16_16816(cb0, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1]);
+                            mma_bf16_16816(cb1, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
+                            mma_bf16_16816(cb0, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                            mma_bf16_16816(cb1, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
                             const float s0 = __half2float(scl[bb * 128 + rib]);
                             const float s8 = __half2float(scl[bb * 128 + rib + 8]);
-                            c[0] = fmaf(s0, cb[0], c[0]);
-                            c[1] = fmaf(s0, cb[1], c[1]);
-                            c[2] = fmaf(s8, cb[2], c[2]);
-                            c[3] = fmaf(s8, cb[3], c[3]);
+                            c[0] = fmaf(s0, cb0[0] + cb1[0], c[0]);
+                            c[1] = fmaf(s0, cb0[1] + cb1[1], c[1]);
+                            c[2] = fmaf(s8, cb0[2] + cb1[2], c[2]);
+                            c[3] = fmaf(s8, cb0[3] + cb1[3], c[3]);
                         }
                     }
                     const int j = j0 + rgb * 16 + g;
