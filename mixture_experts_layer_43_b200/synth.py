@@ -32,8 +32,10 @@ import numpy as np
 
 WFMT_BF16 = 0
 WFMT_Q4_0 = 1
+WFMT_Q8_0 = 2
 Q4_BLOCK = 32          # weights per Q4_0 block
 Q4_BLOCK_BYTES = 18    # 2-byte fp16 scale + 16 bytes of 4-bit codes
+Q8_BLOCK_BYTES = 34    # 2-byte fp16 scale + 32 signed 8-bit codes
 
 
 @dataclasses.dataclass(frozen=True)
@@ -52,6 +54,7 @@ class MoEShape:
     w_std: float = 0.02
     wr_std: float = 0.02
     q4_scale_std: float = 0.005
+    q8_scale_std: float = 0.00035
 
     def replace(self, **kw) -> "MoEShape":
         return dataclasses.replace(self, **kw)
@@ -73,6 +76,16 @@ WORKLOADS = {
     "a3b_q4_T8_d2048_E256k8_F512_S1": MoEShape(
         "a3b_q4_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512,
         S=1, Fs=512, wfmt=WFMT_Q4_0),
+    # the same 35B-A3B layer with Q8_0 weights (another format of the model's mix)
+    "a3b_q8_T1_d2048_E256k8_F512_S1": MoEShape(
+        "a3b_q8_T1_d2048_E256k8_F512_S1", T=1, d=2048, E=256, k=8, F=512,
+        S=1, Fs=512, wfmt=WFMT_Q8_0),
+    "a3b_q8_T8_d2048_E256k8_F512_S1": MoEShape(
+        "a3b_q8_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512,
+        S=1, Fs=512, wfmt=WFMT_Q8_0),
+    # the same 35B-A3B layer in bf16 at T = 8 (about 58 distinct experts, 0.37 GB)
+    "a3b_T8_d2048_E256k8_F512_S1": MoEShape(
+        "a3b_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512, S=1, Fs=512),
     # A smaller case of the Mixtral-shaped decode kernel (same T, d, E, k;
     # F cut to 2048 so the whole layer is 0.4 GB) for detailed profiling.
     "mixtral_small_T8_d4096_E8k2_F2048": MoEShape(
@@ -135,6 +148,24 @@ def q4_0_blocks(rng: np.random.Generator, rows: int, k: int,
     return out
 
 
+def q8_0_blocks(rng: np.random.Generator, rows: int, k: int,
+                scale_std: float) -> np.ndarray:
+    """Canonical Q8_0 blocks [rows][k/32][34] with codes uniform on
+    -128..127 and scales |N(0, scale_std)| stored as fp16."""
+    assert k % Q4_BLOCK == 0
+    nb = k // Q4_BLOCK
+    out = np.empty((rows, nb, Q8_BLOCK_BYTES), dtype=np.uint8)
+    step = max(1, (1 << 22) // max(1, nb))
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        q = rng.integers(0, 256, size=(r1 - r0, nb, Q4_BLOCK), dtype=np.uint8)
+        sc = np.abs(rng.standard_normal((r1 - r0, nb), dtype=np.float32)
+                    * np.float32(scale_std)).astype(np.float16)
+        out[r0:r1, :, 0:2] = sc.view(np.uint8).reshape(r1 - r0, nb, 2)
+        out[r0:r1, :, 2:] = q
+    return out
+
+
 @dataclasses.dataclass
 class MoEInputs:
     shape: MoEShape
@@ -176,20 +207,20 @@ def make_inputs(shape: MoEShape, seed: int = 0,
         else:
             sg = su = sd = None
     else:
-        q = sh.q4_scale_std
-        g = q4_0_blocks(rng(3), sh.E * sh.F, sh.d, q).reshape(
-            sh.E, sh.F, sh.d // 32, 18)
-        u = q4_0_blocks(rng(4), sh.E * sh.F, sh.d, q).reshape(
-            sh.E, sh.F, sh.d // 32, 18)
-        dn = q4_0_blocks(rng(5), sh.E * sh.d, sh.F, q).reshape(
-            sh.E, sh.d, sh.F // 32, 18)
+        if sh.wfmt == WFMT_Q4_0:
+            blocks, q, nbytes = q4_0_blocks, sh.q4_scale_std, Q4_BLOCK_BYTES
+        else:
+            blocks, q, nbytes = q8_0_blocks, sh.q8_scale_std, Q8_BLOCK_BYTES
+
+        def stack(i, mats, rows, kk):
+            return blocks(rng(i), mats * rows, kk, q).reshape(mats, rows, kk // 32, nbytes)
+        g = stack(3, sh.E, sh.F, sh.d)
+        u = stack(4, sh.E, sh.F, sh.d)
+        dn = stack(5, sh.E, sh.d, sh.F)
         if sh.S:
-            sg = q4_0_blocks(rng(6), sh.S * sh.Fs, sh.d, q).reshape(
-                sh.S, sh.Fs, sh.d // 32, 18)
-            su = q4_0_blocks(rng(7), sh.S * sh.Fs, sh.d, q).reshape(
-                sh.S, sh.Fs, sh.d // 32, 18)
-            sd = q4_0_blocks(rng(8), sh.S * sh.d, sh.Fs, q).reshape(
-                sh.S, sh.d, sh.Fs // 32, 18)
+            sg = stack(6, sh.S, sh.Fs, sh.d)
+            su = stack(7, sh.S, sh.Fs, sh.d)
+            sd = stack(8, sh.S, sh.d, sh.Fs)
         else:
             sg = su = sd = None
     return MoEInputs(sh, x, wr, rb, g, u, dn, sg, su, sd)
@@ -201,7 +232,9 @@ def weight_bytes_per_expert(shape: MoEShape, hidden: Optional[int] = None) -> in
     n = 3 * F * shape.d
     if shape.wfmt == WFMT_BF16:
         return 2 * n
-    return n // 32 * 18       # 16 code bytes + 2 scale bytes per 32 weights
+    if shape.wfmt == WFMT_Q4_0:
+        return n // 32 * 18   # 16 code bytes + 2 scale bytes per 32 weights
+    return n // 32 * 34       # 32 code bytes + 2 scale bytes per 32 weights
 
 
 def expert_flops(shape: MoEShape, n_tokens: int, hidden: Optional[int] = None) -> int:
@@ -210,7 +243,7 @@ def expert_flops(shape: MoEShape, n_tokens: int, hidden: Optional[int] = None) -
 
 
 def describe(shape: MoEShape) -> str:
-    fmt = "bf16" if shape.wfmt == WFMT_BF16 else "q4_0"
+    fmt = {WFMT_BF16: "bf16", WFMT_Q4_0: "q4_0", WFMT_Q8_0: "q8_0"}[shape.wfmt]
     s = (f"T={shape.T} d={shape.d} E={shape.E} k={shape.k} F={shape.F} "
          f"S={shape.S} Fs={shape.Fs} {fmt}")
     if shape.zipf_bias:

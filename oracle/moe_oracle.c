@@ -31,13 +31,17 @@
  * The weights are read in the exact formats the GPU sees: bf16 values,
  * fp32 router, and Q4_0 blocks dequantised here as w = d * (q - 8) from the
  * canonical 18-byte blocks (fp16 scale d, then 16 bytes; byte j holds
- * element j in its low nibble and element j+16 in its high nibble).  Every
- * dequantised value is exact in double precision.
+ * element j in its low nibble and element j+16 in its high nibble), and Q8_0
+ * blocks as w = d * q from the canonical 34-byte blocks (fp16 scale d, then
+ * 32 signed bytes q, element j in byte j; the 5090 page names q8_0 among the
+ * formats of the model it measures).  Every dequantised value is exact in
+ * double precision.
  *
  * Layouts (row-major, reduction dimension contiguous):
  *   x [T][d] bf16 bits; Wr [E][d] fp32; b [E] fp32 or NULL
  *   routed gate/up [E][F][d], down [E][d][F]; shared [S][Fs][d], [S][d][Fs]
  *   Q4_0: a row of K weights is K/32 blocks of 18 bytes.
+ *   Q8_0: a row of K weights is K/32 blocks of 34 bytes.
  *
  * The pages print no worked example for the layer output, so the tests pin
  * every function here against what the mathematics fixes instead: brute-force
@@ -55,6 +59,7 @@
 
 #define ORACLE_WFMT_BF16 0
 #define ORACLE_WFMT_Q4_0 1
+#define ORACLE_WFMT_Q8_0 2
 
 /* bfloat16 is the top half of an IEEE binary32. */
 double oracle_bf16_to_f64(uint16_t b) {
@@ -94,6 +99,19 @@ static void q4_0_row(const uint8_t* blocks, int64_t K, double* out) {
     }
 }
 
+/* Dequantise one row of K weights stored as canonical Q8_0 blocks. */
+static void q8_0_row(const uint8_t* blocks, int64_t K, double* out) {
+    for (int64_t b = 0; b < K / 32; ++b) {
+        const uint8_t* blk = blocks + b * 34;
+        uint16_t hd = (uint16_t)(blk[0] | (blk[1] << 8));
+        double dsc = oracle_fp16_to_f64(hd);
+        for (int j = 0; j < 32; ++j) {
+            int q = blk[2 + j] < 128 ? (int)blk[2 + j] : (int)blk[2 + j] - 256;  /* two's complement */
+            out[b * 32 + j] = dsc * (double)q;
+        }
+    }
+}
+
 /* Row r of matrix m (0-based) of a stack of matrices [M][rows][K]. */
 static void load_row(int wfmt, const void* base, int64_t m, int64_t rows,
                      int64_t K, int64_t r, double* out) {
@@ -101,9 +119,12 @@ static void load_row(int wfmt, const void* base, int64_t m, int64_t rows,
     if (wfmt == ORACLE_WFMT_BF16) {
         const uint16_t* p = (const uint16_t*)base + row * K;
         for (int64_t i = 0; i < K; ++i) out[i] = oracle_bf16_to_f64(p[i]);
-    } else {
+    } else if (wfmt == ORACLE_WFMT_Q4_0) {
         const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 18;
         q4_0_row(p, K, out);
+    } else {
+        const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 34;
+        q8_0_row(p, K, out);
     }
 }
 
@@ -236,9 +257,9 @@ int oracle_forward(int d, int E, int k, int F, int S, int Fs, int wfmt,
         !wg || !wu || !wd || !out || !ids || !w || n_tokens < 0)
         return 1;
     if (S > 0 && (Fs <= 0 || !sg || !su || !sd)) return 1;
-    if (wfmt == ORACLE_WFMT_Q4_0 &&
-        (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
-    if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0) return 1;
+    if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0)
+        return 1;
+    if (wfmt != ORACLE_WFMT_BF16 && (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);
 #else

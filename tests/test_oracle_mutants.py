@@ -29,6 +29,10 @@ MUTANTS = {
     "q4_nibbles_swapped": ("int lo = blk[2 + j] & 0x0f;\n            int hi = blk[2 + j] >> 4;",
                            "int hi = blk[2 + j] & 0x0f;\n            int lo = blk[2 + j] >> 4;"),
     "q4_offset_7": ("dsc * (double)(lo - 8);", "dsc * (double)(lo - 7);"),
+    "q8_codes_unsigned": ("int q = blk[2 + j] < 128 ? (int)blk[2 + j] : (int)blk[2 + j] - 256;",
+                          "int q = (int)blk[2 + j];"),
+    "q8_scale_bytes_not_skipped": ("int q = blk[2 + j] < 128 ? (int)blk[2 + j] : (int)blk[2 + j] - 256;",
+                                   "int q = blk[j] < 128 ? (int)blk[j] : (int)blk[j] - 256;"),
     "fp16_exponent_bias": ("ldexp(1024.0 + (double)m, e - 25)", "ldexp(1024.0 + (double)m, e - 24)"),
     "bucket_unstable": ("for (int64_t p = 0; p < n; ++p) {\n            int e = ids[p];",
                         "for (int64_t p = n - 1; p >= 0; --p) {\n            int e = ids[p];"),
@@ -39,6 +43,7 @@ MUTANTS = {
 
 def _pins():
     yield lambda: pins.test_q4_0_golden_blocks()
+    yield lambda: pins.test_q8_0_golden_blocks()
     yield lambda: pins.test_fp16_decode_matches_numpy_all_patterns()
     yield lambda: pins.test_softmax_renormalisation_closed_form()
     yield lambda: pins.test_swiglu_closed_form()

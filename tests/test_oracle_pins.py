@@ -73,6 +73,32 @@ def test_q4_0_rows_are_independent_blocks():
                 assert got[r, 32 * b + 16 + j] == scale * (hi - 8)
 
 
+def test_q8_0_golden_blocks():
+    g = json.load(open(os.path.join(GOLDEN, "q8_0_blocks.json")))
+    for blk in g["blocks"]:
+        raw = np.array(blk["bytes"], dtype=np.uint8)
+        got = oracle.dequant(oracle.WFMT_Q8_0, raw, 1, 32)[0]
+        scale = float(np.array([blk["scale_bits"]], np.uint16).view(np.float16)[0])
+        want = np.array([scale * q for q in blk["codes"]], dtype=np.float64)
+        assert np.array_equal(got, want), blk["name"]
+
+
+def test_q8_0_rows_are_independent_blocks():
+    """A multi-row, multi-block Q8_0 matrix dequantises block by block in
+    row-major block order (checked with Python's struct decoders)."""
+    rng = np.random.default_rng(6)
+    rows, k = 3, 96
+    blocks = synth.q8_0_blocks(rng, rows, k, 0.01)
+    got = oracle.dequant(oracle.WFMT_Q8_0, blocks, rows, k)
+    for r in range(rows):
+        for b in range(k // 32):
+            raw = bytes(blocks[r, b])
+            (scale,) = struct.unpack("<e", raw[:2])
+            codes = struct.unpack("<32b", raw[2:])
+            for j in range(32):
+                assert got[r, 32 * b + j] == scale * codes[j]
+
+
 # ------------------------------------------------- pure-Python brute force
 def _bf16(b):
     return struct.unpack(">f", struct.pack(">I", int(b) << 16))[0]
@@ -93,11 +119,26 @@ def _q4_rows(blocks):
     return out
 
 
+def _q8_rows(blocks):
+    """Pure-Python decode of canonical Q8_0 rows -> list of lists."""
+    out = []
+    for row in blocks:
+        vals = []
+        for blk in row:
+            raw = bytes(blk)
+            (sc,) = struct.unpack("<e", raw[:2])
+            vals.extend(sc * q for q in struct.unpack("<32b", raw[2:]))
+        out.append(vals)
+    return out
+
+
 def _mat(inp_arr, wfmt, m, rows, cols):
     if wfmt == synth.WFMT_BF16:
         a = inp_arr[m]
         return [[_bf16(a[r, c]) for c in range(cols)] for r in range(rows)]
-    return _q4_rows(inp_arr[m])
+    if wfmt == synth.WFMT_Q4_0:
+        return _q4_rows(inp_arr[m])
+    return _q8_rows(inp_arr[m])
 
 
 def _brute_layer(inp):
@@ -156,13 +197,15 @@ TINY = [
     synth.MoEShape("bf16_bias", T=3, d=8, E=7, k=2, F=5, S=1, Fs=3, zipf_bias=1.1),
     synth.MoEShape("q4_shared", T=2, d=32, E=4, k=2, F=32, S=1, Fs=32,
                    wfmt=synth.WFMT_Q4_0),
+    synth.MoEShape("q8_shared", T=2, d=32, E=4, k=2, F=32, S=1, Fs=32,
+                   wfmt=synth.WFMT_Q8_0),
 ]
 
 
 @pytest.mark.parametrize("sh", TINY, ids=[s.name for s in TINY])
 def test_brute_force_tiny(sh):
     # A larger weight std makes the logits spread and the SwiGLU nonlinear.
-    sh = sh.replace(w_std=0.5, wr_std=0.5, q4_scale_std=0.05)
+    sh = sh.replace(w_std=0.5, wr_std=0.5, q4_scale_std=0.05, q8_scale_std=0.004)
     inp = synth.make_inputs(sh, seed=11)
     out, ids, w, logits = oracle.forward(inp)
     bout, bsets, bw, _ = _brute_layer(inp)
@@ -184,6 +227,11 @@ def _f64_stack(arr, wfmt, rows, cols):
     if wfmt == synth.WFMT_BF16:
         t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
         return t.double().numpy().reshape(-1, rows, cols)
+    if wfmt == synth.WFMT_Q8_0:
+        a = np.ascontiguousarray(arr).reshape(-1, rows, cols // 32, 34)
+        sc = a[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
+        q = a[..., 2:].copy().view(np.int8).astype(np.float64)
+        return (q * sc[..., None]).reshape(-1, rows, cols)
     a = np.ascontiguousarray(arr).reshape(-1, rows, cols // 32, 18)
     sc = a[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
     lo = (a[..., 2:] & 15).astype(np.float64) - 8
@@ -204,10 +252,10 @@ def _x64(inp):
     return torch.from_numpy(inp.x.view(np.int16)).view(torch.bfloat16).double().numpy()
 
 
-@pytest.mark.parametrize("wfmt", [synth.WFMT_BF16, synth.WFMT_Q4_0])
+@pytest.mark.parametrize("wfmt", [synth.WFMT_BF16, synth.WFMT_Q4_0, synth.WFMT_Q8_0])
 def test_k_equals_E_is_dense_softmax_mixture(wfmt):
     sh = synth.MoEShape("dense", T=5, d=64, E=4, k=4, F=32, wfmt=wfmt,
-                        wr_std=0.2, w_std=0.2, q4_scale_std=0.02)
+                        wr_std=0.2, w_std=0.2, q4_scale_std=0.02, q8_scale_std=0.002)
     inp = synth.make_inputs(sh, seed=3)
     out, ids, w, logits = oracle.forward(inp)
     x = _x64(inp)
