@@ -114,12 +114,22 @@ moe_status_t check_call(const moe_plan_s* p, const moe_weights_t* w, const void*
 }
 
 // ------------------------------------------------------------ tensor maps
+// L2 promotion no wider than the contiguous bytes one box row reads: a
+// wider promotion fetches the neighbouring columns too (the next work unit's
+// slice of the down matrix), which the evict-first streaming hint may evict
+// again before that unit runs.
+CUtensorMapL2promotion promotion_for(uint32_t row_bytes) {
+    return row_bytes >= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+         : row_bytes >= 128 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                            : CU_TENSOR_MAP_L2_PROMOTION_L2_64B;
+}
+
 bool encode_map(moe_plan_s* p, CUtensorMap* m, CUtensorMapDataType dt, int rank,
                 const void* base, const uint64_t* dims, const uint64_t* strides,
-                const uint32_t* box, CUtensorMapSwizzle sw) {
+                const uint32_t* box, CUtensorMapSwizzle sw, uint32_t row_bytes) {
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
     CUresult r = p->encode(m, dt, rank, const_cast<void*>(base), dims, strides, box, es,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promotion_for(row_bytes),
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -136,7 +146,7 @@ bool map_bf16(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int
     uint64_t strides[1] = {static_cast<uint64_t>(K) * 2};
     uint32_t box[2] = {box_k, box_rows};
     return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
-                      swizzle_for(static_cast<int>(box_k) * 2));
+                      swizzle_for(static_cast<int>(box_k) * 2), box_k * 2);
 }
 
 // Q4_0 packed codes [mats][K/32][N][16] seen as 3D {16, N, mats*K/32}.
@@ -146,7 +156,7 @@ bool map_q4_codes(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats,
     uint64_t strides[2] = {16, static_cast<uint64_t>(N) * 16};
     uint32_t box[3] = {16, box_rows, box_kb};
     return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_NONE);
+                      CU_TENSOR_MAP_SWIZZLE_NONE, 16 * box_rows);   // rows are contiguous
 }
 
 // Q4_0 packed scales [mats][K/32][N] fp16 seen as 2D {N, mats*K/32}.
@@ -156,7 +166,7 @@ bool map_q4_scales(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats
     uint64_t strides[1] = {static_cast<uint64_t>(N) * 2};
     uint32_t box[2] = {box_rows, box_kb};
     return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_NONE);
+                      CU_TENSOR_MAP_SWIZZLE_NONE, 2 * box_rows);
 }
 
 bool same_weights(const moe_weights_t& a, const moe_weights_t& b) {

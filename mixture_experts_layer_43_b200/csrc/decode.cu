@@ -1,25 +1,30 @@
 // decode.cu -- decode-regime kernels (T <= MOE_DECODE_MAX_T tokens per call).
 //
-// Two launches per layer call:
+// moe_forward runs the whole layer as ONE cooperative launch,
+// decode_fused_kernel (its phases are described above the kernel): router
+// logits, a grid barrier, top-k / buckets / work list computed by every CTA,
+// then the experts pipeline.  moe_route + moe_experts (and moe_forward when a
+// cooperative launch cannot place one CTA per SM) use two launches instead:
 //  1. decode_route_kernel: router logits (fp32 FMA), softmax + top-k with
 //     renormalised weights, per-expert buckets (counts, exclusive offsets,
 //     stable slot order), the expert work list, and the zero-fill of `out`.
 //     ("Fused MoE Triton kernel: 5 launches instead of 24" page, fused steps
 //     one and two; its launch table's routing and dispatch rows.)
-//  2. decode_experts_kernel: ONE persistent launch over every active routed
-//     expert and every shared expert ("CUDA: fuse shared experts into MMVQ"
-//     page: shared experts go through the same pass as the routed ones).
-//     Each work unit is (expert, slice of FS hidden rows): it streams the
-//     slice's gate/up rows, forms h = SiLU(gate) * up for the expert's
-//     tokens, streams the matching columns of the down matrix and adds
-//     w * (Wd h) into `out` (the weighted aggregation, fused).  Weights move
-//     HBM -> shared memory by TMA through a ring of stages fed by one
-//     producer warp, so every SM keeps tens of KB in flight ("MoE on RTX 5090
-//     reaches 41% of bandwidth" page: small reads per kernel cap bandwidth;
-//     the fix it predicts is more bytes per launch).  The contraction over
-//     the <= 8 tokens of an expert runs on mma.sync (bf16 in, fp32
-//     accumulate); Q4_0 codes are dequantised in registers and never written
-//     back ("MMVQ" page: read quantised weights once, never expand them).
+//  2. decode_experts_kernel: the experts pipeline alone.
+//
+// The experts pipeline makes ONE pass over every active routed expert and
+// every shared expert ("CUDA: fuse shared experts into MMVQ" page: shared
+// experts go through the same pass as the routed ones).  Each work unit is
+// (expert, slice of FS hidden rows): it streams the slice's gate/up rows,
+// forms h = SiLU(gate) * up for the expert's tokens, streams the matching
+// columns of the down matrix and adds w * (Wd h) into `out` (the weighted
+// aggregation, fused).  Weights move HBM -> shared memory by TMA through a
+// ring of stages fed by one producer warp, so every SM keeps tens of KB in
+// flight ("MoE on RTX 5090 reaches 41% of bandwidth" page: small reads per
+// kernel cap bandwidth; the fix it predicts is more bytes per launch).  The
+// contraction over the <= 8 tokens of an expert runs on mma.sync (bf16 in,
+// fp32 accumulate); Q4_0 codes are dequantised in registers and never
+// written back ("MMVQ" page: read quantised weights once, never expand them).
 #include <float.h>
 #include <math.h>
 
@@ -230,22 +235,21 @@ struct DecodeCfg {
     static constexpr int NB = FS / 32;            // Q4_0 block columns in a slice
     static constexpr int RJ = Q4 ? 32768 / FS : 16384 / FS;   // phase B rows per stage
     static constexpr int HS = FS + 8;             // h row stride (bf16 elements)
+    static constexpr int GS = FS + 4;             // gate/up result row stride (floats)
 };
 
 struct alignas(16) DecodeSmemTail {
-    int tok[kDecodeTok];
-    float w[kDecodeTok];
     int abort_flag;
     int pad[3];
 };
 
-__device__ __forceinline__ uint32_t q4_pair(uint32_t w, int s) {
-    // ((w >> s) & 0x000F000F) puts two codes in the low mantissa bits of two
-    // bf16 values 128 + q; subtracting 136 leaves q - 8 exactly.
-    uint32_t v = ((w >> s) & 0x000F000Fu) | 0x43004300u;
-    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&v);
-    b = __hsub2(b, __floats2bfloat162_rn(136.f, 136.f));
-    return *reinterpret_cast<uint32_t*>(&b);
+// ((w >> s) & 0x000F000F) | 0x43004300 puts two 4-bit codes q in the low
+// mantissa bits of two bf16 values 128 + q (exact).  Q4_0's weight is
+// d * (q - 8) = d * ((128 + q) - 136): instead of subtracting 136 from every
+// weight, the block's accumulator starts at -136 * (sum of the block's 32
+// activations), so one block contributes d * sum((128 + q) x) - 136 d sum(x).
+__device__ __forceinline__ uint32_t q4_raw(uint32_t w, int s) {
+    return ((w >> s) & 0x000F000Fu) | 0x43004300u;
 }
 
 // Work list the experts pipeline reads: generic pointers, so the same code
@@ -261,10 +265,12 @@ struct WorkView {
 // Shared-memory carve-up of the experts pipeline.
 struct DecodeSmem {
     uint8_t* ring;
-    uint8_t* xs;
-    float* gu;
-    __nv_bfloat16* hhi;
+    uint8_t* xs;            // [8][xs_stride]: the T token rows of x, staged once
+    float* xsum;            // [8][d/32]: -136 * block sums of x (Q4_0 only)
+    float* gu;              // [KSPLIT][2][8][GS]: gate / up partial results
+    __nv_bfloat16* hhi;     // [8][HS]: h = hi + lo, per slot
     __nv_bfloat16* hlo;
+    float* hsum;            // [8][2]: -136 * block sums of hi + lo (Q4_0 only)
     DecodeSmemTail* tail;
     uint64_t* full;
     uint64_t* empty;
@@ -278,13 +284,42 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.ring = smem;
     sm.xs = sm.ring + static_cast<size_t>(a.n_stages) * C::STAGE;
-    sm.gu = reinterpret_cast<float*>(sm.xs + kDecodeTok * a.xs_stride);   // [KSPLIT][2][FS][8]
-    sm.hhi = reinterpret_cast<__nv_bfloat16*>(sm.gu + C::KSPLIT * 2 * FS * kDecodeTok);
+    sm.xsum = reinterpret_cast<float*>(sm.xs + kDecodeTok * a.xs_stride);
+    sm.gu = sm.xsum + kDecodeTok * (a.d / 32);
+    sm.hhi = reinterpret_cast<__nv_bfloat16*>(sm.gu + C::KSPLIT * 2 * kDecodeTok * C::GS);
     sm.hlo = sm.hhi + kDecodeTok * C::HS;
-    sm.tail = reinterpret_cast<DecodeSmemTail*>(sm.hlo + kDecodeTok * C::HS);
+    sm.hsum = reinterpret_cast<float*>(sm.hlo + kDecodeTok * C::HS);
+    sm.tail = reinterpret_cast<DecodeSmemTail*>(sm.hsum + kDecodeTok * 2);
     sm.full = reinterpret_cast<uint64_t*>(sm.tail + 1);
     sm.empty = sm.full + a.n_stages;
     return sm;
+}
+
+// Consumer threads copy the T token rows of x into shared memory once per
+// launch; every work unit then addresses its tokens' rows directly.  For
+// Q4_0 the same pass stores -136 * (sum of each 32-wide block of a row), the
+// starting value of that block's accumulator (see q4_raw).
+template <bool Q4>
+__device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& sm, int tid) {
+    const int nkb = a.d / 32;
+    for (int idx = tid; idx < a.T * nkb; idx += kConsumers) {
+        const int t = idx / nkb, kb = idx % nkb;
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + kb * 32);
+        uint4* dst = reinterpret_cast<uint4*>(sm.xs + t * a.xs_stride + kb * 64);
+        float s = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint4 v = __ldg(src + c);
+            dst[c] = v;
+            if constexpr (Q4) {
+                const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    s += __uint_as_float(q[j] << 16) + __uint_as_float(q[j] & 0xffff0000u);
+            }
+        }
+        if constexpr (Q4) sm.xsum[t * nkb + kb] = -136.f * s;
+    }
 }
 
 // The expert stage: work units are (expert, slice of FS hidden rows), shared
@@ -298,7 +333,6 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
     using C = DecodeCfg<FS, Q4>;
     const int ns = a.n_stages;
     uint8_t* ring = sm.ring;
-    uint8_t* xs = sm.xs;
     float* gu = sm.gu;
     __nv_bfloat16* hhi = sm.hhi;
     __nv_bfloat16* hlo = sm.hlo;
@@ -423,9 +457,9 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
     const int g = lane >> 2, tig = lane & 3;
     const int role = warp % C::ROLES, ks = warp / C::ROLES;
     const int mat = role / C::RG, rg = role % C::RG;
-    const uint32_t xs_u = smem_u32(xs);
+    const uint32_t xs_u = smem_u32(sm.xs);
+    const int nkb = d / 32;
     uint32_t it = 0;
-    int prev_item = -1;
 
     // warp-uniform: the ldmatrix / mma.sync that follow are warp-collective
     auto wait_full = [&](int slot, uint32_t parity) -> bool {
@@ -444,32 +478,19 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
         const WorkItem item = wv.items[ii];
         const bool shared = item.expert >= E;
         const int ntok = min(item.count, kDecodeTok);
-
-        if (ii != prev_item) {
-            named_bar_sync(1, kConsumers);
-            if (tid < kDecodeTok) {
-                int t = 0;
-                float w = 0.f;
-                if (tid < ntok) {
-                    if (shared) { t = tid; w = 1.f; }
-                    else { t = wv.slot_token[item.slot_begin + tid]; w = wv.slot_w[item.slot_begin + tid]; }
-                }
-                tail->tok[tid] = t;
-                tail->w[tid] = w;
-            }
-            named_bar_sync(1, kConsumers);
-            const int cpr = d / 8;                       // 16-byte chunks per row
-            for (int idx = tid; idx < kDecodeTok * cpr; idx += kConsumers) {
-                const int t = idx / cpr, c = idx % cpr;
-                uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                if (t < ntok)
-                    v = __ldg(reinterpret_cast<const uint4*>(
-                        a.x + static_cast<size_t>(tail->tok[t]) * d + c * 8));
-                *reinterpret_cast<uint4*>(xs + t * a.xs_stride + c * 16) = v;
-            }
-            named_bar_sync(1, kConsumers);
-            prev_item = ii;
-        }
+        // token slot n of this item -> token row (slots past ntok reuse row 0:
+        // their columns of the mma are computed and never stored)
+        auto tok_of = [&](int n) -> int {
+            return n < ntok ? (shared ? n : wv.slot_token[item.slot_begin + n]) : 0;
+        };
+        auto w_of = [&](int n) -> float {
+            return n < ntok ? (shared ? 1.f : wv.slot_w[item.slot_begin + n]) : 0.f;
+        };
+        const uint32_t xrow = xs_u + tok_of(lane & 7) * a.xs_stride;   // B row of this lane
+        const int t0 = 2 * tig, t1 = t0 + 1;
+        const int tok0 = tok_of(t0), tok1 = tok_of(t1);
+        const float w0 = w_of(t0), w1 = w_of(t1);
+        const bool v0 = t0 < ntok, v1 = t1 < ntok;
 
         // ------------------------------------------- phase A: gate and up
         float cacc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -490,33 +511,32 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         ldsm_x4(tile + (kk >> 2) * (FS * 128) +
                                     swz_offset(arow, (kk & 3) * 2 + (m >> 1), 128),
                                 a0, a1, a2, a3);
-                        ldsm_x2(xs_u + (lane & 7) * a.xs_stride +
-                                    (k0 + kk * 16 + ((lane >> 3) & 1) * 8) * 2,
-                                b0, b1);
+                        ldsm_x2(xrow + (k0 + kk * 16 + ((lane >> 3) & 1) * 8) * 2, b0, b1);
                         mma_bf16_16816(cacc, a0, a1, a2, a3, b0, b1);
                     }
                 } else {
                     const int kb0 = st * C::KB;
-                    const int nkb = min(C::KB, d / 32 - kb0);
+                    const int nkb_st = min(C::KB, nkb - kb0);
                     const uint8_t* mb = stage + mat * (C::KB * FS * 18);
                     const uint32_t* codes = reinterpret_cast<const uint32_t*>(mb);
                     const __half* scl = reinterpret_cast<const __half*>(mb + C::KB * FS * 16);
                     const int r0 = rg * 16 + g;
+                    const float* xsum0 = sm.xsum + tok0 * nkb + kb0;
+                    const float* xsum1 = sm.xsum + tok1 * nkb + kb0;
 #pragma unroll 2
-                    for (int bb = ks; bb < nkb; bb += C::KSPLIT) {
-                        const uint32_t w0 = codes[(bb * FS + r0) * 4 + tig];
-                        const uint32_t w8 = codes[(bb * FS + r0 + 8) * 4 + tig];
+                    for (int bb = ks; bb < nkb_st; bb += C::KSPLIT) {
+                        const uint32_t w0c = codes[(bb * FS + r0) * 4 + tig];
+                        const uint32_t w8c = codes[(bb * FS + r0 + 8) * 4 + tig];
                         uint32_t b0, b1, b2, b3;
-                        ldsm_x4(xs_u + (lane & 7) * a.xs_stride +
-                                    ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2,
-                                b0, b1, b2, b3);
+                        ldsm_x4(xrow + ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
                         // the block's two 16-wide halves go to independent
-                        // accumulators (no mma -> mma dependency inside a block)
-                        float cb0[4] = {0.f, 0.f, 0.f, 0.f}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_bf16_16816(cb0, q4_pair(w0, 0), q4_pair(w8, 0), q4_pair(w0, 4),
-                                       q4_pair(w8, 4), b0, b1);
-                        mma_bf16_16816(cb1, q4_pair(w0, 8), q4_pair(w8, 8), q4_pair(w0, 12),
-                                       q4_pair(w8, 12), b2, b3);
+                        // accumulators; the first starts at -136 * sum(x)
+                        const float c0 = xsum0[bb], c1 = xsum1[bb];
+                        float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_bf16_16816(cb0, q4_raw(w0c, 0), q4_raw(w8c, 0), q4_raw(w0c, 4),
+                                       q4_raw(w8c, 4), b0, b1);
+                        mma_bf16_16816(cb1, q4_raw(w0c, 8), q4_raw(w8c, 8), q4_raw(w0c, 12),
+                                       q4_raw(w8c, 12), b2, b3);
                         const float s0 = __half2float(scl[bb * FS + r0]);
                         const float s8 = __half2float(scl[bb * FS + r0 + 8]);
                         cacc[0] = fmaf(s0, cb0[0] + cb1[0], cacc[0]);
@@ -530,27 +550,38 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             if (lane == 0) mbar_arrive(&empty[slot]);
         }
         {
-            float* gq = gu + ((ks * 2 + mat) * FS) * kDecodeTok;
+            // gate/up partials as [t][f]: row stride GS = FS + 4 keeps the
+            // four token columns of a lane quad in distinct banks
+            float* gq = gu + (ks * 2 + mat) * kDecodeTok * C::GS;
             const int r = rg * 16 + g;
-            gq[r * kDecodeTok + 2 * tig] = cacc[0];
-            gq[r * kDecodeTok + 2 * tig + 1] = cacc[1];
-            gq[(r + 8) * kDecodeTok + 2 * tig] = cacc[2];
-            gq[(r + 8) * kDecodeTok + 2 * tig + 1] = cacc[3];
+            gq[t0 * C::GS + r] = cacc[0];
+            gq[t1 * C::GS + r] = cacc[1];
+            gq[t0 * C::GS + r + 8] = cacc[2];
+            gq[t1 * C::GS + r + 8] = cacc[3];
         }
         named_bar_sync(1, kConsumers);
-        // h = SiLU(gate) * up, kept as a bf16 pair hi + lo (|h - hi - lo| <= 2^-16 |h|)
+        // h = SiLU(gate) * up, kept as a bf16 pair hi + lo (|h - hi - lo| <= 2^-16 |h|).
+        // One warp covers 32 consecutive f of one slot, i.e. one Q4_0 block of
+        // the down matrix (FS * 8 is a multiple of 32: the loop is warp-uniform).
         for (int idx = tid; idx < FS * kDecodeTok; idx += kConsumers) {
-            const int f = idx / kDecodeTok, t = idx % kDecodeTok;
+            const int t = idx / FS, f = idx % FS;
             float gv = 0.f, uv = 0.f;
 #pragma unroll
             for (int q = 0; q < C::KSPLIT; ++q) {
-                gv += gu[((q * 2 + 0) * FS + f) * kDecodeTok + t];
-                uv += gu[((q * 2 + 1) * FS + f) * kDecodeTok + t];
+                gv += gu[((q * 2 + 0) * kDecodeTok + t) * C::GS + f];
+                uv += gu[((q * 2 + 1) * kDecodeTok + t) * C::GS + f];
             }
             const float h = gv / (1.f + expf(-gv)) * uv;
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             hhi[t * C::HS + f] = hi;
-            hlo[t * C::HS + f] = __float2bfloat16_rn(h - __bfloat162float(hi));
+            hlo[t * C::HS + f] = lo;
+            if constexpr (Q4) {
+                float hs = __bfloat162float(hi) + __bfloat162float(lo);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
+                if (lane == 0) sm.hsum[t * 2 + f / 32] = -136.f * hs;
+            }
         }
         named_bar_sync(1, kConsumers);
         uint32_t bh[C::RG][2], bl[C::RG][2];
@@ -560,10 +591,14 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             ldsm_x2(smem_u32(hhi) + off, bh[kk][0], bh[kk][1]);
             ldsm_x2(smem_u32(hlo) + off, bl[kk][0], bl[kk][1]);
         }
-        const int t0 = 2 * tig, t1 = t0 + 1;
-        const int tok0 = tail->tok[t0], tok1 = tail->tok[t1];
-        const float w0 = tail->w[t0], w1 = tail->w[t1];
-        const bool v0 = t0 < ntok, v1 = t1 < ntok;
+        float hs0[C::NB > 0 ? C::NB : 1], hs1[C::NB > 0 ? C::NB : 1];
+        if constexpr (Q4) {
+#pragma unroll
+            for (int bb = 0; bb < C::NB; ++bb) {
+                hs0[bb] = sm.hsum[t0 * 2 + bb];
+                hs1[bb] = sm.hsum[t1 * 2 + bb];
+            }
+        }
 
         // --------------------------------------- phase B: down + combine
         for (int st = 0; st < nB; ++st, ++it) {
@@ -595,12 +630,14 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         for (int bb = 0; bb < C::NB; ++bb) {
                             const uint32_t w0c = codes[(bb * 128 + rib) * 4 + tig];
                             const uint32_t w8c = codes[(bb * 128 + rib + 8) * 4 + tig];
-                            const uint32_t p0 = q4_pair(w0c, 0), q0 = q4_pair(w8c, 0);
-                            const uint32_t p1 = q4_pair(w0c, 4), q1 = q4_pair(w8c, 4);
-                            const uint32_t p2 = q4_pair(w0c, 8), q2 = q4_pair(w8c, 8);
-                            const uint32_t p3 = q4_pair(w0c, 12), q3 = q4_pair(w8c, 12);
-                            // two independent accumulator chains (halves of the block)
-                            float cb0[4] = {0.f, 0.f, 0.f, 0.f}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+                            const uint32_t p0 = q4_raw(w0c, 0), q0 = q4_raw(w8c, 0);
+                            const uint32_t p1 = q4_raw(w0c, 4), q1 = q4_raw(w8c, 4);
+                            const uint32_t p2 = q4_raw(w0c, 8), q2 = q4_raw(w8c, 8);
+                            const uint32_t p3 = q4_raw(w0c, 12), q3 = q4_raw(w8c, 12);
+                            // two independent accumulator chains (halves of the
+                            // block); the first starts at -136 * sum(hi + lo)
+                            float cb0[4] = {hs0[bb], hs1[bb], hs0[bb], hs1[bb]};
+                            float cb1[4] = {0.f, 0.f, 0.f, 0.f};
                             mma_bf16_16816(cb0, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1]);
                             mma_bf16_16816(cb1, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
                             mma_bf16_16816(cb0, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
@@ -644,6 +681,7 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
         sm.tail->abort_flag = 0;
         fence_mbar_init();
     }
+    if (threadIdx.x < kConsumers) stage_x<Q4>(a, sm, threadIdx.x);
     __syncthreads();
     const WorkView wv{a.n_items[0], a.n_items[1], a.items, a.slot_token, a.slot_w};
     experts_pipeline<FS, Q4>(a, sm, wv);
@@ -721,8 +759,9 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
     }
     __syncthreads();
 
-    // ---- R: logits of this CTA's experts; zero-fill of out
+    // ---- R: logits of this CTA's experts; zero-fill of out; x staged for X
     if (warp < kConsumerWarps) {
+        stage_x<Q4>(a, sm, tid);
         {
             float4* o = reinterpret_cast<float4*>(a.out);
             const int n4 = (T * d) >> 2;
@@ -873,8 +912,10 @@ size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages) {
     size_t b = 1024;                                            // alignment slack
     b += static_cast<size_t>(n_stages) * decode_stage_bytes(fs, q4);
     b += static_cast<size_t>(kDecodeTok) * (d * 2 + 16);       // staged x
-    b += static_cast<size_t>(ksplit) * 2 * fs * kDecodeTok * 4;  // gate/up results
+    b += static_cast<size_t>(kDecodeTok) * (d / 32) * 4;       // block sums of x
+    b += static_cast<size_t>(ksplit) * 2 * kDecodeTok * (fs + 4) * 4;  // gate/up results
     b += 2ull * kDecodeTok * (fs + 8) * 2;                      // h hi/lo
+    b += static_cast<size_t>(kDecodeTok) * 2 * 4;              // block sums of h
     b += sizeof(DecodeSmemTail);
     b += 2ull * n_stages * 8;                                   // barriers
     return b;

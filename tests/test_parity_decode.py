@@ -58,7 +58,8 @@ def _check(sh, seed=0, T=None, split=False):
 
 @pytest.mark.parametrize("name", ["tiny_T4_d256_E8k2_F512", "a3b_T1_d2048_E256k8_F512_S1",
                                   "a3b_q4_T1_d2048_E256k8_F512_S1",
-                                  "a3b_q4_T8_d2048_E256k8_F512_S1"])
+                                  "a3b_q4_T8_d2048_E256k8_F512_S1",
+                                  "a3b_T8_d2048_E256k8_F512_S1"])
 def test_decode_workloads_full_size(name):
     err = _check(W[name])
     print(f"{name}: rel L2 {err:.3e}")
