@@ -59,14 +59,21 @@ typedef enum moe_status {
  *   bandwidth" page names Q4_0, measurement-setup paragraph; the MMVQ page
  *   asks that quantised weights be read once and never expanded, section
  *   "what MMVQ is").  The kernels read the packed form written by
- *   moe_q4_0_pack, not the canonical 18-byte blocks. */
+ *   moe_q4_0_pack, not the canonical 18-byte blocks.
+ * MOE_WFMT_Q8_0: blocks of 32 consecutive weights along the reduction dim,
+ *   each an fp16 scale d and 32 signed 8-bit codes q, weight = d * q (the
+ *   5090 page lists q8_0 among the formats of the 35B-A3B model it measures;
+ *   it prints no layout, and the canonical 34-byte block is the reading
+ *   taken).  The kernels read the packed form written by moe_q8_0_pack.
+ * The quantised formats run in the decode regime only (T <= MOE_DECODE_MAX_T). */
 typedef enum moe_wfmt {
     MOE_WFMT_BF16 = 0,
-    MOE_WFMT_Q4_0 = 1
+    MOE_WFMT_Q4_0 = 1,
+    MOE_WFMT_Q8_0 = 2
 } moe_wfmt_t;
 
 /* Execution regime.  AUTO picks DECODE for T <= MOE_DECODE_MAX_T (and for
- * every T with Q4_0 weights, up to MOE_DECODE_MAX_T) and PREFILL otherwise.
+ * every T with quantised weights, up to MOE_DECODE_MAX_T) and PREFILL otherwise.
  * DECODE streams every active expert's weights once, through a TMA ring,
  * with the <= 8 tokens of an expert as the N side of mma.sync and the
  * weighted combine fused.  PREFILL runs grouped GEMMs on tcgen05 tensor
@@ -95,8 +102,8 @@ typedef struct moe_config {
 } moe_config_t;
 
 /* One stack of expert matrices.  bf16: `data` is the bf16 stack, `scales`
- * must be NULL.  Q4_0: `data` = packed codes, `scales` = packed fp16 scales
- * (both from moe_q4_0_pack). */
+ * must be NULL.  Q4_0 / Q8_0: `data` = packed codes, `scales` = packed fp16
+ * scales (both from moe_q4_0_pack / moe_q8_0_pack). */
 typedef struct moe_matrix {
     const void* data;
     const void* scales;
@@ -203,13 +210,14 @@ int32_t moe_last_launch_count(moe_plan_t plan);
 moe_status_t moe_get_device_status(moe_plan_t plan);
 
 /* Failure-path check (the pages have no counterpart): make the next fused
- * decode launch of `plan` unable to pass its grid barrier, by writing an
- * arrival count no launch can complete into the plan's barrier word (an
- * async memset on `stream`).  That launch waits the bounded 2 s, skips its
- * expert work, and exits; moe_get_device_status then returns
- * MOE_ERR_TIMEOUT and resets the barrier, after which the plan works
- * normally again.  Nothing hangs and nothing faults.  UNSUPPORTED if the
- * device cannot run the fused (cooperative) launch. */
+ * decode launch of `plan` unable to pass its grid barrier, by setting the
+ * plan's barrier count to 1 (async memsets on `stream`), a value the
+ * launch's arrivals cannot bring to the last CTA's target.  That CTA waits
+ * the bounded 2 s, skips its expert work, and exits, so the call's `out` is
+ * incomplete; moe_get_device_status then returns MOE_ERR_TIMEOUT and resets
+ * the barrier, after which the plan works normally again.  Nothing hangs and
+ * nothing faults.  UNSUPPORTED if the device cannot run the fused
+ * (cooperative) launch. */
 moe_status_t moe_debug_stall_barrier(moe_plan_t plan, void* stream);
 
 /* Bytes of the packed Q4_0 form of n_mats matrices of [rows][k] weights.
@@ -226,6 +234,26 @@ moe_status_t moe_q4_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
  * Same 4.5 bits per weight.  All pointers are device pointers; `blocks`
  * needs no alignment, `codes`/`scales` 16 bytes.  Enqueued on `stream`. */
 moe_status_t moe_q4_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
+                           int64_t k, void* codes, void* scales, void* stream);
+
+/* Bytes of the packed Q8_0 form of n_mats matrices of [rows][k] weights
+ * (32 code bytes and one fp16 scale per block).  k must be a multiple of 32.
+ * Returns INVALID_ARG otherwise. */
+moe_status_t moe_q8_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
+                                   size_t* code_bytes, size_t* scale_bytes);
+
+/* Repack canonical Q8_0 blocks ([n_mats][rows][k/32] blocks of 34 bytes: a
+ * little-endian fp16 scale, then 32 signed bytes, element j in byte j) into
+ * the kernel layout:
+ *   codes  [n_mats][k/32][rows][32 bytes]: each code biased to q + 128 and
+ *          split into two 4-bit planes, each permuted like the Q4_0 codes,
+ *          the planes' 32-bit words interleaved (low, high, low, high, ...);
+ *   scales [n_mats][k/32][rows] fp16.
+ * Same 8.5 bits per weight.  All pointers are device pointers; `blocks`
+ * needs no alignment, `codes`/`scales` 16 bytes.  Enqueued on `stream`.
+ * The pages have no counterpart to this repacking (it serves the kernels'
+ * tensor-core fragments). */
+moe_status_t moe_q8_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
                            int64_t k, void* codes, void* scales, void* stream);
 
 /* Static description of a status code (never NULL). */

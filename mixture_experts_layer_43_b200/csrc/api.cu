@@ -66,7 +66,8 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->n_shared < 0 || c->n_shared > kMaxShared) return MOE_ERR_INVALID_ARG;
     if (c->n_shared > 0 && (c->d_ff_shared < 32 || c->d_ff_shared % 32 != 0))
         return MOE_ERR_INVALID_ARG;
-    if (c->wfmt != MOE_WFMT_BF16 && c->wfmt != MOE_WFMT_Q4_0) return MOE_ERR_INVALID_ARG;
+    if (c->wfmt != MOE_WFMT_BF16 && c->wfmt != MOE_WFMT_Q4_0 && c->wfmt != MOE_WFMT_Q8_0)
+        return MOE_ERR_INVALID_ARG;
     if (c->regime < MOE_REGIME_AUTO || c->regime > MOE_REGIME_PREFILL) return MOE_ERR_INVALID_ARG;
     if (c->device < 0) return MOE_ERR_INVALID_ARG;
     // 2^31 limits of the int32 index arithmetic in the kernels
@@ -75,19 +76,19 @@ moe_status_t check_config(const moe_config_t* c) {
     if (static_cast<int64_t>(c->n_experts) * c->d_ff >= (1ll << 31) ||
         static_cast<int64_t>(c->n_experts) * c->d_model >= (1ll << 31))
         return MOE_ERR_INVALID_ARG;
-    if (c->wfmt == MOE_WFMT_Q4_0 && c->regime == MOE_REGIME_PREFILL) return MOE_ERR_UNSUPPORTED;
+    if (c->wfmt != MOE_WFMT_BF16 && c->regime == MOE_REGIME_PREFILL) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
 bool use_decode(const moe_plan_s* p, int T) {
     if (p->cfg.regime == MOE_REGIME_DECODE) return true;
     if (p->cfg.regime == MOE_REGIME_PREFILL) return false;
-    return T <= MOE_DECODE_MAX_T || p->cfg.wfmt == MOE_WFMT_Q4_0;
+    return T <= MOE_DECODE_MAX_T || p->cfg.wfmt != MOE_WFMT_BF16;
 }
 
-moe_status_t check_matrix(const moe_matrix_t& m, bool q4) {
+moe_status_t check_matrix(const moe_matrix_t& m, bool quant) {
     if (!m.data || !aligned16(m.data)) return MOE_ERR_INVALID_ARG;
-    if (q4 ? (!m.scales || !aligned16(m.scales)) : (m.scales != nullptr)) return MOE_ERR_INVALID_ARG;
+    if (quant ? (!m.scales || !aligned16(m.scales)) : (m.scales != nullptr)) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 
@@ -99,17 +100,17 @@ moe_status_t check_call(const moe_plan_s* p, const moe_weights_t* w, const void*
     if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
     if (!w->router_w || !aligned16(w->router_w)) return MOE_ERR_INVALID_ARG;
     if (w->router_b && (reinterpret_cast<uintptr_t>(w->router_b) & 3u)) return MOE_ERR_INVALID_ARG;
-    const bool q4 = p->cfg.wfmt == MOE_WFMT_Q4_0;
+    const bool quant = p->cfg.wfmt != MOE_WFMT_BF16;     // quantised: codes + scales
     moe_status_t s;
-    if ((s = check_matrix(w->gate, q4)) || (s = check_matrix(w->up, q4)) ||
-        (s = check_matrix(w->down, q4)))
+    if ((s = check_matrix(w->gate, quant)) || (s = check_matrix(w->up, quant)) ||
+        (s = check_matrix(w->down, quant)))
         return s;
     if (p->cfg.n_shared > 0 &&
-        ((s = check_matrix(w->shared_gate, q4)) || (s = check_matrix(w->shared_up, q4)) ||
-         (s = check_matrix(w->shared_down, q4))))
+        ((s = check_matrix(w->shared_gate, quant)) || (s = check_matrix(w->shared_up, quant)) ||
+         (s = check_matrix(w->shared_down, quant))))
         return s;
     if (use_decode(p, T) && T > MOE_DECODE_MAX_T) return MOE_ERR_UNSUPPORTED;
-    if (!use_decode(p, T) && q4) return MOE_ERR_UNSUPPORTED;
+    if (!use_decode(p, T) && quant) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
@@ -149,18 +150,19 @@ bool map_bf16(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int
                       swizzle_for(static_cast<int>(box_k) * 2), box_k * 2);
 }
 
-// Q4_0 packed codes [mats][K/32][N][16] seen as 3D {16, N, mats*K/32}.
-bool map_q4_codes(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
-                  int64_t K, uint32_t box_rows, uint32_t box_kb) {
-    uint64_t dims[3] = {16, static_cast<uint64_t>(N), static_cast<uint64_t>(mats * (K / 32))};
-    uint64_t strides[2] = {16, static_cast<uint64_t>(N) * 16};
-    uint32_t box[3] = {16, box_rows, box_kb};
+// Q4_0 / Q8_0 packed codes [mats][K/32][N][cb] (cb = 16 / 32 bytes per
+// block row) seen as 3D {cb, N, mats*K/32}.
+bool map_quant_codes(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
+                     int64_t K, uint32_t box_rows, uint32_t box_kb, uint32_t cb) {
+    uint64_t dims[3] = {cb, static_cast<uint64_t>(N), static_cast<uint64_t>(mats * (K / 32))};
+    uint64_t strides[2] = {cb, static_cast<uint64_t>(N) * cb};
+    uint32_t box[3] = {cb, box_rows, box_kb};
     return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, 16 * box_rows);   // rows are contiguous
+                      CU_TENSOR_MAP_SWIZZLE_NONE, cb * box_rows);   // rows are contiguous
 }
 
-// Q4_0 packed scales [mats][K/32][N] fp16 seen as 2D {N, mats*K/32}.
-bool map_q4_scales(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
+// Q4_0 / Q8_0 packed scales [mats][K/32][N] fp16 seen as 2D {N, mats*K/32}.
+bool map_quant_scales(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
                    int64_t K, uint32_t box_rows, uint32_t box_kb) {
     uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(mats * (K / 32))};
     uint64_t strides[1] = {static_cast<uint64_t>(N) * 2};
@@ -214,19 +216,20 @@ DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
         }
     } else {
         const uint32_t kb = 512 / fs, nb = fs / 32;
-        ok &= map_q4_codes(p, &a.tm_gate, w->gate.data, E, F, d, fs, kb);
-        ok &= map_q4_codes(p, &a.tm_up, w->up.data, E, F, d, fs, kb);
-        ok &= map_q4_codes(p, &a.tm_down, w->down.data, E, d, F, 128, nb);
-        ok &= map_q4_scales(p, &a.tm_gate_sc, w->gate.scales, E, F, d, fs, kb);
-        ok &= map_q4_scales(p, &a.tm_up_sc, w->up.scales, E, F, d, fs, kb);
-        ok &= map_q4_scales(p, &a.tm_down_sc, w->down.scales, E, d, F, 128, nb);
+        const uint32_t cb = c.wfmt == MOE_WFMT_Q8_0 ? 32 : 16;
+        ok &= map_quant_codes(p, &a.tm_gate, w->gate.data, E, F, d, fs, kb, cb);
+        ok &= map_quant_codes(p, &a.tm_up, w->up.data, E, F, d, fs, kb, cb);
+        ok &= map_quant_codes(p, &a.tm_down, w->down.data, E, d, F, kQuantDownBoxRows, nb, cb);
+        ok &= map_quant_scales(p, &a.tm_gate_sc, w->gate.scales, E, F, d, fs, kb);
+        ok &= map_quant_scales(p, &a.tm_up_sc, w->up.scales, E, F, d, fs, kb);
+        ok &= map_quant_scales(p, &a.tm_down_sc, w->down.scales, E, d, F, kQuantDownBoxRows, nb);
         if (S) {
-            ok &= map_q4_codes(p, &a.tm_sgate, w->shared_gate.data, S, Fs, d, fs, kb);
-            ok &= map_q4_codes(p, &a.tm_sup, w->shared_up.data, S, Fs, d, fs, kb);
-            ok &= map_q4_codes(p, &a.tm_sdown, w->shared_down.data, S, d, Fs, 128, nb);
-            ok &= map_q4_scales(p, &a.tm_sgate_sc, w->shared_gate.scales, S, Fs, d, fs, kb);
-            ok &= map_q4_scales(p, &a.tm_sup_sc, w->shared_up.scales, S, Fs, d, fs, kb);
-            ok &= map_q4_scales(p, &a.tm_sdown_sc, w->shared_down.scales, S, d, Fs, 128, nb);
+            ok &= map_quant_codes(p, &a.tm_sgate, w->shared_gate.data, S, Fs, d, fs, kb, cb);
+            ok &= map_quant_codes(p, &a.tm_sup, w->shared_up.data, S, Fs, d, fs, kb, cb);
+            ok &= map_quant_codes(p, &a.tm_sdown, w->shared_down.data, S, d, Fs, kQuantDownBoxRows, nb, cb);
+            ok &= map_quant_scales(p, &a.tm_sgate_sc, w->shared_gate.scales, S, Fs, d, fs, kb);
+            ok &= map_quant_scales(p, &a.tm_sup_sc, w->shared_up.scales, S, Fs, d, fs, kb);
+            ok &= map_quant_scales(p, &a.tm_sdown_sc, w->shared_down.scales, S, d, Fs, kQuantDownBoxRows, nb);
         }
     }
     if (!ok) return nullptr;
@@ -257,7 +260,6 @@ moe_status_t route_decode(moe_plan_s* p, const moe_weights_t* w, const void* x, 
 moe_status_t decode_args(moe_plan_s* p, const moe_weights_t* w, const void* x, int T, float* out,
                          bool fused, DecodeArgs** out_args, int* out_fs, size_t* out_smem) {
     const moe_config_t& c = p->cfg;
-    const bool q4 = c.wfmt == MOE_WFMT_Q4_0;
     const int fs = pick_fs(p, T);
     DecodeArgs* ap = build_decode_maps(p, w, fs);
     if (!ap) return MOE_ERR_INVALID_ARG;
@@ -282,8 +284,8 @@ moe_status_t decode_args(moe_plan_s* p, const moe_weights_t* w, const void* x, i
     a.ws = p->ws;
     a.gbar = p->ws.gbar;
     const size_t extra = fused ? decode_fused_extra_smem() : 0;
-    const size_t fixed = decode_smem_bytes(fs, q4, c.d_model, 0) + extra;
-    const int stage = decode_stage_bytes(fs, q4);
+    const size_t fixed = decode_smem_bytes(fs, c.wfmt, c.d_model, 0) + extra;
+    const int stage = decode_stage_bytes(fs, c.wfmt);
     int ns = static_cast<int>((p->smem_optin - fixed) / (stage + 16));
     if (ns > 8) ns = 8;
     if (ns < 2) return MOE_ERR_UNSUPPORTED;
@@ -293,7 +295,7 @@ moe_status_t decode_args(moe_plan_s* p, const moe_weights_t* w, const void* x, i
     a.n_stages = ns;
     *out_args = ap;
     *out_fs = fs;
-    *out_smem = decode_smem_bytes(fs, q4, c.d_model, ns) + extra;
+    *out_smem = decode_smem_bytes(fs, c.wfmt, c.d_model, ns) + extra;
     return MOE_OK;
 }
 
@@ -304,8 +306,7 @@ moe_status_t experts_decode(moe_plan_s* p, const moe_weights_t* w, const void* x
     size_t smem = 0;
     moe_status_t s = decode_args(p, w, x, T, out, false, &a, &fs, &smem);
     if (s) return s;
-    return cuda_status(launch_decode_experts(*a, fs, p->cfg.wfmt == MOE_WFMT_Q4_0, p->num_sms,
-                                             smem, st));
+    return cuda_status(launch_decode_experts(*a, fs, p->cfg.wfmt, p->num_sms, smem, st));
 }
 
 moe_status_t forward_decode_fused(moe_plan_s* p, const moe_weights_t* w, const void* x, int T,
@@ -315,8 +316,7 @@ moe_status_t forward_decode_fused(moe_plan_s* p, const moe_weights_t* w, const v
     size_t smem = 0;
     moe_status_t s = decode_args(p, w, x, T, out, true, &a, &fs, &smem);
     if (s) return s;
-    return cuda_status(launch_decode_fused(*a, fs, p->cfg.wfmt == MOE_WFMT_Q4_0, p->num_sms, smem,
-                                           st));
+    return cuda_status(launch_decode_fused(*a, fs, p->cfg.wfmt, p->num_sms, smem, st));
 }
 
 moe_status_t copy_routing(moe_plan_s* p, int T, moe_routing_t* r, cudaStream_t st) {
@@ -566,8 +566,12 @@ moe_status_t moe_debug_stall_barrier(moe_plan_t p, void* stream) {
     if (!p) return MOE_ERR_INVALID_ARG;
     if (!p->coop) return MOE_ERR_UNSUPPORTED;
     DeviceGuard dg(p->cfg.device);
-    // an arrival count no launch can complete (each arrival adds 1)
-    return cuda_status(cudaMemsetAsync(p->ws.gbar, 0x40, 4, static_cast<cudaStream_t>(stream)));
+    // an arrival count of 1 (not a multiple of the grid): after the next
+    // launch's G arrivals the count is G + 1, short of the target 2G of the
+    // CTA that arrives last, whose bounded wait runs out
+    cudaError_t e = cudaMemsetAsync(p->ws.gbar, 0, 16, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess) e = cudaMemsetAsync(p->ws.gbar, 0x01, 1, static_cast<cudaStream_t>(stream));
+    return cuda_status(e);
 }
 
 moe_status_t moe_q4_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k, size_t* code_bytes,
@@ -586,6 +590,27 @@ moe_status_t moe_q4_0_pack(const void* blocks, int64_t n_mats, int64_t rows, int
     if (!blocks || !codes || !scales || !aligned16(codes) || !aligned16(scales))
         return MOE_ERR_INVALID_ARG;
     return cuda_status(launch_q4_0_pack(static_cast<const uint8_t*>(blocks), n_mats, rows, k,
+                                        static_cast<uint8_t*>(codes),
+                                        static_cast<uint16_t*>(scales),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_q8_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k, size_t* code_bytes,
+                                   size_t* scale_bytes) {
+    if (n_mats < 0 || rows < 0 || k < 0 || k % 32 != 0) return MOE_ERR_INVALID_ARG;
+    const int64_t blocks = n_mats * rows * (k / 32);
+    if (code_bytes) *code_bytes = static_cast<size_t>(blocks) * 32;
+    if (scale_bytes) *scale_bytes = static_cast<size_t>(blocks) * 2;
+    return MOE_OK;
+}
+
+moe_status_t moe_q8_0_pack(const void* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                           void* codes, void* scales, void* stream) {
+    if (n_mats < 0 || rows < 0 || k < 0 || k % 32 != 0) return MOE_ERR_INVALID_ARG;
+    if (n_mats * rows * k == 0) return MOE_OK;
+    if (!blocks || !codes || !scales || !aligned16(codes) || !aligned16(scales))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_q8_0_pack(static_cast<const uint8_t*>(blocks), n_mats, rows, k,
                                         static_cast<uint8_t*>(codes),
                                         static_cast<uint16_t*>(scales),
                                         static_cast<cudaStream_t>(stream)));

@@ -220,20 +220,34 @@ constexpr int kConsumerWarps = 16;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumers + 32;   // + one producer warp
 
-template <int FS, bool Q4>
+// Weight formats of the decode kernels (the values of moe_wfmt_t).
+constexpr int kWfBf16 = 0, kWfQ4 = 1, kWfQ8 = 2;
+
+// The constant that turns the bf16 "128 + nibble" operands back into signed
+// codes (see q4_raw): Q4_0 subtracts 128 + 8; Q8_0, whose biased byte
+// u = q + 128 = 16 hi + lo enters as two nibble planes weighted 1 and 16,
+// subtracts 128 + 16 * 128 + 128.
+constexpr float quant_offset(int wf) { return wf == kWfQ8 ? 2304.f : 136.f; }
+
+template <int FS, int WF>
 struct DecodeCfg {
     static constexpr int RG = FS / 16;            // 16-row groups in a slice
     static constexpr int ROLES = 2 * RG;          // (matrix, row group) pairs of phase A
     static constexpr int KSPLIT = kConsumerWarps / ROLES;
     static_assert(KSPLIT >= 1 && ROLES * KSPLIT == kConsumerWarps, "warp roles");
-    static_assert(!Q4 || FS >= 32, "Q4_0 slices hold whole blocks");
+    static constexpr bool QUANT = WF != kWfBf16;
+    static_assert(!QUANT || FS >= 32, "quantised slices hold whole blocks");
+    static constexpr int CB = WF == kWfQ8 ? 32 : 16;   // code bytes of one block row
+    static constexpr int BR = CB + 2;                  // + its fp16 scale
     // bf16: phase A stage = gate+up [FS rows][KT cols]; phase B = down [RJ rows][FS cols]
-    // Q4_0: phase A stage = gate+up [KB block cols][FS rows]; phase B = [NB][RJ rows]
-    static constexpr int STAGE = Q4 ? 2 * 512 * 18 : 32768;
+    // Q4_0 / Q8_0: phase A stage = gate+up [KB block cols][FS rows];
+    //              phase B = [NB block cols][RJ rows]; codes, then the scales
+    static constexpr int STAGE = QUANT ? 2 * 512 * BR : 32768;
     static constexpr int KT = 8192 / FS;          // bf16 phase A k columns
-    static constexpr int KB = 512 / FS;           // Q4_0 phase A block columns
-    static constexpr int NB = FS / 32;            // Q4_0 block columns in a slice
-    static constexpr int RJ = Q4 ? 32768 / FS : 16384 / FS;   // phase B rows per stage
+    static constexpr int KB = 512 / FS;           // quantised phase A block columns
+    static constexpr int NB = FS / 32;            // quantised block columns in a slice
+    static constexpr int RJ = QUANT ? 32768 / FS : 16384 / FS;   // phase B rows per stage
+    static_assert(!QUANT || RJ % kQuantDownBoxRows == 0, "whole down boxes per stage");
     static constexpr int HS = FS + 8;             // h row stride (bf16 elements)
     static constexpr int GS = FS + 4;             // gate/up result row stride (floats)
 };
@@ -252,6 +266,83 @@ __device__ __forceinline__ uint32_t q4_raw(uint32_t w, int s) {
     return ((w >> s) & 0x000F000Fu) | 0x43004300u;
 }
 
+// One quantised block (32 weights along k) of rows r and r+8 of an mma A
+// tile, times the B fragment of the same 32 k (b0 b1: k 0-15, b2 b3: k
+// 16-31).  row_r / row_r8 point at the rows' packed code words; c0, c1 are
+// the accumulator start values of the lane's two token columns.  v gets the
+// block's four dot products before the block scale.
+//   Q4_0: one word per lane holds 8 codes, both 16-wide halves;
+//   Q8_0: the biased byte u = q + 128 is two Q4_0-packed nibble planes
+//         (words 2 tig = low nibbles, 2 tig + 1 = high nibbles), weighted 1
+//         and 16.
+template <int WF>
+__device__ __forceinline__ void quant_block_a(const uint32_t* row_r, const uint32_t* row_r8,
+                                              int tig, float c0, float c1, uint32_t b0,
+                                              uint32_t b1, uint32_t b2, uint32_t b3, float v[4]) {
+    if constexpr (WF == kWfQ4) {
+        const uint32_t w0 = row_r[tig], w8 = row_r8[tig];
+        // the two halves go to independent accumulators; the first starts at c
+        float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_bf16_16816(cb0, q4_raw(w0, 0), q4_raw(w8, 0), q4_raw(w0, 4), q4_raw(w8, 4), b0, b1);
+        mma_bf16_16816(cb1, q4_raw(w0, 8), q4_raw(w8, 8), q4_raw(w0, 12), q4_raw(w8, 12), b2, b3);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = cb0[i] + cb1[i];
+    } else {
+        const uint2 p = reinterpret_cast<const uint2*>(row_r)[tig];
+        const uint2 q = reinterpret_cast<const uint2*>(row_r8)[tig];
+        float cl[4] = {c0, c1, c0, c1}, ch[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_bf16_16816(cl, q4_raw(p.x, 0), q4_raw(q.x, 0), q4_raw(p.x, 4), q4_raw(q.x, 4), b0, b1);
+        mma_bf16_16816(ch, q4_raw(p.y, 0), q4_raw(q.y, 0), q4_raw(p.y, 4), q4_raw(q.y, 4), b0, b1);
+        mma_bf16_16816(cl, q4_raw(p.x, 8), q4_raw(q.x, 8), q4_raw(p.x, 12), q4_raw(q.x, 12), b2, b3);
+        mma_bf16_16816(ch, q4_raw(p.y, 8), q4_raw(q.y, 8), q4_raw(p.y, 12), q4_raw(q.y, 12), b2, b3);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = fmaf(16.f, ch[i], cl[i]);
+    }
+}
+
+// The same for the down contraction, whose B operand is h as a bf16 pair:
+// bh / bl hold the hi and lo fragments of the block's two 16-wide halves.
+template <int WF>
+__device__ __forceinline__ void quant_block_b(const uint32_t* row_r, const uint32_t* row_r8,
+                                              int tig, float c0, float c1, const uint32_t* bh0,
+                                              const uint32_t* bh1, const uint32_t* bl0,
+                                              const uint32_t* bl1, float v[4]) {
+    if constexpr (WF == kWfQ4) {
+        const uint32_t w0 = row_r[tig], w8 = row_r8[tig];
+        const uint32_t p0 = q4_raw(w0, 0), q0 = q4_raw(w8, 0), p1 = q4_raw(w0, 4), q1 = q4_raw(w8, 4);
+        const uint32_t p2 = q4_raw(w0, 8), q2 = q4_raw(w8, 8), p3 = q4_raw(w0, 12), q3 = q4_raw(w8, 12);
+        float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_bf16_16816(cb0, p0, q0, p1, q1, bh0[0], bh0[1]);
+        mma_bf16_16816(cb1, p2, q2, p3, q3, bh1[0], bh1[1]);
+        mma_bf16_16816(cb0, p0, q0, p1, q1, bl0[0], bl0[1]);
+        mma_bf16_16816(cb1, p2, q2, p3, q3, bl1[0], bl1[1]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = cb0[i] + cb1[i];
+    } else {
+        const uint2 p = reinterpret_cast<const uint2*>(row_r)[tig];
+        const uint2 q = reinterpret_cast<const uint2*>(row_r8)[tig];
+        float cl[4] = {c0, c1, c0, c1}, ch[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const uint32_t p0 = q4_raw(p.x, 0), q0 = q4_raw(q.x, 0), p1 = q4_raw(p.x, 4), q1 = q4_raw(q.x, 4);
+            const uint32_t p2 = q4_raw(p.x, 8), q2 = q4_raw(q.x, 8), p3 = q4_raw(p.x, 12), q3 = q4_raw(q.x, 12);
+            mma_bf16_16816(cl, p0, q0, p1, q1, bh0[0], bh0[1]);
+            mma_bf16_16816(cl, p2, q2, p3, q3, bh1[0], bh1[1]);
+            mma_bf16_16816(cl, p0, q0, p1, q1, bl0[0], bl0[1]);
+            mma_bf16_16816(cl, p2, q2, p3, q3, bl1[0], bl1[1]);
+        }
+        {
+            const uint32_t p0 = q4_raw(p.y, 0), q0 = q4_raw(q.y, 0), p1 = q4_raw(p.y, 4), q1 = q4_raw(q.y, 4);
+            const uint32_t p2 = q4_raw(p.y, 8), q2 = q4_raw(q.y, 8), p3 = q4_raw(p.y, 12), q3 = q4_raw(q.y, 12);
+            mma_bf16_16816(ch, p0, q0, p1, q1, bh0[0], bh0[1]);
+            mma_bf16_16816(ch, p2, q2, p3, q3, bh1[0], bh1[1]);
+            mma_bf16_16816(ch, p0, q0, p1, q1, bl0[0], bl0[1]);
+            mma_bf16_16816(ch, p2, q2, p3, q3, bl1[0], bl1[1]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[i] = fmaf(16.f, ch[i], cl[i]);
+    }
+}
+
 // Work list the experts pipeline reads: generic pointers, so the same code
 // serves the two-launch path (global memory, written by the router kernel)
 // and the fused kernel (shared memory, computed by every CTA itself).
@@ -266,19 +357,19 @@ struct WorkView {
 struct DecodeSmem {
     uint8_t* ring;
     uint8_t* xs;            // [8][xs_stride]: the T token rows of x, staged once
-    float* xsum;            // [8][d/32]: -136 * block sums of x (Q4_0 only)
+    float* xsum;            // [8][d/32]: -offset * block sums of x (quantised formats)
     float* gu;              // [KSPLIT][2][8][GS]: gate / up partial results
     __nv_bfloat16* hhi;     // [8][HS]: h = hi + lo, per slot
     __nv_bfloat16* hlo;
-    float* hsum;            // [8][2]: -136 * block sums of hi + lo (Q4_0 only)
+    float* hsum;            // [8][2]: -offset * block sums of hi + lo (quantised formats)
     DecodeSmemTail* tail;
     uint64_t* full;
     uint64_t* empty;
 };
 
-template <int FS, bool Q4>
+template <int FS, int WF>
 __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const DecodeArgs& a) {
-    using C = DecodeCfg<FS, Q4>;
+    using C = DecodeCfg<FS, WF>;
     DecodeSmem sm;
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -297,9 +388,10 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
 
 // Consumer threads copy the T token rows of x into shared memory once per
 // launch; every work unit then addresses its tokens' rows directly.  For
-// Q4_0 the same pass stores -136 * (sum of each 32-wide block of a row), the
-// starting value of that block's accumulator (see q4_raw).
-template <bool Q4>
+// the quantised formats the same pass stores -offset * (sum of each 32-wide
+// block of a row), the starting value of that block's accumulator (see
+// q4_raw and quant_offset).
+template <int WF>
 __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& sm, int tid) {
     const int nkb = a.d / 32;
     for (int idx = tid; idx < a.T * nkb; idx += kConsumers) {
@@ -311,14 +403,14 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
         for (int c = 0; c < 4; ++c) {
             const uint4 v = __ldg(src + c);
             dst[c] = v;
-            if constexpr (Q4) {
+            if constexpr (WF != kWfBf16) {
                 const uint32_t q[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     s += __uint_as_float(q[j] << 16) + __uint_as_float(q[j] & 0xffff0000u);
             }
         }
-        if constexpr (Q4) sm.xsum[t * nkb + kb] = -136.f * s;
+        if constexpr (WF != kWfBf16) sm.xsum[t * nkb + kb] = -quant_offset(WF) * s;
     }
 }
 
@@ -327,10 +419,10 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
 // (assignment to CTAs: see experts_pipeline).  The last warp (lane 0) is the
 // TMA producer, the others consume.  Barriers must be initialised by the
 // caller.
-template <int FS, bool Q4>
+template <int FS, int WF>
 __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const DecodeSmem& sm,
                                                  const WorkView& wv) {
-    using C = DecodeCfg<FS, Q4>;
+    using C = DecodeCfg<FS, WF>;
     const int ns = a.n_stages;
     uint8_t* ring = sm.ring;
     float* gu = sm.gu;
@@ -346,21 +438,19 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
     const int sl_r = a.F / FS, sl_s = a.S ? a.Fs / FS : 0;
     const int n_su = n_shared * sl_s;
     const int n_units = n_su + n_routed * sl_r;
-    const int nA = Q4 ? (d / 32 + C::KB - 1) / C::KB : (d + C::KT - 1) / C::KT;
+    const int nA = C::QUANT ? (d / 32 + C::KB - 1) / C::KB : (d + C::KT - 1) / C::KT;
     const int nB = (d + C::RJ - 1) / C::RJ;
     volatile int* abort_flag = &tail->abort_flag;
 
-    // Unit assignment.  When an expert has at least as many slices as there
-    // are CTAs, CTA b takes units b, b+G, ...: the CTAs stream neighbouring
-    // slices of one expert together and each keeps its x rows staged across
-    // units.  Otherwise CTA b takes the contiguous range [b*U/G, (b+1)*U/G),
-    // so that its consecutive units still share an expert.
-    const bool interleave = sl_r >= static_cast<int>(gridDim.x);
-    const int u_begin = interleave ? static_cast<int>(blockIdx.x)
-        : static_cast<int>((static_cast<long long>(blockIdx.x) * n_units) / gridDim.x);
-    const int u_end = interleave ? n_units
-        : static_cast<int>((static_cast<long long>(blockIdx.x + 1) * n_units) / gridDim.x);
-    const int u_step = interleave ? static_cast<int>(gridDim.x) : 1;
+    // Unit assignment: CTA b takes units b, b+G, b+2G, ...  At any moment the
+    // CTAs stream neighbouring slices of the same expert, so DRAM pages and
+    // L2 lines are shared by requests that arrive together.  (Every unit
+    // reads its tokens' rows of x from the copy staged once per CTA, so
+    // nothing is lost when consecutive units of a CTA belong to different
+    // experts.)
+    const int u_begin = static_cast<int>(blockIdx.x);
+    const int u_end = n_units;
+    const int u_step = static_cast<int>(gridDim.x);
 
     // unit -> (item index, slice): shared units first
     auto unit_item = [&](int u, int& ii, int& sl) {
@@ -374,6 +464,12 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             prefetch_tensormap(&a.tm_down);
             if (a.S) { prefetch_tensormap(&a.tm_sgate); prefetch_tensormap(&a.tm_sup);
                        prefetch_tensormap(&a.tm_sdown); }
+            if constexpr (C::QUANT) {
+                prefetch_tensormap(&a.tm_gate_sc); prefetch_tensormap(&a.tm_up_sc);
+                prefetch_tensormap(&a.tm_down_sc);
+                if (a.S) { prefetch_tensormap(&a.tm_sgate_sc); prefetch_tensormap(&a.tm_sup_sc);
+                           prefetch_tensormap(&a.tm_sdown_sc); }
+            }
             const uint64_t pol = l2_policy_evict_first();
             uint32_t it = 0;
             bool ok = true;
@@ -400,7 +496,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                     }
                     uint8_t* dst = ring + static_cast<size_t>(slot) * C::STAGE;
                     if (st < nA) {
-                        if constexpr (!Q4) {
+                        if constexpr (!C::QUANT) {
                             const int k0 = st * C::KT;
                             const int nbox = min(C::KT, d - k0) / 64;
                             mbar_arrive_expect_tx(&full[slot], 2 * nbox * FS * 128);
@@ -413,30 +509,34 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         } else {
                             const int kb0 = st * C::KB;
                             const int c2 = ex * (d / 32) + kb0;
-                            mbar_arrive_expect_tx(&full[slot], 2 * C::KB * FS * 18);
+                            mbar_arrive_expect_tx(&full[slot], 2 * C::KB * FS * C::BR);
                             uint8_t* g = dst;
-                            uint8_t* u2 = dst + C::KB * FS * 18;
+                            uint8_t* u2 = dst + C::KB * FS * C::BR;
                             tma_load_3d(g, mg, &full[slot], 0, f0, c2, pol);
-                            tma_load_2d(g + C::KB * FS * 16, mgs, &full[slot], f0, c2, pol);
+                            tma_load_2d(g + C::KB * FS * C::CB, mgs, &full[slot], f0, c2, pol);
                             tma_load_3d(u2, mu, &full[slot], 0, f0, c2, pol);
-                            tma_load_2d(u2 + C::KB * FS * 16, mus, &full[slot], f0, c2, pol);
+                            tma_load_2d(u2 + C::KB * FS * C::CB, mus, &full[slot], f0, c2, pol);
                         }
                     } else {
                         const int j0 = (st - nA) * C::RJ;
-                        const int nbox = min(C::RJ, d - j0) / 128;
-                        if constexpr (!Q4) {
+                        if constexpr (!C::QUANT) {
+                            const int nbox = min(C::RJ, d - j0) / 128;
                             mbar_arrive_expect_tx(&full[slot], nbox * 128 * FS * 2);
                             for (int b = 0; b < nbox; ++b)
                                 tma_load_2d(dst + b * 128 * FS * 2, md, &full[slot], f0,
                                             ex * d + j0 + 128 * b, pol);
                         } else {
+                            // boxes of QB rows; rows past d (d is a multiple of 128)
+                            // are out of the map and arrive as zeros
+                            constexpr int QB = kQuantDownBoxRows;
+                            const int nbox = (min(C::RJ, d - j0) + QB - 1) / QB;
                             const int c2 = ex * (Fh / 32) + f0 / 32;
-                            mbar_arrive_expect_tx(&full[slot], nbox * C::NB * 128 * 18);
+                            mbar_arrive_expect_tx(&full[slot], nbox * C::NB * QB * C::BR);
                             for (int b = 0; b < nbox; ++b) {
-                                uint8_t* bd = dst + b * (C::NB * 128 * 18);
-                                tma_load_3d(bd, md, &full[slot], 0, j0 + 128 * b, c2, pol);
-                                tma_load_2d(bd + C::NB * 128 * 16, mds, &full[slot],
-                                            j0 + 128 * b, c2, pol);
+                                uint8_t* bd = dst + b * (C::NB * QB * C::BR);
+                                tma_load_3d(bd, md, &full[slot], 0, j0 + QB * b, c2, pol);
+                                tma_load_2d(bd + C::NB * QB * C::CB, mds, &full[slot],
+                                            j0 + QB * b, c2, pol);
                             }
                         }
                     }
@@ -499,7 +599,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             const bool ok = wait_full(slot, (it / ns) & 1);
             const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
             if (ok) {
-                if constexpr (!Q4) {
+                if constexpr (!C::QUANT) {
                     const int k0 = st * C::KT;
                     const int kmax = min(C::KT, d - k0) / 16;
                     const uint32_t tile = smem_u32(stage) + mat * (FS * C::KT * 2);
@@ -517,32 +617,27 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                 } else {
                     const int kb0 = st * C::KB;
                     const int nkb_st = min(C::KB, nkb - kb0);
-                    const uint8_t* mb = stage + mat * (C::KB * FS * 18);
-                    const uint32_t* codes = reinterpret_cast<const uint32_t*>(mb);
-                    const __half* scl = reinterpret_cast<const __half*>(mb + C::KB * FS * 16);
+                    const uint8_t* mb = stage + mat * (C::KB * FS * C::BR);
+                    const uint32_t* codes = reinterpret_cast<const uint32_t*>(mb);   // [KB][FS][CB]
+                    const __half* scl = reinterpret_cast<const __half*>(mb + C::KB * FS * C::CB);
                     const int r0 = rg * 16 + g;
                     const float* xsum0 = sm.xsum + tok0 * nkb + kb0;
                     const float* xsum1 = sm.xsum + tok1 * nkb + kb0;
 #pragma unroll 2
                     for (int bb = ks; bb < nkb_st; bb += C::KSPLIT) {
-                        const uint32_t w0c = codes[(bb * FS + r0) * 4 + tig];
-                        const uint32_t w8c = codes[(bb * FS + r0 + 8) * 4 + tig];
+                        const uint32_t* row = codes + (bb * FS + r0) * (C::CB / 4);
                         uint32_t b0, b1, b2, b3;
                         ldsm_x4(xrow + ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
-                        // the block's two 16-wide halves go to independent
-                        // accumulators; the first starts at -136 * sum(x)
-                        const float c0 = xsum0[bb], c1 = xsum1[bb];
-                        float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_bf16_16816(cb0, q4_raw(w0c, 0), q4_raw(w8c, 0), q4_raw(w0c, 4),
-                                       q4_raw(w8c, 4), b0, b1);
-                        mma_bf16_16816(cb1, q4_raw(w0c, 8), q4_raw(w8c, 8), q4_raw(w0c, 12),
-                                       q4_raw(w8c, 12), b2, b3);
+                        float v[4];
+                        // the accumulator starts at -offset * sum(x) of the block
+                        quant_block_a<WF>(row, row + 8 * (C::CB / 4), tig, xsum0[bb], xsum1[bb],
+                                          b0, b1, b2, b3, v);
                         const float s0 = __half2float(scl[bb * FS + r0]);
                         const float s8 = __half2float(scl[bb * FS + r0 + 8]);
-                        cacc[0] = fmaf(s0, cb0[0] + cb1[0], cacc[0]);
-                        cacc[1] = fmaf(s0, cb0[1] + cb1[1], cacc[1]);
-                        cacc[2] = fmaf(s8, cb0[2] + cb1[2], cacc[2]);
-                        cacc[3] = fmaf(s8, cb0[3] + cb1[3], cacc[3]);
+                        cacc[0] = fmaf(s0, v[0], cacc[0]);
+                        cacc[1] = fmaf(s0, v[1], cacc[1]);
+                        cacc[2] = fmaf(s8, v[2], cacc[2]);
+                        cacc[3] = fmaf(s8, v[3], cacc[3]);
                     }
                 }
             }
@@ -576,11 +671,11 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             hhi[t * C::HS + f] = hi;
             hlo[t * C::HS + f] = lo;
-            if constexpr (Q4) {
+            if constexpr (C::QUANT) {
                 float hs = __bfloat162float(hi) + __bfloat162float(lo);
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
-                if (lane == 0) sm.hsum[t * 2 + f / 32] = -136.f * hs;
+                if (lane == 0) sm.hsum[t * 2 + f / 32] = -quant_offset(WF) * hs;
             }
         }
         named_bar_sync(1, kConsumers);
@@ -592,7 +687,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             ldsm_x2(smem_u32(hlo) + off, bl[kk][0], bl[kk][1]);
         }
         float hs0[C::NB > 0 ? C::NB : 1], hs1[C::NB > 0 ? C::NB : 1];
-        if constexpr (Q4) {
+        if constexpr (C::QUANT) {
 #pragma unroll
             for (int bb = 0; bb < C::NB; ++bb) {
                 hs0[bb] = sm.hsum[t0 * 2 + bb];
@@ -610,7 +705,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             if (ok) {
                 for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
                     float c[4] = {0.f, 0.f, 0.f, 0.f};
-                    if constexpr (!Q4) {
+                    if constexpr (!C::QUANT) {
                         const uint32_t tile = smem_u32(stage);
                         const int m = lane >> 3, r = lane & 7;
                         const uint32_t arow = rgb * 16 + ((m & 1) << 3) + r;
@@ -622,32 +717,24 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                             mma_bf16_16816(c, a0, a1, a2, a3, bl[kk][0], bl[kk][1]);
                         }
                     } else {
-                        const uint8_t* bbase = stage + (rgb >> 3) * (C::NB * 128 * 18);
-                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);
-                        const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * 128 * 16);
-                        const int rib = (rgb & 7) * 16 + g;
+                        constexpr int QB = kQuantDownBoxRows;
+                        const uint8_t* bbase = stage + (rgb / (QB / 16)) * (C::NB * QB * C::BR);
+                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);   // [NB][128][CB]
+                        const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * QB * C::CB);
+                        const int rib = (rgb % (QB / 16)) * 16 + g;
 #pragma unroll
                         for (int bb = 0; bb < C::NB; ++bb) {
-                            const uint32_t w0c = codes[(bb * 128 + rib) * 4 + tig];
-                            const uint32_t w8c = codes[(bb * 128 + rib + 8) * 4 + tig];
-                            const uint32_t p0 = q4_raw(w0c, 0), q0 = q4_raw(w8c, 0);
-                            const uint32_t p1 = q4_raw(w0c, 4), q1 = q4_raw(w8c, 4);
-                            const uint32_t p2 = q4_raw(w0c, 8), q2 = q4_raw(w8c, 8);
-                            const uint32_t p3 = q4_raw(w0c, 12), q3 = q4_raw(w8c, 12);
-                            // two independent accumulator chains (halves of the
-                            // block); the first starts at -136 * sum(hi + lo)
-                            float cb0[4] = {hs0[bb], hs1[bb], hs0[bb], hs1[bb]};
-                            float cb1[4] = {0.f, 0.f, 0.f, 0.f};
-                            mma_bf16_16816(cb0, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1]);
-                            mma_bf16_16816(cb1, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
-                            mma_bf16_16816(cb0, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
-                            mma_bf16_16816(cb1, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
-                            const float s0 = __half2float(scl[bb * 128 + rib]);
-                            const float s8 = __half2float(scl[bb * 128 + rib + 8]);
-                            c[0] = fmaf(s0, cb0[0] + cb1[0], c[0]);
-                            c[1] = fmaf(s0, cb0[1] + cb1[1], c[1]);
-                            c[2] = fmaf(s8, cb0[2] + cb1[2], c[2]);
-                            c[3] = fmaf(s8, cb0[3] + cb1[3], c[3]);
+                            const uint32_t* row = codes + (bb * QB + rib) * (C::CB / 4);
+                            float v[4];
+                            // the accumulator starts at -offset * sum(hi + lo) of the block
+                            quant_block_b<WF>(row, row + 8 * (C::CB / 4), tig, hs0[bb], hs1[bb],
+                                              bh[2 * bb], bh[2 * bb + 1], bl[2 * bb], bl[2 * bb + 1], v);
+                            const float s0 = __half2float(scl[bb * QB + rib]);
+                            const float s8 = __half2float(scl[bb * QB + rib + 8]);
+                            c[0] = fmaf(s0, v[0], c[0]);
+                            c[1] = fmaf(s0, v[1], c[1]);
+                            c[2] = fmaf(s8, v[2], c[2]);
+                            c[3] = fmaf(s8, v[3], c[3]);
                         }
                     }
                     const int j = j0 + rgb * 16 + g;
@@ -668,11 +755,11 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
 }
 
 
-template <int FS, bool Q4>
+template <int FS, int WF>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const DecodeSmem sm = decode_smem<FS, Q4>(smem_raw, a);
+    const DecodeSmem sm = decode_smem<FS, WF>(smem_raw, a);
     if (threadIdx.x == 0) {
         for (int s = 0; s < a.n_stages; ++s) {
             mbar_init(&sm.full[s], 1);
@@ -681,10 +768,10 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
         sm.tail->abort_flag = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x < kConsumers) stage_x<Q4>(a, sm, threadIdx.x);
+    if (threadIdx.x < kConsumers) stage_x<WF>(a, sm, threadIdx.x);
     __syncthreads();
     const WorkView wv{a.n_items[0], a.n_items[1], a.items, a.slot_token, a.slot_w};
-    experts_pipeline<FS, Q4>(a, sm, wv);
+    experts_pipeline<FS, WF>(a, sm, wv);
 }
 
 // ====================================================== fused decode ===
@@ -708,10 +795,8 @@ struct alignas(16) FusedRouteSmem {
     float w[kFusedMaxPairs];
     int slot_token[kFusedMaxPairs];
     float slot_w[kFusedMaxPairs];
-    int lt[kFusedMaxPairs];
-    int cnt[kFusedMaxPairs];
-    int first[kFusedMaxPairs];
     float sel[kDecodeTok][kMaxTopK];
+    uint32_t emask[kMaxExperts / 32];   // bit e: expert e was selected by some token
     int n_routed;
     int pad[3];
 };
@@ -719,32 +804,30 @@ struct alignas(16) FusedRouteSmem {
 size_t decode_fused_extra_smem() { return sizeof(FusedRouteSmem); }
 
 // Grid-wide barrier of a cooperative launch; thread 0 of each CTA calls it.
+// gbar[0..1] is a 64-bit arrival counter that only grows: the G CTAs of one
+// launch raise it from n*G to (n+1)*G.  Each CTA takes its launch's target
+// from the value its own arrival returned and polls until the counter
+// reaches it (one atomic per CTA, no reset, no second word to publish).
+// The count starts at a multiple of G as long as every earlier launch
+// arrived completely; after a timed-out wait the host resets it to 0.
 __device__ __forceinline__ bool grid_barrier(uint32_t* gbar, uint32_t nblocks) {
-    volatile uint32_t* gen_p = gbar + 1;
-    const uint32_t gen = *gen_p;
-    __threadfence();
-    const uint32_t arrived = atomicAdd(gbar, 1u);
-    if (arrived == nblocks - 1) {
-        *gbar = 0u;                  // ready for the next launch
-        __threadfence();
-        atomicAdd(gbar + 1, 1u);
-        return true;
-    }
+    unsigned long long* ctr = reinterpret_cast<unsigned long long*>(gbar);
+    __threadfence();                       // this CTA's logits before its arrival
+    const unsigned long long old = atomicAdd(ctr, 1ull);
+    const unsigned long long target = old - old % nblocks + nblocks;
     const uint64_t t0 = globaltimer_ns();
-    while (*gen_p == gen) {
+    while (ld_acquire_u64(ctr) < target) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
-        __nanosleep(64);
     }
-    __threadfence();
     return true;
 }
 
-template <int FS, bool Q4>
+template <int FS, int WF>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
-    using C = DecodeCfg<FS, Q4>;
+    using C = DecodeCfg<FS, WF>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    const DecodeSmem sm = decode_smem<FS, Q4>(smem_raw, a);
+    const DecodeSmem sm = decode_smem<FS, WF>(smem_raw, a);
     FusedRouteSmem* rs = reinterpret_cast<FusedRouteSmem*>(sm.empty + a.n_stages);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = a.T, d = a.d, E = a.E, k = a.k, S = a.S;
@@ -759,9 +842,24 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
     }
     __syncthreads();
 
+    // the producer warp idles through R and T: fetch the tensor maps now, so
+    // the first TMA of phase X does not wait for them
+    if (warp == kConsumerWarps && lane == 0) {
+        prefetch_tensormap(&a.tm_gate); prefetch_tensormap(&a.tm_up); prefetch_tensormap(&a.tm_down);
+        if (S) { prefetch_tensormap(&a.tm_sgate); prefetch_tensormap(&a.tm_sup);
+                 prefetch_tensormap(&a.tm_sdown); }
+        if constexpr (C::QUANT) {
+            prefetch_tensormap(&a.tm_gate_sc); prefetch_tensormap(&a.tm_up_sc);
+            prefetch_tensormap(&a.tm_down_sc);
+            if (S) { prefetch_tensormap(&a.tm_sgate_sc); prefetch_tensormap(&a.tm_sup_sc);
+                     prefetch_tensormap(&a.tm_sdown_sc); }
+        }
+    }
+
     // ---- R: logits of this CTA's experts; zero-fill of out; x staged for X
     if (warp < kConsumerWarps) {
-        stage_x<Q4>(a, sm, tid);
+        stage_x<WF>(a, sm, tid);
+        if (tid < kMaxExperts / 32) rs->emask[tid] = 0u;
         {
             float4* o = reinterpret_cast<float4*>(a.out);
             const int n4 = (T * d) >> 2;
@@ -842,10 +940,14 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
                 float wj = expf(rs->sel[t][lane] - m) / den;
                 if (!(m > -INFINITY)) wj = 1.f / k;
                 rs->w[t * k + lane] = wj;
+                const int e = rs->ids[t * k + lane];
+                atomicOr(&rs->emask[e >> 5], 1u << (e & 31));
             }
         }
         named_bar_sync(1, kConsumers);
-        // stable slots: pairs with a smaller expert id come first, ties by pair index
+        // stable slots: pairs with a smaller expert id come first, ties by pair
+        // index; the first pair of each expert writes its work item, whose
+        // index is the number of selected experts below it (mask popcount)
         for (int p = tid; p < P; p += kConsumers) {
             const int e = rs->ids[p];
             int lt = 0, before = 0, cnt = 0;
@@ -858,9 +960,11 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
             const int slot = lt + before;
             rs->slot_token[slot] = p / k;
             rs->slot_w[slot] = rs->w[p];
-            rs->lt[p] = lt;
-            rs->cnt[p] = cnt;
-            rs->first[p] = before == 0;
+            if (before == 0) {
+                int idx = __popc(rs->emask[e >> 5] & ((1u << (e & 31)) - 1u));
+                for (int wd = 0; wd < (e >> 5); ++wd) idx += __popc(rs->emask[wd]);
+                rs->items[idx] = WorkItem{e, lt, cnt, 0};
+            }
             if (b == 0) {
                 a.ws.slot_pair[slot] = p;
                 a.ws.slot_token[slot] = p / k;
@@ -869,17 +973,9 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
                 a.ws.wts[p] = rs->w[p];
             }
         }
-        named_bar_sync(1, kConsumers);
-        for (int p = tid; p < P; p += kConsumers) {
-            if (!rs->first[p]) continue;
-            const int e = rs->ids[p];
-            int idx = 0;
-            for (int q = 0; q < P; ++q) idx += rs->first[q] & (rs->ids[q] < e);
-            rs->items[idx] = WorkItem{e, rs->lt[p], rs->cnt[p], 0};
-        }
-        if (tid == 0) {
+        if (tid == kConsumers - 1) {     // a thread the pair loop above rarely uses
             int n = 0;
-            for (int q = 0; q < P; ++q) n += rs->first[q];
+            for (int wd = 0; wd < (E + 31) / 32; ++wd) n += __popc(rs->emask[wd]);
             rs->n_routed = n;
             for (int s2 = 0; s2 < S; ++s2) rs->items[n + s2] = WorkItem{E + s2, -1, T, 0};
         }
@@ -897,20 +993,20 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
     }
     __syncthreads();
     const WorkView wv{rs->n_routed, S, rs->items, rs->slot_token, rs->slot_w};
-    experts_pipeline<FS, Q4>(a, sm, wv);
-    (void)sizeof(C);
+    experts_pipeline<FS, WF>(a, sm, wv);
 }
 
-int decode_stage_bytes(int fs, bool q4) {
-    if (q4) return 2 * 512 * 18;
+int decode_stage_bytes(int fs, int wfmt) {
     (void)fs;
+    if (wfmt == kWfQ4) return 2 * 512 * 18;
+    if (wfmt == kWfQ8) return 2 * 512 * 34;
     return 32768;
 }
 
-size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages) {
+size_t decode_smem_bytes(int fs, int wfmt, int d, int n_stages) {
     const int ksplit = kConsumerWarps / (2 * (fs / 16));
     size_t b = 1024;                                            // alignment slack
-    b += static_cast<size_t>(n_stages) * decode_stage_bytes(fs, q4);
+    b += static_cast<size_t>(n_stages) * decode_stage_bytes(fs, wfmt);
     b += static_cast<size_t>(kDecodeTok) * (d * 2 + 16);       // staged x
     b += static_cast<size_t>(kDecodeTok) * (d / 32) * 4;       // block sums of x
     b += static_cast<size_t>(ksplit) * 2 * kDecodeTok * (fs + 4) * 4;  // gate/up results
@@ -921,9 +1017,9 @@ size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages) {
     return b;
 }
 
-template <int FS, bool Q4>
+template <int FS, int WF>
 static cudaError_t launch_one(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
-    auto* k = decode_experts_kernel<FS, Q4>;
+    auto* k = decode_experts_kernel<FS, WF>;
     // the dynamic shared memory limit is raised once per device (and again
     // only if a later launch needs more)
     static int set_bytes[64] = {0};
@@ -940,9 +1036,9 @@ static cudaError_t launch_one(const DecodeArgs& a, int grid, size_t smem, cudaSt
     return cudaGetLastError();
 }
 
-template <int FS, bool Q4>
+template <int FS, int WF>
 static cudaError_t launch_fused_one(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
-    auto* k = decode_fused_kernel<FS, Q4>;
+    auto* k = decode_fused_kernel<FS, WF>;
     static int set_bytes[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -967,28 +1063,30 @@ static cudaError_t launch_fused_one(const DecodeArgs& a, int grid, size_t smem, 
     return cudaLaunchKernelEx(&cfg, k, a);
 }
 
-cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, bool q4, int grid, size_t smem,
+cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, int wfmt, int grid, size_t smem,
                                 cudaStream_t stream) {
-    if (q4) {
-        if (fs == 64) return launch_fused_one<64, true>(a, grid, smem, stream);
-        if (fs == 32) return launch_fused_one<32, true>(a, grid, smem, stream);
-    } else {
-        if (fs == 64) return launch_fused_one<64, false>(a, grid, smem, stream);
-        if (fs == 32) return launch_fused_one<32, false>(a, grid, smem, stream);
+    switch (wfmt * 100 + fs) {
+        case kWfBf16 * 100 + 64: return launch_fused_one<64, kWfBf16>(a, grid, smem, stream);
+        case kWfBf16 * 100 + 32: return launch_fused_one<32, kWfBf16>(a, grid, smem, stream);
+        case kWfQ4 * 100 + 64: return launch_fused_one<64, kWfQ4>(a, grid, smem, stream);
+        case kWfQ4 * 100 + 32: return launch_fused_one<32, kWfQ4>(a, grid, smem, stream);
+        case kWfQ8 * 100 + 64: return launch_fused_one<64, kWfQ8>(a, grid, smem, stream);
+        case kWfQ8 * 100 + 32: return launch_fused_one<32, kWfQ8>(a, grid, smem, stream);
+        default: return cudaErrorInvalidValue;
     }
-    return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, bool q4, int grid, size_t smem,
+cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, int wfmt, int grid, size_t smem,
                                   cudaStream_t stream) {
-    if (q4) {
-        if (fs == 64) return launch_one<64, true>(a, grid, smem, stream);
-        if (fs == 32) return launch_one<32, true>(a, grid, smem, stream);
-    } else {
-        if (fs == 64) return launch_one<64, false>(a, grid, smem, stream);
-        if (fs == 32) return launch_one<32, false>(a, grid, smem, stream);
+    switch (wfmt * 100 + fs) {
+        case kWfBf16 * 100 + 64: return launch_one<64, kWfBf16>(a, grid, smem, stream);
+        case kWfBf16 * 100 + 32: return launch_one<32, kWfBf16>(a, grid, smem, stream);
+        case kWfQ4 * 100 + 64: return launch_one<64, kWfQ4>(a, grid, smem, stream);
+        case kWfQ4 * 100 + 32: return launch_one<32, kWfQ4>(a, grid, smem, stream);
+        case kWfQ8 * 100 + 64: return launch_one<64, kWfQ8>(a, grid, smem, stream);
+        case kWfQ8 * 100 + 32: return launch_one<32, kWfQ8>(a, grid, smem, stream);
+        default: return cudaErrorInvalidValue;
     }
-    return cudaErrorInvalidValue;
 }
 
 }  // namespace moe

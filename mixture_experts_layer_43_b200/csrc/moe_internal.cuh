@@ -50,7 +50,7 @@ struct Workspace {
     int32_t* n_items;      // [2]: routed items, shared items
     uint32_t* ticket;      // last-CTA ticket of the decode router
     uint32_t* err;         // sticky device error word
-    uint32_t* gbar;        // grid barrier of the fused decode kernel: arrivals, generation
+    uint32_t* gbar;        // grid barrier of the fused decode kernel: 64-bit arrival count (8-aligned)
     // prefill
     uint16_t* x_perm;      // [t_max*k][d] bf16 rows gathered per slot
     uint16_t* h_routed;    // [t_max*k][F] bf16
@@ -70,11 +70,15 @@ struct RouteArgs {
     int experts_per_cta;   // 1, 2, 4 or 8
 };
 
+// Rows of one TMA box of a quantised down matrix in the decode kernels (the
+// host builds the tensor maps with the same box).
+constexpr int kQuantDownBoxRows = 256;
+
 struct DecodeArgs {
-    // bf16: 2D maps over the weight stacks.  Q4_0: 3D maps over the codes.
+    // bf16: 2D maps over the weight stacks.  Q4_0 / Q8_0: 3D maps over the codes.
     CUtensorMap tm_gate, tm_up, tm_down;
     CUtensorMap tm_sgate, tm_sup, tm_sdown;
-    // Q4_0 only: 2D maps over the scales.
+    // Q4_0 / Q8_0 only: 2D maps over the scales.
     CUtensorMap tm_gate_sc, tm_up_sc, tm_down_sc;
     CUtensorMap tm_sgate_sc, tm_sup_sc, tm_sdown_sc;
     const uint16_t* x;          // [T][d] bf16
@@ -87,32 +91,40 @@ struct DecodeArgs {
     int T, d, F, Fs, E, S;
     int n_stages;               // ring depth
     int xs_stride;              // bytes per token row of the staged x
-    int kt;                     // phase A: k columns (bf16) / block columns (Q4_0) per stage
+    int kt;                     // phase A: k columns (bf16) / block columns (quantised) per stage
     int rj;                     // phase B: output rows per stage
     // fused single-launch path only: router inputs, routing tables, grid barrier
     const float* wr;            // [E][d]
     const float* br;            // [E] or nullptr
     int k;
     Workspace ws;
-    uint32_t* gbar;             // [0] arrivals, [1] generation
+    uint32_t* gbar;             // [0..1] 64-bit arrival count of the grid barrier
 };
 
-// Host launchers (decode.cu, q4_pack.cu).
+// Host launchers (decode.cu, quant_pack.cu).
 cudaError_t launch_decode_route(const RouteArgs& a, cudaStream_t stream);
-cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, bool q4, int grid,
+cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, int wfmt, int grid,
                                   size_t smem, cudaStream_t stream);
-size_t decode_smem_bytes(int fs, bool q4, int d, int n_stages);
-cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, bool q4, int grid, size_t smem,
+size_t decode_smem_bytes(int fs, int wfmt, int d, int n_stages);
+cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, int wfmt, int grid, size_t smem,
                                 cudaStream_t stream);
 size_t decode_fused_extra_smem();
-int decode_stage_bytes(int fs, bool q4);
+int decode_stage_bytes(int fs, int wfmt);
 cudaError_t launch_q4_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint16_t* scales, cudaStream_t stream);
+cudaError_t launch_q8_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
                              uint8_t* codes, uint16_t* scales, cudaStream_t stream);
 
 // --------------------------------------------------------- device helpers
 #ifdef __CUDACC__
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -324,9 +336,18 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float
 }
 
 // --------------------------------------------------------- warp top-k
+// Warp-wide float maximum (sm_100a: one redux.sync instead of five shuffle
+// rounds).
+__device__ __forceinline__ float warp_max_f32(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
 // Top-k of one token's E logits (shared memory, E <= 32 * PER) by one warp.
 // Each lane keeps logits lane, lane+32, ... in registers; a bitmask marks the
-// ones already taken, so a round is a register scan plus one shuffle argmax.
+// ones already taken.  A round is a register scan, a warp max of the lanes'
+// best values and a warp min over the indices holding that max.
 // Order: descending logit, equal logits -> lower expert index; NaN counts as
 // -inf.  Lane 0 writes ids[j] and the selected logits sel[j].
 template <int PER>
@@ -351,23 +372,18 @@ __device__ __forceinline__ void warp_topk(const float* row, int E, int k, int* i
         float bv = -INFINITY;
         int bi = 0x7fffffff;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) {
-            const int x = lane + 32 * i;
-            if (!((taken >> i) & 1u) && (v[i] > bv || (v[i] == bv && x < bi))) { bv = v[i]; bi = x; }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if (bi >= E) {                 // cannot happen for k <= E; keep ids in range
+        for (int i = 0; i < PER; ++i)   // strict '>': the lowest index wins inside a lane
+            if (!((taken >> i) & 1u) && (v[i] > bv || bi == 0x7fffffff)) { bv = v[i]; bi = lane + 32 * i; }
+        const float m = warp_max_f32(bv);
+        const uint32_t cand = (bv == m) ? static_cast<uint32_t>(bi) : 0xffffffffu;
+        int w = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
+        if (w < 0 || w >= E) {         // cannot happen for k <= E; keep ids in range
             if (lane == 0) atomicOr(err, kErrBadId);
-            bi = 0;
-        } else if ((bi & 31) == lane) {
-            taken |= 1u << (bi >> 5);
+            w = 0;
+        } else if ((w & 31) == lane) {
+            taken |= 1u << (w >> 5);
         }
-        if (lane == 0) { ids[j] = bi; sel[j] = bv; }
+        if (lane == 0) { ids[j] = w; sel[j] = m; }
     }
 }
 

@@ -1,9 +1,10 @@
 // prefill.cu -- prefill regime (T > MOE_DECODE_MAX_T tokens, bf16 weights).
 //
 // Four launches per layer call:
-//  1. prefill_router_kernel: router logits for 32 tokens per CTA with fp32
-//     FMAs, top-k with renormalised weights, the CTA's per-expert histogram,
-//     and the zero-fill of its rows of `out`.
+//  1. prefill_router_kernel: router logits for 32 tokens per CTA on the
+//     tensor cores, as accurate as fp32 FMAs (the fp32 router weights are
+//     split exactly into three bf16 parts), top-k with renormalised weights,
+//     the CTA's per-expert histogram, and the zero-fill of its rows of `out`.
 //     ("Fused MoE Triton kernel: 5 launches instead of 24" page, fused steps
 //     one and two.)
 //  2. prefill_scatter_kernel: every CTA reduces the histograms to its chunk's

@@ -1,0 +1,136 @@
+// quant_pack.cu -- repack canonical Q4_0 and Q8_0 blocks into the decode
+// kernels' layout.
+//
+// ---- Q4_0
+// Canonical block (32 weights along the reduction dim, 18 bytes): little-endian
+// fp16 scale d, then 16 bytes; byte j holds code j (low nibble) and code j+16
+// (high nibble); weight = d * (q - 8).  This is the Q4_0 the "MoE on RTX 5090
+// reaches 41% of bandwidth" page measures (measurement-setup paragraph), with
+// the block layout of the 35B-A3B Q4_0 workload.
+//
+// Kernel layout (same 4.5 bits per weight):
+//   codes  [mat][k/32][rows][16 B]   block-column major, so an expert's slice
+//                                    of rows, or a slice of block columns, is
+//                                    one contiguous run for TMA
+//   scales [mat][k/32][rows] fp16
+// Inside a block the 32 codes are permuted so that 32-bit word `tig` (0..3)
+// holds exactly the 8 codes lane tig of an mma.sync m16n8k16 A fragment needs
+// for both 16-wide halves of the block:
+//   bits  0- 3 code 2tig      bits 16-19 code 2tig+1
+//   bits  4- 7 code 2tig+8    bits 20-23 code 2tig+9
+//   bits  8-11 code 2tig+16   bits 24-27 code 2tig+17
+//   bits 12-15 code 2tig+24   bits 28-31 code 2tig+25
+#include "moe_internal.cuh"
+
+namespace moe {
+
+__global__ void q4_0_pack_kernel(const uint8_t* __restrict__ blocks, int64_t n_mats, int64_t rows,
+                                 int64_t nkb, uint8_t* __restrict__ codes,
+                                 uint16_t* __restrict__ scales) {
+    const int64_t total = n_mats * rows * nkb;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t kb = i % nkb;
+        const int64_t r = (i / nkb) % rows;
+        const int64_t m = i / (nkb * rows);
+        const uint8_t* src = blocks + i * 18;            // [m][r][kb] canonical
+        uint8_t q[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const uint8_t b = src[2 + j];
+            q[j] = b & 0x0f;
+            q[j + 16] = b >> 4;
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int e = 2 * t;
+            w[t] = static_cast<uint32_t>(q[e]) | (static_cast<uint32_t>(q[e + 8]) << 4) |
+                   (static_cast<uint32_t>(q[e + 16]) << 8) | (static_cast<uint32_t>(q[e + 24]) << 12) |
+                   (static_cast<uint32_t>(q[e + 1]) << 16) | (static_cast<uint32_t>(q[e + 9]) << 20) |
+                   (static_cast<uint32_t>(q[e + 17]) << 24) | (static_cast<uint32_t>(q[e + 25]) << 28);
+        }
+        const int64_t dst = (m * nkb + kb) * rows + r;   // [m][kb][r]
+        *reinterpret_cast<uint4*>(codes + dst * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        scales[dst] = static_cast<uint16_t>(src[0] | (src[1] << 8));
+    }
+}
+
+cudaError_t launch_q4_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint16_t* scales, cudaStream_t stream) {
+    const int64_t total = n_mats * rows * (k / 32);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t want = (total + threads - 1) / threads;
+    const int grid = static_cast<int>(want < 65536 ? want : 65536);
+    q4_0_pack_kernel<<<grid, threads, 0, stream>>>(blocks, n_mats, rows, k / 32, codes, scales);
+    return cudaGetLastError();
+}
+
+
+// ---- Q8_0
+// Canonical block (32 weights, 34 bytes): little-endian fp16 scale d, then 32
+// signed bytes q (element j in byte j); weight = d * q.  (The 5090 page lists
+// q8_0 among the formats of the model it measures; the byte layout is the
+// canonical llama.cpp one, a reading.)
+//
+// Kernel layout (same 8.5 bits per weight):
+//   codes  [mat][k/32][rows][32 B]
+//   scales [mat][k/32][rows] fp16
+// Each code is biased to u = q + 128 (0..255) and split into its nibbles
+// u = 16 hi + lo.  Both nibble planes are packed exactly like Q4_0 codes
+// above (one 32-bit word per lane holds the 8 values of the lane's A
+// fragment for both halves of the block); the 8 words of a block row are
+// interleaved as lo0 hi0 lo1 hi1 lo2 hi2 lo3 hi3, so lane tig fetches both
+// of its words with one 64-bit load.
+__device__ __forceinline__ uint32_t pack_q4_lane(const uint8_t* q, int t) {
+    const int e = 2 * t;
+    return static_cast<uint32_t>(q[e]) | (static_cast<uint32_t>(q[e + 8]) << 4) |
+           (static_cast<uint32_t>(q[e + 16]) << 8) | (static_cast<uint32_t>(q[e + 24]) << 12) |
+           (static_cast<uint32_t>(q[e + 1]) << 16) | (static_cast<uint32_t>(q[e + 9]) << 20) |
+           (static_cast<uint32_t>(q[e + 17]) << 24) | (static_cast<uint32_t>(q[e + 25]) << 28);
+}
+
+__global__ void q8_0_pack_kernel(const uint8_t* __restrict__ blocks, int64_t n_mats, int64_t rows,
+                                 int64_t nkb, uint8_t* __restrict__ codes,
+                                 uint16_t* __restrict__ scales) {
+    const int64_t total = n_mats * rows * nkb;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t kb = i % nkb;
+        const int64_t r = (i / nkb) % rows;
+        const int64_t m = i / (nkb * rows);
+        const uint8_t* src = blocks + i * 34;            // [m][r][kb] canonical
+        uint8_t lo[32], hi[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const uint8_t u = static_cast<uint8_t>(src[2 + j] ^ 0x80u);   // q + 128
+            lo[j] = u & 0x0f;
+            hi[j] = u >> 4;
+        }
+        uint32_t w[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            w[2 * t] = pack_q4_lane(lo, t);
+            w[2 * t + 1] = pack_q4_lane(hi, t);
+        }
+        const int64_t dst = (m * nkb + kb) * rows + r;   // [m][kb][r]
+        uint4* o = reinterpret_cast<uint4*>(codes + dst * 32);
+        o[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        o[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        scales[dst] = static_cast<uint16_t>(src[0] | (src[1] << 8));
+    }
+}
+
+cudaError_t launch_q8_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint16_t* scales, cudaStream_t stream) {
+    const int64_t total = n_mats * rows * (k / 32);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t want = (total + threads - 1) / threads;
+    const int grid = static_cast<int>(want < 65536 ? want : 65536);
+    q8_0_pack_kernel<<<grid, threads, 0, stream>>>(blocks, n_mats, rows, k / 32, codes, scales);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,6 +1,7 @@
 """Device-memory plumbing around the C ABI: upload a layer's tensors with
-PyTorch (device memory and streams only), repack Q4_0 through the library's
-own moe_q4_0_pack kernel, and fill the moe_weights_t / moe_config_t structs.
+PyTorch (device memory and streams only), repack Q4_0 / Q8_0 through the
+library's own moe_q4_0_pack / moe_q8_0_pack kernels, and fill the
+moe_weights_t / moe_config_t structs.
 No arithmetic of the layer happens here."""
 from __future__ import annotations
 
@@ -28,7 +29,10 @@ class DeviceLayer:
         sh = inp.shape
         self.shape = sh
         self.device = torch.device(device)
-        self.q4 = sh.wfmt == synth.WFMT_Q4_0
+        self.q4 = sh.wfmt != synth.WFMT_BF16          # quantised: codes + scales
+        q8 = sh.wfmt == synth.WFMT_Q8_0
+        packed_bytes = B.moe_q8_0_packed_bytes if q8 else B.moe_q4_0_packed_bytes
+        pack = B.moe_q8_0_pack if q8 else B.moe_q4_0_pack
         st = stream if stream is not None else torch.cuda.current_stream(self.device)
         self.router_w = _dev(inp.router_w.astype(np.float32), self.device)
         self.router_b = None if inp.router_b is None else _dev(inp.router_b.astype(np.float32),
@@ -43,11 +47,11 @@ class DeviceLayer:
                 self._keep.append(t)
                 return B.moe_matrix_t(t.data_ptr(), None)
             canon = _dev(arr.reshape(-1), self.device)
-            cb, sb = B.moe_q4_0_packed_bytes(n_mats, rows, k)
+            cb, sb = packed_bytes(n_mats, rows, k)
             codes = torch.empty(cb, dtype=torch.uint8, device=self.device)
             scales = torch.empty(sb // 2, dtype=torch.int16, device=self.device)
-            B.moe_q4_0_pack(canon.data_ptr(), n_mats, rows, k, codes.data_ptr(),
-                            scales.data_ptr(), st.cuda_stream)
+            pack(canon.data_ptr(), n_mats, rows, k, codes.data_ptr(), scales.data_ptr(),
+                 st.cuda_stream)
             st.synchronize()
             del canon
             self._keep += [codes, scales]

@@ -46,7 +46,7 @@ def _cfg(**kw):
     dict(t_max=0), dict(d_model=100), dict(d_model=192), dict(d_ff=48), dict(n_experts=0),
     dict(n_experts=2000), dict(top_k=0), dict(top_k=9), dict(n_experts=32, top_k=17),
     dict(n_shared=-1), dict(n_shared=9), dict(n_shared=1, d_ff_shared=0),
-    dict(n_shared=1, d_ff_shared=40), dict(wfmt=2), dict(regime=3), dict(device=-1),
+    dict(n_shared=1, d_ff_shared=40), dict(wfmt=3), dict(regime=3), dict(device=-1),
 ])
 def test_plan_create_rejects_bad_config(L, kw):
     plan = ctypes.c_void_p(123)
@@ -58,6 +58,8 @@ def test_plan_create_rejects_bad_config(L, kw):
 def test_plan_create_q4_prefill_unsupported(L):
     plan = ctypes.c_void_p()
     s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=1, regime=2)), ctypes.byref(plan))
+    assert s == B.MOE_ERR_UNSUPPORTED
+    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=2, regime=2)), ctypes.byref(plan))
     assert s == B.MOE_ERR_UNSUPPORTED
 
 
@@ -88,3 +90,18 @@ def test_q4_pack_rejects_bad_args_without_gpu(L):
     assert L.moe_q4_0_pack(16, 1, 1, 32, 17, 32, None) == B.MOE_ERR_INVALID_ARG
     # empty is a no-op
     assert L.moe_q4_0_pack(None, 0, 4, 32, None, None, None) == B.MOE_OK
+
+
+def test_q8_packed_bytes(L):
+    assert B.moe_q8_0_packed_bytes(256, 512, 2048) == (256 * 512 * 64 * 32, 256 * 512 * 64 * 2)
+    assert B.moe_q8_0_packed_bytes(0, 5, 32) == (0, 0)
+    cb = ctypes.c_size_t()
+    assert L.moe_q8_0_packed_bytes(1, 1, 33, ctypes.byref(cb), None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q8_0_packed_bytes(-1, 1, 32, None, None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_q8_pack_rejects_bad_args_without_gpu(L):
+    assert L.moe_q8_0_pack(None, 1, 1, 33, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q8_0_pack(None, 1, 1, 32, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q8_0_pack(16, 1, 1, 32, 17, 32, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q8_0_pack(None, 0, 4, 32, None, None, None) == B.MOE_OK

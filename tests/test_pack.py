@@ -1,0 +1,73 @@
+"""GPU test of the two repacking kernels (moe_q4_0_pack, moe_q8_0_pack):
+byte work, so bit-exact.  The packed arrays are decoded here with numpy by
+inverting the layout include/moe.h documents, and the codes and scales must
+equal those of the canonical blocks exactly."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_43_b200 import binding as B
+from mixture_experts_layer_43_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+# (bit offset in the 32-bit word, element of the 32-wide block) for lane word t
+def _word_slots(t):
+    e = 2 * t
+    return [(0, e), (4, e + 8), (8, e + 16), (12, e + 24),
+            (16, e + 1), (20, e + 9), (24, e + 17), (28, e + 25)]
+
+
+def _unpack_nibble_words(words):
+    """[..., 4] uint32 words of one block row -> [..., 32] 4-bit values."""
+    out = np.zeros(words.shape[:-1] + (32,), np.uint8)
+    for t in range(4):
+        for shift, idx in _word_slots(t):
+            out[..., idx] = (words[..., t] >> shift) & 15
+    return out
+
+
+def _pack_on_gpu(fn_bytes, fn_pack, canon, n_mats, rows, k):
+    cb, sb = fn_bytes(n_mats, rows, k)
+    src = torch.from_numpy(np.ascontiguousarray(canon).reshape(-1)).cuda()
+    codes = torch.zeros(cb, dtype=torch.uint8, device="cuda")
+    scales = torch.zeros(sb // 2, dtype=torch.int16, device="cuda")
+    fn_pack(src.data_ptr(), n_mats, rows, k, codes.data_ptr(), scales.data_ptr(),
+            torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("n_mats,rows,k", [(1, 1, 32), (3, 40, 96), (2, 128, 512)])
+def test_q4_0_pack_is_the_documented_permutation(n_mats, rows, k):
+    rng = np.random.default_rng(n_mats * 1000 + rows)
+    canon = synth.q4_0_blocks(rng, n_mats * rows, k, 0.01).reshape(n_mats, rows, k // 32, 18)
+    codes, scales = _pack_on_gpu(B.moe_q4_0_packed_bytes, B.moe_q4_0_pack, canon, n_mats, rows, k)
+    words = codes.view(np.uint32).reshape(n_mats, k // 32, rows, 4)
+    got = _unpack_nibble_words(words).transpose(0, 2, 1, 3)          # [m][r][kb][32]
+    want = np.concatenate([canon[..., 2:] & 15, canon[..., 2:] >> 4], axis=-1)
+    assert np.array_equal(got, want)
+    want_sc = canon[..., :2].copy().view(np.uint16)[..., 0]          # [m][r][kb]
+    assert np.array_equal(scales.reshape(n_mats, k // 32, rows).transpose(0, 2, 1), want_sc)
+
+
+@pytest.mark.parametrize("n_mats,rows,k", [(1, 1, 32), (3, 40, 96), (2, 128, 512)])
+def test_q8_0_pack_is_the_documented_planes(n_mats, rows, k):
+    rng = np.random.default_rng(n_mats * 1000 + rows + 7)
+    canon = synth.q8_0_blocks(rng, n_mats * rows, k, 0.01).reshape(n_mats, rows, k // 32, 34)
+    codes, scales = _pack_on_gpu(B.moe_q8_0_packed_bytes, B.moe_q8_0_pack, canon, n_mats, rows, k)
+    words = codes.view(np.uint32).reshape(n_mats, k // 32, rows, 8)
+    lo = _unpack_nibble_words(words[..., 0::2]).astype(np.int32)
+    hi = _unpack_nibble_words(words[..., 1::2]).astype(np.int32)
+    got = (16 * hi + lo - 128).transpose(0, 2, 1, 3)                # signed codes [m][r][kb][32]
+    want = canon[..., 2:].copy().view(np.int8).astype(np.int32)
+    assert np.array_equal(got, want)
+    want_sc = canon[..., :2].copy().view(np.uint16)[..., 0]
+    assert np.array_equal(scales.reshape(n_mats, k // 32, rows).transpose(0, 2, 1), want_sc)

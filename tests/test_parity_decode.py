@@ -29,6 +29,11 @@ SMALL = [
     synth.MoEShape("multi_unit_q4", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512,
                    wfmt=synth.WFMT_Q4_0),
     synth.MoEShape("biased", T=8, d=512, E=64, k=6, F=128, S=2, Fs=128, zipf_bias=1.1),
+    synth.MoEShape("ragged_q8", T=3, d=384, E=5, k=3, F=96, S=1, Fs=64, wfmt=synth.WFMT_Q8_0),
+    synth.MoEShape("two_shared_q8", T=7, d=256, E=16, k=2, F=64, S=2, Fs=96,
+                   wfmt=synth.WFMT_Q8_0),
+    synth.MoEShape("multi_unit_q8", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512,
+                   wfmt=synth.WFMT_Q8_0),
 ]
 
 
@@ -59,7 +64,9 @@ def _check(sh, seed=0, T=None, split=False):
 @pytest.mark.parametrize("name", ["tiny_T4_d256_E8k2_F512", "a3b_T1_d2048_E256k8_F512_S1",
                                   "a3b_q4_T1_d2048_E256k8_F512_S1",
                                   "a3b_q4_T8_d2048_E256k8_F512_S1",
-                                  "a3b_T8_d2048_E256k8_F512_S1"])
+                                  "a3b_T8_d2048_E256k8_F512_S1",
+                                  "a3b_q8_T1_d2048_E256k8_F512_S1",
+                                  "a3b_q8_T8_d2048_E256k8_F512_S1"])
 def test_decode_workloads_full_size(name):
     err = _check(W[name])
     print(f"{name}: rel L2 {err:.3e}")
@@ -75,8 +82,10 @@ def test_decode_small_shapes(sh):
     _check(sh, seed=1)
 
 
-@pytest.mark.parametrize("sh", SMALL[:6] + [W["a3b_q4_T8_d2048_E256k8_F512_S1"]],
-                         ids=[s.name for s in SMALL[:6]] + ["a3b_q4_T8"])
+SPLIT = SMALL[:6] + [SMALL[10], W["a3b_q4_T8_d2048_E256k8_F512_S1"]]
+
+
+@pytest.mark.parametrize("sh", SPLIT, ids=[s.name for s in SPLIT[:-1]] + ["a3b_q4_T8"])
 def test_decode_two_launch_path(sh):
     _check(sh, seed=5, split=True)
 
