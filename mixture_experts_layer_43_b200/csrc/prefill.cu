@@ -3,8 +3,9 @@
 // Four launches per layer call:
 //  1. prefill_router_kernel: router logits for 32 tokens per CTA on the
 //     tensor cores, as accurate as fp32 FMAs (the fp32 router weights are
-//     split exactly into three bf16 parts), top-k with renormalised weights,
-//     the CTA's per-expert histogram, and the zero-fill of its rows of `out`.
+//     split exactly into three bf16 parts; x and router chunks stream in by
+//     cp.async three chunks ahead), top-k with renormalised weights, the
+//     CTA's per-expert histogram, and the zero-fill of its rows of `out`.
 //     ("Fused MoE Triton kernel: 5 launches instead of 24" page, fused steps
 //     one and two.)
 //  2. prefill_scatter_kernel: every CTA reduces the histograms to its chunk's
@@ -53,12 +54,29 @@ struct PrefillRouteArgs {
 
 constexpr int kRouterXTile = kChunkTok * kRouterPitch;          // bf16 elements
 constexpr int kRouterWTile = kRouterEC * kRouterPitch;          // bf16 elements, one part
+constexpr int kRouterStages = 4;                                // raw chunks in flight
+constexpr int kRouterRawW = kRouterEC * kRouterKC;             // fp32 elements of one raw w chunk
 
 size_t router_smem_bytes(int E) {
     return static_cast<size_t>(kChunkTok) * E * 4 +                      // logits
-           2ull * (kRouterXTile + 3 * kRouterWTile) * 2 +                 // x, 3 w parts, x2
+           static_cast<size_t>(kRouterStages) * (kRouterXTile * 2 + kRouterRawW * 4) +  // raw ring
+           2ull * 3 * kRouterWTile * 2 +                                  // 3 w parts, x2
            (kChunkTok * kMaxTopK + E) * 4 +                               // ids, histogram
            static_cast<size_t>(kChunkTok) * kMaxTopK * 4;                 // selected logits
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only); src_bytes < 16
+// zero-fills the rest of the destination (0: a row past the end).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+                 :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory");
 }
 
 // ============================================================ router ===
@@ -67,17 +85,20 @@ size_t router_smem_bytes(int E) {
 // split into three bf16 parts hi + mid + lo that sum to w exactly (each part
 // holds the next 8 significant bits), so every x*part product (bf16 x) is
 // exact in fp32 and mma.sync accumulates the three partial logits in fp32.
-// (TF32 would instead round w to 10 bits.)  64-column chunks of x and of
-// the split router matrix are double-buffered in shared memory; the next
-// chunk's global loads are in flight while the current one is multiplied.
+// (TF32 would instead round w to 10 bits.)  64-column chunks of x and of the
+// fp32 router arrive by cp.async in a ring of four (three chunks in flight
+// while one is used); each chunk is split into the double-buffered bf16
+// tiles the mma's read.
 // Warp w handles tokens 16*(w/4).. and experts 16*(w%4)..  of the pass.
 __global__ void __launch_bounds__(kRouterThreads)
 prefill_router_kernel(const PrefillRouteArgs a) {
     extern __shared__ __align__(1024) uint8_t sm_raw[];
     const int E = a.E, d = a.d, k = a.k, T = a.T;
     float* s_log = reinterpret_cast<float*>(sm_raw);                   // [32][E]
-    __nv_bfloat16* s_x = reinterpret_cast<__nv_bfloat16*>(s_log + kChunkTok * E);   // [2][32][pitch]
-    __nv_bfloat16* s_w = s_x + 2 * kRouterXTile;                        // [2][3][64][pitch]
+    // raw ring: x chunk [32][pitch] bf16 (read by ldmatrix as is), w chunk [64][64] fp32
+    __nv_bfloat16* s_xr = reinterpret_cast<__nv_bfloat16*>(s_log + kChunkTok * E);
+    float* s_wr = reinterpret_cast<float*>(s_xr + kRouterStages * kRouterXTile);
+    __nv_bfloat16* s_w = reinterpret_cast<__nv_bfloat16*>(s_wr + kRouterStages * kRouterRawW);  // [2][3][64][pitch]
     int* s_ids = reinterpret_cast<int*>(s_w + 2 * 3 * kRouterWTile);    // [32*k]
     int* s_hist = s_ids + kChunkTok * kMaxTopK;                         // [E]
 
@@ -93,69 +114,75 @@ prefill_router_kernel(const PrefillRouteArgs a) {
     }
     for (int e = tid; e < E; e += kRouterThreads) s_hist[e] = 0;
 
-    // loader roles: x -- token tid/8, 8 columns at (tid%8)*8; w -- expert
-    // tid/4, 16 columns at (tid%4)*16
-    const int xt = tid >> 3, xk = (tid & 7) * 8;
-    const int we = tid >> 2, wk = (tid & 3) * 16;
     const int tg = warp >> 2, eq = warp & 3;
     const int g = lane >> 2, tig = lane & 3;
     const int nkc = d / kRouterKC;
     for (int e0 = 0; e0 < E; e0 += kRouterEC) {
         const int ne = min(kRouterEC, E - e0);
-        uint4 xr;
-        float4 wr4[4];
-        auto gload = [&](int kc) {
-            const int kb = kc * kRouterKC;
-            xr = make_uint4(0u, 0u, 0u, 0u);
-            if (xt < nt)
-                xr = __ldg(reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + xt) * d + kb + xk));
-            if (we < ne) {
-                const float4* src = reinterpret_cast<const float4*>(
-                    a.wr + static_cast<size_t>(e0 + we) * d + kb + wk);
+        // chunk kc -> ring stage kc % kRouterStages, by cp.async: x row tid/8,
+        // 16 bytes at (tid%8)*16; w: 4 x 16 bytes, row c/16, floats (c%16)*4
+        auto issue = [&](int kc) {
+            const int st = kc % kRouterStages, kb = kc * kRouterKC;
+            {
+                const int r = tid >> 3, c8 = (tid & 7) * 8;
+                const bool ok = r < nt;
+                cp_async_16(smem_u32(s_xr + st * kRouterXTile + r * kRouterPitch + c8),
+                            a.x + static_cast<size_t>(t0 + (ok ? r : 0)) * d + kb + c8, ok ? 16 : 0);
+            }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) wr4[q] = __ldg(src + q);
-            } else {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) wr4[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int q = 0; q < kRouterRawW / 4 / kRouterThreads; ++q) {
+                const int c = q * kRouterThreads + tid, r = c >> 4, c4 = (c & 15) * 4;
+                const bool ok = r < ne;
+                cp_async_16(smem_u32(s_wr + st * kRouterRawW + r * kRouterKC + c4),
+                            a.wr + static_cast<size_t>(e0 + (ok ? r : 0)) * d + kb + c4, ok ? 16 : 0);
             }
         };
-        auto sstore = [&](int buf) {
-            *reinterpret_cast<uint4*>(s_x + buf * kRouterXTile + xt * kRouterPitch + xk) = xr;
-            const float wf[16] = {wr4[0].x, wr4[0].y, wr4[0].z, wr4[0].w, wr4[1].x, wr4[1].y,
-                                  wr4[1].z, wr4[1].w, wr4[2].x, wr4[2].y, wr4[2].z, wr4[2].w,
-                                  wr4[3].x, wr4[3].y, wr4[3].z, wr4[3].w};
-            uint32_t hi[8], mid[8], lo[8];
+        // exact split of a raw fp32 chunk into the hi / mid / lo bf16 tiles
+        auto split = [&](int kc, int buf) {
+            const float* raw = s_wr + (kc % kRouterStages) * kRouterRawW;
+            __nv_bfloat16* wb = s_w + buf * 3 * kRouterWTile;
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float p0 = wf[2 * q], p1 = wf[2 * q + 1];
-                const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-                p0 -= __low2float(h);                 // exact: fp32 minus its bf16 rounding
-                p1 -= __high2float(h);
-                const __nv_bfloat162 m = __floats2bfloat162_rn(p0, p1);
-                p0 -= __low2float(m);
-                p1 -= __high2float(m);
-                const __nv_bfloat162 l = __floats2bfloat162_rn(p0, p1);   // exact: <= 8 bits left
-                hi[q] = *reinterpret_cast<const uint32_t*>(&h);
-                mid[q] = *reinterpret_cast<const uint32_t*>(&m);
-                lo[q] = *reinterpret_cast<const uint32_t*>(&l);
+            for (int q = 0; q < kRouterRawW / 4 / kRouterThreads; ++q) {
+                const int i = (q * kRouterThreads + tid) * 4, r = i / kRouterKC, c = i % kRouterKC;
+                const float4 f = *reinterpret_cast<const float4*>(raw + i);
+                const float p[4] = {f.x, f.y, f.z, f.w};
+                uint32_t hi[2], mid[2], lo[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    float p0 = p[2 * h2], p1 = p[2 * h2 + 1];
+                    const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                    p0 -= __low2float(h);             // exact: fp32 minus its bf16 rounding
+                    p1 -= __high2float(h);
+                    const __nv_bfloat162 m = __floats2bfloat162_rn(p0, p1);
+                    p0 -= __low2float(m);
+                    p1 -= __high2float(m);
+                    const __nv_bfloat162 l = __floats2bfloat162_rn(p0, p1);   // exact: <= 8 bits left
+                    hi[h2] = *reinterpret_cast<const uint32_t*>(&h);
+                    mid[h2] = *reinterpret_cast<const uint32_t*>(&m);
+                    lo[h2] = *reinterpret_cast<const uint32_t*>(&l);
+                }
+                const int o = r * kRouterPitch + c;
+                *reinterpret_cast<uint2*>(wb + o) = make_uint2(hi[0], hi[1]);
+                *reinterpret_cast<uint2*>(wb + kRouterWTile + o) = make_uint2(mid[0], mid[1]);
+                *reinterpret_cast<uint2*>(wb + 2 * kRouterWTile + o) = make_uint2(lo[0], lo[1]);
             }
-            __nv_bfloat16* wb = s_w + buf * 3 * kRouterWTile + we * kRouterPitch + wk;
-            uint4* d0 = reinterpret_cast<uint4*>(wb);
-            uint4* d1 = reinterpret_cast<uint4*>(wb + kRouterWTile);
-            uint4* d2 = reinterpret_cast<uint4*>(wb + 2 * kRouterWTile);
-            d0[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);   d0[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-            d1[0] = make_uint4(mid[0], mid[1], mid[2], mid[3]); d1[1] = make_uint4(mid[4], mid[5], mid[6], mid[7]);
-            d2[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);   d2[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
         };
         float acc[2][4] = {};
-        __syncthreads();
-        gload(0);
-        sstore(0);
-        __syncthreads();
+        __syncthreads();                           // previous pass done with the ring
+#pragma unroll
+        for (int kc = 0; kc < kRouterStages - 1; ++kc) {
+            if (kc < nkc) issue(kc);
+            cp_async_commit();
+        }
         for (int kc = 0; kc < nkc; ++kc) {
+            cp_async_wait<kRouterStages - 2>();   // this thread's copies of chunk kc landed
+            __syncthreads();                       // everyone's; chunk kc-1 fully consumed
+            if (kc + kRouterStages - 1 < nkc) issue(kc + kRouterStages - 1);   // into kc-1's stage
+            cp_async_commit();
             const int buf = kc & 1;
-            if (kc + 1 < nkc) gload(kc + 1);           // in flight during the MMAs
-            const uint32_t xs = smem_u32(s_x + buf * kRouterXTile);
+            split(kc, buf);
+            __syncthreads();
+            const uint32_t xs = smem_u32(s_xr + (kc % kRouterStages) * kRouterXTile);
             const uint32_t ws = smem_u32(s_w + buf * 3 * kRouterWTile);
 #pragma unroll
             for (int kk = 0; kk < kRouterKC / 16; ++kk) {
@@ -177,9 +204,8 @@ prefill_router_kernel(const PrefillRouteArgs a) {
                     }
                 }
             }
-            if (kc + 1 < nkc) sstore(buf ^ 1);
-            __syncthreads();
         }
+        cp_async_wait<0>();
         // C fragment: rows (tokens) g, g+8; columns (experts) 2tig, 2tig+1
 #pragma unroll
         for (int n8 = 0; n8 < 2; ++n8)
@@ -326,7 +352,15 @@ __global__ void __launch_bounds__(kScatterThreads) prefill_scatter_kernel(const 
     for (int i = warp; i < np; i += kScatterThreads / 32) {
         const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + i / k) * a.d);
         uint4* dst = reinterpret_cast<uint4*>(a.ws.x_perm + static_cast<size_t>(s_slot[i]) * a.d);
-        for (int c = lane; c < cpr; c += 32) dst[c] = __ldg(src + c);
+        for (int cb = lane; cb < cpr; cb += 32 * 8) {     // 8 independent loads in flight
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (cb + 32 * u < cpr) v[u] = __ldg(src + cb + 32 * u);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (cb + 32 * u < cpr) dst[cb + 32 * u] = v[u];
+        }
     }
 }
 
