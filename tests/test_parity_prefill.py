@@ -65,6 +65,9 @@ SMALL = [
     synth.MoEShape("one_token", T=1, d=256, E=8, k=2, F=128, S=1, Fs=128),
     synth.MoEShape("many_tiles", T=1000, d=1024, E=32, k=6, F=704, S=2, Fs=704,
                    zipf_bias=1.1),
+    # >= 1024 rows per expert on average: the GEMMs run as CTA pairs (256-row
+    # tiles, tcgen05.mma.cta_group::2); a ragged T and tail tiles of both kinds
+    synth.MoEShape("cta_pairs", T=2300, d=512, E=4, k=2, F=384, S=1, Fs=256),
 ]
 
 
