@@ -34,6 +34,11 @@ SMALL = [
                    wfmt=synth.WFMT_Q8_0),
     synth.MoEShape("multi_unit_q8", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512,
                    wfmt=synth.WFMT_Q8_0),
+    # the interface's limits: E = 1024 experts, k = 16, 8 shared experts, T = 8
+    # (128 token-expert pairs, a 32-word expert mask, the widest register top-k)
+    synth.MoEShape("max_limits", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32),
+    synth.MoEShape("max_limits_q4", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32,
+                   wfmt=synth.WFMT_Q4_0),
 ]
 
 

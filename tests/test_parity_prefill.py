@@ -68,6 +68,8 @@ SMALL = [
     # >= 1024 rows per expert on average: the GEMMs run as CTA pairs (256-row
     # tiles, tcgen05.mma.cta_group::2); a ragged T and tail tiles of both kinds
     synth.MoEShape("cta_pairs", T=2300, d=512, E=4, k=2, F=384, S=1, Fs=256),
+    # the prefill limit E = 256: four 64-expert router passes, k = 8
+    synth.MoEShape("E256", T=300, d=256, E=256, k=8, F=128, S=1, Fs=128, zipf_bias=1.1),
 ]
 
 
