@@ -136,7 +136,8 @@ typedef struct moe_plan_s* moe_plan_t;
  * success *out receives the plan; on failure *out is NULL and nothing is
  * left allocated.  This is the only entry point that allocates device
  * memory.  Errors: INVALID_ARG (shape limits above), UNSUPPORTED (PREFILL
- * regime with Q4_0, or a device that is not sm_100), CUDA, OOM. */
+ * regime with Q4_0 or Q8_0 weights, or a device that is not sm_100), CUDA,
+ * OOM. */
 moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out);
 
 /* Free the plan's workspace.  The caller must make sure no work enqueued

@@ -779,7 +779,7 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
 //   R  every CTA computes the router logits of experts b, b+G, ... (fp32 FMA,
 //      each dot product split over 8 warps and summed in a fixed order) and
 //      zero-fills its share of `out`;
-//   -  grid barrier (arrival counter + generation word, bounded wait);
+//   -  grid barrier (a 64-bit arrival count that only grows, bounded wait);
 //   T  every CTA reads all T x E logits and computes the same top-k,
 //      renormalised weights, stable slots and work list in its own shared
 //      memory (no second barrier); CTA 0 also writes the routing tables;
