@@ -4,7 +4,7 @@
 //  1. prefill_router_kernel: router logits for 32 tokens per CTA on the
 //     tensor cores, as accurate as fp32 FMAs (the fp32 router weights are
 //     split exactly into three bf16 parts; x and router chunks stream in by
-//     cp.async three chunks ahead), top-k with renormalised weights, the
+//     cp.async, two chunks in flight), top-k with renormalised weights, the
 //     CTA's per-expert histogram, and the zero-fill of its rows of `out`.
 //     ("Fused MoE Triton kernel: 5 launches instead of 24" page, fused steps
 //     one and two.)
@@ -86,9 +86,9 @@ __device__ __forceinline__ void cp_async_wait() {
 // holds the next 8 significant bits), so every x*part product (bf16 x) is
 // exact in fp32 and mma.sync accumulates the three partial logits in fp32.
 // (TF32 would instead round w to 10 bits.)  64-column chunks of x and of the
-// fp32 router arrive by cp.async in a ring of four (three chunks in flight
-// while one is used); each chunk is split into the double-buffered bf16
-// tiles the mma's read.
+// fp32 router arrive by cp.async in a ring of four (two chunks in flight
+// while one is split and used); each chunk is split into the double-buffered
+// bf16 tiles the mma's read.
 // Warp w handles tokens 16*(w/4).. and experts 16*(w%4)..  of the pass.
 __global__ void __launch_bounds__(kRouterThreads)
 prefill_router_kernel(const PrefillRouteArgs a) {
