@@ -321,16 +321,23 @@ def run_b200(args, sh):
 
         # The timed loop replays a CUDA graph of S whole steps (router +
         # experts per step, cycling the instances), so host launch overhead
-        # cannot starve the GPU.  A second graph of the same steps carries
-        # an event node on each side of every experts launch, for that
-        # kernel's own duration.
+        # cannot starve the GPU: R full replays and one graph of the
+        # remaining K - R*S steps time exactly K = --steps steps.  A second
+        # graph of S steps carries an event node on each side of every
+        # experts launch, for that kernel's own duration.
         S = n_inst * max(1, -(-32 // n_inst))
-        R = max(1, -(-args.steps // S))
-        K = R * S
+        K = max(1, args.steps)
+        R, rem = divmod(K, S)
         g_steps = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_steps, stream=stream):
             for i in range(S):
                 step(i)
+        g_rem = None
+        if rem:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem, stream=stream):
+                for i in range(rem):
+                    step(i)
         ev_a = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(S)]
         ev_b = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(S)]
         g_kern = torch.cuda.CUDAGraph()
@@ -340,6 +347,8 @@ def run_b200(args, sh):
         for _ in range(2):
             g_steps.replay()
             g_kern.replay()
+            if g_rem is not None:
+                g_rem.replay()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         uuid = str(torch.cuda.get_device_properties(dev).uuid)
@@ -352,6 +361,8 @@ def run_b200(args, sh):
             t_start.record(stream)
             for _ in range(R):
                 g_steps.replay()
+            if g_rem is not None:
+                g_rem.replay()
             t_end.record(stream)
             torch.cuda.synchronize(dev)
             kern_ms = []
@@ -367,7 +378,7 @@ def run_b200(args, sh):
         status = B.moe_get_device_status(plan)
         if status != B.MOE_OK:
             raise RuntimeError("device status after timing: " + B.moe_status_string(status))
-        del g_steps, g_kern
+        del g_steps, g_kern, g_rem
 
         # e2e: pinned host x in, pinned host out back, every step
         x_host = torch.from_numpy(base.x.view(np.int16)).pin_memory()
