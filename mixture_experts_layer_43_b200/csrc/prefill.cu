@@ -37,6 +37,7 @@
 namespace moe {
 
 constexpr int kChunkTok = 32;        // tokens per router / scatter CTA
+constexpr int kMaxDevices = 64;      // per-device launch attributes
 constexpr int kRouterThreads = 256;
 constexpr int kRouterKC = 64;        // d columns per router k-chunk (double-buffered)
 constexpr int kRouterEC = 64;        // experts per router pass
@@ -894,12 +895,15 @@ moe_status_t prefill_route(PrefillState* st, const moe_config_t& c, const Worksp
     r.F = c.d_ff; r.Fs = c.n_shared ? c.d_ff_shared : 0;
     const int nch = (T + kChunkTok - 1) / kChunkTok;
     const size_t smem = router_smem_bytes(c.n_experts);
-    static int set_smem = 0;
-    if (static_cast<int>(smem) > set_smem) {
+    // the shared-memory limit is a per-device attribute: raise it once per device
+    static int set_smem[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    if (static_cast<int>(smem) > set_smem[dev]) {
         if (cudaFuncSetAttribute(prefill_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess)
             return MOE_ERR_CUDA;
-        set_smem = static_cast<int>(smem);
+        set_smem[dev] = static_cast<int>(smem);
     }
     prefill_router_kernel<<<nch, kRouterThreads, smem, stream>>>(r);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
@@ -967,14 +971,16 @@ moe_status_t prefill_experts(PrefillState* st, const moe_config_t& c, const Work
     const int cg = prefill_pick_cg(st, num_sms);
     const size_t smem = gemm_smem_bytes(E, cg);
     if (cg == 1) {
-        static bool attr = false;
-        if (!attr) {
+        static bool attr[kMaxDevices] = {false};
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+        if (!attr[dev]) {
             if (cudaFuncSetAttribute(prefill_gemm_kernel<kGateUp, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(gemm_smem_bytes(kMaxExperts, 1))) != cudaSuccess ||
                 cudaFuncSetAttribute(prefill_gemm_kernel<kDown, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(gemm_smem_bytes(kMaxExperts, 1))) != cudaSuccess)
                 return MOE_ERR_CUDA;
-            attr = true;
+            attr[dev] = true;
         }
         prefill_gemm_kernel<kGateUp, 1><<<num_sms, kGemmThreads, smem, stream>>>(st->g1);
         if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
