@@ -64,3 +64,29 @@ def test_reduce_is_identity_without_process_group():
     import bench
     assert bench.reduce_max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
     assert bench.job_tokens_per_s(1, 8, 100, 50.0) == pytest.approx(16000.0)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """`bench.py --impl reference` runs the oracle on the host (no GPU): one
+    JSON line with the contract's keys, its own cpu_baseline and an e2e
+    block with no host-device copies."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny_T4_d256_E8k2_F512", "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 3 and d["warmup"] == 3
+    assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "tiny_T4_d256_E8k2_F512"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
