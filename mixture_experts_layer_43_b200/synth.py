@@ -21,6 +21,10 @@ Storage conventions (the C ABI's, see include/moe.h):
   Q4_0      canonical 18-byte blocks along the reduction dim:
             [rows][K/32][18] = fp16 scale (little endian) + 16 code bytes,
             byte j holding element j (low nibble) and element j+16 (high).
+  Q8_0      [rows][K/32][34] = fp16 scale + 32 signed code bytes.
+  Q5_0      [rows][K/32][22] = fp16 scale + 32-bit little-endian word of
+            fifth bits (bit j for element j) + 16 bytes of low nibbles
+            packed as in Q4_0.
 """
 from __future__ import annotations
 
@@ -33,9 +37,11 @@ import numpy as np
 WFMT_BF16 = 0
 WFMT_Q4_0 = 1
 WFMT_Q8_0 = 2
+WFMT_Q5_0 = 3
 Q4_BLOCK = 32          # weights per Q4_0 block
 Q4_BLOCK_BYTES = 18    # 2-byte fp16 scale + 16 bytes of 4-bit codes
 Q8_BLOCK_BYTES = 34    # 2-byte fp16 scale + 32 signed 8-bit codes
+Q5_BLOCK_BYTES = 22    # 2-byte fp16 scale + 4 bytes of fifth bits + 16 bytes of nibbles
 
 
 @dataclasses.dataclass(frozen=True)
@@ -55,6 +61,7 @@ class MoEShape:
     wr_std: float = 0.02
     q4_scale_std: float = 0.005
     q8_scale_std: float = 0.00035
+    q5_scale_std: float = 0.0025
 
     def replace(self, **kw) -> "MoEShape":
         return dataclasses.replace(self, **kw)
@@ -83,6 +90,13 @@ WORKLOADS = {
     "a3b_q8_T8_d2048_E256k8_F512_S1": MoEShape(
         "a3b_q8_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512,
         S=1, Fs=512, wfmt=WFMT_Q8_0),
+    # ... and with Q5_0 weights (also in the model's mix)
+    "a3b_q5_T1_d2048_E256k8_F512_S1": MoEShape(
+        "a3b_q5_T1_d2048_E256k8_F512_S1", T=1, d=2048, E=256, k=8, F=512,
+        S=1, Fs=512, wfmt=WFMT_Q5_0),
+    "a3b_q5_T8_d2048_E256k8_F512_S1": MoEShape(
+        "a3b_q5_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512,
+        S=1, Fs=512, wfmt=WFMT_Q5_0),
     # the same 35B-A3B layer in bf16 at T = 8 (about 58 distinct experts, 0.37 GB)
     "a3b_T8_d2048_E256k8_F512_S1": MoEShape(
         "a3b_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512, S=1, Fs=512),
@@ -166,15 +180,37 @@ def q8_0_blocks(rng: np.random.Generator, rows: int, k: int,
     return out
 
 
+def q5_0_blocks(rng: np.random.Generator, rows: int, k: int,
+                scale_std: float) -> np.ndarray:
+    """Canonical Q5_0 blocks [rows][k/32][22] with codes uniform on 0..31
+    and scales |N(0, scale_std)| stored as fp16."""
+    assert k % Q4_BLOCK == 0
+    nb = k // Q4_BLOCK
+    out = np.empty((rows, nb, Q5_BLOCK_BYTES), dtype=np.uint8)
+    step = max(1, (1 << 22) // max(1, nb))
+    bit = (np.uint32(1) << np.arange(32, dtype=np.uint32)).astype(np.uint32)
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        q = rng.integers(0, 32, size=(r1 - r0, nb, Q4_BLOCK), dtype=np.uint8)
+        sc = np.abs(rng.standard_normal((r1 - r0, nb), dtype=np.float32)
+                    * np.float32(scale_std)).astype(np.float16)
+        qh = ((q >> 4).astype(np.uint32) * bit).sum(axis=2, dtype=np.uint32)
+        lo = q & 15
+        out[r0:r1, :, 0:2] = sc.view(np.uint8).reshape(r1 - r0, nb, 2)
+        out[r0:r1, :, 2:6] = qh.astype("<u4").view(np.uint8).reshape(r1 - r0, nb, 4)
+        out[r0:r1, :, 6:] = lo[:, :, :16] | (lo[:, :, 16:] << 4)
+    return out
+
+
 @dataclasses.dataclass
 class MoEInputs:
     shape: MoEShape
     x: np.ndarray                 # uint16 bf16 bits [T][d]
     router_w: np.ndarray          # float32 [E][d]
     router_b: Optional[np.ndarray]  # float32 [E] or None
-    gate: np.ndarray              # bf16 bits [E][F][d] or Q4_0 blocks [E][F][d/32][18]
+    gate: np.ndarray              # bf16 bits [E][F][d] or blocks [E][F][d/32][block bytes]
     up: np.ndarray
-    down: np.ndarray              # bf16 bits [E][d][F] or Q4_0 blocks [E][d][F/32][18]
+    down: np.ndarray              # bf16 bits [E][d][F] or blocks [E][d][F/32][block bytes]
     shared_gate: Optional[np.ndarray]
     shared_up: Optional[np.ndarray]
     shared_down: Optional[np.ndarray]
@@ -207,10 +243,10 @@ def make_inputs(shape: MoEShape, seed: int = 0,
         else:
             sg = su = sd = None
     else:
-        if sh.wfmt == WFMT_Q4_0:
-            blocks, q, nbytes = q4_0_blocks, sh.q4_scale_std, Q4_BLOCK_BYTES
-        else:
-            blocks, q, nbytes = q8_0_blocks, sh.q8_scale_std, Q8_BLOCK_BYTES
+        blocks, q, nbytes = {
+            WFMT_Q4_0: (q4_0_blocks, sh.q4_scale_std, Q4_BLOCK_BYTES),
+            WFMT_Q8_0: (q8_0_blocks, sh.q8_scale_std, Q8_BLOCK_BYTES),
+            WFMT_Q5_0: (q5_0_blocks, sh.q5_scale_std, Q5_BLOCK_BYTES)}[sh.wfmt]
 
         def stack(i, mats, rows, kk):
             return blocks(rng(i), mats * rows, kk, q).reshape(mats, rows, kk // 32, nbytes)
@@ -234,6 +270,8 @@ def weight_bytes_per_expert(shape: MoEShape, hidden: Optional[int] = None) -> in
         return 2 * n
     if shape.wfmt == WFMT_Q4_0:
         return n // 32 * 18   # 16 code bytes + 2 scale bytes per 32 weights
+    if shape.wfmt == WFMT_Q5_0:
+        return n // 32 * 22   # 16 nibble bytes + 4 fifth-bit bytes + 2 scale bytes
     return n // 32 * 34       # 32 code bytes + 2 scale bytes per 32 weights
 
 
@@ -243,7 +281,8 @@ def expert_flops(shape: MoEShape, n_tokens: int, hidden: Optional[int] = None) -
 
 
 def describe(shape: MoEShape) -> str:
-    fmt = {WFMT_BF16: "bf16", WFMT_Q4_0: "q4_0", WFMT_Q8_0: "q8_0"}[shape.wfmt]
+    fmt = {WFMT_BF16: "bf16", WFMT_Q4_0: "q4_0", WFMT_Q8_0: "q8_0",
+           WFMT_Q5_0: "q5_0"}[shape.wfmt]
     s = (f"T={shape.T} d={shape.d} E={shape.E} k={shape.k} F={shape.F} "
          f"S={shape.S} Fs={shape.Fs} {fmt}")
     if shape.zipf_bias:

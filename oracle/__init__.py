@@ -24,6 +24,7 @@ _lib = None
 WFMT_BF16 = 0
 WFMT_Q4_0 = 1
 WFMT_Q8_0 = 2
+WFMT_Q5_0 = 3
 
 
 def build(force: bool = False) -> str:
@@ -116,8 +117,8 @@ def fp16_to_f64(bits: int) -> float:
 
 
 def dequant(wfmt: int, w: np.ndarray, rows: int, k: int) -> np.ndarray:
-    """Rows x k matrix of a bf16 (uint16 bits), canonical-Q4_0 or canonical-Q8_0
-    array, fp64."""
+    """Rows x k matrix of a bf16 (uint16 bits), canonical-Q4_0, canonical-Q8_0
+    or canonical-Q5_0 array, fp64."""
     out = np.empty((rows, k), dtype=np.float64)
     _L().oracle_dequant_rows(wfmt, _p(np.ascontiguousarray(w)), rows, k, _p(out))
     return out

@@ -34,14 +34,18 @@
  * element j in its low nibble and element j+16 in its high nibble), and Q8_0
  * blocks as w = d * q from the canonical 34-byte blocks (fp16 scale d, then
  * 32 signed bytes q, element j in byte j; the 5090 page names q8_0 among the
- * formats of the model it measures).  Every dequantised value is exact in
- * double precision.
+ * formats of the model it measures), and Q5_0 blocks as w = d * (q - 16) from
+ * the canonical 22-byte blocks (fp16 scale d, a little-endian 32-bit word qh
+ * of fifth bits, then 16 bytes of low nibbles as in Q4_0; element j takes
+ * bit j of qh as its fifth bit; q5_0 is in the same list of formats).  Every
+ * dequantised value is exact in double precision.
  *
  * Layouts (row-major, reduction dimension contiguous):
  *   x [T][d] bf16 bits; Wr [E][d] fp32; b [E] fp32 or NULL
  *   routed gate/up [E][F][d], down [E][d][F]; shared [S][Fs][d], [S][d][Fs]
  *   Q4_0: a row of K weights is K/32 blocks of 18 bytes.
  *   Q8_0: a row of K weights is K/32 blocks of 34 bytes.
+ *   Q5_0: a row of K weights is K/32 blocks of 22 bytes.
  *
  * The pages print no worked example for the layer output, so the tests pin
  * every function here against what the mathematics fixes instead: brute-force
@@ -60,6 +64,7 @@
 #define ORACLE_WFMT_BF16 0
 #define ORACLE_WFMT_Q4_0 1
 #define ORACLE_WFMT_Q8_0 2
+#define ORACLE_WFMT_Q5_0 3
 
 /* bfloat16 is the top half of an IEEE binary32. */
 double oracle_bf16_to_f64(uint16_t b) {
@@ -112,6 +117,23 @@ static void q8_0_row(const uint8_t* blocks, int64_t K, double* out) {
     }
 }
 
+/* Dequantise one row of K weights stored as canonical Q5_0 blocks. */
+static void q5_0_row(const uint8_t* blocks, int64_t K, double* out) {
+    for (int64_t b = 0; b < K / 32; ++b) {
+        const uint8_t* blk = blocks + b * 22;
+        uint16_t hd = (uint16_t)(blk[0] | (blk[1] << 8));
+        double dsc = oracle_fp16_to_f64(hd);
+        uint32_t qh = (uint32_t)blk[2] | ((uint32_t)blk[3] << 8) | ((uint32_t)blk[4] << 16) |
+                      ((uint32_t)blk[5] << 24);
+        for (int j = 0; j < 16; ++j) {
+            int lo = (blk[6 + j] & 0x0f) | (int)(((qh >> j) & 1u) << 4);
+            int hi = (blk[6 + j] >> 4) | (int)(((qh >> (j + 16)) & 1u) << 4);
+            out[b * 32 + j] = dsc * (double)(lo - 16);
+            out[b * 32 + j + 16] = dsc * (double)(hi - 16);
+        }
+    }
+}
+
 /* Row r of matrix m (0-based) of a stack of matrices [M][rows][K]. */
 static void load_row(int wfmt, const void* base, int64_t m, int64_t rows,
                      int64_t K, int64_t r, double* out) {
@@ -122,9 +144,12 @@ static void load_row(int wfmt, const void* base, int64_t m, int64_t rows,
     } else if (wfmt == ORACLE_WFMT_Q4_0) {
         const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 18;
         q4_0_row(p, K, out);
-    } else {
+    } else if (wfmt == ORACLE_WFMT_Q8_0) {
         const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 34;
         q8_0_row(p, K, out);
+    } else {
+        const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 22;
+        q5_0_row(p, K, out);
     }
 }
 
@@ -257,7 +282,8 @@ int oracle_forward(int d, int E, int k, int F, int S, int Fs, int wfmt,
         !wg || !wu || !wd || !out || !ids || !w || n_tokens < 0)
         return 1;
     if (S > 0 && (Fs <= 0 || !sg || !su || !sd)) return 1;
-    if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0)
+    if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0 &&
+        wfmt != ORACLE_WFMT_Q5_0)
         return 1;
     if (wfmt != ORACLE_WFMT_BF16 && (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
 #ifdef _OPENMP

@@ -33,6 +33,10 @@ MUTANTS = {
                           "int q = (int)blk[2 + j];"),
     "q8_scale_bytes_not_skipped": ("int q = blk[2 + j] < 128 ? (int)blk[2 + j] : (int)blk[2 + j] - 256;",
                                    "int q = blk[j] < 128 ? (int)blk[j] : (int)blk[j] - 256;"),
+    "q5_fifth_bits_swapped_halves": ("int lo = (blk[6 + j] & 0x0f) | (int)(((qh >> j) & 1u) << 4);",
+                                     "int lo = (blk[6 + j] & 0x0f) | (int)(((qh >> (j + 16)) & 1u) << 4);"),
+    "q5_offset_15": ("out[b * 32 + j] = dsc * (double)(lo - 16);", "out[b * 32 + j] = dsc * (double)(lo - 15);"),
+    "q5_qh_bytes_not_skipped": ("int lo = (blk[6 + j] & 0x0f)", "int lo = (blk[2 + j] & 0x0f)"),
     "fp16_exponent_bias": ("ldexp(1024.0 + (double)m, e - 25)", "ldexp(1024.0 + (double)m, e - 24)"),
     "bucket_unstable": ("for (int64_t p = 0; p < n; ++p) {\n            int e = ids[p];",
                         "for (int64_t p = n - 1; p >= 0; --p) {\n            int e = ids[p];"),
@@ -44,6 +48,7 @@ MUTANTS = {
 def _pins():
     yield lambda: pins.test_q4_0_golden_blocks()
     yield lambda: pins.test_q8_0_golden_blocks()
+    yield lambda: pins.test_q5_0_golden_blocks()
     yield lambda: pins.test_fp16_decode_matches_numpy_all_patterns()
     yield lambda: pins.test_softmax_renormalisation_closed_form()
     yield lambda: pins.test_swiglu_closed_form()

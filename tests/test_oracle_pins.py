@@ -99,6 +99,44 @@ def test_q8_0_rows_are_independent_blocks():
                 assert got[r, 32 * b + j] == scale * codes[j]
 
 
+def test_q5_0_golden_blocks():
+    g = json.load(open(os.path.join(GOLDEN, "q5_0_blocks.json")))
+    for blk in g["blocks"]:
+        raw = np.array(blk["bytes"], dtype=np.uint8)
+        got = oracle.dequant(oracle.WFMT_Q5_0, raw, 1, 32)[0]
+        scale = float(np.array([blk["scale_bits"]], np.uint16).view(np.float16)[0])
+        want = np.array([scale * (q - 16) for q in blk["codes"]], dtype=np.float64)
+        assert np.array_equal(got, want), blk["name"]
+
+
+def _q5_codes(raw):
+    """The 32 codes of one canonical Q5_0 block, with Python's struct and
+    integer operations: bit j of the little-endian word after the scale is
+    element j's fifth bit."""
+    (qh,) = struct.unpack("<I", raw[2:6])
+    qs = raw[6:22]
+    low = [c & 15 for c in qs] + [c >> 4 for c in qs]
+    return [low[j] + 16 * ((qh >> j) & 1) for j in range(32)]
+
+
+def test_q5_0_rows_are_independent_blocks():
+    """A multi-row, multi-block Q5_0 matrix dequantises block by block in
+    row-major block order (checked with Python's struct decoders)."""
+    rng = np.random.default_rng(7)
+    rows, k = 3, 96
+    blocks = synth.q5_0_blocks(rng, rows, k, 0.01)
+    got = oracle.dequant(oracle.WFMT_Q5_0, blocks, rows, k)
+    seen = set()
+    for r in range(rows):
+        for b in range(k // 32):
+            raw = bytes(blocks[r, b])
+            (scale,) = struct.unpack("<e", raw[:2])
+            for j, q in enumerate(_q5_codes(raw)):
+                assert got[r, 32 * b + j] == scale * (q - 16)
+                seen.add(q)
+    assert min(seen) < 16 <= max(seen)     # both values of the fifth bit occur
+
+
 # ------------------------------------------------- pure-Python brute force
 def _bf16(b):
     return struct.unpack(">f", struct.pack(">I", int(b) << 16))[0]
@@ -132,12 +170,27 @@ def _q8_rows(blocks):
     return out
 
 
+def _q5_rows(blocks):
+    """Pure-Python decode of canonical Q5_0 rows -> list of lists."""
+    out = []
+    for row in blocks:
+        vals = []
+        for blk in row:
+            raw = bytes(blk)
+            (sc,) = struct.unpack("<e", raw[:2])
+            vals.extend(sc * (q - 16) for q in _q5_codes(raw))
+        out.append(vals)
+    return out
+
+
 def _mat(inp_arr, wfmt, m, rows, cols):
     if wfmt == synth.WFMT_BF16:
         a = inp_arr[m]
         return [[_bf16(a[r, c]) for c in range(cols)] for r in range(rows)]
     if wfmt == synth.WFMT_Q4_0:
         return _q4_rows(inp_arr[m])
+    if wfmt == synth.WFMT_Q5_0:
+        return _q5_rows(inp_arr[m])
     return _q8_rows(inp_arr[m])
 
 
@@ -199,13 +252,16 @@ TINY = [
                    wfmt=synth.WFMT_Q4_0),
     synth.MoEShape("q8_shared", T=2, d=32, E=4, k=2, F=32, S=1, Fs=32,
                    wfmt=synth.WFMT_Q8_0),
+    synth.MoEShape("q5_shared", T=2, d=32, E=4, k=2, F=32, S=1, Fs=32,
+                   wfmt=synth.WFMT_Q5_0),
 ]
 
 
 @pytest.mark.parametrize("sh", TINY, ids=[s.name for s in TINY])
 def test_brute_force_tiny(sh):
     # A larger weight std makes the logits spread and the SwiGLU nonlinear.
-    sh = sh.replace(w_std=0.5, wr_std=0.5, q4_scale_std=0.05, q8_scale_std=0.004)
+    sh = sh.replace(w_std=0.5, wr_std=0.5, q4_scale_std=0.05, q8_scale_std=0.004,
+                    q5_scale_std=0.025)
     inp = synth.make_inputs(sh, seed=11)
     out, ids, w, logits = oracle.forward(inp)
     bout, bsets, bw, _ = _brute_layer(inp)
@@ -232,6 +288,14 @@ def _f64_stack(arr, wfmt, rows, cols):
         sc = a[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
         q = a[..., 2:].copy().view(np.int8).astype(np.float64)
         return (q * sc[..., None]).reshape(-1, rows, cols)
+    if wfmt == synth.WFMT_Q5_0:
+        a = np.ascontiguousarray(arr).reshape(-1, rows, cols // 32, 22)
+        sc = a[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
+        qh = a[..., 2:6].copy().view("<u4")[..., 0]
+        fifth = (qh[..., None] >> np.arange(32, dtype=np.uint32)) & 1
+        low = np.concatenate([a[..., 6:] & 15, a[..., 6:] >> 4], axis=-1)
+        q = low.astype(np.float64) + 16.0 * fifth - 16.0
+        return (q * sc[..., None]).reshape(-1, rows, cols)
     a = np.ascontiguousarray(arr).reshape(-1, rows, cols // 32, 18)
     sc = a[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
     lo = (a[..., 2:] & 15).astype(np.float64) - 8
@@ -252,10 +316,12 @@ def _x64(inp):
     return torch.from_numpy(inp.x.view(np.int16)).view(torch.bfloat16).double().numpy()
 
 
-@pytest.mark.parametrize("wfmt", [synth.WFMT_BF16, synth.WFMT_Q4_0, synth.WFMT_Q8_0])
+@pytest.mark.parametrize("wfmt", [synth.WFMT_BF16, synth.WFMT_Q4_0, synth.WFMT_Q8_0,
+                                  synth.WFMT_Q5_0])
 def test_k_equals_E_is_dense_softmax_mixture(wfmt):
     sh = synth.MoEShape("dense", T=5, d=64, E=4, k=4, F=32, wfmt=wfmt,
-                        wr_std=0.2, w_std=0.2, q4_scale_std=0.02, q8_scale_std=0.002)
+                        wr_std=0.2, w_std=0.2, q4_scale_std=0.02, q8_scale_std=0.002,
+                        q5_scale_std=0.01)
     inp = synth.make_inputs(sh, seed=3)
     out, ids, w, logits = oracle.forward(inp)
     x = _x64(inp)
