@@ -443,7 +443,7 @@ def run_b200(args, sh):
         "ms_per_step": t_max / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": {synth.WFMT_BF16: "bf16", synth.WFMT_Q4_0: "q4_0/bf16",
-                  synth.WFMT_Q8_0: "q8_0/bf16"}[sh.wfmt],
+                  synth.WFMT_Q8_0: "q8_0/bf16", synth.WFMT_Q5_0: "q5_0/bf16"}[sh.wfmt],
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x; no trained weights)",
         "config": {"workload": sh.name, "shape": synth.describe(sh), "T": T,
                    "instances": n_inst, "graph_steps": S,

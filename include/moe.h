@@ -65,11 +65,17 @@ typedef enum moe_status {
  *   5090 page lists q8_0 among the formats of the 35B-A3B model it measures;
  *   it prints no layout, and the canonical 34-byte block is the reading
  *   taken).  The kernels read the packed form written by moe_q8_0_pack.
+ * MOE_WFMT_Q5_0: blocks of 32 consecutive weights along the reduction dim,
+ *   each an fp16 scale d and 32 codes q in 0..31, weight = d * (q - 16) (the
+ *   5090 page lists q5_0 in the same list of formats; the canonical 22-byte
+ *   block is the reading taken).  The kernels read the packed form written by
+ *   moe_q5_0_pack.
  * The quantised formats run in the decode regime only (T <= MOE_DECODE_MAX_T). */
 typedef enum moe_wfmt {
     MOE_WFMT_BF16 = 0,
     MOE_WFMT_Q4_0 = 1,
-    MOE_WFMT_Q8_0 = 2
+    MOE_WFMT_Q8_0 = 2,
+    MOE_WFMT_Q5_0 = 3
 } moe_wfmt_t;
 
 /* Execution regime.  AUTO picks DECODE for T <= MOE_DECODE_MAX_T (and for
@@ -102,8 +108,9 @@ typedef struct moe_config {
 } moe_config_t;
 
 /* One stack of expert matrices.  bf16: `data` is the bf16 stack, `scales`
- * must be NULL.  Q4_0 / Q8_0: `data` = packed codes, `scales` = packed fp16
- * scales (both from moe_q4_0_pack / moe_q8_0_pack). */
+ * must be NULL.  Q4_0 / Q8_0 / Q5_0: `data` = packed codes, `scales` = the
+ * packed fp16 scales (Q5_0: the packed records of scales and fifth bits),
+ * both from moe_q4_0_pack / moe_q8_0_pack / moe_q5_0_pack. */
 typedef struct moe_matrix {
     const void* data;
     const void* scales;
@@ -136,7 +143,7 @@ typedef struct moe_plan_s* moe_plan_t;
  * success *out receives the plan; on failure *out is NULL and nothing is
  * left allocated.  This is the only entry point that allocates device
  * memory.  Errors: INVALID_ARG (shape limits above), UNSUPPORTED (PREFILL
- * regime with Q4_0 or Q8_0 weights, or a device that is not sm_100), CUDA,
+ * regime with quantised weights, or a device that is not sm_100), CUDA,
  * OOM. */
 moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out);
 
@@ -255,6 +262,33 @@ moe_status_t moe_q8_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
  * The pages have no counterpart to this repacking (it serves the kernels'
  * tensor-core fragments). */
 moe_status_t moe_q8_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
+                           int64_t k, void* codes, void* scales, void* stream);
+
+/* Bytes of the packed Q5_0 form of n_mats matrices of [rows][k] weights
+ * (16 code bytes per block; 6 bytes of scale and fifth bits per block in
+ * `scale_bytes`).  k must be a multiple of 32 and rows of 8 (every matrix of
+ * a layer qualifies: d is a multiple of 128, F and Fs of 32).  Returns
+ * INVALID_ARG otherwise. */
+moe_status_t moe_q5_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
+                                   size_t* code_bytes, size_t* scale_bytes);
+
+/* Repack canonical Q5_0 blocks ([n_mats][rows][k/32] blocks of 22 bytes: a
+ * little-endian fp16 scale, a little-endian 32-bit word whose bit j is the
+ * fifth bit of element j, then 16 bytes whose byte j holds the low 4 bits of
+ * element j in the low nibble and of element j+16 in the high nibble) into
+ * the kernel layout:
+ *   codes  [n_mats][k/32][rows][16 bytes]: the low 4 bits, permuted exactly
+ *          like the Q4_0 codes;
+ *   scales [n_mats][k/32][rows/8][48 bytes]: for 8 consecutive rows their 8
+ *          fp16 scales, then their 8 32-bit words of fifth bits; in a row's
+ *          word, bits 4t+n and 16+4t+n (t, n = 0..3) are the fifth bits of
+ *          the codes that bits 4n..4n+3 and 16+4n..16+4n+3 of the row's code
+ *          word t hold.
+ * Same 5.5 bits per weight.  All pointers are device pointers; `blocks`
+ * needs no alignment, `codes`/`scales` 16 bytes.  Enqueued on `stream`.  The
+ * pages have no counterpart to this repacking (it serves the kernels'
+ * tensor-core fragments). */
+moe_status_t moe_q5_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
                            int64_t k, void* codes, void* scales, void* stream);
 
 /* Static description of a status code (never NULL). */

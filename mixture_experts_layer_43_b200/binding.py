@@ -27,6 +27,7 @@ MOE_ERR_TIMEOUT = 6
 MOE_WFMT_BF16 = 0
 MOE_WFMT_Q4_0 = 1
 MOE_WFMT_Q8_0 = 2
+MOE_WFMT_Q5_0 = 3
 MOE_REGIME_AUTO = 0
 MOE_REGIME_DECODE = 1
 MOE_REGIME_PREFILL = 2
@@ -110,6 +111,11 @@ def lib() -> ctypes.CDLL:
     L.moe_q8_0_packed_bytes.restype = S
     L.moe_q8_0_pack.argtypes = [P, I64, I64, I64, P, P, P]
     L.moe_q8_0_pack.restype = S
+    L.moe_q5_0_packed_bytes.argtypes = [I64, I64, I64, ctypes.POINTER(ctypes.c_size_t),
+                                        ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_q5_0_packed_bytes.restype = S
+    L.moe_q5_0_pack.argtypes = [P, I64, I64, I64, P, P, P]
+    L.moe_q5_0_pack.restype = S
     _lib = L
     return L
 
@@ -201,3 +207,15 @@ def moe_q8_0_packed_bytes(n_mats: int, rows: int, k: int):
 def moe_q8_0_pack(blocks: int, n_mats: int, rows: int, k: int, codes: int, scales: int,
                   stream: int = 0) -> None:
     _check(lib().moe_q8_0_pack(blocks, n_mats, rows, k, codes, scales, stream), "moe_q8_0_pack")
+
+
+def moe_q5_0_packed_bytes(n_mats: int, rows: int, k: int):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().moe_q5_0_packed_bytes(n_mats, rows, k, ctypes.byref(cb), ctypes.byref(sb)),
+           "moe_q5_0_packed_bytes")
+    return cb.value, sb.value
+
+
+def moe_q5_0_pack(blocks: int, n_mats: int, rows: int, k: int, codes: int, scales: int,
+                  stream: int = 0) -> None:
+    _check(lib().moe_q5_0_pack(blocks, n_mats, rows, k, codes, scales, stream), "moe_q5_0_pack")

@@ -66,7 +66,8 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->n_shared < 0 || c->n_shared > kMaxShared) return MOE_ERR_INVALID_ARG;
     if (c->n_shared > 0 && (c->d_ff_shared < 32 || c->d_ff_shared % 32 != 0))
         return MOE_ERR_INVALID_ARG;
-    if (c->wfmt != MOE_WFMT_BF16 && c->wfmt != MOE_WFMT_Q4_0 && c->wfmt != MOE_WFMT_Q8_0)
+    if (c->wfmt != MOE_WFMT_BF16 && c->wfmt != MOE_WFMT_Q4_0 && c->wfmt != MOE_WFMT_Q8_0 &&
+        c->wfmt != MOE_WFMT_Q5_0)
         return MOE_ERR_INVALID_ARG;
     if (c->regime < MOE_REGIME_AUTO || c->regime > MOE_REGIME_PREFILL) return MOE_ERR_INVALID_ARG;
     if (c->device < 0) return MOE_ERR_INVALID_ARG;
@@ -150,8 +151,8 @@ bool map_bf16(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int
                       swizzle_for(static_cast<int>(box_k) * 2), box_k * 2);
 }
 
-// Q4_0 / Q8_0 packed codes [mats][K/32][N][cb] (cb = 16 / 32 bytes per
-// block row) seen as 3D {cb, N, mats*K/32}.
+// Q4_0 / Q8_0 / Q5_0 packed codes [mats][K/32][N][cb] (cb = 16 / 32 / 16
+// bytes per block row) seen as 3D {cb, N, mats*K/32}.
 bool map_quant_codes(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
                      int64_t K, uint32_t box_rows, uint32_t box_kb, uint32_t cb) {
     uint64_t dims[3] = {cb, static_cast<uint64_t>(N), static_cast<uint64_t>(mats * (K / 32))};
@@ -169,6 +170,17 @@ bool map_quant_scales(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t m
     uint32_t box[2] = {box_rows, box_kb};
     return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_NONE, 2 * box_rows);
+}
+
+// Q5_0 packed scales and fifth bits [mats][K/32][N/8][48 bytes] seen as 3D
+// {48, N/8, mats*K/32}; a box of box_rows rows reads box_rows/8 records.
+bool map_q5_aux(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
+                int64_t K, uint32_t box_rows, uint32_t box_kb) {
+    uint64_t dims[3] = {48, static_cast<uint64_t>(N / 8), static_cast<uint64_t>(mats * (K / 32))};
+    uint64_t strides[2] = {48, static_cast<uint64_t>(N / 8) * 48};
+    uint32_t box[3] = {48, box_rows / 8, box_kb};
+    return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, 6 * box_rows);   // records are contiguous
 }
 
 bool same_weights(const moe_weights_t& a, const moe_weights_t& b) {
@@ -217,19 +229,25 @@ DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
     } else {
         const uint32_t kb = 512 / fs, nb = fs / 32;
         const uint32_t cb = c.wfmt == MOE_WFMT_Q8_0 ? 32 : 16;
+        // scales: fp16 [mats][K/32][N], or Q5_0's 48-byte records of 8 rows
+        auto scales = [&](CUtensorMap* m, const void* base, int64_t mats, int64_t N, int64_t K,
+                          uint32_t box_rows, uint32_t box_kb) {
+            return c.wfmt == MOE_WFMT_Q5_0 ? map_q5_aux(p, m, base, mats, N, K, box_rows, box_kb)
+                                           : map_quant_scales(p, m, base, mats, N, K, box_rows, box_kb);
+        };
         ok &= map_quant_codes(p, &a.tm_gate, w->gate.data, E, F, d, fs, kb, cb);
         ok &= map_quant_codes(p, &a.tm_up, w->up.data, E, F, d, fs, kb, cb);
         ok &= map_quant_codes(p, &a.tm_down, w->down.data, E, d, F, kQuantDownBoxRows, nb, cb);
-        ok &= map_quant_scales(p, &a.tm_gate_sc, w->gate.scales, E, F, d, fs, kb);
-        ok &= map_quant_scales(p, &a.tm_up_sc, w->up.scales, E, F, d, fs, kb);
-        ok &= map_quant_scales(p, &a.tm_down_sc, w->down.scales, E, d, F, kQuantDownBoxRows, nb);
+        ok &= scales(&a.tm_gate_sc, w->gate.scales, E, F, d, fs, kb);
+        ok &= scales(&a.tm_up_sc, w->up.scales, E, F, d, fs, kb);
+        ok &= scales(&a.tm_down_sc, w->down.scales, E, d, F, kQuantDownBoxRows, nb);
         if (S) {
             ok &= map_quant_codes(p, &a.tm_sgate, w->shared_gate.data, S, Fs, d, fs, kb, cb);
             ok &= map_quant_codes(p, &a.tm_sup, w->shared_up.data, S, Fs, d, fs, kb, cb);
             ok &= map_quant_codes(p, &a.tm_sdown, w->shared_down.data, S, d, Fs, kQuantDownBoxRows, nb, cb);
-            ok &= map_quant_scales(p, &a.tm_sgate_sc, w->shared_gate.scales, S, Fs, d, fs, kb);
-            ok &= map_quant_scales(p, &a.tm_sup_sc, w->shared_up.scales, S, Fs, d, fs, kb);
-            ok &= map_quant_scales(p, &a.tm_sdown_sc, w->shared_down.scales, S, d, Fs, kQuantDownBoxRows, nb);
+            ok &= scales(&a.tm_sgate_sc, w->shared_gate.scales, S, Fs, d, fs, kb);
+            ok &= scales(&a.tm_sup_sc, w->shared_up.scales, S, Fs, d, fs, kb);
+            ok &= scales(&a.tm_sdown_sc, w->shared_down.scales, S, d, Fs, kQuantDownBoxRows, nb);
         }
     }
     if (!ok) return nullptr;
@@ -613,6 +631,26 @@ moe_status_t moe_q8_0_pack(const void* blocks, int64_t n_mats, int64_t rows, int
     return cuda_status(launch_q8_0_pack(static_cast<const uint8_t*>(blocks), n_mats, rows, k,
                                         static_cast<uint8_t*>(codes),
                                         static_cast<uint16_t*>(scales),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_q5_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k, size_t* code_bytes,
+                                   size_t* scale_bytes) {
+    if (n_mats < 0 || rows < 0 || rows % 8 != 0 || k < 0 || k % 32 != 0) return MOE_ERR_INVALID_ARG;
+    const int64_t blocks = n_mats * rows * (k / 32);
+    if (code_bytes) *code_bytes = static_cast<size_t>(blocks) * 16;
+    if (scale_bytes) *scale_bytes = static_cast<size_t>(blocks) * 6;
+    return MOE_OK;
+}
+
+moe_status_t moe_q5_0_pack(const void* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                           void* codes, void* scales, void* stream) {
+    if (n_mats < 0 || rows < 0 || rows % 8 != 0 || k < 0 || k % 32 != 0) return MOE_ERR_INVALID_ARG;
+    if (n_mats * rows * k == 0) return MOE_OK;
+    if (!blocks || !codes || !scales || !aligned16(codes) || !aligned16(scales))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_q5_0_pack(static_cast<const uint8_t*>(blocks), n_mats, rows, k,
+                                        static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
                                         static_cast<cudaStream_t>(stream)));
 }
 

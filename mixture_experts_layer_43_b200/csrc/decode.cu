@@ -222,12 +222,14 @@ constexpr int kDecodeThreads = kConsumers + 32;   // + one producer warp
 
 // Weight formats of the decode kernels (the values of moe_wfmt_t).
 constexpr int kWfBf16 = 0, kWfQ4 = 1, kWfQ8 = 2;
+constexpr int kWfQ5 = 3;
 
 // The constant that turns the bf16 "128 + nibble" operands back into signed
 // codes (see q4_raw): Q4_0 subtracts 128 + 8; Q8_0, whose biased byte
 // u = q + 128 = 16 hi + lo enters as two nibble planes weighted 1 and 16,
-// subtracts 128 + 16 * 128 + 128.
-constexpr float quant_offset(int wf) { return wf == kWfQ8 ? 2304.f : 136.f; }
+// subtracts 128 + 16 * 128 + 128; Q5_0 (operands 128 + q, q < 32, see
+// q5_raw) subtracts 128 + 16.
+constexpr float quant_offset(int wf) { return wf == kWfQ8 ? 2304.f : wf == kWfQ5 ? 144.f : 136.f; }
 
 template <int FS, int WF>
 struct DecodeCfg {
@@ -238,10 +240,13 @@ struct DecodeCfg {
     static constexpr bool QUANT = WF != kWfBf16;
     static_assert(!QUANT || FS >= 32, "quantised slices hold whole blocks");
     static constexpr int CB = WF == kWfQ8 ? 32 : 16;   // code bytes of one block row
-    static constexpr int BR = CB + 2;                  // + its fp16 scale
+    // + its fp16 scale (Q5_0: + its 32-bit word of fifth bits; scale and word
+    // sit in 48-byte records of 8 rows, see q5_aux)
+    static constexpr int BR = CB + (WF == kWfQ5 ? 6 : 2);
     // bf16: phase A stage = gate+up [FS rows][KT cols]; phase B = down [RJ rows][FS cols]
-    // Q4_0 / Q8_0: phase A stage = gate+up [KB block cols][FS rows];
+    // Q4_0 / Q8_0 / Q5_0: phase A stage = gate+up [KB block cols][FS rows];
     //              phase B = [NB block cols][RJ rows]; codes, then the scales
+    //              (Q5_0: the 48-byte records of scales and fifth bits)
     static constexpr int STAGE = QUANT ? 2 * 512 * BR : 32768;
     static constexpr int KT = 8192 / FS;          // bf16 phase A k columns
     static constexpr int KB = 512 / FS;           // quantised phase A block columns
@@ -341,6 +346,69 @@ __device__ __forceinline__ void quant_block_b(const uint32_t* row_r, const uint3
 #pragma unroll
         for (int i = 0; i < 4; ++i) v[i] = fmaf(16.f, ch[i], cl[i]);
     }
+}
+
+// ---- Q5_0.  The low 4 bits of each code are packed exactly like Q4_0
+// codes.  The fifth bits of a block row form one 32-bit word in which lane
+// tig owns bits 4 tig + n (the code in nibble n of its code word, n = 0..3)
+// and bits 16 + 4 tig + n (nibble n + 4).  q5_lane_bits moves the lane's
+// eight bits to bits 4-7 and 20-23, so that (e >> n) & 0x00100010 is the
+// fifth bit, worth 16, of the two codes q4_raw(w, 4n) extracts: q5_raw is
+// then two bf16 values 128 + q, q in 0..31 (exact; Q5_0's weight is
+// d * (q - 16), the 16 folded into quant_offset like Q4_0's 8).
+__device__ __forceinline__ uint32_t q5_lane_bits(uint32_t word, int tig) {
+    return ((word >> (4 * tig)) & 0x000F000Fu) << 4;
+}
+
+__device__ __forceinline__ uint32_t q5_raw(uint32_t w, uint32_t e, int n) {
+    return q4_raw(w, 4 * n) | ((e >> n) & 0x00100010u);
+}
+
+// Scale and fifth-bit word of rows r and r + 8 (r % 16 < 8) of block column
+// bb in a stage region of 48-byte records [block columns][rows / 8]: a record
+// holds the 8 fp16 scales of 8 consecutive rows, then their 8 words.
+__device__ __forceinline__ void q5_aux(const uint8_t* aux, int bb, int nrows, int r, float& s0,
+                                       float& s8, uint32_t& h0, uint32_t& h8) {
+    const uint8_t* rec = aux + (bb * (nrows / 8) + (r >> 3)) * 48;
+    const int i = r & 7;
+    s0 = __half2float(*reinterpret_cast<const __half*>(rec + 2 * i));
+    s8 = __half2float(*reinterpret_cast<const __half*>(rec + 48 + 2 * i));
+    h0 = *reinterpret_cast<const uint32_t*>(rec + 16 + 4 * i);
+    h8 = *reinterpret_cast<const uint32_t*>(rec + 48 + 16 + 4 * i);
+}
+
+// quant_block_a / quant_block_b for Q5_0: e0, e8 are q5_lane_bits of rows r
+// and r + 8.
+__device__ __forceinline__ void q5_block_a(const uint32_t* row_r, const uint32_t* row_r8,
+                                           uint32_t e0, uint32_t e8, int tig, float c0, float c1,
+                                           uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3,
+                                           float v[4]) {
+    const uint32_t w0 = row_r[tig], w8 = row_r8[tig];
+    float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_bf16_16816(cb0, q5_raw(w0, e0, 0), q5_raw(w8, e8, 0), q5_raw(w0, e0, 1), q5_raw(w8, e8, 1),
+                   b0, b1);
+    mma_bf16_16816(cb1, q5_raw(w0, e0, 2), q5_raw(w8, e8, 2), q5_raw(w0, e0, 3), q5_raw(w8, e8, 3),
+                   b2, b3);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = cb0[i] + cb1[i];
+}
+
+__device__ __forceinline__ void q5_block_b(const uint32_t* row_r, const uint32_t* row_r8,
+                                           uint32_t e0, uint32_t e8, int tig, float c0, float c1,
+                                           const uint32_t* bh0, const uint32_t* bh1,
+                                           const uint32_t* bl0, const uint32_t* bl1, float v[4]) {
+    const uint32_t w0 = row_r[tig], w8 = row_r8[tig];
+    const uint32_t p0 = q5_raw(w0, e0, 0), q0 = q5_raw(w8, e8, 0);
+    const uint32_t p1 = q5_raw(w0, e0, 1), q1 = q5_raw(w8, e8, 1);
+    const uint32_t p2 = q5_raw(w0, e0, 2), q2 = q5_raw(w8, e8, 2);
+    const uint32_t p3 = q5_raw(w0, e0, 3), q3 = q5_raw(w8, e8, 3);
+    float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
+    mma_bf16_16816(cb0, p0, q0, p1, q1, bh0[0], bh0[1]);
+    mma_bf16_16816(cb1, p2, q2, p3, q3, bh1[0], bh1[1]);
+    mma_bf16_16816(cb0, p0, q0, p1, q1, bl0[0], bl0[1]);
+    mma_bf16_16816(cb1, p2, q2, p3, q3, bl1[0], bl1[1]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = cb0[i] + cb1[i];
 }
 
 // Work list the experts pipeline reads: generic pointers, so the same code
@@ -513,9 +581,15 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                             uint8_t* g = dst;
                             uint8_t* u2 = dst + C::KB * FS * C::BR;
                             tma_load_3d(g, mg, &full[slot], 0, f0, c2, pol);
-                            tma_load_2d(g + C::KB * FS * C::CB, mgs, &full[slot], f0, c2, pol);
                             tma_load_3d(u2, mu, &full[slot], 0, f0, c2, pol);
-                            tma_load_2d(u2 + C::KB * FS * C::CB, mus, &full[slot], f0, c2, pol);
+                            if constexpr (WF == kWfQ5) {
+                                // 48-byte records of 8 rows: {48 bytes, rows / 8, block columns}
+                                tma_load_3d(g + C::KB * FS * C::CB, mgs, &full[slot], 0, f0 / 8, c2, pol);
+                                tma_load_3d(u2 + C::KB * FS * C::CB, mus, &full[slot], 0, f0 / 8, c2, pol);
+                            } else {
+                                tma_load_2d(g + C::KB * FS * C::CB, mgs, &full[slot], f0, c2, pol);
+                                tma_load_2d(u2 + C::KB * FS * C::CB, mus, &full[slot], f0, c2, pol);
+                            }
                         }
                     } else {
                         const int j0 = (st - nA) * C::RJ;
@@ -535,8 +609,12 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                             for (int b = 0; b < nbox; ++b) {
                                 uint8_t* bd = dst + b * (C::NB * QB * C::BR);
                                 tma_load_3d(bd, md, &full[slot], 0, j0 + QB * b, c2, pol);
-                                tma_load_2d(bd + C::NB * QB * C::CB, mds, &full[slot],
-                                            j0 + QB * b, c2, pol);
+                                if constexpr (WF == kWfQ5)
+                                    tma_load_3d(bd + C::NB * QB * C::CB, mds, &full[slot], 0,
+                                                (j0 + QB * b) / 8, c2, pol);
+                                else
+                                    tma_load_2d(bd + C::NB * QB * C::CB, mds, &full[slot],
+                                                j0 + QB * b, c2, pol);
                             }
                         }
                     }
@@ -629,15 +707,28 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         uint32_t b0, b1, b2, b3;
                         ldsm_x4(xrow + ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
                         float v[4];
-                        // the accumulator starts at -offset * sum(x) of the block
-                        quant_block_a<WF>(row, row + 8 * (C::CB / 4), tig, xsum0[bb], xsum1[bb],
-                                          b0, b1, b2, b3, v);
-                        const float s0 = __half2float(scl[bb * FS + r0]);
-                        const float s8 = __half2float(scl[bb * FS + r0 + 8]);
-                        cacc[0] = fmaf(s0, v[0], cacc[0]);
-                        cacc[1] = fmaf(s0, v[1], cacc[1]);
-                        cacc[2] = fmaf(s8, v[2], cacc[2]);
-                        cacc[3] = fmaf(s8, v[3], cacc[3]);
+                        if constexpr (WF == kWfQ5) {
+                            float s0, s8;
+                            uint32_t h0, h8;
+                            q5_aux(reinterpret_cast<const uint8_t*>(scl), bb, FS, r0, s0, s8, h0, h8);
+                            q5_block_a(row, row + 8 * (C::CB / 4), q5_lane_bits(h0, tig),
+                                       q5_lane_bits(h8, tig), tig, xsum0[bb], xsum1[bb], b0, b1, b2,
+                                       b3, v);
+                            cacc[0] = fmaf(s0, v[0], cacc[0]);
+                            cacc[1] = fmaf(s0, v[1], cacc[1]);
+                            cacc[2] = fmaf(s8, v[2], cacc[2]);
+                            cacc[3] = fmaf(s8, v[3], cacc[3]);
+                        } else {
+                            // the accumulator starts at -offset * sum(x) of the block
+                            quant_block_a<WF>(row, row + 8 * (C::CB / 4), tig, xsum0[bb], xsum1[bb],
+                                              b0, b1, b2, b3, v);
+                            const float s0 = __half2float(scl[bb * FS + r0]);
+                            const float s8 = __half2float(scl[bb * FS + r0 + 8]);
+                            cacc[0] = fmaf(s0, v[0], cacc[0]);
+                            cacc[1] = fmaf(s0, v[1], cacc[1]);
+                            cacc[2] = fmaf(s8, v[2], cacc[2]);
+                            cacc[3] = fmaf(s8, v[3], cacc[3]);
+                        }
                     }
                 }
             }
@@ -726,15 +817,28 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         for (int bb = 0; bb < C::NB; ++bb) {
                             const uint32_t* row = codes + (bb * QB + rib) * (C::CB / 4);
                             float v[4];
-                            // the accumulator starts at -offset * sum(hi + lo) of the block
-                            quant_block_b<WF>(row, row + 8 * (C::CB / 4), tig, hs0[bb], hs1[bb],
-                                              bh[2 * bb], bh[2 * bb + 1], bl[2 * bb], bl[2 * bb + 1], v);
-                            const float s0 = __half2float(scl[bb * QB + rib]);
-                            const float s8 = __half2float(scl[bb * QB + rib + 8]);
-                            c[0] = fmaf(s0, v[0], c[0]);
-                            c[1] = fmaf(s0, v[1], c[1]);
-                            c[2] = fmaf(s8, v[2], c[2]);
-                            c[3] = fmaf(s8, v[3], c[3]);
+                            if constexpr (WF == kWfQ5) {
+                                float s0, s8;
+                                uint32_t h0, h8;
+                                q5_aux(reinterpret_cast<const uint8_t*>(scl), bb, QB, rib, s0, s8, h0, h8);
+                                q5_block_b(row, row + 8 * (C::CB / 4), q5_lane_bits(h0, tig),
+                                           q5_lane_bits(h8, tig), tig, hs0[bb], hs1[bb], bh[2 * bb],
+                                           bh[2 * bb + 1], bl[2 * bb], bl[2 * bb + 1], v);
+                                c[0] = fmaf(s0, v[0], c[0]);
+                                c[1] = fmaf(s0, v[1], c[1]);
+                                c[2] = fmaf(s8, v[2], c[2]);
+                                c[3] = fmaf(s8, v[3], c[3]);
+                            } else {
+                                // the accumulator starts at -offset * sum(hi + lo) of the block
+                                quant_block_b<WF>(row, row + 8 * (C::CB / 4), tig, hs0[bb], hs1[bb],
+                                                  bh[2 * bb], bh[2 * bb + 1], bl[2 * bb], bl[2 * bb + 1], v);
+                                const float s0 = __half2float(scl[bb * QB + rib]);
+                                const float s8 = __half2float(scl[bb * QB + rib + 8]);
+                                c[0] = fmaf(s0, v[0], c[0]);
+                                c[1] = fmaf(s0, v[1], c[1]);
+                                c[2] = fmaf(s8, v[2], c[2]);
+                                c[3] = fmaf(s8, v[3], c[3]);
+                            }
                         }
                     }
                     const int j = j0 + rgb * 16 + g;
@@ -1000,6 +1104,7 @@ int decode_stage_bytes(int fs, int wfmt) {
     (void)fs;
     if (wfmt == kWfQ4) return 2 * 512 * 18;
     if (wfmt == kWfQ8) return 2 * 512 * 34;
+    if (wfmt == kWfQ5) return 2 * 512 * 22;
     return 32768;
 }
 
@@ -1072,6 +1177,8 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, int wfmt, int grid,
         case kWfQ4 * 100 + 32: return launch_fused_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_fused_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_fused_one<32, kWfQ8>(a, grid, smem, stream);
+        case kWfQ5 * 100 + 64: return launch_fused_one<64, kWfQ5>(a, grid, smem, stream);
+        case kWfQ5 * 100 + 32: return launch_fused_one<32, kWfQ5>(a, grid, smem, stream);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -1085,6 +1192,8 @@ cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, int wfmt, int gri
         case kWfQ4 * 100 + 32: return launch_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_one<32, kWfQ8>(a, grid, smem, stream);
+        case kWfQ5 * 100 + 64: return launch_one<64, kWfQ5>(a, grid, smem, stream);
+        case kWfQ5 * 100 + 32: return launch_one<32, kWfQ5>(a, grid, smem, stream);
         default: return cudaErrorInvalidValue;
     }
 }

@@ -114,6 +114,8 @@ cudaError_t launch_q4_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
                              uint8_t* codes, uint16_t* scales, cudaStream_t stream);
 cudaError_t launch_q8_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
                              uint8_t* codes, uint16_t* scales, cudaStream_t stream);
+cudaError_t launch_q5_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint8_t* aux, cudaStream_t stream);
 
 // --------------------------------------------------------- device helpers
 #ifdef __CUDACC__

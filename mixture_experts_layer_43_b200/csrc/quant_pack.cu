@@ -1,5 +1,5 @@
-// quant_pack.cu -- repack canonical Q4_0 and Q8_0 blocks into the decode
-// kernels' layout.
+// quant_pack.cu -- repack canonical Q4_0, Q8_0 and Q5_0 blocks into the
+// decode kernels' layout.
 //
 // ---- Q4_0
 // Canonical block (32 weights along the reduction dim, 18 bytes): little-endian
@@ -130,6 +130,70 @@ cudaError_t launch_q8_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
     const int64_t want = (total + threads - 1) / threads;
     const int grid = static_cast<int>(want < 65536 ? want : 65536);
     q8_0_pack_kernel<<<grid, threads, 0, stream>>>(blocks, n_mats, rows, k / 32, codes, scales);
+    return cudaGetLastError();
+}
+
+
+
+// ---- Q5_0
+// Canonical block (32 weights, 22 bytes): little-endian fp16 scale d, a
+// little-endian 32-bit word qh whose bit j is the fifth bit of element j,
+// then 16 bytes; byte j holds the low 4 bits of element j (low nibble) and of
+// element j+16 (high nibble); q = low bits + 16 * fifth bit, weight =
+// d * (q - 16).  (The 5090 page lists q5_0 among the formats of the model it
+// measures; the byte layout is the canonical llama.cpp one, a reading.)
+//
+// Kernel layout (same 5.5 bits per weight):
+//   codes  [mat][k/32][rows][16 B]        the low 4 bits, packed like Q4_0
+//   aux    [mat][k/32][rows/8][48 B]      per 8 consecutive rows: their 8
+//                                         fp16 scales, then their 8 32-bit
+//                                         words of fifth bits
+// In a row's word of fifth bits, lane t (0..3) owns bits 4t+n and 16+4t+n
+// (n = 0..3): the fifth bits of the codes in nibbles n and n+4 of its code
+// word (elements 2t+8n and 2t+1+8n).
+__global__ void q5_0_pack_kernel(const uint8_t* __restrict__ blocks, int64_t n_mats, int64_t rows,
+                                 int64_t nkb, uint8_t* __restrict__ codes, uint8_t* __restrict__ aux) {
+    const int64_t total = n_mats * rows * nkb;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t kb = i % nkb;
+        const int64_t r = (i / nkb) % rows;
+        const int64_t m = i / (nkb * rows);
+        const uint8_t* src = blocks + i * 22;            // [m][r][kb] canonical
+        const uint32_t qh = static_cast<uint32_t>(src[2]) | (static_cast<uint32_t>(src[3]) << 8) |
+                            (static_cast<uint32_t>(src[4]) << 16) | (static_cast<uint32_t>(src[5]) << 24);
+        uint8_t lo[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            lo[j] = src[6 + j] & 0x0f;
+            lo[j + 16] = src[6 + j] >> 4;
+        }
+        uint32_t w[4], fifth = 0;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            w[t] = pack_q4_lane(lo, t);
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                fifth |= ((qh >> (2 * t + 8 * n)) & 1u) << (4 * t + n);
+                fifth |= ((qh >> (2 * t + 1 + 8 * n)) & 1u) << (16 + 4 * t + n);
+            }
+        }
+        const int64_t dst = (m * nkb + kb) * rows + r;   // [m][kb][r]
+        *reinterpret_cast<uint4*>(codes + dst * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        uint8_t* rec = aux + ((m * nkb + kb) * (rows / 8) + r / 8) * 48;
+        *reinterpret_cast<uint16_t*>(rec + 2 * (r % 8)) = static_cast<uint16_t>(src[0] | (src[1] << 8));
+        *reinterpret_cast<uint32_t*>(rec + 16 + 4 * (r % 8)) = fifth;
+    }
+}
+
+cudaError_t launch_q5_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint8_t* aux, cudaStream_t stream) {
+    const int64_t total = n_mats * rows * (k / 32);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t want = (total + threads - 1) / threads;
+    const int grid = static_cast<int>(want < 65536 ? want : 65536);
+    q5_0_pack_kernel<<<grid, threads, 0, stream>>>(blocks, n_mats, rows, k / 32, codes, aux);
     return cudaGetLastError();
 }
 

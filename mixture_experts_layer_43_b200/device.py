@@ -1,8 +1,8 @@
 """Device-memory plumbing around the C ABI: upload a layer's tensors with
-PyTorch (device memory and streams only), repack Q4_0 / Q8_0 through the
-library's own moe_q4_0_pack / moe_q8_0_pack kernels, and fill the
-moe_weights_t / moe_config_t structs.
-No arithmetic of the layer happens here."""
+PyTorch (device memory and streams only), repack Q4_0 / Q8_0 / Q5_0 through
+the library's own moe_q4_0_pack / moe_q8_0_pack / moe_q5_0_pack kernels, and
+fill the moe_weights_t / moe_config_t structs.  No arithmetic of the layer
+happens here."""
 from __future__ import annotations
 
 from typing import Optional
@@ -30,9 +30,11 @@ class DeviceLayer:
         self.shape = sh
         self.device = torch.device(device)
         self.q4 = sh.wfmt != synth.WFMT_BF16          # quantised: codes + scales
-        q8 = sh.wfmt == synth.WFMT_Q8_0
-        packed_bytes = B.moe_q8_0_packed_bytes if q8 else B.moe_q4_0_packed_bytes
-        pack = B.moe_q8_0_pack if q8 else B.moe_q4_0_pack
+        packed_bytes, pack = {
+            synth.WFMT_BF16: (None, None),
+            synth.WFMT_Q4_0: (B.moe_q4_0_packed_bytes, B.moe_q4_0_pack),
+            synth.WFMT_Q8_0: (B.moe_q8_0_packed_bytes, B.moe_q8_0_pack),
+            synth.WFMT_Q5_0: (B.moe_q5_0_packed_bytes, B.moe_q5_0_pack)}[sh.wfmt]
         st = stream if stream is not None else torch.cuda.current_stream(self.device)
         self.router_w = _dev(inp.router_w.astype(np.float32), self.device)
         self.router_b = None if inp.router_b is None else _dev(inp.router_b.astype(np.float32),

@@ -46,7 +46,7 @@ def _cfg(**kw):
     dict(t_max=0), dict(d_model=100), dict(d_model=192), dict(d_ff=48), dict(n_experts=0),
     dict(n_experts=2000), dict(top_k=0), dict(top_k=9), dict(n_experts=32, top_k=17),
     dict(n_shared=-1), dict(n_shared=9), dict(n_shared=1, d_ff_shared=0),
-    dict(n_shared=1, d_ff_shared=40), dict(wfmt=3), dict(regime=3), dict(device=-1),
+    dict(n_shared=1, d_ff_shared=40), dict(wfmt=4), dict(regime=3), dict(device=-1),
 ])
 def test_plan_create_rejects_bad_config(L, kw):
     plan = ctypes.c_void_p(123)
@@ -60,6 +60,8 @@ def test_plan_create_q4_prefill_unsupported(L):
     s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=1, regime=2)), ctypes.byref(plan))
     assert s == B.MOE_ERR_UNSUPPORTED
     s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=2, regime=2)), ctypes.byref(plan))
+    assert s == B.MOE_ERR_UNSUPPORTED
+    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=3, regime=2)), ctypes.byref(plan))
     assert s == B.MOE_ERR_UNSUPPORTED
 
 
@@ -105,3 +107,23 @@ def test_q8_pack_rejects_bad_args_without_gpu(L):
     assert L.moe_q8_0_pack(None, 1, 1, 32, None, None, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_q8_0_pack(16, 1, 1, 32, 17, 32, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_q8_0_pack(None, 0, 4, 32, None, None, None) == B.MOE_OK
+
+
+def test_q5_packed_bytes(L):
+    # 16 code bytes and 6 bytes of scale + fifth bits per block
+    assert B.moe_q5_0_packed_bytes(256, 512, 2048) == (256 * 512 * 64 * 16, 256 * 512 * 64 * 6)
+    assert B.moe_q5_0_packed_bytes(0, 8, 32) == (0, 0)
+    cb = ctypes.c_size_t()
+    assert L.moe_q5_0_packed_bytes(1, 8, 33, ctypes.byref(cb), None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q5_0_packed_bytes(-1, 8, 32, None, None) == B.MOE_ERR_INVALID_ARG
+    # records of 8 rows: rows must be a multiple of 8
+    assert L.moe_q5_0_packed_bytes(1, 12, 32, ctypes.byref(cb), None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_q5_pack_rejects_bad_args_without_gpu(L):
+    assert L.moe_q5_0_pack(None, 1, 8, 33, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q5_0_pack(None, 1, 8, 32, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q5_0_pack(None, 1, 4, 32, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q5_0_pack(16, 1, 8, 32, 17, 32, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q5_0_pack(None, 0, 8, 32, None, None, None) == B.MOE_OK
+

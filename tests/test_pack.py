@@ -1,4 +1,4 @@
-"""GPU test of the two repacking kernels (moe_q4_0_pack, moe_q8_0_pack):
+"""GPU test of the repacking kernels (moe_q4_0_pack, moe_q8_0_pack, moe_q5_0_pack):
 byte work, so bit-exact.  The packed arrays are decoded here with numpy by
 inverting the layout include/moe.h documents, and the codes and scales must
 equal those of the canonical blocks exactly."""
@@ -31,6 +31,17 @@ def _unpack_nibble_words(words):
     for t in range(4):
         for shift, idx in _word_slots(t):
             out[..., idx] = (words[..., t] >> shift) & 15
+    return out
+
+
+def _unpack_fifth_words(words):
+    """[...] uint32 words of fifth bits of one block row -> [..., 32] bits:
+    lane t's bits 4t+n and 16+4t+n belong to elements 2t+8n and 2t+1+8n."""
+    out = np.zeros(words.shape + (32,), np.uint8)
+    for t in range(4):
+        for n in range(4):
+            out[..., 2 * t + 8 * n] = (words >> (4 * t + n)) & 1
+            out[..., 2 * t + 1 + 8 * n] = (words >> (16 + 4 * t + n)) & 1
     return out
 
 
@@ -71,3 +82,22 @@ def test_q8_0_pack_is_the_documented_planes(n_mats, rows, k):
     assert np.array_equal(got, want)
     want_sc = canon[..., :2].copy().view(np.uint16)[..., 0]
     assert np.array_equal(scales.reshape(n_mats, k // 32, rows).transpose(0, 2, 1), want_sc)
+
+
+@pytest.mark.parametrize("n_mats,rows,k", [(1, 8, 32), (3, 40, 96), (2, 128, 512)])
+def test_q5_0_pack_is_the_documented_records(n_mats, rows, k):
+    rng = np.random.default_rng(n_mats * 1000 + rows + 13)
+    canon = synth.q5_0_blocks(rng, n_mats * rows, k, 0.01).reshape(n_mats, rows, k // 32, 22)
+    codes, aux = _pack_on_gpu(B.moe_q5_0_packed_bytes, B.moe_q5_0_pack, canon, n_mats, rows, k)
+    low = _unpack_nibble_words(codes.view(np.uint32).reshape(n_mats, k // 32, rows, 4))
+    rec = aux.view(np.uint8).reshape(n_mats, k // 32, rows // 8, 48)
+    sc = rec[..., :16].copy().view(np.uint16).reshape(n_mats, k // 32, rows)
+    fifth = _unpack_fifth_words(rec[..., 16:].copy().view(np.uint32).reshape(n_mats, k // 32, rows))
+    got = (low.astype(np.int32) + 16 * fifth).transpose(0, 2, 1, 3)    # [m][r][kb][32]
+    qh = canon[..., 2:6].copy().view("<u4")[..., 0]
+    want = np.concatenate([canon[..., 6:] & 15, canon[..., 6:] >> 4], axis=-1).astype(np.int32)
+    want += 16 * ((qh[..., None] >> np.arange(32, dtype=np.uint32)) & 1).astype(np.int32)
+    assert np.array_equal(got, want)
+    want_sc = canon[..., :2].copy().view(np.uint16)[..., 0]
+    assert np.array_equal(sc.transpose(0, 2, 1), want_sc)
+

@@ -39,6 +39,15 @@ SMALL = [
     synth.MoEShape("max_limits", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32),
     synth.MoEShape("max_limits_q4", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32,
                    wfmt=synth.WFMT_Q4_0),
+    # Q5_0: 32-row slices with a partial last down box (d = 384), two shared
+    # experts of another size, 64-row slices over several stages, the limits
+    synth.MoEShape("ragged_q5", T=3, d=384, E=5, k=3, F=96, S=1, Fs=64, wfmt=synth.WFMT_Q5_0),
+    synth.MoEShape("two_shared_q5", T=7, d=256, E=16, k=2, F=64, S=2, Fs=96,
+                   wfmt=synth.WFMT_Q5_0),
+    synth.MoEShape("multi_unit_q5", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512,
+                   wfmt=synth.WFMT_Q5_0),
+    synth.MoEShape("max_limits_q5", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32,
+                   wfmt=synth.WFMT_Q5_0),
 ]
 
 
@@ -71,7 +80,9 @@ def _check(sh, seed=0, T=None, split=False):
                                   "a3b_q4_T8_d2048_E256k8_F512_S1",
                                   "a3b_T8_d2048_E256k8_F512_S1",
                                   "a3b_q8_T1_d2048_E256k8_F512_S1",
-                                  "a3b_q8_T8_d2048_E256k8_F512_S1"])
+                                  "a3b_q8_T8_d2048_E256k8_F512_S1",
+                                  "a3b_q5_T1_d2048_E256k8_F512_S1",
+                                  "a3b_q5_T8_d2048_E256k8_F512_S1"])
 def test_decode_workloads_full_size(name):
     err = _check(W[name])
     print(f"{name}: rel L2 {err:.3e}")
@@ -87,10 +98,10 @@ def test_decode_small_shapes(sh):
     _check(sh, seed=1)
 
 
-SPLIT = SMALL[:6] + [SMALL[10], W["a3b_q4_T8_d2048_E256k8_F512_S1"]]
+SPLIT = SMALL[:6] + [SMALL[10], SMALL[-4], W["a3b_q4_T8_d2048_E256k8_F512_S1"]]
 
 
-@pytest.mark.parametrize("sh", SPLIT, ids=[s.name for s in SPLIT[:-1]] + ["a3b_q4_T8"])
+@pytest.mark.parametrize("sh", SPLIT, ids=[s.name for s in SPLIT])
 def test_decode_two_launch_path(sh):
     _check(sh, seed=5, split=True)
 
