@@ -75,10 +75,11 @@ struct RouteArgs {
 constexpr int kQuantDownBoxRows = 256;
 
 struct DecodeArgs {
-    // bf16: 2D maps over the weight stacks.  Q4_0 / Q8_0: 3D maps over the codes.
+    // bf16: 2D maps over the weight stacks.  Quantised: 3D maps over the codes.
     CUtensorMap tm_gate, tm_up, tm_down;
     CUtensorMap tm_sgate, tm_sup, tm_sdown;
-    // Q4_0 / Q8_0 only: 2D maps over the scales.
+    // Quantised only: Q4_0 / Q8_0 2D maps over the scales, Q5_0 3D maps over
+    // the 48-byte records of scales and fifth bits.
     CUtensorMap tm_gate_sc, tm_up_sc, tm_down_sc;
     CUtensorMap tm_sgate_sc, tm_sup_sc, tm_sdown_sc;
     const uint16_t* x;          // [T][d] bf16
