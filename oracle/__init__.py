@@ -119,6 +119,13 @@ def fp16_to_f64(bits: int) -> float:
 def dequant(wfmt: int, w: np.ndarray, rows: int, k: int) -> np.ndarray:
     """Rows x k matrix of a bf16 (uint16 bits), canonical-Q4_0, canonical-Q8_0
     or canonical-Q5_0 array, fp64."""
+    block_bytes = {WFMT_BF16: None, WFMT_Q4_0: 18, WFMT_Q8_0: 34, WFMT_Q5_0: 22}
+    if wfmt not in block_bytes:
+        raise ValueError(f"unknown weight format {wfmt}")
+    nb = block_bytes[wfmt]
+    need = rows * k * 2 if nb is None else rows * (k // 32) * nb
+    if (nb is not None and k % 32) or np.asarray(w).nbytes < need:
+        raise ValueError("array too small for the requested rows x k")
     out = np.empty((rows, k), dtype=np.float64)
     _L().oracle_dequant_rows(wfmt, _p(np.ascontiguousarray(w)), rows, k, _p(out))
     return out
