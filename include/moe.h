@@ -30,6 +30,11 @@
  *    routed gate/up [E][F][d], down [E][d][F];  shared gate/up [S][Fs][d],
  *    down [S][d][Fs];  out [T][d] fp32.
  *  - bf16 values are raw IEEE bfloat16 bit patterns (uint16).
+ *  - Host threads: the library keeps per-process state (each kernel's
+ *    shared-memory limit, raised once per device) and per-plan state (the
+ *    tensor-map caches, the launch count).  Calls must not run concurrently
+ *    on several host threads; serialise them.  Work from one plan must also
+ *    not overlap on the GPU (see moe_forward).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
