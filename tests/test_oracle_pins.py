@@ -46,6 +46,16 @@ def test_fp16_decode_matches_numpy_all_patterns():
     assert np.array_equal(got[~nan], ref[~nan])
 
 
+def test_golden_fixtures_match_their_encoder():
+    """The committed fixtures are exactly what make_golden.py (plain struct
+    packing of the hand-chosen codes, no oracle code) writes."""
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(GOLDEN, "make_golden.py"), "--check"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def test_q4_0_golden_blocks():
     g = json.load(open(os.path.join(GOLDEN, "q4_0_blocks.json")))
     for blk in g["blocks"]:
