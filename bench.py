@@ -287,14 +287,14 @@ def run_b200(args, sh):
         if not prefill:
             if ev_a is not None:
                 ev_a.record(stream)
-            B.moe_forward(plan, L.weights, x.data_ptr(), T, out.data_ptr(), None, st)
+            B.moe_forward(plan, L.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), None, st)
             if ev_b is not None:
                 ev_b.record(stream)
             return
-        B.moe_route(plan, L.weights, x.data_ptr(), T, out.data_ptr(), st)
+        B.moe_route(plan, L.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), st)
         if ev_a is not None:
             ev_a.record(stream)
-        B.moe_experts(plan, L.weights, x.data_ptr(), T, out.data_ptr(), st)
+        B.moe_experts(plan, L.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), st)
         if ev_b is not None:
             ev_b.record(stream)
 
@@ -306,7 +306,7 @@ def run_b200(args, sh):
         acts = []
         act_flops = []
         for i in range(n_inst):
-            B.moe_forward(plan, layers[i].weights, x.data_ptr(), T, out.data_ptr(),
+            B.moe_forward(plan, layers[i].weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(),
                           routing.struct, st)
             stream.synchronize()
             cnt = routing.counts.cpu().numpy()
@@ -390,7 +390,7 @@ def run_b200(args, sh):
         e_start.record(stream)
         for i in range(K2):
             x.copy_(x_host, non_blocking=True)
-            B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, out.data_ptr(),
+            B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(),
                           None, st)
             out_host.copy_(out, non_blocking=True)
         e_end.record(stream)
@@ -492,7 +492,7 @@ def run_sweep(args):
         plan = B.moe_plan_create(base.config(sh.T))
         routing = D.Routing(sh.T, sh.k, sh.E, dev)
         with torch.cuda.stream(stream):
-            B.moe_forward(plan, base.weights, x.data_ptr(), sh.T, out.data_ptr(), routing.struct, st)
+            B.moe_forward(plan, base.weights, x.data_ptr(), sh.T, sh.k, sh.wfmt, out.data_ptr(), routing.struct, st)
         stream.synchronize()
         act, n_act = _active_bytes(sh, routing.counts.cpu().numpy(), 0)
         act += sh.E * sh.d * 4
@@ -502,12 +502,12 @@ def run_sweep(args):
         S = n_inst * max(1, -(-64 // n_inst))
         with torch.cuda.stream(stream):
             for i in range(args.warmup):
-                B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), sh.T, out.data_ptr(), None, st)
+                B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), sh.T, sh.k, sh.wfmt, out.data_ptr(), None, st)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for i in range(S):
-                    B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), sh.T,
-                                  out.data_ptr(), None, st)
+                    B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), sh.T, sh.k,
+                                  sh.wfmt, out.data_ptr(), None, st)
             g.replay()
             stream.synchronize()
             R = max(3, min(200, -(-args.steps // S)))
@@ -558,11 +558,11 @@ def run_sweep_t(args):
         S = n_inst * 2
         with torch.cuda.stream(stream):
             for i in range(args.warmup):
-                B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, out.data_ptr(), None, st)
+                B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), None, st)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 for i in range(S):
-                    B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, out.data_ptr(),
+                    B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(),
                                   None, st)
             g.replay()
             stream.synchronize()

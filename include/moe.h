@@ -144,7 +144,11 @@ typedef struct moe_routing {
 typedef struct moe_plan_s* moe_plan_t;
 
 /* Validate `cfg`, select the device, size and allocate the plan workspace
- * for cfg->t_max tokens and resolve the driver's tensor-map encoder.  On
+ * for cfg->t_max tokens and resolve the driver's tensor-map encoder.  The
+ * pages have no counterpart to the plan itself: it owns the tables that the
+ * fused steps of the "Fused MoE Triton kernel: 5 launches instead of 24" page
+ * pass between them (routing weights, the dispatch buckets), so that the
+ * compute calls below allocate nothing.  On
  * success *out receives the plan; on failure *out is NULL and nothing is
  * left allocated.  This is the only entry point that allocates device
  * memory.  Errors: INVALID_ARG (shape limits above), UNSUPPORTED (PREFILL
@@ -153,11 +157,20 @@ typedef struct moe_plan_s* moe_plan_t;
 moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out);
 
 /* Free the plan's workspace.  The caller must make sure no work enqueued
- * with the plan is still running.  NULL is ignored. */
+ * with the plan is still running.  NULL is ignored.  (No counterpart on the
+ * pages: the pair of moe_plan_create.) */
 void moe_plan_destroy(moe_plan_t plan);
 
-/* The whole layer: route, bucket, experts, weighted combine.
+/* The whole layer: route, bucket, experts, weighted combine -- the four
+ * fused steps of the "Fused MoE Triton kernel: 5 launches instead of 24"
+ * page (list of fused steps), with the always-on shared experts of the
+ * "CUDA: fuse shared experts into MMVQ" page (section on shared experts) in
+ * the same pass.
  * x [T][d] bf16, out [T][d] fp32 (overwritten), 0 <= T <= t_max.
+ * top_k and wfmt are the call's k and weight format (moe_wfmt_t); they must
+ * equal the plan's (cfg->top_k, cfg->wfmt), else MOE_ERR_INVALID_ARG and
+ * nothing is enqueued (the plan's workspace and tensor maps are sized and
+ * built for one k and one format).
  * `routing` may be NULL; when given, the routing tables are copied to it
  * (device-to-device, on `stream`).  T = 0 enqueues nothing.
  * Launches: decode regime -- 1 cooperative kernel (router, top-k, buckets,
@@ -168,19 +181,26 @@ void moe_plan_destroy(moe_plan_t plan);
  * weighted combine).  Work enqueued with one plan must not overlap on the
  * GPU with other work of the same plan (they share the workspace). */
 moe_status_t moe_forward(moe_plan_t plan, const moe_weights_t* w,
-                         const void* x, int32_t T, float* out,
-                         moe_routing_t* routing, void* stream);
+                         const void* x, int32_t T, int32_t top_k, int32_t wfmt,
+                         float* out, moe_routing_t* routing, void* stream);
 
 /* The same layer as moe_forward in two steps, for callers that time or
  * schedule them separately.  moe_route: router, top-k, buckets and work
  * list into the plan's workspace; also zero-fills `out` (decode: 1 kernel;
- * prefill: 2, including the gather of x rows per expert).  moe_experts:
- * expert FFNs and the weighted combine into `out`, reading what moe_route
- * wrote with the same T (decode: 1 kernel; prefill: 2 GEMM kernels). */
+ * prefill: 2, including the gather of x rows per expert) -- the Triton
+ * page's fused steps one and two (routing weights, dispatch; its launch
+ * table's routing and dispatch rows).  moe_experts: expert FFNs and the
+ * weighted combine into `out`, reading what moe_route wrote with the same T
+ * (decode: 1 kernel; prefill: 2 GEMM kernels) -- the Triton page's steps
+ * three and four (parallel expert compute, weighted aggregation), shared
+ * experts in the same pass as on the MMVQ page.  top_k and wfmt as for
+ * moe_forward. */
 moe_status_t moe_route(moe_plan_t plan, const moe_weights_t* w,
-                       const void* x, int32_t T, float* out, void* stream);
+                       const void* x, int32_t T, int32_t top_k, int32_t wfmt,
+                       float* out, void* stream);
 moe_status_t moe_experts(moe_plan_t plan, const moe_weights_t* w,
-                         const void* x, int32_t T, float* out, void* stream);
+                         const void* x, int32_t T, int32_t top_k, int32_t wfmt,
+                         float* out, void* stream);
 
 /* moe_route_noalloc: moe_route for callers that cannot allocate device
  * memory (no plan needed).  The source pages have no counterpart to this
@@ -199,27 +219,49 @@ moe_status_t moe_experts(moe_plan_t plan, const moe_weights_t* w,
  * `routing` (all five required) filled as moe_routing_get would.
  * 0 <= T <= MOE_DECODE_MAX_T; a larger T returns MOE_ERR_INVALID_ARG (the
  * scratch array holds at most that many tokens).  Runs on the current
- * device.  The first call on a device resolves the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * device.  The first call in a CUDA context resolves the array's device
+ * address (cudaGetSymbolAddress) and caches it with the context's id; make
+ * that first call before any stream capture.  With CUDA's lazy module
+ * loading (the default) the first call on a device may also be the one that
+ * loads the library's module, and loading a module allocates device memory
+ * (for this array and the kernels): make a first call at start-up, outside
+ * the section that must not allocate.
  * Every call on a device shares the one array, so calls whose work overlaps
- * on the GPU race: serialise them. */
+ * on the GPU race: serialise them.  Device-side flags (an out-of-range id)
+ * are not returned by this call; they stay in the array's error word until
+ * moe_route_noalloc_status reads them. */
 moe_status_t moe_route_noalloc(const moe_config_t* cfg, const moe_weights_t* w,
                                const void* x, int32_t T, float* out,
                                moe_routing_t* routing, void* stream);
 
+/* Read and clear the error word of moe_route_noalloc on the current device
+ * (synchronises the device): OK, or DEVICE_FLAG if a router kernel of an
+ * earlier call saw an out-of-range id or an expert with more tokens than a
+ * decode pass holds.  Allocates nothing.  No counterpart on the pages. */
+moe_status_t moe_route_noalloc_status(void);
+
 /* Copy the routing tables of the last moe_route/moe_forward (T tokens) from
- * the workspace to `routing` (device pointers; NULL members skipped). */
+ * the workspace to `routing` (device pointers; NULL members skipped): the
+ * routing weights and dispatch buckets of the Triton page's fused steps one
+ * and two. */
 moe_status_t moe_routing_get(moe_plan_t plan, int32_t T, moe_routing_t* routing,
                              void* stream);
 
-/* Number of kernels the last moe_forward/moe_route/moe_experts call enqueued. */
+/* Number of kernels the last moe_forward/moe_route/moe_experts call enqueued
+ * (what the Triton page's launch-count table counts: 24 launches per layer
+ * for PyTorch, 16 for Megablocks, 5 for the fused kernel).  -1 for NULL. */
 int32_t moe_last_launch_count(moe_plan_t plan);
 
 /* Read and clear the sticky device error word (synchronises `plan`'s device).
+ * The pages have no counterpart (they describe no failure handling).
  * OK, DEVICE_FLAG (a kernel saw an out-of-range id or count) or TIMEOUT (a
  * bounded wait -- of a pipeline stage or the fused kernel's grid barrier --
  * gave up, after at most 2 s; the kernel then skipped its remaining work, so
- * that call's `out` is incomplete; the plan's barrier state is reset). */
+ * that call's `out` is incomplete).  A fused decode launch that starts while
+ * such a timeout is still unread does no work at all: it writes NaN to its
+ * `out` and the next read of this word also returns TIMEOUT (a timed-out
+ * grid barrier may have been left mid-round, and computing on it could
+ * route on stale logits).  Reading the word resets the plan's barrier. */
 moe_status_t moe_get_device_status(moe_plan_t plan);
 
 /* Failure-path check (the pages have no counterpart): make the next fused
@@ -234,11 +276,14 @@ moe_status_t moe_get_device_status(moe_plan_t plan);
 moe_status_t moe_debug_stall_barrier(moe_plan_t plan, void* stream);
 
 /* Bytes of the packed Q4_0 form of n_mats matrices of [rows][k] weights.
- * k must be a multiple of 32.  Returns INVALID_ARG otherwise. */
+ * k must be a multiple of 32.  Returns INVALID_ARG otherwise.  (The 5090
+ * page's Q4_0, measurement-setup paragraph; the sizes serve moe_q4_0_pack.) */
 moe_status_t moe_q4_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
                                    size_t* code_bytes, size_t* scale_bytes);
 
-/* Repack canonical Q4_0 blocks ([n_mats][rows][k/32] blocks of 18 bytes: a
+/* Repack canonical Q4_0 blocks (the 5090 page's Q4_0, measurement-setup
+ * paragraph; the MMVQ page's "read quantised weights once" is why the
+ * kernels read this packed form directly) ([n_mats][rows][k/32] blocks of 18 bytes: a
  * little-endian fp16 scale, then 16 bytes whose byte j holds code j in the
  * low nibble and code j+16 in the high nibble) into the kernel layout:
  *   codes  [n_mats][k/32][rows][16 bytes], the 32 codes of each block
@@ -251,7 +296,8 @@ moe_status_t moe_q4_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
 
 /* Bytes of the packed Q8_0 form of n_mats matrices of [rows][k] weights
  * (32 code bytes and one fp16 scale per block).  k must be a multiple of 32.
- * Returns INVALID_ARG otherwise. */
+ * Returns INVALID_ARG otherwise.  (q8_0 is in the 5090 page's list of the
+ * model's formats; the sizes serve moe_q8_0_pack.) */
 moe_status_t moe_q8_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
                                    size_t* code_bytes, size_t* scale_bytes);
 
@@ -273,7 +319,8 @@ moe_status_t moe_q8_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
  * (16 code bytes per block; 6 bytes of scale and fifth bits per block in
  * `scale_bytes`).  k must be a multiple of 32 and rows of 8 (every matrix of
  * a layer qualifies: d is a multiple of 128, F and Fs of 32).  Returns
- * INVALID_ARG otherwise. */
+ * INVALID_ARG otherwise.  (q5_0 is in the 5090 page's list of the model's
+ * formats; the sizes serve moe_q5_0_pack.) */
 moe_status_t moe_q5_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
                                    size_t* code_bytes, size_t* scale_bytes);
 
@@ -296,7 +343,8 @@ moe_status_t moe_q5_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
 moe_status_t moe_q5_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
                            int64_t k, void* codes, void* scales, void* stream);
 
-/* Static description of a status code (never NULL). */
+/* Static description of a status code (never NULL).  No counterpart on the
+ * pages. */
 const char* moe_status_string(moe_status_t status);
 
 #ifdef __cplusplus

@@ -83,16 +83,17 @@ def lib() -> ctypes.CDLL:
     L.moe_plan_create.restype = S
     L.moe_plan_destroy.argtypes = [P]
     L.moe_plan_destroy.restype = None
-    for name in ("moe_forward",):
-        getattr(L, name).argtypes = [P, ctypes.POINTER(moe_weights_t), P, I32, P,
-                                     ctypes.POINTER(moe_routing_t), P]
-        getattr(L, name).restype = S
+    L.moe_forward.argtypes = [P, ctypes.POINTER(moe_weights_t), P, I32, I32, I32, P,
+                              ctypes.POINTER(moe_routing_t), P]
+    L.moe_forward.restype = S
     for name in ("moe_route", "moe_experts"):
-        getattr(L, name).argtypes = [P, ctypes.POINTER(moe_weights_t), P, I32, P, P]
+        getattr(L, name).argtypes = [P, ctypes.POINTER(moe_weights_t), P, I32, I32, I32, P, P]
         getattr(L, name).restype = S
     L.moe_route_noalloc.argtypes = [ctypes.POINTER(moe_config_t), ctypes.POINTER(moe_weights_t),
                                     P, I32, P, ctypes.POINTER(moe_routing_t), P]
     L.moe_route_noalloc.restype = S
+    L.moe_route_noalloc_status.argtypes = []
+    L.moe_route_noalloc_status.restype = S
     L.moe_routing_get.argtypes = [P, I32, ctypes.POINTER(moe_routing_t), P]
     L.moe_routing_get.restype = S
     L.moe_last_launch_count.argtypes = [P]
@@ -146,19 +147,22 @@ def moe_plan_destroy(plan: int) -> None:
     lib().moe_plan_destroy(plan)
 
 
-def moe_forward(plan: int, w: moe_weights_t, x: int, T: int, out: int,
+def moe_forward(plan: int, w: moe_weights_t, x: int, T: int, top_k: int, wfmt: int, out: int,
                 routing: Optional[moe_routing_t] = None, stream: int = 0) -> None:
-    _check(lib().moe_forward(plan, ctypes.byref(w), x, T, out,
+    _check(lib().moe_forward(plan, ctypes.byref(w), x, T, top_k, wfmt, out,
                              ctypes.byref(routing) if routing is not None else None, stream),
            "moe_forward")
 
 
-def moe_route(plan: int, w: moe_weights_t, x: int, T: int, out: int, stream: int = 0) -> None:
-    _check(lib().moe_route(plan, ctypes.byref(w), x, T, out, stream), "moe_route")
+def moe_route(plan: int, w: moe_weights_t, x: int, T: int, top_k: int, wfmt: int, out: int,
+              stream: int = 0) -> None:
+    _check(lib().moe_route(plan, ctypes.byref(w), x, T, top_k, wfmt, out, stream), "moe_route")
 
 
-def moe_experts(plan: int, w: moe_weights_t, x: int, T: int, out: int, stream: int = 0) -> None:
-    _check(lib().moe_experts(plan, ctypes.byref(w), x, T, out, stream), "moe_experts")
+def moe_experts(plan: int, w: moe_weights_t, x: int, T: int, top_k: int, wfmt: int, out: int,
+                stream: int = 0) -> None:
+    _check(lib().moe_experts(plan, ctypes.byref(w), x, T, top_k, wfmt, out, stream),
+           "moe_experts")
 
 
 def moe_route_noalloc(cfg: moe_config_t, w: moe_weights_t, x: int, T: int, out: int,
@@ -166,6 +170,12 @@ def moe_route_noalloc(cfg: moe_config_t, w: moe_weights_t, x: int, T: int, out: 
     """moe_route without a plan: scratch in the library's static device array."""
     _check(lib().moe_route_noalloc(ctypes.byref(cfg), ctypes.byref(w), x, T, out,
                                    ctypes.byref(routing), stream), "moe_route_noalloc")
+
+
+def moe_route_noalloc_status() -> int:
+    """Raw status of moe_route_noalloc's sticky error word on the current
+    device (not raised)."""
+    return lib().moe_route_noalloc_status()
 
 
 def moe_routing_get(plan: int, T: int, routing: moe_routing_t, stream: int = 0) -> None:

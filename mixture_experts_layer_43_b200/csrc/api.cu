@@ -93,9 +93,12 @@ moe_status_t check_matrix(const moe_matrix_t& m, bool quant) {
     return MOE_OK;
 }
 
+// top_k and wfmt restate the plan's: a call whose k or weight format differs
+// from the plan it runs on is rejected before anything is enqueued.
 moe_status_t check_call(const moe_plan_s* p, const moe_weights_t* w, const void* x, int32_t T,
-                        const float* out) {
+                        int32_t top_k, int32_t wfmt, const float* out) {
     if (!p || !w) return MOE_ERR_INVALID_ARG;
+    if (top_k != p->cfg.top_k || wfmt != p->cfg.wfmt) return MOE_ERR_INVALID_ARG;
     if (T < 0 || T > p->cfg.t_max) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
@@ -484,9 +487,9 @@ void moe_plan_destroy(moe_plan_t p) {
     delete p;
 }
 
-moe_status_t moe_route(moe_plan_t p, const moe_weights_t* w, const void* x, int32_t T, float* out,
-                       void* stream) {
-    moe_status_t s = check_call(p, w, x, T, out);
+moe_status_t moe_route(moe_plan_t p, const moe_weights_t* w, const void* x, int32_t T,
+                       int32_t top_k, int32_t wfmt, float* out, void* stream) {
+    moe_status_t s = check_call(p, w, x, T, top_k, wfmt, out);
     if (s) return s;
     p->last_launches = 0;
     if (T == 0) return MOE_OK;
@@ -505,8 +508,8 @@ moe_status_t moe_route(moe_plan_t p, const moe_weights_t* w, const void* x, int3
 }
 
 moe_status_t moe_experts(moe_plan_t p, const moe_weights_t* w, const void* x, int32_t T,
-                         float* out, void* stream) {
-    moe_status_t s = check_call(p, w, x, T, out);
+                         int32_t top_k, int32_t wfmt, float* out, void* stream) {
+    moe_status_t s = check_call(p, w, x, T, top_k, wfmt, out);
     if (s) return s;
     p->last_launches = 0;
     if (T == 0) return MOE_OK;
@@ -524,9 +527,10 @@ moe_status_t moe_experts(moe_plan_t p, const moe_weights_t* w, const void* x, in
     return s;
 }
 
-moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const void* x, int32_t T, float* out,
-                         moe_routing_t* routing, void* stream) {
-    moe_status_t s = check_call(p, w, x, T, out);
+moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const void* x, int32_t T,
+                         int32_t top_k, int32_t wfmt, float* out, moe_routing_t* routing,
+                         void* stream) {
+    moe_status_t s = check_call(p, w, x, T, top_k, wfmt, out);
     if (s) return s;
     p->last_launches = 0;
     if (T == 0) return MOE_OK;
@@ -542,10 +546,10 @@ moe_status_t moe_forward(moe_plan_t p, const moe_weights_t* w, const void* x, in
         if (s != MOE_ERR_UNSUPPORTED) return s;
         // fall through to the two-launch path (same kernels, separate router)
     }
-    s = moe_route(p, w, x, T, out, stream);
+    s = moe_route(p, w, x, T, top_k, wfmt, out, stream);
     if (s) return s;
     const int l1 = p->last_launches;
-    s = moe_experts(p, w, x, T, out, stream);
+    s = moe_experts(p, w, x, T, top_k, wfmt, out, stream);
     if (s) return s;
     p->last_launches += l1;
     if (routing) {
@@ -571,8 +575,9 @@ moe_status_t moe_get_device_status(moe_plan_t p) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaMemcpy(&v, p->ws.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
     if (v && cudaMemset(p->ws.err, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
-    if (v & kErrTimeout) {
-        // a launch gave up waiting: leave the grid barrier words clean for the next one
+    if (v & (kErrTimeout | kErrSkipped)) {
+        // a launch gave up waiting (or skipped its work because of an earlier
+        // timeout): leave the grid barrier words clean for the next one
         if (cudaMemset(p->ws.gbar, 0, 16) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_ERR_TIMEOUT;
     }

@@ -936,6 +936,28 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int T = a.T, d = a.d, E = a.E, k = a.k, S = a.S;
     const int G = gridDim.x, b = blockIdx.x;
+
+    // A timeout of an earlier launch that the host has not yet read (and
+    // cleared, resetting the barrier) may have left the grid barrier's count
+    // short of a whole round, so that some CTAs of this launch would pass it
+    // before every CTA has written its logits.  Every CTA reads the sticky
+    // error word first; if a timeout is pending, the whole launch skips its
+    // work, writes NaN to `out` (so a caller that ignores the status cannot
+    // take the result for a valid one) and records kErrSkipped.
+    __shared__ int s_skip;
+    if (tid == 0)
+        s_skip = (*reinterpret_cast<volatile uint32_t*>(a.err) & (kErrTimeout | kErrSkipped)) != 0;
+    __syncthreads();
+    if (s_skip) {
+        float4* o = reinterpret_cast<float4*>(a.out);
+        const float qnan = __uint_as_float(0x7fc00000u);
+        const int n4 = (T * d) >> 2;
+        for (int i = b * kDecodeThreads + tid; i < n4; i += G * kDecodeThreads)
+            o[i] = make_float4(qnan, qnan, qnan, qnan);
+        if (b == 0 && tid == 0) atomicOr(a.err, kErrSkipped);
+        return;
+    }
+
     if (tid == 0) {
         for (int s = 0; s < a.n_stages; ++s) {
             mbar_init(&sm.full[s], 1);

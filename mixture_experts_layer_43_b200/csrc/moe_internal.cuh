@@ -24,6 +24,12 @@ static_assert(MOE_DECODE_MAX_T <= kDecodeTok, "decode pass holds every token");
 constexpr uint32_t kErrBadId = 1u;        // an expert id or count out of range
 constexpr uint32_t kErrTimeout = 2u;      // a bounded wait ran out
 constexpr uint32_t kErrTooManyTok = 4u;   // an expert got more tokens than a pass holds
+// A fused decode launch found kErrTimeout (or this bit) already set when it
+// started: an earlier launch's grid barrier may have been left short of a
+// whole round, so the launch did no routing or expert work and wrote NaN to
+// `out`.  Cleared with the timeout by moe_get_device_status, which also
+// resets the barrier.
+constexpr uint32_t kErrSkipped = 8u;
 
 // Bounded waits give up after this long (a healthy wait lasts microseconds).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

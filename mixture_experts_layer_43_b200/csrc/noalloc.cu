@@ -12,11 +12,16 @@
 //
 // The array is a module global: every GPU that loads the library holds its
 // own copy (kNoAllocScratchBytes) until the process exits, and every call on
-// that GPU shares it.  The ticket and error word are cleared before each
-// launch; the rest is fully rewritten by each call, so the array keeps only
-// the last call's contents.  Two calls whose work overlaps on the GPU (other
-// streams, other threads) race on the array and must be serialised by the
-// caller.
+// that GPU shares it.  The ticket is cleared before each launch; the error
+// word is sticky until moe_route_noalloc_status reads it; the rest is fully
+// rewritten by each call, so the array keeps only the last call's contents.
+// Two calls whose work overlaps on the GPU (other streams, other threads)
+// race on the array and must be serialised by the caller.
+//
+// The array's device address is resolved once per CUDA context (the first
+// call in a context, with its device current) and cached with the context's
+// id: after a cudaDeviceReset, or in another context on the same device, the
+// module global lives at a different address, and the cache is refreshed.
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -33,7 +38,8 @@ constexpr int kMaxDevices = 64;
 
 struct NoAllocDevice {
     bool ready = false;
-    uint8_t* scratch = nullptr;   // device address of g_route_scratch on that device
+    unsigned long long ctx_id = 0;  // CUDA context the address below belongs to
+    uint8_t* scratch = nullptr;     // device address of g_route_scratch in that context
     int num_sms = 0;
 };
 
@@ -51,13 +57,46 @@ constexpr size_t kOffErr = kOffTicket + 16;
 constexpr size_t kScratchUsed = kOffErr + 16;
 static_assert(kScratchUsed <= kNoAllocScratchBytes, "scratch layout exceeds the array");
 
-// First call on a device (that device current): resolve the array's device
-// address and the SM count.  Neither allocates.
+// Id of the calling thread's current CUDA context, through the driver entry
+// points (the library links no driver stub).  0 when it cannot be read.
+unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static bool resolved = false;
+    if (!resolved) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1{}, q2{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+            q1 == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) == cudaSuccess &&
+            q2 == cudaDriverEntryPointSuccess) {
+            get_current = reinterpret_cast<GetCurrent>(f1);
+            get_id = reinterpret_cast<GetId>(f2);
+        }
+        cudaGetLastError();
+        resolved = true;
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// First call in a context (its device current): resolve the array's device
+// address and the SM count.  Neither allocates.  A context id that cannot be
+// read (0) resolves the address again on every call.
 moe_status_t setup_device(int dev, NoAllocDevice** out) {
     if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(g_mu);
     NoAllocDevice& d = g_dev[dev];
-    if (!d.ready) {
+    const unsigned long long ctx = current_context_id();
+    if (!d.ready || ctx == 0 || ctx != d.ctx_id) {
+        d.ready = false;
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess || !ptr) {
             cudaGetLastError();
@@ -68,6 +107,7 @@ moe_status_t setup_device(int dev, NoAllocDevice** out) {
             return MOE_ERR_CUDA;
         d.scratch = static_cast<uint8_t*>(ptr);
         d.num_sms = sms;
+        d.ctx_id = ctx;
         d.ready = true;
     }
     *out = &d;
@@ -131,7 +171,21 @@ extern "C" moe_status_t moe_route_noalloc(const moe_config_t* cfg, const moe_wei
     while (epc < 8 && (E + epc - 1) / epc > nd->num_sms) epc *= 2;
     r.experts_per_cta = epc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the ticket and the error word must start at zero
-    if (cudaMemsetAsync(sc + kOffTicket, 0, 32, st) != cudaSuccess) return MOE_ERR_CUDA;
+    // the last-CTA ticket must start at zero (the error word stays sticky)
+    if (cudaMemsetAsync(sc + kOffTicket, 0, 16, st) != cudaSuccess) return MOE_ERR_CUDA;
     return launch_decode_route(r, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" moe_status_t moe_route_noalloc_status(void) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    NoAllocDevice* nd = nullptr;
+    moe_status_t s = setup_device(dev, &nd);
+    if (s) return s;
+    uint32_t v = 0;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(&v, nd->scratch + kOffErr, 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (v && cudaMemset(nd->scratch + kOffErr, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+    return v ? MOE_ERR_DEVICE_FLAG : MOE_OK;
 }

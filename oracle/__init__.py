@@ -56,6 +56,8 @@ def _bind(path: str):
     L.oracle_buckets.restype = I
     L.oracle_forward.argtypes = [I] * 7 + [P, I] + [P] * 8 + [P, I] + [P] * 4 + [I]
     L.oracle_forward.restype = I
+    L.oracle_forward_routed.argtypes = [I] * 7 + [P, I] + [P] * 6 + [P, I, P, P, P, I]
+    L.oracle_forward_routed.restype = I
     L.oracle_max_threads.argtypes = []
     L.oracle_max_threads.restype = I
     return L
@@ -191,6 +193,33 @@ def forward(inp, tokens: Optional[Sequence[int]] = None, n_threads: int = 0):
     if rc:
         raise ValueError(f"oracle_forward failed ({rc})")
     return out, ids, w, logits
+
+
+def forward_routed(inp, ids: np.ndarray, w: np.ndarray,
+                   tokens: Optional[Sequence[int]] = None, n_threads: int = 0) -> np.ndarray:
+    """Layer output (fp64 [n][d]) for the listed tokens (default: all) with
+    the routing given by ids (int [n][k]) and weights ([n][k]) instead of the
+    oracle's own router: steps 6-7 only."""
+    sh = inp.shape
+    T = inp.x.shape[0]
+    tok = None
+    n = T
+    if tokens is not None:
+        tok = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        n = tok.shape[0]
+    ids = np.ascontiguousarray(np.asarray(ids, dtype=np.int32).reshape(n, sh.k))
+    w = np.ascontiguousarray(np.asarray(w, dtype=np.float64).reshape(n, sh.k))
+    out = np.empty((n, sh.d), dtype=np.float64)
+    S = sh.S if inp.shared_gate is not None else 0
+    rc = _L().oracle_forward_routed(
+        sh.d, sh.E, sh.k, sh.F, S, sh.Fs if S else 0, sh.wfmt,
+        _p(np.ascontiguousarray(inp.x)), T,
+        _p(inp.gate), _p(inp.up), _p(inp.down),
+        _p(inp.shared_gate), _p(inp.shared_up), _p(inp.shared_down),
+        _p(tok), n, _p(ids), _p(w), _p(out), int(n_threads))
+    if rc:
+        raise ValueError(f"oracle_forward_routed failed ({rc})")
+    return out
 
 
 def max_threads() -> int:

@@ -317,6 +317,55 @@ int oracle_forward(int d, int E, int k, int F, int S, int Fs, int wfmt,
     return 0;
 }
 
+/* Steps 6-7 alone, for routing decided elsewhere: out_t = sum_j w_j
+ * FFN_{ids_j}(x_t) + sum_s FFN_s(x_t) for the listed tokens, with the given
+ * ids [n_tokens][k] and weights [n_tokens][k] (fp64) in place of steps 1-4.
+ * The parity tests use it to check the output of a token whose k-th and
+ * (k+1)-th logits nearly tie, where fp32 and fp64 may pick different experts:
+ * the GPU's own choice is then evaluated exactly. */
+int oracle_forward_routed(int d, int E, int k, int F, int S, int Fs, int wfmt,
+                          const uint16_t* x, int T,
+                          const void* wg, const void* wu, const void* wd,
+                          const void* sg, const void* su, const void* sd,
+                          const int32_t* tokens, int n_tokens, const int32_t* ids,
+                          const double* w, double* out, int n_threads) {
+    if (d <= 0 || E <= 0 || k <= 0 || F <= 0 || S < 0 || !x || !wg || !wu || !wd || !ids ||
+        !w || !out || n_tokens < 0)
+        return 1;
+    if (S > 0 && (Fs <= 0 || !sg || !su || !sd)) return 1;
+    if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0 &&
+        wfmt != ORACLE_WFMT_Q5_0)
+        return 1;
+    if (wfmt != ORACLE_WFMT_BF16 && (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#else
+    (void)n_threads;
+#endif
+    double* xt = (double*)malloc(sizeof(double) * (size_t)d);
+    double* y = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int n = 0; n < n_tokens; ++n) {
+        int t = tokens ? tokens[n] : n;
+        if (t < 0 || t >= T) { free(xt); free(y); return 2; }
+        x_row(x, d, t, xt);
+        double* o = out + (int64_t)n * d;
+        for (int j = 0; j < d; ++j) o[j] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int e = ids[(int64_t)n * k + j];
+            if (e < 0 || e >= E) { free(xt); free(y); return 3; }
+            expert_ffn(wfmt, d, F, wg, wu, wd, e, xt, y);
+            for (int i = 0; i < d; ++i) o[i] += w[(int64_t)n * k + j] * y[i];
+        }
+        for (int s2 = 0; s2 < S; ++s2) {
+            expert_ffn(wfmt, d, Fs, sg, su, sd, s2, xt, y);
+            for (int i = 0; i < d; ++i) o[i] += y[i];
+        }
+    }
+    free(xt);
+    free(y);
+    return 0;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -4,16 +4,21 @@ it element by element with the fp64 oracle on the same seeded inputs.
 Acceptance (the contract of the layer):
   * expert ids bit-exact, except for a token whose oracle gap between the
     k-th and (k+1)-th largest logit is below 1e-5 * |k-th logit| (a near tie
-    that fp32 and fp64 may order differently);
+    that fp32 and fp64 may order differently); there the GPU's experts must
+    still lie inside the tie band;
   * counts, offsets and the slot order bit-exact against the oracle's
     bucketing of the GPU's own ids (they are a pure function of the ids);
-  * routing weights within relative 16*sqrt(d)*2^-24: the GPU sums the d
+  * routing weights within relative 5*sqrt(d)*2^-24: the GPU sums the d
     products of a logit in fp32, whose rounding error grows like sqrt(d)*2^-24
     times the partial sums (|partial sums| <~ 1 here), and a renormalised
-    weight's relative error is the difference of two such logit errors; the
-    factor 16 is the margin (observed <= 4.2e-6 at d = 2048, bound 4.3e-5);
-  * out within relative L2 2e-3 (bf16 weights) or 5e-3 (Q4_0, Q8_0 and Q5_0 weights),
-    over all tokens whose ids matched.
+    weight's relative error is the difference of two such logit errors
+    (observed 1.6*sqrt(d)*2^-24 at d = 2048: a margin of about 3);
+  * out within relative L2 2e-3 (bf16 weights) or 5e-3 (Q4_0, Q8_0 and Q5_0
+    weights) over every token: a token whose ids differ from the oracle's
+    (a waived near tie) is compared with the oracle evaluated on the GPU's own
+    ids and weights.  Callers may add a tighter tripwire: the decode kernels
+    measure about 5e-6 in every format, so a regression of 20x fails long
+    before the contract bound would.
 """
 from __future__ import annotations
 
@@ -31,9 +36,12 @@ GAP_REL = 1e-5
 W_ABS = 1e-7
 
 
+DECODE_TRIPWIRE = 1e-4
+
+
 def w_rtol(d: int) -> float:
     """Relative tolerance of the renormalised routing weights (see above)."""
-    return 16.0 * np.sqrt(d) * 2.0 ** -24
+    return 5.0 * np.sqrt(d) * 2.0 ** -24
 
 
 def run_gpu(layer: D.DeviceLayer, x_bits: np.ndarray, T: int, regime=B.MOE_REGIME_AUTO,
@@ -51,7 +59,7 @@ def run_gpu(layer: D.DeviceLayer, x_bits: np.ndarray, T: int, regime=B.MOE_REGIM
                              device=layer.device)
         r = D.Routing(max(T, 1), sh.k, sh.E, layer.device)
         st = torch.cuda.current_stream(layer.device).cuda_stream
-        B.moe_forward(plan, layer.weights, x.data_ptr(), T, out.data_ptr(), r.struct, st)
+        B.moe_forward(plan, layer.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), r.struct, st)
         launches = B.moe_last_launch_count(plan)
         torch.cuda.synchronize(layer.device)
         status = B.moe_get_device_status(plan)
@@ -71,9 +79,9 @@ def run_gpu_split(layer: D.DeviceLayer, x_bits: np.ndarray, T: int, regime=B.MOE
         out = torch.full((T, sh.d), float("nan"), dtype=torch.float32, device=layer.device)
         r = D.Routing(T, sh.k, sh.E, layer.device)
         st = torch.cuda.current_stream(layer.device).cuda_stream
-        B.moe_route(plan, layer.weights, x.data_ptr(), T, out.data_ptr(), st)
+        B.moe_route(plan, layer.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), st)
         n1 = B.moe_last_launch_count(plan)
-        B.moe_experts(plan, layer.weights, x.data_ptr(), T, out.data_ptr(), st)
+        B.moe_experts(plan, layer.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), st)
         n2 = B.moe_last_launch_count(plan)
         B.moe_routing_get(plan, T, r.struct, st)
         torch.cuda.synchronize(layer.device)
@@ -93,8 +101,21 @@ def waived_tokens(logits: np.ndarray, k: int) -> np.ndarray:
     return gap < GAP_REL * np.abs(s[:, k - 1])
 
 
-def compare(inp: synth.MoEInputs, gpu_out, routing, oracle_res, tokens=None, tol=None):
-    """Check one GPU call against the oracle; returns the relative L2 error."""
+def check_tie_choice(logits: np.ndarray, ids, k: int):
+    """On a waived near-tie token the GPU may order the tied experts
+    differently, but every expert it picked must lie in the tie band of the
+    oracle's k-th largest logit, and the picks must be distinct."""
+    s = -np.sort(-logits)
+    kth = s[k - 1]
+    band = GAP_REL * abs(kth)
+    assert len(set(np.asarray(ids).tolist())) == k
+    assert all(logits[e] >= kth - band for e in ids), (ids, kth)
+
+
+def compare(inp: synth.MoEInputs, gpu_out, routing, oracle_res, tokens=None, tol=None,
+            tripwire=None):
+    """Check one GPU call against the oracle; returns the relative L2 error
+    over every token checked."""
     sh = inp.shape
     o_out, o_ids, o_w, o_logits = oracle_res
     ids, w, counts, offsets, slot_pair = routing
@@ -114,9 +135,17 @@ def compare(inp: synth.MoEInputs, gpu_out, routing, oracle_res, tokens=None, tol
         assert np.array_equal(counts, c)
         assert np.array_equal(offsets, o)
         assert np.array_equal(slot_pair, sp)
-    ref = o_out[ok_ids]
-    err = float(np.linalg.norm(g_out[ok_ids] - ref) / max(np.linalg.norm(ref), 1e-300))
+    ref = np.array(o_out, dtype=np.float64, copy=True)
+    flip = np.where(~ok_ids)[0]
+    if len(flip):
+        for i in flip:
+            check_tie_choice(o_logits[i], g_ids[i], sh.k)
+        ref[flip] = oracle.forward_routed(inp, g_ids[flip], g_w[flip].astype(np.float64),
+                                          tokens=tok[flip])
+    err = float(np.linalg.norm(g_out - ref) / max(np.linalg.norm(ref), 1e-300))
     lim = TOL[sh.wfmt] if tol is None else tol
     assert err <= lim, f"relative L2 error {err:.3e} > {lim:.1e}"
+    if tripwire is not None:
+        assert err <= tripwire, f"relative L2 error {err:.3e} above the regression tripwire {tripwire:.1e}"
     assert np.all(np.isfinite(gpu_out))
     return err

@@ -68,9 +68,10 @@ def test_plan_create_q4_prefill_unsupported(L):
 def test_null_arguments(L):
     assert L.moe_plan_create(None, None) == B.MOE_ERR_INVALID_ARG
     w = B.moe_weights_t()
-    assert L.moe_forward(None, ctypes.byref(w), None, 1, None, None, None) == B.MOE_ERR_INVALID_ARG
-    assert L.moe_route(None, ctypes.byref(w), None, 1, None, None) == B.MOE_ERR_INVALID_ARG
-    assert L.moe_experts(None, None, None, 1, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_forward(None, ctypes.byref(w), None, 1, 2, 0, None, None, None) == \
+        B.MOE_ERR_INVALID_ARG
+    assert L.moe_route(None, ctypes.byref(w), None, 1, 2, 0, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_experts(None, None, None, 1, 2, 0, None, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_routing_get(None, 1, None, None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_get_device_status(None) == B.MOE_ERR_INVALID_ARG
     assert L.moe_last_launch_count(None) == -1

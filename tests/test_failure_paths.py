@@ -32,9 +32,17 @@ def test_grid_barrier_timeout_is_reported_and_recovered():
         out = torch.zeros((sh.T, sh.d), device="cuda")
         st = torch.cuda.current_stream().cuda_stream
         B.moe_debug_stall_barrier(plan, st)
-        B.moe_forward(plan, layer.weights, x.data_ptr(), sh.T, out.data_ptr(), None, st)
+        B.moe_forward(plan, layer.weights, x.data_ptr(), sh.T, sh.k, sh.wfmt, out.data_ptr(), None, st)
         assert B.moe_last_launch_count(plan) == 1
         torch.cuda.synchronize()                       # the launch ends by itself
+        # a second call before the status is read must not compute on the
+        # barrier the timeout left mid-round: it skips its work and its out
+        # is NaN, never a plausible wrong value
+        out2 = torch.zeros((sh.T, sh.d), device="cuda")
+        B.moe_forward(plan, layer.weights, x.data_ptr(), sh.T, sh.k, sh.wfmt, out2.data_ptr(),
+                      None, st)
+        torch.cuda.synchronize()
+        assert torch.all(torch.isnan(out2))
         assert B.moe_get_device_status(plan) == B.MOE_ERR_TIMEOUT
         assert B.moe_get_device_status(plan) == B.MOE_OK   # read-and-clear
         # the context and the plan are usable again: full parity on the next call

@@ -42,6 +42,12 @@ MUTANTS = {
                         "for (int64_t p = n - 1; p >= 0; --p) {\n            int e = ids[p];"),
     "softmax_temperature": ("p[e] = exp(l[e] - mx); z += p[e];",
                             "p[e] = exp(0.5 * (l[e] - mx)); z += p[e];"),
+    "routed_weight_ignored": ("o[i] += w[(int64_t)n * k + j] * y[i];", "o[i] += y[i];"),
+    "routed_shared_dropped": (
+        "expert_ffn(wfmt, d, Fs, sg, su, sd, s2, xt, y);\n"
+        "            for (int i = 0; i < d; ++i) o[i] += y[i];",
+        "expert_ffn(wfmt, d, Fs, sg, su, sd, s2, xt, y);\n"
+        "            for (int i = 0; i < d; ++i) o[i] += 0.0 * y[i];"),
 }
 
 
@@ -59,6 +65,7 @@ def _pins():
     yield lambda: pins.test_k_equals_E_is_dense_softmax_mixture(synth.WFMT_BF16)
     yield lambda: pins.test_single_expert_is_plain_swiglu()
     yield lambda: pins.test_shared_only_when_routed_down_is_zero()
+    yield lambda: pins.test_forward_routed_is_weighted_sum_of_ffns(synth.WFMT_BF16)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -384,6 +384,35 @@ def test_single_expert_is_plain_swiglu():
     np.testing.assert_allclose(out, _np_ffn(G, U, D, x), rtol=1e-12, atol=1e-14)
 
 
+@pytest.mark.parametrize("wfmt", [synth.WFMT_BF16, synth.WFMT_Q4_0])
+def test_forward_routed_is_weighted_sum_of_ffns(wfmt):
+    """Steps 6-7 with routing given from outside: arbitrary ids (repeats and
+    any order allowed by the definition) and weights, plus the shared
+    experts, against numpy float64 matmuls."""
+    sh = synth.MoEShape("routed", T=4, d=64, E=5, k=3, F=32, S=1, Fs=32, wfmt=wfmt,
+                        w_std=0.2, q4_scale_std=0.02)
+    inp = synth.make_inputs(sh, seed=8)
+    ids = np.array([[4, 0, 2], [1, 1, 3], [2, 4, 0], [3, 0, 1]], dtype=np.int32)
+    w = np.array([[0.5, 0.25, 0.25], [0.125, 0.375, 0.5], [1.0, 0.0, 0.0],
+                  [0.3, 0.3, 0.4]])
+    x = _x64(inp)
+    G = _f64_stack(inp.gate, wfmt, sh.F, sh.d)
+    U = _f64_stack(inp.up, wfmt, sh.F, sh.d)
+    D = _f64_stack(inp.down, wfmt, sh.d, sh.F)
+    want = _np_ffn(_f64_stack(inp.shared_gate, wfmt, sh.Fs, sh.d)[0],
+                   _f64_stack(inp.shared_up, wfmt, sh.Fs, sh.d)[0],
+                   _f64_stack(inp.shared_down, wfmt, sh.d, sh.Fs)[0], x)
+    for t in range(sh.T):
+        for j in range(sh.k):
+            e = ids[t, j]
+            want[t] += w[t, j] * _np_ffn(G[e], U[e], D[e], x[t:t + 1])[0]
+    got = oracle.forward_routed(inp, ids, w)
+    np.testing.assert_allclose(got, want, rtol=1e-11, atol=1e-13)
+    # a subset of tokens, in any order
+    sub = oracle.forward_routed(inp, ids[[3, 1]], w[[3, 1]], tokens=[3, 1])
+    np.testing.assert_allclose(sub, want[[3, 1]], rtol=1e-11, atol=1e-13)
+
+
 def test_shared_only_when_routed_down_is_zero():
     sh = synth.MoEShape("sh", T=3, d=32, E=5, k=2, F=16, S=2, Fs=8, w_std=0.3)
     inp = synth.make_inputs(sh, seed=6)

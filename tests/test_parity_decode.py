@@ -11,7 +11,7 @@ from mixture_experts_layer_43_b200 import binding as B
 from mixture_experts_layer_43_b200 import device as D
 from mixture_experts_layer_43_b200 import synth
 
-from gpu_util import compare, run_gpu, run_gpu_split
+from gpu_util import DECODE_TRIPWIRE, compare, run_gpu, run_gpu_split
 
 pytestmark = pytest.mark.gpu
 
@@ -72,7 +72,7 @@ def _check(sh, seed=0, T=None, split=False):
     sub = synth.MoEInputs(sh, inp.x[:T], inp.router_w, inp.router_b, inp.gate, inp.up,
                           inp.down, inp.shared_gate, inp.shared_up, inp.shared_down)
     res = oracle.forward(sub)
-    return compare(sub, out, routing, res)
+    return compare(sub, out, routing, res, tripwire=DECODE_TRIPWIRE)
 
 
 @pytest.mark.parametrize("name", ["tiny_T4_d256_E8k2_F512", "a3b_T1_d2048_E256k8_F512_S1",
@@ -119,7 +119,7 @@ def test_decode_T0_enqueues_nothing():
     try:
         out = torch.full((1, sh.d), 7.0, device="cuda")
         x = D.upload_x(inp.x, "cuda")
-        B.moe_forward(plan, layer.weights, x.data_ptr(), 0, out.data_ptr())
+        B.moe_forward(plan, layer.weights, x.data_ptr(), 0, sh.k, sh.wfmt, out.data_ptr())
         assert B.moe_last_launch_count(plan) == 0
         torch.cuda.synchronize()
         assert torch.all(out == 7.0)
@@ -153,14 +153,24 @@ def test_decode_invalid_call_enqueues_nothing():
         x = D.upload_x(inp.x, "cuda")
         out = torch.zeros((2, sh.d), device="cuda")
         with pytest.raises(B.MoeError) as e:
-            B.moe_forward(plan, layer.weights, x.data_ptr(), 3, out.data_ptr())   # T > t_max
+            B.moe_forward(plan, layer.weights, x.data_ptr(), 3, sh.k, sh.wfmt, out.data_ptr())  # T > t_max
         assert e.value.status == B.MOE_ERR_INVALID_ARG
         with pytest.raises(B.MoeError):
-            B.moe_forward(plan, layer.weights, x.data_ptr() + 2, 2, out.data_ptr())  # misaligned
+            B.moe_forward(plan, layer.weights, x.data_ptr() + 2, 2, sh.k, sh.wfmt,
+                          out.data_ptr())                                  # misaligned
         w = B.moe_weights_t()
         w.router_w = layer.weights.router_w
         with pytest.raises(B.MoeError):
-            B.moe_forward(plan, w, x.data_ptr(), 2, out.data_ptr())          # missing weights
+            B.moe_forward(plan, w, x.data_ptr(), 2, sh.k, sh.wfmt, out.data_ptr())  # missing weights
+        # k and the weight format restate the plan's: a mismatch is rejected
+        for k, wfmt in ((sh.k + 1, sh.wfmt), (sh.k - 1, sh.wfmt), (sh.k, B.MOE_WFMT_Q4_0),
+                        (sh.k, 7)):
+            for call in (B.moe_forward, B.moe_route, B.moe_experts):
+                with pytest.raises(B.MoeError) as e:
+                    call(plan, layer.weights, x.data_ptr(), 2, k, wfmt, out.data_ptr())
+                assert e.value.status == B.MOE_ERR_INVALID_ARG
+        torch.cuda.synchronize()
+        assert torch.all(out == 0.0)                                      # nothing ran
         assert B.moe_get_device_status(plan) == B.MOE_OK
     finally:
         B.moe_plan_destroy(plan)
