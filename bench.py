@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -241,119 +242,145 @@ def run_reference(args, sh):
     return 0
 
 
-def run_b200(args, sh):
-    import torch
-    from mixture_experts_layer_43_b200 import binding as B
-    from mixture_experts_layer_43_b200 import device as D
+# Every seeded workload of the layer measured by the default run, under the
+# same protocol (CUDA-graph replays, cold weights, events on the launching
+# stream): the decode layers of the Mixtral-8x7B and 35B-A3B shapes (bf16
+# and Q4_0, T = 1 and 8), the tiny parity layer, and the DeepSeek-MoE-16B
+# prefill layer.  The first is the headline line's workload.
+ALL_WORKLOADS = ("mixtral_T8_d4096_E8k2_F14336", "tiny_T4_d256_E8k2_F512",
+                 "a3b_T1_d2048_E256k8_F512_S1", "a3b_q4_T1_d2048_E256k8_F512_S1",
+                 "a3b_q4_T8_d2048_E256k8_F512_S1", "deepseek_T4096_d2048_E64k6_F1408_S2")
+MIN_TIMED_MS = 150.0      # per-workload entries time at least this long (clock samples)
 
-    ws, rank, local = _dist()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = _peaks()
 
-    # layer instances: distinct device copies, enough of them that the
-    # weights one step reads are cold in L2 (>= 4x L2 over the rotation)
-    base = synth.make_inputs(sh, seed=args.seed)
-    layers = [D.DeviceLayer(base, device=str(dev))]
-    E_act = sh.E * (1.0 - (1.0 - sh.k / sh.E) ** sh.T)
-    active_est = (E_act * synth.weight_bytes_per_expert(sh) + sh.S * (
-        synth.weight_bytes_per_expert(sh, sh.Fs) if sh.S else 0) + sh.E * sh.d * 4)
-    per_inst = layers[0].weight_bytes() + sh.E * sh.d * 4
-    n_inst = args.instances or int(min(128, max(1, -(-4 * L2_BYTES // int(active_est)))))
-    n_inst = max(1, min(n_inst, int(60e9 // per_inst)))
-    for _ in range(1, n_inst):
-        layers.append(layers[0].clone())
-    torch.cuda.synchronize(dev)
-    T = sh.T
-    x = D.upload_x(base.x, dev)
-    out = torch.empty((T, sh.d), dtype=torch.float32, device=dev)
-    stream = torch.cuda.Stream(device=dev)
-    st = stream.cuda_stream
-    plan = B.moe_plan_create(layers[0].config(T))
-    routing = D.Routing(T, sh.k, sh.E, dev)
+class _Setup:
+    """A workload resident on the device: layer instances, x, out, plan."""
 
-    prefill = T > B.MOE_DECODE_MAX_T and sh.wfmt == synth.WFMT_BF16
+    def __init__(self, sh, args, dev, stream, host_inputs):
+        import torch
+        from mixture_experts_layer_43_b200 import binding as B
+        from mixture_experts_layer_43_b200 import device as D
+        self.sh, self.dev, self.stream = sh, dev, stream
+        if host_inputs:
+            self.base = synth.make_inputs(sh, seed=args.seed)
+            first = D.DeviceLayer(self.base, device=str(dev))
+            x_bits = self.base.x
+        else:
+            self.base = None
+            first = D.random_layer(sh, seed=args.seed, device=str(dev))
+            x_bits = synth.make_inputs(sh, seed=args.seed, x_only=True).x
+        self.x_bits = x_bits
+        E_act = sh.E * (1.0 - (1.0 - sh.k / sh.E) ** sh.T)
+        active_est = (E_act * synth.weight_bytes_per_expert(sh) + sh.S * (
+            synth.weight_bytes_per_expert(sh, sh.Fs) if sh.S else 0) + sh.E * sh.d * 4)
+        self.per_inst = first.weight_bytes() + sh.E * sh.d * 4
+        # distinct device copies, enough that the weights one step reads are
+        # cold in L2 (>= 4x L2 over the rotation)
+        n_inst = args.instances or int(min(128, max(1, -(-4 * L2_BYTES // int(active_est)))))
+        self.n_inst = max(1, min(n_inst, int(40e9 // self.per_inst)))
+        self.layers = [first] + [first.clone() for _ in range(1, self.n_inst)]
+        torch.cuda.synchronize(dev)
+        self.x = D.upload_x(x_bits, dev)
+        self.out = torch.empty((sh.T, sh.d), dtype=torch.float32, device=dev)
+        self.plan = B.moe_plan_create(first.config(sh.T))
+        self.routing = D.Routing(sh.T, sh.k, sh.E, dev)
+        self.prefill = sh.T > B.MOE_DECODE_MAX_T and sh.wfmt == synth.WFMT_BF16
 
-    def step(i, ev_a=None, ev_b=None):
+    def step(self, i, ev_a=None, ev_b=None):
         """One layer call.  Decode: moe_forward (the single fused launch),
         events around it.  Prefill: router + scatter, then events around the
         two GEMM launches."""
-        L = layers[i % n_inst]
-        if not prefill:
+        from mixture_experts_layer_43_b200 import binding as B
+        sh, L, st = self.sh, self.layers[i % self.n_inst], self.stream.cuda_stream
+        xp, op = self.x.data_ptr(), self.out.data_ptr()
+        if not self.prefill:
             if ev_a is not None:
-                ev_a.record(stream)
-            B.moe_forward(plan, L.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), None, st)
+                ev_a.record(self.stream)
+            B.moe_forward(self.plan, L.weights, xp, sh.T, sh.k, sh.wfmt, op, None, st)
             if ev_b is not None:
-                ev_b.record(stream)
+                ev_b.record(self.stream)
             return
-        B.moe_route(plan, L.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), st)
+        B.moe_route(self.plan, L.weights, xp, sh.T, sh.k, sh.wfmt, op, st)
         if ev_a is not None:
-            ev_a.record(stream)
-        B.moe_experts(plan, L.weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(), st)
+            ev_a.record(self.stream)
+        B.moe_experts(self.plan, L.weights, xp, sh.T, sh.k, sh.wfmt, op, st)
         if ev_b is not None:
-            ev_b.record(stream)
+            ev_b.record(self.stream)
 
+    def destroy(self):
+        from mixture_experts_layer_43_b200 import binding as B
+        B.moe_plan_destroy(self.plan)
+        self.layers = []
+
+
+def _measure(su: "_Setup", args, uuid, exact_steps=None, min_ms=0.0, ws=1):
+    """Time one workload.  exact_steps: time exactly that many steps (the
+    headline line); else at least --steps steps and at least min_ms.
+    Returns the measurement as a dict (max over ranks where it matters)."""
+    import torch
+    from mixture_experts_layer_43_b200 import binding as B
+    sh, dev, stream = su.sh, su.dev, su.stream
+    T, st = sh.T, stream.cuda_stream
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            step(i)
-        # algorithmic bytes: from each instance's own routing on this x
-        act_bytes = []
-        acts = []
-        act_flops = []
-        for i in range(n_inst):
-            B.moe_forward(plan, layers[i].weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(),
-                          routing.struct, st)
+            su.step(i)
+        # algorithmic bytes and FLOPs: from each instance's own routing on this x
+        act_bytes, acts, act_flops = [], [], []
+        for i in range(su.n_inst):
+            B.moe_forward(su.plan, su.layers[i].weights, su.x.data_ptr(), T, sh.k, sh.wfmt,
+                          su.out.data_ptr(), su.routing.struct, st)
             stream.synchronize()
-            cnt = routing.counts.cpu().numpy()
-            b, a = _active_bytes(sh, cnt, layers[i].n_shared)
+            cnt = su.routing.counts.cpu().numpy()
+            b, a = _active_bytes(sh, cnt, su.layers[i].n_shared)
             act_bytes.append(b)
             acts.append(a)
-            act_flops.append(_expert_flops(sh, cnt, layers[i].n_shared))
-        launches_per_step = B.moe_last_launch_count(plan)
-        status = B.moe_get_device_status(plan)
+            act_flops.append(_expert_flops(sh, cnt, su.layers[i].n_shared))
+        launches_per_step = B.moe_last_launch_count(su.plan)
+        status = B.moe_get_device_status(su.plan)
         if status != B.MOE_OK:
-            raise RuntimeError("device status after warm-up: " + B.moe_status_string(status))
+            raise RuntimeError(f"{sh.name}: device status after warm-up: "
+                               + B.moe_status_string(status))
 
         # The timed loop replays a CUDA graph of S whole steps (router +
         # experts per step, cycling the instances), so host launch overhead
-        # cannot starve the GPU: R full replays and one graph of the
-        # remaining K - R*S steps time exactly K = --steps steps.  A second
-        # graph of S steps carries an event node on each side of every
-        # experts launch, for that kernel's own duration.
-        S = n_inst * max(1, -(-32 // n_inst))
-        K = max(1, args.steps)
-        R, rem = divmod(K, S)
+        # cannot starve the GPU.  A second graph of S steps carries an event
+        # node on each side of every experts launch, for that kernel's own
+        # duration.
+        S = su.n_inst * max(1, -(-32 // su.n_inst))
         g_steps = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_steps, stream=stream):
             for i in range(S):
-                step(i)
-        g_rem = None
-        if rem:
-            g_rem = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_rem, stream=stream):
-                for i in range(rem):
-                    step(i)
+                su.step(i)
         ev_a = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(S)]
         ev_b = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(S)]
         g_kern = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g_kern, stream=stream):
             for i in range(S):
-                step(i, ev_a[i], ev_b[i])
+                su.step(i, ev_a[i], ev_b[i])
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
         for _ in range(2):
             g_steps.replay()
             g_kern.replay()
-            if g_rem is not None:
-                g_rem.replay()
+        t0.record(stream)
+        g_steps.replay()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        est_ms = max(t0.elapsed_time(t1) / S, 1e-4)
+        if exact_steps is not None:
+            K = exact_steps
+        else:
+            K = max(args.steps, int(math.ceil(min_ms / est_ms)))
+        R, rem = divmod(K, S)
+        g_rem = None
+        if rem:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem, stream=stream):
+                for i in range(rem):
+                    su.step(i)
+            g_rem.replay()
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        if uuid and not uuid.startswith("GPU-"):
-            uuid = "GPU-" + uuid
         if ws > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize(dev)
@@ -374,14 +401,15 @@ def run_b200(args, sh):
             torch.distributed.barrier()
         clocks = clk.summary()
         total_ms = t_start.elapsed_time(t_end)
-        launches = launches_per_step * K
-        status = B.moe_get_device_status(plan)
+        status = B.moe_get_device_status(su.plan)
         if status != B.MOE_OK:
-            raise RuntimeError("device status after timing: " + B.moe_status_string(status))
+            raise RuntimeError(f"{sh.name}: device status after timing: "
+                               + B.moe_status_string(status))
         del g_steps, g_kern, g_rem
 
-        # e2e: pinned host x in, pinned host out back, every step
-        x_host = torch.from_numpy(base.x.view(np.int16)).pin_memory()
+        # e2e: pinned host x in, pinned host out back, every step, through
+        # the public moe_forward call
+        x_host = torch.from_numpy(su.x_bits.view(np.int16)).pin_memory()
         out_host = torch.empty((T, sh.d), dtype=torch.float32).pin_memory()
         e_start = torch.cuda.Event(enable_timing=True)
         e_end = torch.cuda.Event(enable_timing=True)
@@ -389,26 +417,35 @@ def run_b200(args, sh):
         torch.cuda.synchronize(dev)
         e_start.record(stream)
         for i in range(K2):
-            x.copy_(x_host, non_blocking=True)
-            B.moe_forward(plan, layers[i % n_inst].weights, x.data_ptr(), T, sh.k, sh.wfmt, out.data_ptr(),
-                          None, st)
-            out_host.copy_(out, non_blocking=True)
+            su.x.copy_(x_host, non_blocking=True)
+            B.moe_forward(su.plan, su.layers[i % su.n_inst].weights, su.x.data_ptr(), T, sh.k,
+                          sh.wfmt, su.out.data_ptr(), None, st)
+            out_host.copy_(su.out, non_blocking=True)
         e_end.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = e_start.elapsed_time(e_end)
 
     t_max, e2e_max = reduce_max_over_ranks([total_ms, e2e_ms], device=dev)
-    B.moe_plan_destroy(plan)
+    return {"K": K, "K2": K2, "S": S, "t_max": t_max, "e2e_max": e2e_max, "kern_ms": kern_ms,
+            "launches": launches_per_step * K, "launches_per_step": launches_per_step,
+            "act_bytes": act_bytes, "acts": acts, "act_flops": act_flops, "clocks": clocks}
 
-    tokens_per_s = job_tokens_per_s(ws, T, K, t_max)
-    kern_evt_s = float(np.mean(kern_ms)) / 1e3
+
+def _entry(su: "_Setup", m: dict, ws: int, peaks):
+    """The JSON fields of one measured workload."""
+    from mixture_experts_layer_43_b200 import binding as B  # noqa: F401
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = peaks
+    sh, K, n_inst = su.sh, m["K"], su.n_inst
+    T = sh.T
+    tokens_per_s = job_tokens_per_s(ws, T, K, m["t_max"])
+    kern_evt_s = float(np.mean(m["kern_ms"])) / 1e3
     # A decode step is exactly one launch (the fused kernel), so its duration
     # is the graph step time (event nodes around such short kernels add
     # their own overhead); prefill: event nodes around the two GEMM launches.
-    kern_avg_s = kern_evt_s if prefill else min(kern_evt_s, total_ms / K / 1e3)
-    alg_bytes = float(np.mean([act_bytes[i % n_inst] for i in range(K)]))
-    alg_flops = float(np.mean([act_flops[i % n_inst] for i in range(K)]))
-    if prefill:
+    kern_avg_s = kern_evt_s if su.prefill else min(kern_evt_s, m["t_max"] / K / 1e3)
+    alg_bytes = float(np.mean([m["act_bytes"][i % n_inst] for i in range(K)]))
+    alg_flops = float(np.mean([m["act_flops"][i % n_inst] for i in range(K)]))
+    if su.prefill:
         src_sha = _kernel_src_sha(["prefill.cu", "moe_internal.cuh"])
         achieved = alg_flops / kern_avg_s / 1e12
         roof = {"bound": "tensor", "kernel": "prefill_gemm_kernel (gate/up + down launches)",
@@ -420,7 +457,7 @@ def run_b200(args, sh):
                 "frac_of_burst_peak": achieved / bf16_tf,
                 "peak_source": (f"{peak_src} (MEASURED_PEAKS.json bf16_tflops_sustained; "
                                 "the GEMMs run inside a seconds-long loop)")}
-        l2 = (f"inputs larger than L2: each step reads {per_inst / 1e9:.2f} GB of expert "
+        l2 = (f"inputs larger than L2: each step reads {su.per_inst / 1e9:.2f} GB of expert "
               f"weights and {T * sh.d * 2 / 1e6:.1f} MB of x; {n_inst} instance(s)")
     else:
         src_sha = _kernel_src_sha(["decode.cu", "moe_internal.cuh"])
@@ -437,28 +474,93 @@ def run_b200(args, sh):
         l2 = ("inputs larger than L2: each step streams "
               f"{alg_bytes / 1e9:.3f} GB of distinct expert weights; "
               f"{n_inst} layer instance(s) rotated")
-    line = {
-        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": ws,
-        "steps": K, "steps_requested": args.steps, "warmup": args.warmup,
-        "ms_per_step": t_max / K,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": {synth.WFMT_BF16: "bf16", synth.WFMT_Q4_0: "q4_0/bf16",
-                  synth.WFMT_Q8_0: "q8_0/bf16", synth.WFMT_Q5_0: "q5_0/bf16"}[sh.wfmt],
-        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x; no trained weights)",
+    return {
+        "value": tokens_per_s, "unit": "tokens/s", "steps": K, "ms_per_step": m["t_max"] / K,
+        "dtype": _dtype(sh),
         "config": {"workload": sh.name, "shape": synth.describe(sh), "T": T,
-                   "instances": n_inst, "graph_steps": S,
+                   "instances": n_inst, "graph_steps": m["S"],
                    "timing": ("CUDA-graph replays of whole steps; kernel time from event "
                               "nodes in a second graph around each moe_forward (decode: the "
                               "single fused kernel) or moe_experts (prefill: the two GEMMs)"),
                    "l2": l2,
-                   "active_experts_per_step": float(np.mean(acts)),
-                   "parallelism": f"replicas x{ws}" if ws > 1 else "single GPU"},
+                   "active_experts_per_step": float(np.mean(m["acts"])),
+                   "weights": ("host-generated by synth" if su.base is not None else
+                               "drawn on the device with the workload's distributions")},
         "roofline": roof,
-        "e2e": {"value": job_tokens_per_s(ws, T, K2, e2e_max), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(ws, T, m["K2"], m["e2e_max"]), "unit": "tokens/s",
                 "h2d_bytes_per_step": T * sh.d * 2, "d2h_bytes_per_step": T * sh.d * 4},
-        "gpu_launches": launches,
-        "clocks": clocks,
+        "gpu_launches": m["launches"],
+        "clocks": m["clocks"],
     }
+
+
+def _dtype(sh):
+    return {synth.WFMT_BF16: "bf16", synth.WFMT_Q4_0: "q4_0/bf16",
+            synth.WFMT_Q8_0: "q8_0/bf16", synth.WFMT_Q5_0: "q5_0/bf16"}[sh.wfmt]
+
+
+def run_b200(args, sh):
+    import torch
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks = _peaks()
+    stream = torch.cuda.Stream(device=dev)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    if uuid and not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+
+    # the headline workload: exactly --steps timed steps
+    su = _Setup(sh, args, dev, stream, host_inputs=True)
+    m = _measure(su, args, uuid, exact_steps=max(1, args.steps), ws=ws)
+    head = _entry(su, m, ws, peaks)
+    base = su.base
+    su.destroy()
+    del su
+    torch.cuda.empty_cache()
+
+    # the other seeded workloads, each its own entry
+    configs = {}
+    if not args.only_workload:
+        for name in ALL_WORKLOADS:
+            if name == sh.name:
+                continue
+            wsh = synth.WORKLOADS[name]
+            small = wsh.name.startswith("tiny")
+            su = _Setup(wsh, args, dev, stream, host_inputs=small)
+            mm = _measure(su, args, uuid, min_ms=MIN_TIMED_MS, ws=ws)
+            configs[name] = _entry(su, mm, ws, peaks)
+            su.destroy()
+            del su
+            torch.cuda.empty_cache()
+
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": ws,
+        "steps": head["steps"], "steps_requested": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": head["dtype"],
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) x; no trained weights)",
+        "config": dict(head["config"],
+                       parallelism=f"replicas x{ws}" if ws > 1 else "single GPU"),
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+    }
+    if configs:
+        configs[sh.name] = {k: head[k] for k in head}
+        line["configs"] = configs
+        line["configs_note"] = (
+            "one entry per seeded workload, keyed by workload name, each timed with the same "
+            f"protocol; entries other than the headline time max(--steps, {MIN_TIMED_MS:.0f} ms "
+            "worth of) steps so the clock sampler sees the timed region")
     if ws == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = _cpu_baseline(base, sh)
     if rank == 0:
@@ -594,6 +696,8 @@ def main(argv=None):
     ap.add_argument("--instances", type=int, default=0)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-workload", action="store_true",
+                    help="measure only --workload (no per-workload `configs` entries)")
     ap.add_argument("--sweep-bytes", action="store_true",
                     help="bandwidth vs bytes per launch of the decode kernel, one JSON line per point")
     ap.add_argument("--sweep-t", action="store_true",

@@ -239,6 +239,9 @@ struct DecodeCfg {
     static_assert(KSPLIT >= 1 && ROLES * KSPLIT == kConsumerWarps, "warp roles");
     static constexpr bool QUANT = WF != kWfBf16;
     static_assert(!QUANT || FS >= 32, "quantised slices hold whole blocks");
+    // fp16 tensor-core operands (see q4h_lo): x staged as fp16, h as an fp16
+    // hi + lo pair, per-block corrections with two code bases
+    static constexpr bool F16 = WF == kWfQ4;
     static constexpr int CB = WF == kWfQ8 ? 32 : 16;   // code bytes of one block row
     // + its fp16 scale (Q5_0: + its 32-bit word of fifth bits; scale and word
     // sit in 48-byte records of 8 rows, see q5_aux)
@@ -270,6 +273,20 @@ struct alignas(16) DecodeSmemTail {
 __device__ __forceinline__ uint32_t q4_raw(uint32_t w, int s) {
     return ((w >> s) & 0x000F000Fu) | 0x43004300u;
 }
+
+// The fp16 form of the same operands, one LOP3 per register (Q4_0).  In an
+// fp16 value whose exponent makes the unit in the last place 1 (base 1024,
+// 0x6400), a code in mantissa bits 0-3 reads as 1024 + q; with base 64
+// (0x5400, ulp 1/16) a code in bits 4-7 reads as 64 + q.  Both are exact.
+// So the word's codes in bits 0-3 / 16-19 (k pair 2t, 2t+1 of the first
+// 16-wide half) and 4-7 / 20-23 (k pair 2t+8, 2t+9) need no shift; one
+// shift by 8 brings the second half's codes to the same places.  Within a
+// block, k % 16 < 8 has base 1024 and k % 16 >= 8 base 64, and the block's
+// accumulator starts at -sum((base_k + 8) x_k), so that the block adds
+// sum((q - 8) x) before its scale.
+__device__ __forceinline__ uint32_t q4h_lo(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
+__device__ __forceinline__ uint32_t q4h_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x54005400u; }
+constexpr float kF16BaseLo = 1024.f, kF16BaseHi = 64.f;
 
 // One quantised block (32 weights along k) of rows r and r+8 of an mma A
 // tile, times the B fragment of the same 32 k (b0 b1: k 0-15, b2 b3: k
@@ -462,6 +479,35 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
 template <int WF>
 __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& sm, int tid) {
     const int nkb = a.d / 32;
+    if constexpr (WF == kWfQ4) {
+        // fp16 copy of x (exact for |x| >= 2^-17; below, off by at most 2^-25)
+        // and each block's accumulator start -sum((base_k + 8) x_k), base_k
+        // 1024 for k % 16 < 8 and 64 otherwise (see q4h_lo)
+        for (int idx = tid; idx < a.T * nkb; idx += kConsumers) {
+            const int t = idx / nkb, kb = idx % nkb;
+            const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + kb * 32);
+            uint4* dst = reinterpret_cast<uint4*>(sm.xs + t * a.xs_stride + kb * 64);
+            float s_lo = 0.f, s_hi = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = __ldg(src + c);
+                const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+                uint32_t h[4];
+                float s = 0.f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float lo = __uint_as_float(q[j] << 16), hi = __uint_as_float(q[j] & 0xffff0000u);
+                    s += lo + hi;
+                    __half2 hv = __floats2half2_rn(lo, hi);
+                    h[j] = *reinterpret_cast<uint32_t*>(&hv);
+                }
+                dst[c] = make_uint4(h[0], h[1], h[2], h[3]);
+                if (c & 1) s_hi += s; else s_lo += s;      // elements 8c .. 8c+7
+            }
+            sm.xsum[t * nkb + kb] = -((kF16BaseLo + 8.f) * s_lo + (kF16BaseHi + 8.f) * s_hi);
+        }
+        return;
+    }
     for (int idx = tid; idx < a.T * nkb; idx += kConsumers) {
         const int t = idx / nkb, kb = idx % nkb;
         const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + kb * 32);
@@ -701,6 +747,28 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                     const int r0 = rg * 16 + g;
                     const float* xsum0 = sm.xsum + tok0 * nkb + kb0;
                     const float* xsum1 = sm.xsum + tok1 * nkb + kb0;
+                    if constexpr (C::F16) {
+                        // fp16 operands: one chain per block from its correction
+#pragma unroll 4
+                        for (int bb = ks; bb < nkb_st; bb += C::KSPLIT) {
+                            const uint32_t* row = codes + (bb * FS + r0) * 4;
+                            const uint32_t w0 = row[tig], w8 = row[32 + tig];
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4(xrow + ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
+                            const float c0 = xsum0[bb], c1 = xsum1[bb];
+                            float v[4];
+                            mma_f16_16816(v, q4h_lo(w0), q4h_lo(w8), q4h_hi(w0), q4h_hi(w8), b0, b1,
+                                          c0, c1, c0, c1);
+                            const uint32_t u0 = w0 >> 8, u8 = w8 >> 8;
+                            mma_f16_16816_acc(v, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8), b2, b3);
+                            const float s0 = __half2float(scl[bb * FS + r0]);
+                            const float s8 = __half2float(scl[bb * FS + r0 + 8]);
+                            cacc[0] = fmaf(s0, v[0], cacc[0]);
+                            cacc[1] = fmaf(s0, v[1], cacc[1]);
+                            cacc[2] = fmaf(s8, v[2], cacc[2]);
+                            cacc[3] = fmaf(s8, v[3], cacc[3]);
+                        }
+                    } else {
 #pragma unroll 2
                     for (int bb = ks; bb < nkb_st; bb += C::KSPLIT) {
                         const uint32_t* row = codes + (bb * FS + r0) * (C::CB / 4);
@@ -730,6 +798,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                             cacc[3] = fmaf(s8, v[3], cacc[3]);
                         }
                     }
+                    }
                 }
             }
             __syncwarp();
@@ -758,6 +827,20 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                 uv += gu[((q * 2 + 1) * kDecodeTok + t) * C::GS + f];
             }
             const float h = gv / (1.f + expf(-gv)) * uv;
+            if constexpr (C::F16) {
+                // fp16 pair hi + lo; the down block's accumulator starts at
+                // -sum((base_f + 8)(hi + lo)) (bases as in q4h_lo)
+                const __half hi = __float2half_rn(h);
+                const __half lo = __float2half_rn(h - __half2float(hi));
+                reinterpret_cast<__half*>(hhi)[t * C::HS + f] = hi;
+                reinterpret_cast<__half*>(hlo)[t * C::HS + f] = lo;
+                const float base = (f & 15) < 8 ? kF16BaseLo : kF16BaseHi;
+                float hs = (base + 8.f) * (__half2float(hi) + __half2float(lo));
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
+                if (lane == 0) sm.hsum[t * 2 + f / 32] = -hs;
+                continue;
+            }
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             hhi[t * C::HS + f] = hi;
@@ -813,6 +896,31 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);   // [NB][128][CB]
                         const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * QB * C::CB);
                         const int rib = (rgb % (QB / 16)) * 16 + g;
+                        if constexpr (C::F16) {
+#pragma unroll
+                            for (int bb = 0; bb < C::NB; ++bb) {
+                                const uint32_t* row = codes + (bb * QB + rib) * 4;
+                                const uint32_t w0 = row[tig], w8 = row[32 + tig];
+                                const uint32_t u0 = w0 >> 8, u8 = w8 >> 8;
+                                const uint32_t p0 = q4h_lo(w0), q0 = q4h_lo(w8);
+                                const uint32_t p1 = q4h_hi(w0), q1 = q4h_hi(w8);
+                                const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
+                                const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
+                                float v[4];
+                                // one chain from the block's correction: hi then lo parts of h
+                                mma_f16_16816(v, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
+                                              hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
+                                mma_f16_16816_acc(v, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
+                                mma_f16_16816_acc(v, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                                mma_f16_16816_acc(v, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                                const float s0 = __half2float(scl[bb * QB + rib]);
+                                const float s8 = __half2float(scl[bb * QB + rib + 8]);
+                                c[0] = fmaf(s0, v[0], c[0]);
+                                c[1] = fmaf(s0, v[1], c[1]);
+                                c[2] = fmaf(s8, v[2], c[2]);
+                                c[3] = fmaf(s8, v[3], c[3]);
+                            }
+                        } else {
 #pragma unroll
                         for (int bb = 0; bb < C::NB; ++bb) {
                             const uint32_t* row = codes + (bb * QB + rib) * (C::CB / 4);
@@ -839,6 +947,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                                 c[2] = fmaf(s8, v[2], c[2]);
                                 c[3] = fmaf(s8, v[3], c[3]);
                             }
+                        }
                         }
                     }
                     const int j = j0 + rgb * 16 + g;
@@ -902,7 +1011,8 @@ struct alignas(16) FusedRouteSmem {
     float sel[kDecodeTok][kMaxTopK];
     uint32_t emask[kMaxExperts / 32];   // bit e: expert e was selected by some token
     int n_routed;
-    int pad[3];
+    int skip;                           // this launch does no work (see decode_fused_kernel)
+    int pad[2];
 };
 
 size_t decode_fused_extra_smem() { return sizeof(FusedRouteSmem); }
@@ -944,11 +1054,13 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
     // error word first; if a timeout is pending, the whole launch skips its
     // work, writes NaN to `out` (so a caller that ignores the status cannot
     // take the result for a valid one) and records kErrSkipped.
-    __shared__ int s_skip;
+    // (The flag lives in the dynamic shared memory: a static __shared__
+    // variable would add a 1 KB block, the dynamic block's alignment, on top
+    // of a launch sized to the opt-in limit.)
     if (tid == 0)
-        s_skip = (*reinterpret_cast<volatile uint32_t*>(a.err) & (kErrTimeout | kErrSkipped)) != 0;
+        rs->skip = (*reinterpret_cast<volatile uint32_t*>(a.err) & (kErrTimeout | kErrSkipped)) != 0;
     __syncthreads();
-    if (s_skip) {
+    if (rs->skip) {
         float4* o = reinterpret_cast<float4*>(a.out);
         const float qnan = __uint_as_float(0x7fc00000u);
         const int n4 = (T * d) >> 2;

@@ -141,6 +141,85 @@ def random_bf16_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") 
     return L, inp.x
 
 
+def random_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") -> DeviceLayer:
+    """A layer of any weight format whose router and x come from synth (the
+    same routing as make_inputs with this seed) and whose expert weights are
+    drawn on the device from a seeded generator with the workload's
+    distributions -- bf16 N(0, w_std); Q4_0 / Q8_0 / Q5_0 canonical blocks
+    with codes uniform on their range and scales |N(0, std)| as fp16, then
+    repacked by the library's own packer.  For timing, where the weight
+    values do not matter and host generation would dominate."""
+    if shape.wfmt == synth.WFMT_BF16:
+        return random_bf16_layer(shape, seed, device)[0]
+    inp = synth.make_inputs(shape, seed=seed, x_only=True)
+    dev = torch.device(device)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    packed_bytes, pack, std = {
+        synth.WFMT_Q4_0: (B.moe_q4_0_packed_bytes, B.moe_q4_0_pack, shape.q4_scale_std),
+        synth.WFMT_Q8_0: (B.moe_q8_0_packed_bytes, B.moe_q8_0_pack, shape.q8_scale_std),
+        synth.WFMT_Q5_0: (B.moe_q5_0_packed_bytes, B.moe_q5_0_pack, shape.q5_scale_std)}[shape.wfmt]
+    st = torch.cuda.current_stream(dev)
+
+    def blocks(n_rows: int, k: int) -> torch.Tensor:
+        nb = k // 32
+        sc = (torch.randn((n_rows, nb), generator=gen, device=dev) * std).abs().half()
+        sc = sc.view(torch.uint8).reshape(n_rows, nb, 2)
+        if shape.wfmt == synth.WFMT_Q8_0:
+            q = torch.randint(0, 256, (n_rows, nb, 32), generator=gen, device=dev,
+                              dtype=torch.int32).to(torch.uint8)
+            return torch.cat([sc, q], dim=2)
+        if shape.wfmt == synth.WFMT_Q4_0:
+            q = torch.randint(0, 16, (n_rows, nb, 32), generator=gen, device=dev,
+                              dtype=torch.int32)
+            qs = (q[:, :, :16] | (q[:, :, 16:] << 4)).to(torch.uint8)
+            return torch.cat([sc, qs], dim=2)
+        q = torch.randint(0, 32, (n_rows, nb, 32), generator=gen, device=dev, dtype=torch.int64)
+        bit = torch.arange(32, device=dev, dtype=torch.int64)
+        qh = ((q >> 4) << bit).sum(dim=2)                               # fifth bits, bit j
+        qh = torch.stack([(qh >> (8 * i)) & 255 for i in range(4)], dim=2).to(torch.uint8)
+        lo = q & 15
+        qs = (lo[:, :, :16] | (lo[:, :, 16:] << 4)).to(torch.uint8)
+        return torch.cat([sc, qh, qs], dim=2)
+
+    L = DeviceLayer.__new__(DeviceLayer)
+    L.shape, L.device, L.q4 = shape, dev, True
+    L.router_w = _dev(inp.router_w.astype(np.float32), dev)
+    L.router_b = None if inp.router_b is None else _dev(inp.router_b.astype(np.float32), dev)
+    L._keep = []
+
+    def mat(n_mats, rows, k):
+        cb, sb = packed_bytes(n_mats, rows, k)
+        codes = torch.empty(cb, dtype=torch.uint8, device=dev)
+        scales = torch.empty(sb // 2, dtype=torch.int16, device=dev)
+        step = max(1, (1 << 26) // (rows * k))                  # bound the temporaries
+        per_c, per_s = cb // n_mats, sb // n_mats
+        for m0 in range(0, n_mats, step):
+            m1 = min(n_mats, m0 + step)
+            canon = blocks((m1 - m0) * rows, k)
+            pack(canon.data_ptr(), m1 - m0, rows, k, codes.data_ptr() + m0 * per_c,
+                 scales.data_ptr() + m0 * per_s, st.cuda_stream)
+            st.synchronize()
+        L._keep += [codes, scales]
+        return B.moe_matrix_t(codes.data_ptr(), scales.data_ptr())
+
+    E, F, d, S, Fs = shape.E, shape.F, shape.d, shape.S, shape.Fs
+    w = B.moe_weights_t()
+    w.router_w = L.router_w.data_ptr()
+    w.router_b = L.router_b.data_ptr() if L.router_b is not None else None
+    w.gate = mat(E, F, d)
+    w.up = mat(E, F, d)
+    w.down = mat(E, d, F)
+    L.n_shared = 0
+    if S:
+        w.shared_gate = mat(S, Fs, d)
+        w.shared_up = mat(S, Fs, d)
+        w.shared_down = mat(S, d, Fs)
+        L.n_shared = S
+    L.weights = w
+    return L
+
+
 def upload_x(x_bits: np.ndarray, device) -> torch.Tensor:
     return _dev(x_bits, torch.device(device))
 
