@@ -25,6 +25,12 @@ Storage conventions (the C ABI's, see include/moe.h):
   Q5_0      [rows][K/32][22] = fp16 scale + 32-bit little-endian word of
             fifth bits (bit j for element j) + 16 bytes of low nibbles
             packed as in Q4_0.
+  q6_K      [rows][K/256][210] super-blocks of 256 weights = ql[128] (low 4
+            bits) + qh[64] (high 2 bits) + 16 signed 8-bit sub-block scales
+            + fp16 super-block scale; element i of a super-block takes its
+            low bits from the low (quarter c = (i%128)/32 < 2) or high nibble
+            of ql[64*(i//128) + 32*(c%2) + i%32] and its high bits from bits
+            2c, 2c+1 of qh[32*(i//128) + i%32]; weight d*sc[i//16]*(q-32).
 """
 from __future__ import annotations
 
@@ -38,10 +44,13 @@ WFMT_BF16 = 0
 WFMT_Q4_0 = 1
 WFMT_Q8_0 = 2
 WFMT_Q5_0 = 3
+WFMT_Q6_K = 4
 Q4_BLOCK = 32          # weights per Q4_0 block
 Q4_BLOCK_BYTES = 18    # 2-byte fp16 scale + 16 bytes of 4-bit codes
 Q8_BLOCK_BYTES = 34    # 2-byte fp16 scale + 32 signed 8-bit codes
 Q5_BLOCK_BYTES = 22    # 2-byte fp16 scale + 4 bytes of fifth bits + 16 bytes of nibbles
+Q6_SUPER = 256         # weights per q6_K super-block
+Q6_SUPER_BYTES = 210   # 128 + 64 code bytes, 16 sub-block scales, 2-byte fp16 scale
 
 
 @dataclasses.dataclass(frozen=True)
@@ -62,6 +71,7 @@ class MoEShape:
     q4_scale_std: float = 0.005
     q8_scale_std: float = 0.00035
     q5_scale_std: float = 0.0025
+    q6_scale_std: float = 1.5e-5     # super-block scale; sub-scales uniform on -128..127
 
     def replace(self, **kw) -> "MoEShape":
         return dataclasses.replace(self, **kw)
@@ -97,6 +107,13 @@ WORKLOADS = {
     "a3b_q5_T8_d2048_E256k8_F512_S1": MoEShape(
         "a3b_q5_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512,
         S=1, Fs=512, wfmt=WFMT_Q5_0),
+    # ... and with q6_K weights (also in the model's mix; 256-weight super-blocks)
+    "a3b_q6_T1_d2048_E256k8_F512_S1": MoEShape(
+        "a3b_q6_T1_d2048_E256k8_F512_S1", T=1, d=2048, E=256, k=8, F=512,
+        S=1, Fs=512, wfmt=WFMT_Q6_K),
+    "a3b_q6_T8_d2048_E256k8_F512_S1": MoEShape(
+        "a3b_q6_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512,
+        S=1, Fs=512, wfmt=WFMT_Q6_K),
     # the same 35B-A3B layer in bf16 at T = 8 (about 58 distinct experts, 0.37 GB)
     "a3b_T8_d2048_E256k8_F512_S1": MoEShape(
         "a3b_T8_d2048_E256k8_F512_S1", T=8, d=2048, E=256, k=8, F=512, S=1, Fs=512),
@@ -202,6 +219,37 @@ def q5_0_blocks(rng: np.random.Generator, rows: int, k: int,
     return out
 
 
+def q6_k_blocks(rng: np.random.Generator, rows: int, k: int,
+                scale_std: float) -> np.ndarray:
+    """Canonical q6_K super-blocks [rows][k/256][210] with codes uniform on
+    0..63, sub-block scales uniform on -128..127 and super-block scales
+    |N(0, scale_std)| stored as fp16."""
+    assert k % Q6_SUPER == 0
+    nb = k // Q6_SUPER
+    out = np.empty((rows, nb, Q6_SUPER_BYTES), dtype=np.uint8)
+    step = max(1, (1 << 20) // max(1, nb))
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        n = r1 - r0
+        q = rng.integers(0, 64, size=(n, nb, Q6_SUPER), dtype=np.uint8)
+        sc = rng.integers(-128, 128, size=(n, nb, 16), dtype=np.int16).astype(np.int8)
+        d = np.abs(rng.standard_normal((n, nb), dtype=np.float32)
+                   * np.float32(scale_std)).astype(np.float16)
+        # element i = 128 h + 32 c + l
+        qq = q.reshape(n, nb, 2, 4, 32)                         # [h][c][l]
+        low, high = qq & 15, qq >> 4
+        ql = np.empty((n, nb, 2, 2, 32), dtype=np.uint8)        # [h][c % 2][l]
+        ql[:, :, :, 0] = low[:, :, :, 0] | (low[:, :, :, 2] << 4)
+        ql[:, :, :, 1] = low[:, :, :, 1] | (low[:, :, :, 3] << 4)
+        qh = (high[:, :, :, 0] | (high[:, :, :, 1] << 2) | (high[:, :, :, 2] << 4)
+              | (high[:, :, :, 3] << 6))                        # [h][l]
+        out[r0:r1, :, 0:128] = ql.reshape(n, nb, 128)
+        out[r0:r1, :, 128:192] = qh.reshape(n, nb, 64)
+        out[r0:r1, :, 192:208] = sc.view(np.uint8)
+        out[r0:r1, :, 208:210] = d.view(np.uint8).reshape(n, nb, 2)
+    return out
+
+
 @dataclasses.dataclass
 class MoEInputs:
     shape: MoEShape
@@ -243,13 +291,14 @@ def make_inputs(shape: MoEShape, seed: int = 0,
         else:
             sg = su = sd = None
     else:
-        blocks, q, nbytes = {
-            WFMT_Q4_0: (q4_0_blocks, sh.q4_scale_std, Q4_BLOCK_BYTES),
-            WFMT_Q8_0: (q8_0_blocks, sh.q8_scale_std, Q8_BLOCK_BYTES),
-            WFMT_Q5_0: (q5_0_blocks, sh.q5_scale_std, Q5_BLOCK_BYTES)}[sh.wfmt]
+        blocks, q, nbytes, per = {
+            WFMT_Q4_0: (q4_0_blocks, sh.q4_scale_std, Q4_BLOCK_BYTES, Q4_BLOCK),
+            WFMT_Q8_0: (q8_0_blocks, sh.q8_scale_std, Q8_BLOCK_BYTES, Q4_BLOCK),
+            WFMT_Q5_0: (q5_0_blocks, sh.q5_scale_std, Q5_BLOCK_BYTES, Q4_BLOCK),
+            WFMT_Q6_K: (q6_k_blocks, sh.q6_scale_std, Q6_SUPER_BYTES, Q6_SUPER)}[sh.wfmt]
 
         def stack(i, mats, rows, kk):
-            return blocks(rng(i), mats * rows, kk, q).reshape(mats, rows, kk // 32, nbytes)
+            return blocks(rng(i), mats * rows, kk, q).reshape(mats, rows, kk // per, nbytes)
         g = stack(3, sh.E, sh.F, sh.d)
         u = stack(4, sh.E, sh.F, sh.d)
         dn = stack(5, sh.E, sh.d, sh.F)
@@ -272,6 +321,8 @@ def weight_bytes_per_expert(shape: MoEShape, hidden: Optional[int] = None) -> in
         return n // 32 * 18   # 16 code bytes + 2 scale bytes per 32 weights
     if shape.wfmt == WFMT_Q5_0:
         return n // 32 * 22   # 16 nibble bytes + 4 fifth-bit bytes + 2 scale bytes
+    if shape.wfmt == WFMT_Q6_K:
+        return n // 256 * 210  # 192 code bytes + 16 sub-scales + 2 scale bytes
     return n // 32 * 34       # 32 code bytes + 2 scale bytes per 32 weights
 
 
@@ -282,7 +333,7 @@ def expert_flops(shape: MoEShape, n_tokens: int, hidden: Optional[int] = None) -
 
 def describe(shape: MoEShape) -> str:
     fmt = {WFMT_BF16: "bf16", WFMT_Q4_0: "q4_0", WFMT_Q8_0: "q8_0",
-           WFMT_Q5_0: "q5_0"}[shape.wfmt]
+           WFMT_Q5_0: "q5_0", WFMT_Q6_K: "q6_k"}[shape.wfmt]
     s = (f"T={shape.T} d={shape.d} E={shape.E} k={shape.k} F={shape.F} "
          f"S={shape.S} Fs={shape.Fs} {fmt}")
     if shape.zipf_bias:

@@ -25,6 +25,7 @@ WFMT_BF16 = 0
 WFMT_Q4_0 = 1
 WFMT_Q8_0 = 2
 WFMT_Q5_0 = 3
+WFMT_Q6_K = 4
 
 
 def build(force: bool = False) -> str:
@@ -119,14 +120,16 @@ def fp16_to_f64(bits: int) -> float:
 
 
 def dequant(wfmt: int, w: np.ndarray, rows: int, k: int) -> np.ndarray:
-    """Rows x k matrix of a bf16 (uint16 bits), canonical-Q4_0, canonical-Q8_0
-    or canonical-Q5_0 array, fp64."""
-    block_bytes = {WFMT_BF16: None, WFMT_Q4_0: 18, WFMT_Q8_0: 34, WFMT_Q5_0: 22}
-    if wfmt not in block_bytes:
+    """Rows x k matrix of a bf16 (uint16 bits), canonical-Q4_0, canonical-Q8_0,
+    canonical-Q5_0 or canonical-q6_K array, fp64."""
+    # (bytes per block, weights per block)
+    blocks = {WFMT_BF16: None, WFMT_Q4_0: (18, 32), WFMT_Q8_0: (34, 32), WFMT_Q5_0: (22, 32),
+              WFMT_Q6_K: (210, 256)}
+    if wfmt not in blocks:
         raise ValueError(f"unknown weight format {wfmt}")
-    nb = block_bytes[wfmt]
-    need = rows * k * 2 if nb is None else rows * (k // 32) * nb
-    if (nb is not None and k % 32) or np.asarray(w).nbytes < need:
+    nb = blocks[wfmt]
+    need = rows * k * 2 if nb is None else rows * (k // nb[1]) * nb[0]
+    if (nb is not None and k % nb[1]) or np.asarray(w).nbytes < need:
         raise ValueError("array too small for the requested rows x k")
     out = np.empty((rows, k), dtype=np.float64)
     _L().oracle_dequant_rows(wfmt, _p(np.ascontiguousarray(w)), rows, k, _p(out))

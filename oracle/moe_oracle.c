@@ -37,8 +37,10 @@
  * formats of the model it measures), and Q5_0 blocks as w = d * (q - 16) from
  * the canonical 22-byte blocks (fp16 scale d, a little-endian 32-bit word qh
  * of fifth bits, then 16 bytes of low nibbles as in Q4_0; element j takes
- * bit j of qh as its fifth bit; q5_0 is in the same list of formats).  Every
- * dequantised value is exact in double precision.
+ * bit j of qh as its fifth bit; q5_0 is in the same list of formats), and
+ * q6_K super-blocks as w = d * sc * (q - 32) from the canonical 210-byte
+ * super-blocks of 256 weights (see q6_k_row; q6_K is in the same list).
+ * Every dequantised value is exact in double precision.
  *
  * Layouts (row-major, reduction dimension contiguous):
  *   x [T][d] bf16 bits; Wr [E][d] fp32; b [E] fp32 or NULL
@@ -46,6 +48,7 @@
  *   Q4_0: a row of K weights is K/32 blocks of 18 bytes.
  *   Q8_0: a row of K weights is K/32 blocks of 34 bytes.
  *   Q5_0: a row of K weights is K/32 blocks of 22 bytes.
+ *   q6_K: a row of K weights is K/256 super-blocks of 210 bytes.
  *
  * The pages print no worked example for the layer output, so the tests pin
  * every function here against what the mathematics fixes instead: brute-force
@@ -65,6 +68,7 @@
 #define ORACLE_WFMT_Q4_0 1
 #define ORACLE_WFMT_Q8_0 2
 #define ORACLE_WFMT_Q5_0 3
+#define ORACLE_WFMT_Q6_K 4
 
 /* bfloat16 is the top half of an IEEE binary32. */
 double oracle_bf16_to_f64(uint16_t b) {
@@ -134,6 +138,37 @@ static void q5_0_row(const uint8_t* blocks, int64_t K, double* out) {
     }
 }
 
+/* Dequantise one row of K weights stored as canonical q6_K super-blocks (K a
+ * multiple of 256; 210 bytes per 256 weights: ql[128] low 4 bits, qh[64]
+ * high 2 bits, 16 signed 8-bit sub-block scales, then a little-endian fp16
+ * super-block scale d; the 5090 page names q6_K among the formats of the
+ * model it measures and prints no layout -- this is the reading taken).
+ * Element i of a super-block: h = i / 128 (which half), r = i % 128,
+ * c = r / 32 (which quarter of the half), l = r % 32.  Its low 4 bits are
+ * the low nibble (c = 0, 1) or the high nibble (c = 2, 3) of byte
+ * ql[64 h + l] (c even) or ql[64 h + 32 + l] (c odd); its high 2 bits are
+ * bits 2c, 2c+1 of qh[32 h + l]; its sub-block is i / 16.
+ * weight = d * sc[i / 16] * (q - 32), q = low + 16 * high in 0..63. */
+static void q6_k_row(const uint8_t* blocks, int64_t K, double* out) {
+    for (int64_t b = 0; b < K / 256; ++b) {
+        const uint8_t* blk = blocks + b * 210;
+        const uint8_t* ql = blk;
+        const uint8_t* qh = blk + 128;
+        const uint8_t* sc = blk + 192;
+        uint16_t hd = (uint16_t)(blk[208] | (blk[209] << 8));
+        double dsc = oracle_fp16_to_f64(hd);
+        for (int i = 0; i < 256; ++i) {
+            int h = i / 128, r = i % 128, c = r / 32, l = r % 32;
+            int byte = ql[64 * h + ((c & 1) ? 32 : 0) + l];
+            int low = (c >= 2) ? (byte >> 4) : (byte & 0x0f);
+            int high = (qh[32 * h + l] >> (2 * c)) & 3;
+            int q = low | (high << 4);
+            int s8 = sc[i / 16] < 128 ? (int)sc[i / 16] : (int)sc[i / 16] - 256;  /* two's complement */
+            out[b * 256 + i] = dsc * (double)s8 * (double)(q - 32);
+        }
+    }
+}
+
 /* Row r of matrix m (0-based) of a stack of matrices [M][rows][K]. */
 static void load_row(int wfmt, const void* base, int64_t m, int64_t rows,
                      int64_t K, int64_t r, double* out) {
@@ -147,9 +182,12 @@ static void load_row(int wfmt, const void* base, int64_t m, int64_t rows,
     } else if (wfmt == ORACLE_WFMT_Q8_0) {
         const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 34;
         q8_0_row(p, K, out);
-    } else {
+    } else if (wfmt == ORACLE_WFMT_Q5_0) {
         const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 22;
         q5_0_row(p, K, out);
+    } else {
+        const uint8_t* p = (const uint8_t*)base + row * (K / 256) * 210;
+        q6_k_row(p, K, out);
     }
 }
 
@@ -283,9 +321,10 @@ int oracle_forward(int d, int E, int k, int F, int S, int Fs, int wfmt,
         return 1;
     if (S > 0 && (Fs <= 0 || !sg || !su || !sd)) return 1;
     if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0 &&
-        wfmt != ORACLE_WFMT_Q5_0)
+        wfmt != ORACLE_WFMT_Q5_0 && wfmt != ORACLE_WFMT_Q6_K)
         return 1;
     if (wfmt != ORACLE_WFMT_BF16 && (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
+    if (wfmt == ORACLE_WFMT_Q6_K && (d % 256 || F % 256 || (S > 0 && Fs % 256))) return 1;
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);
 #else
@@ -334,9 +373,10 @@ int oracle_forward_routed(int d, int E, int k, int F, int S, int Fs, int wfmt,
         return 1;
     if (S > 0 && (Fs <= 0 || !sg || !su || !sd)) return 1;
     if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0 &&
-        wfmt != ORACLE_WFMT_Q5_0)
+        wfmt != ORACLE_WFMT_Q5_0 && wfmt != ORACLE_WFMT_Q6_K)
         return 1;
     if (wfmt != ORACLE_WFMT_BF16 && (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
+    if (wfmt == ORACLE_WFMT_Q6_K && (d % 256 || F % 256 || (S > 0 && Fs % 256))) return 1;
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);
 #else

@@ -16,6 +16,11 @@ but print no layout; the canonical llama.cpp blocks are the reading taken):
   Q5_0  2-byte scale, a little-endian 32-bit word whose bit j is the fifth
         bit of element j, then 16 bytes of low nibbles as in Q4_0;
         weight d*(q-16).
+  q6_K  super-blocks of 256 weights in 210 bytes: ql[128], qh[64], 16
+        signed 8-bit sub-block scales, then the 2-byte fp16 scale d.  Element
+        i = 128 h + 32 c + l takes its low 4 bits from the low (c < 2) or high
+        (c >= 2) nibble of ql[64 h + 32 (c % 2) + l] and its high 2 bits from
+        bits 2c, 2c+1 of qh[32 h + l]; weight d * sc[i // 16] * (q - 32).
 """
 from __future__ import annotations
 
@@ -109,8 +114,51 @@ def pack_q5_0(scale_bits: int, codes) -> bytes:
 
 PACK = {"q4_0": pack_q4_0, "q8_0": pack_q8_0, "q5_0": pack_q5_0}
 
+ABOUT["q6_k"] = (
+    "Hand-built canonical q6_K super-blocks. The 'MoE on RTX 5090 reaches 41% of bandwidth' "
+    "page names q6_K among the quantisation formats of the 35B-A3B model it measures "
+    "(measurement-setup paragraph) but prints no layout; our reading is the canonical "
+    "llama.cpp super-block of 256 weights in 210 bytes: ql[128] (low 4 bits), qh[64] (high 2 "
+    "bits), 16 signed 8-bit sub-block scales, then a little-endian fp16 super-block scale d. "
+    "Element i = 128h + 32c + l takes its low 4 bits from the low (c < 2) or high (c >= 2) "
+    "nibble of ql[64h + 32(c%2) + l] and its high 2 bits from bits 2c, 2c+1 of qh[32h + l]; "
+    "weight = d * sc[i/16] * (q - 32). Each entry lists the 210 bytes and, separately, the "
+    "256 codes, the 16 sub-scales and the scale bits they were built from.")
+
+# (name, fp16 scale bits, 16 sub-scales, 256 codes)
+SPECS_Q6K = [
+    ("ramp 0..63 four times, sub-scales 1..16, scale 1", 0x3C00, list(range(1, 17)),
+     [i % 64 for i in range(256)]),
+    ("codes 0 / 63 alternating, sub-scales -128 / 127 alternating, scale 0.5", 0x3800,
+     [-128, 127] * 8, [0, 63] * 128),
+    ("smallest subnormal scale, all codes 63, sub-scales -1", 0x0001, [-1] * 16, [63] * 256),
+    ("largest normal scale 65504, code 63 at element 0 and 0 at element 255, 32 elsewhere, "
+     "sub-scales 1", 0x7BFF, [1] * 16, [63] + [32] * 254 + [0]),
+    ("scrambled codes (37 i mod 64), sub-scales j - 8, scale -0.25", 0xB400,
+     [j - 8 for j in range(16)], [(37 * i) % 64 for i in range(256)]),
+]
+
+
+def pack_q6_k(scale_bits: int, sub_scales, codes) -> bytes:
+    assert len(codes) == 256 and all(0 <= q < 64 for q in codes)
+    assert len(sub_scales) == 16 and all(-128 <= s < 128 for s in sub_scales)
+    ql = [0] * 128
+    qh = [0] * 64
+    for i, q in enumerate(codes):
+        h, r = divmod(i, 128)
+        c, l = divmod(r, 32)
+        j = 64 * h + 32 * (c % 2) + l
+        ql[j] |= (q & 15) << (4 if c >= 2 else 0)
+        qh[32 * h + l] |= (q >> 4) << (2 * c)
+    return bytes(ql) + bytes(qh) + struct.pack("<16b", *sub_scales) + struct.pack("<H", scale_bits)
+
 
 def fixture(fmt: str) -> dict:
+    if fmt == "q6_k":
+        blocks = [{"name": name, "bytes": list(pack_q6_k(sb, scs, codes)), "scale_bits": sb,
+                   "sub_scales": list(scs), "codes": list(codes)}
+                  for name, sb, scs, codes in SPECS_Q6K]
+        return {"about": ABOUT[fmt], "blocks": blocks}
     blocks = [{"name": name, "bytes": list(PACK[fmt](sb, codes)), "scale_bits": sb,
                "codes": list(codes)} for name, sb, codes in SPECS[fmt]]
     return {"about": ABOUT[fmt], "blocks": blocks}
@@ -123,7 +171,7 @@ def text(fmt: str) -> str:
 def main(argv) -> int:
     check = "--check" in argv
     bad = 0
-    for fmt in SPECS:
+    for fmt in list(SPECS) + ["q6_k"]:
         path = os.path.join(HERE, f"{fmt}_blocks.json")
         want = text(fmt)
         if check:

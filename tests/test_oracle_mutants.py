@@ -42,6 +42,16 @@ MUTANTS = {
                         "for (int64_t p = n - 1; p >= 0; --p) {\n            int e = ids[p];"),
     "softmax_temperature": ("p[e] = exp(l[e] - mx); z += p[e];",
                             "p[e] = exp(0.5 * (l[e] - mx)); z += p[e];"),
+    "q6_nibble_halves_swapped": ("int low = (c >= 2) ? (byte >> 4) : (byte & 0x0f);",
+                                 "int low = (c >= 2) ? (byte & 0x0f) : (byte >> 4);"),
+    "q6_high_bits_shift": ("int high = (qh[32 * h + l] >> (2 * c)) & 3;",
+                           "int high = (qh[32 * h + l] >> c) & 3;"),
+    "q6_offset_31": ("out[b * 256 + i] = dsc * (double)s8 * (double)(q - 32);",
+                     "out[b * 256 + i] = dsc * (double)s8 * (double)(q - 31);"),
+    "q6_sub_scales_unsigned": ("int s8 = sc[i / 16] < 128 ? (int)sc[i / 16] : (int)sc[i / 16] - 256;",
+                               "int s8 = (int)sc[i / 16];"),
+    "q6_sub_scale_index": ("int s8 = sc[i / 16] < 128", "int s8 = sc[i / 32] < 128"),
+    "q6_odd_quarter_offset": ("ql[64 * h + ((c & 1) ? 32 : 0) + l]", "ql[64 * h + ((c & 1) ? 16 : 0) + l]"),
     "routed_weight_ignored": ("o[i] += w[(int64_t)n * k + j] * y[i];", "o[i] += y[i];"),
     "routed_shared_dropped": (
         "expert_ffn(wfmt, d, Fs, sg, su, sd, s2, xt, y);\n"
@@ -55,6 +65,7 @@ def _pins():
     yield lambda: pins.test_q4_0_golden_blocks()
     yield lambda: pins.test_q8_0_golden_blocks()
     yield lambda: pins.test_q5_0_golden_blocks()
+    yield lambda: pins.test_q6_k_golden_blocks()
     yield lambda: pins.test_fp16_decode_matches_numpy_all_patterns()
     yield lambda: pins.test_softmax_renormalisation_closed_form()
     yield lambda: pins.test_swiglu_closed_form()

@@ -148,6 +148,55 @@ def test_q5_0_rows_are_independent_blocks():
 
 
 # ------------------------------------------------- pure-Python brute force
+def test_q6_k_golden_blocks():
+    g = json.load(open(os.path.join(GOLDEN, "q6_k_blocks.json")))
+    for blk in g["blocks"]:
+        raw = np.array(blk["bytes"], dtype=np.uint8)
+        got = oracle.dequant(oracle.WFMT_Q6_K, raw, 1, 256)[0]
+        scale = float(np.array([blk["scale_bits"]], np.uint16).view(np.float16)[0])
+        want = np.array([scale * blk["sub_scales"][i // 16] * (q - 32)
+                         for i, q in enumerate(blk["codes"])], dtype=np.float64)
+        assert np.array_equal(got, want), blk["name"]
+
+
+def _q6_codes(raw):
+    """The 256 codes and 16 sub-scales of one canonical q6_K super-block,
+    decoded with Python's struct and integer operations, element by element
+    from the layout statement: element i = 128 h + 32 c + l."""
+    ql, qh = raw[:128], raw[128:192]
+    subs = struct.unpack("<16b", raw[192:208])
+    codes = []
+    for i in range(256):
+        h, r = divmod(i, 128)
+        c, l = divmod(r, 32)
+        byte = ql[64 * h + 32 * (c % 2) + l]
+        low = (byte >> 4) if c >= 2 else (byte & 15)
+        high = (qh[32 * h + l] >> (2 * c)) & 3
+        codes.append(low + 16 * high)
+    return codes, subs
+
+
+def test_q6_k_rows_are_independent_blocks():
+    """A multi-row, multi-super-block q6_K matrix dequantises super-block by
+    super-block in row-major order (checked with Python's struct decoders)."""
+    rng = np.random.default_rng(8)
+    rows, k = 2, 512
+    blocks = synth.q6_k_blocks(rng, rows, k, 0.01)
+    got = oracle.dequant(oracle.WFMT_Q6_K, blocks, rows, k)
+    for r in range(rows):
+        for b in range(k // 256):
+            raw = bytes(blocks[r, b])
+            (scale,) = struct.unpack("<e", raw[208:210])
+            codes, subs = _q6_codes(raw)
+            for i in range(256):
+                assert got[r, 256 * b + i] == scale * subs[i // 16] * (codes[i] - 32)
+
+
+def test_q6_k_rejects_ragged_rows():
+    with pytest.raises(ValueError):
+        oracle.dequant(oracle.WFMT_Q6_K, np.zeros(420, np.uint8), 1, 288)
+
+
 def _bf16(b):
     return struct.unpack(">f", struct.pack(">I", int(b) << 16))[0]
 
@@ -193,10 +242,26 @@ def _q5_rows(blocks):
     return out
 
 
+def _q6_rows(blocks):
+    """Pure-Python decode of canonical q6_K rows -> list of lists."""
+    out = []
+    for row in blocks:
+        vals = []
+        for blk in row:
+            raw = bytes(blk)
+            (sc,) = struct.unpack("<e", raw[208:210])
+            codes, subs = _q6_codes(raw)
+            vals.extend(sc * subs[i // 16] * (q - 32) for i, q in enumerate(codes))
+        out.append(vals)
+    return out
+
+
 def _mat(inp_arr, wfmt, m, rows, cols):
     if wfmt == synth.WFMT_BF16:
         a = inp_arr[m]
         return [[_bf16(a[r, c]) for c in range(cols)] for r in range(rows)]
+    if wfmt == synth.WFMT_Q6_K:
+        return _q6_rows(inp_arr[m])
     if wfmt == synth.WFMT_Q4_0:
         return _q4_rows(inp_arr[m])
     if wfmt == synth.WFMT_Q5_0:
@@ -264,6 +329,8 @@ TINY = [
                    wfmt=synth.WFMT_Q8_0),
     synth.MoEShape("q5_shared", T=2, d=32, E=4, k=2, F=32, S=1, Fs=32,
                    wfmt=synth.WFMT_Q5_0),
+    synth.MoEShape("q6_shared", T=2, d=256, E=3, k=2, F=256, S=1, Fs=256,
+                   wfmt=synth.WFMT_Q6_K),
 ]
 
 
@@ -271,7 +338,7 @@ TINY = [
 def test_brute_force_tiny(sh):
     # A larger weight std makes the logits spread and the SwiGLU nonlinear.
     sh = sh.replace(w_std=0.5, wr_std=0.5, q4_scale_std=0.05, q8_scale_std=0.004,
-                    q5_scale_std=0.025)
+                    q5_scale_std=0.025, q6_scale_std=2e-4)
     inp = synth.make_inputs(sh, seed=11)
     out, ids, w, logits = oracle.forward(inp)
     bout, bsets, bw, _ = _brute_layer(inp)
@@ -298,6 +365,18 @@ def _f64_stack(arr, wfmt, rows, cols):
         sc = a[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
         q = a[..., 2:].copy().view(np.int8).astype(np.float64)
         return (q * sc[..., None]).reshape(-1, rows, cols)
+    if wfmt == synth.WFMT_Q6_K:
+        a = np.ascontiguousarray(arr).reshape(-1, rows, cols // 256, 210)
+        d = a[..., 208:210].copy().view(np.float16)[..., 0].astype(np.float64)
+        sub = a[..., 192:208].copy().view(np.int8).astype(np.float64)          # [..][16]
+        ql = a[..., :128].reshape(a.shape[:-1] + (2, 2, 32))                  # [h][c%2][l]
+        qh = a[..., 128:192].reshape(a.shape[:-1] + (2, 32))                  # [h][l]
+        low = np.stack([ql[..., 0, :] & 15, ql[..., 1, :] & 15,
+                        ql[..., 0, :] >> 4, ql[..., 1, :] >> 4], axis=-2)      # [h][c][l]
+        high = np.stack([(qh >> (2 * c)) & 3 for c in range(4)], axis=-2)      # [h][c][l]
+        q = (low.astype(np.float64) + 16.0 * high).reshape(a.shape[:-1] + (256,)) - 32.0
+        w = q * np.repeat(sub, 16, axis=-1) * d[..., None]
+        return w.reshape(-1, rows, cols)
     if wfmt == synth.WFMT_Q5_0:
         a = np.ascontiguousarray(arr).reshape(-1, rows, cols // 32, 22)
         sc = a[..., :2].copy().view(np.float16)[..., 0].astype(np.float64)
@@ -327,11 +406,13 @@ def _x64(inp):
 
 
 @pytest.mark.parametrize("wfmt", [synth.WFMT_BF16, synth.WFMT_Q4_0, synth.WFMT_Q8_0,
-                                  synth.WFMT_Q5_0])
+                                  synth.WFMT_Q5_0, synth.WFMT_Q6_K])
 def test_k_equals_E_is_dense_softmax_mixture(wfmt):
-    sh = synth.MoEShape("dense", T=5, d=64, E=4, k=4, F=32, wfmt=wfmt,
-                        wr_std=0.2, w_std=0.2, q4_scale_std=0.02, q8_scale_std=0.002,
-                        q5_scale_std=0.01)
+    big = wfmt == synth.WFMT_Q6_K          # 256-weight super-blocks
+    sh = synth.MoEShape("dense", T=5, d=256 if big else 64, E=4, k=4, F=256 if big else 32,
+                        wfmt=wfmt, wr_std=0.2 if not big else 0.1, w_std=0.2,
+                        q4_scale_std=0.02, q8_scale_std=0.002, q5_scale_std=0.01,
+                        q6_scale_std=1e-4)
     inp = synth.make_inputs(sh, seed=3)
     out, ids, w, logits = oracle.forward(inp)
     x = _x64(inp)
