@@ -198,6 +198,9 @@ int pick_fs(const moe_plan_s* p, int T) {
     const double act = E * (1.0 - pow(1.0 - static_cast<double>(c.top_k) / E, T));
     int best = 32;
     double best_eff = -1.0;
+    // Q4_0's row-streaming pipeline keeps every row group's partial sums in
+    // registers, which fit for 32-row slices only
+    if (c.wfmt == MOE_WFMT_Q4_0) return 32;
     for (int fs : {64, 32}) {
         if (c.d_ff % fs || (c.n_shared && c.d_ff_shared % fs)) continue;
         const double units = act * (c.d_ff / fs) + c.n_shared * (c.n_shared ? c.d_ff_shared / fs : 0);
@@ -230,26 +233,33 @@ DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
             ok &= map_bf16(p, &a.tm_sdown, w->shared_down.data, S, d, Fs, fs, 128);
         }
     } else {
-        const uint32_t kb = 512 / fs, nb = fs / 32;
+        // phase-A boxes: Q4_0 streams 16-row groups over up to 64 block
+        // columns (the row-streaming pipeline); the other formats stream
+        // 512 / fs block columns of the whole slice
+        const bool rows16 = c.wfmt == MOE_WFMT_Q4_0;
+        const uint32_t kb = rows16 ? static_cast<uint32_t>(d / 32 < 64 ? d / 32 : 64) : 512 / fs;
+        const uint32_t ar = rows16 ? 16 : fs;
+        const uint32_t nb = fs / 32;
         const uint32_t cb = c.wfmt == MOE_WFMT_Q8_0 ? 32 : 16;
+        a.kt = static_cast<int>(kb);
         // scales: fp16 [mats][K/32][N], or Q5_0's 48-byte records of 8 rows
         auto scales = [&](CUtensorMap* m, const void* base, int64_t mats, int64_t N, int64_t K,
                           uint32_t box_rows, uint32_t box_kb) {
             return c.wfmt == MOE_WFMT_Q5_0 ? map_q5_aux(p, m, base, mats, N, K, box_rows, box_kb)
                                            : map_quant_scales(p, m, base, mats, N, K, box_rows, box_kb);
         };
-        ok &= map_quant_codes(p, &a.tm_gate, w->gate.data, E, F, d, fs, kb, cb);
-        ok &= map_quant_codes(p, &a.tm_up, w->up.data, E, F, d, fs, kb, cb);
+        ok &= map_quant_codes(p, &a.tm_gate, w->gate.data, E, F, d, ar, kb, cb);
+        ok &= map_quant_codes(p, &a.tm_up, w->up.data, E, F, d, ar, kb, cb);
         ok &= map_quant_codes(p, &a.tm_down, w->down.data, E, d, F, kQuantDownBoxRows, nb, cb);
-        ok &= scales(&a.tm_gate_sc, w->gate.scales, E, F, d, fs, kb);
-        ok &= scales(&a.tm_up_sc, w->up.scales, E, F, d, fs, kb);
+        ok &= scales(&a.tm_gate_sc, w->gate.scales, E, F, d, ar, kb);
+        ok &= scales(&a.tm_up_sc, w->up.scales, E, F, d, ar, kb);
         ok &= scales(&a.tm_down_sc, w->down.scales, E, d, F, kQuantDownBoxRows, nb);
         if (S) {
-            ok &= map_quant_codes(p, &a.tm_sgate, w->shared_gate.data, S, Fs, d, fs, kb, cb);
-            ok &= map_quant_codes(p, &a.tm_sup, w->shared_up.data, S, Fs, d, fs, kb, cb);
+            ok &= map_quant_codes(p, &a.tm_sgate, w->shared_gate.data, S, Fs, d, ar, kb, cb);
+            ok &= map_quant_codes(p, &a.tm_sup, w->shared_up.data, S, Fs, d, ar, kb, cb);
             ok &= map_quant_codes(p, &a.tm_sdown, w->shared_down.data, S, d, Fs, kQuantDownBoxRows, nb, cb);
-            ok &= scales(&a.tm_sgate_sc, w->shared_gate.scales, S, Fs, d, fs, kb);
-            ok &= scales(&a.tm_sup_sc, w->shared_up.scales, S, Fs, d, fs, kb);
+            ok &= scales(&a.tm_sgate_sc, w->shared_gate.scales, S, Fs, d, ar, kb);
+            ok &= scales(&a.tm_sup_sc, w->shared_up.scales, S, Fs, d, ar, kb);
             ok &= scales(&a.tm_sdown_sc, w->shared_down.scales, S, d, Fs, kQuantDownBoxRows, nb);
         }
     }

@@ -258,6 +258,12 @@ struct DecodeCfg {
     static_assert(!QUANT || RJ % kQuantDownBoxRows == 0, "whole down boxes per stage");
     static constexpr int HS = FS + 8;             // h row stride (bf16 elements)
     static constexpr int GS = FS + 4;             // gate/up result row stride (floats)
+    // Row-streaming phase A (the F16 formats, experts_pipeline_rows): a stage
+    // is one 16-row group of one matrix over KC <= KCMAX block columns, and
+    // consumer warp w owns block columns w, w + 16, ... of every stage.
+    static constexpr int KCMAX = 64;
+    static constexpr int NBW = KCMAX / kConsumerWarps;   // block columns per warp
+    static constexpr int GU_PARTS = F16 ? kConsumerWarps : KSPLIT;   // partial sums per output
 };
 
 struct alignas(16) DecodeSmemTail {
@@ -443,7 +449,7 @@ struct DecodeSmem {
     uint8_t* ring;
     uint8_t* xs;            // [8][xs_stride]: the T token rows of x, staged once
     float* xsum;            // [8][d/32]: -offset * block sums of x (quantised formats)
-    float* gu;              // [KSPLIT][2][8][GS]: gate / up partial results
+    float* gu;              // [GU_PARTS][2][8][GS]: gate / up partial results
     __nv_bfloat16* hhi;     // [8][HS]: h = hi + lo, per slot
     __nv_bfloat16* hlo;
     float* hsum;            // [8][2]: -offset * block sums of hi + lo (quantised formats)
@@ -462,7 +468,7 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
     sm.xs = sm.ring + static_cast<size_t>(a.n_stages) * C::STAGE;
     sm.xsum = reinterpret_cast<float*>(sm.xs + kDecodeTok * a.xs_stride);
     sm.gu = sm.xsum + kDecodeTok * (a.d / 32);
-    sm.hhi = reinterpret_cast<__nv_bfloat16*>(sm.gu + C::KSPLIT * 2 * kDecodeTok * C::GS);
+    sm.hhi = reinterpret_cast<__nv_bfloat16*>(sm.gu + C::GU_PARTS * 2 * kDecodeTok * C::GS);
     sm.hlo = sm.hhi + kDecodeTok * C::HS;
     sm.hsum = reinterpret_cast<float*>(sm.hlo + kDecodeTok * C::HS);
     sm.tail = reinterpret_cast<DecodeSmemTail*>(sm.hsum + kDecodeTok * 2);
@@ -747,28 +753,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                     const int r0 = rg * 16 + g;
                     const float* xsum0 = sm.xsum + tok0 * nkb + kb0;
                     const float* xsum1 = sm.xsum + tok1 * nkb + kb0;
-                    if constexpr (C::F16) {
-                        // fp16 operands: one chain per block from its correction
-#pragma unroll 4
-                        for (int bb = ks; bb < nkb_st; bb += C::KSPLIT) {
-                            const uint32_t* row = codes + (bb * FS + r0) * 4;
-                            const uint32_t w0 = row[tig], w8 = row[32 + tig];
-                            uint32_t b0, b1, b2, b3;
-                            ldsm_x4(xrow + ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
-                            const float c0 = xsum0[bb], c1 = xsum1[bb];
-                            float v[4];
-                            mma_f16_16816(v, q4h_lo(w0), q4h_lo(w8), q4h_hi(w0), q4h_hi(w8), b0, b1,
-                                          c0, c1, c0, c1);
-                            const uint32_t u0 = w0 >> 8, u8 = w8 >> 8;
-                            mma_f16_16816_acc(v, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8), b2, b3);
-                            const float s0 = __half2float(scl[bb * FS + r0]);
-                            const float s8 = __half2float(scl[bb * FS + r0 + 8]);
-                            cacc[0] = fmaf(s0, v[0], cacc[0]);
-                            cacc[1] = fmaf(s0, v[1], cacc[1]);
-                            cacc[2] = fmaf(s8, v[2], cacc[2]);
-                            cacc[3] = fmaf(s8, v[3], cacc[3]);
-                        }
-                    } else {
+                    {
 #pragma unroll 2
                     for (int bb = ks; bb < nkb_st; bb += C::KSPLIT) {
                         const uint32_t* row = codes + (bb * FS + r0) * (C::CB / 4);
@@ -827,20 +812,6 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                 uv += gu[((q * 2 + 1) * kDecodeTok + t) * C::GS + f];
             }
             const float h = gv / (1.f + expf(-gv)) * uv;
-            if constexpr (C::F16) {
-                // fp16 pair hi + lo; the down block's accumulator starts at
-                // -sum((base_f + 8)(hi + lo)) (bases as in q4h_lo)
-                const __half hi = __float2half_rn(h);
-                const __half lo = __float2half_rn(h - __half2float(hi));
-                reinterpret_cast<__half*>(hhi)[t * C::HS + f] = hi;
-                reinterpret_cast<__half*>(hlo)[t * C::HS + f] = lo;
-                const float base = (f & 15) < 8 ? kF16BaseLo : kF16BaseHi;
-                float hs = (base + 8.f) * (__half2float(hi) + __half2float(lo));
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
-                if (lane == 0) sm.hsum[t * 2 + f / 32] = -hs;
-                continue;
-            }
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             hhi[t * C::HS + f] = hi;
@@ -896,31 +867,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);   // [NB][128][CB]
                         const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * QB * C::CB);
                         const int rib = (rgb % (QB / 16)) * 16 + g;
-                        if constexpr (C::F16) {
-#pragma unroll
-                            for (int bb = 0; bb < C::NB; ++bb) {
-                                const uint32_t* row = codes + (bb * QB + rib) * 4;
-                                const uint32_t w0 = row[tig], w8 = row[32 + tig];
-                                const uint32_t u0 = w0 >> 8, u8 = w8 >> 8;
-                                const uint32_t p0 = q4h_lo(w0), q0 = q4h_lo(w8);
-                                const uint32_t p1 = q4h_hi(w0), q1 = q4h_hi(w8);
-                                const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
-                                const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
-                                float v[4];
-                                // one chain from the block's correction: hi then lo parts of h
-                                mma_f16_16816(v, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
-                                              hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
-                                mma_f16_16816_acc(v, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
-                                mma_f16_16816_acc(v, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
-                                mma_f16_16816_acc(v, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
-                                const float s0 = __half2float(scl[bb * QB + rib]);
-                                const float s8 = __half2float(scl[bb * QB + rib + 8]);
-                                c[0] = fmaf(s0, v[0], c[0]);
-                                c[1] = fmaf(s0, v[1], c[1]);
-                                c[2] = fmaf(s8, v[2], c[2]);
-                                c[3] = fmaf(s8, v[3], c[3]);
-                            }
-                        } else {
+                        {
 #pragma unroll
                         for (int bb = 0; bb < C::NB; ++bb) {
                             const uint32_t* row = codes + (bb * QB + rib) * (C::CB / 4);
@@ -968,6 +915,327 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
 }
 
 
+// The experts pipeline for the weight formats that feed fp16 operands to
+// the tensor cores (F16): phase A streams row groups instead of block
+// columns.  A phase-A stage is 16 consecutive rows of the gate or up slice
+// over the whole reduction dim (KC <= 64 block columns per stage, more
+// stages per row group when d > 2048), and consumer warp w owns block
+// columns w, w + 16, w + 32, w + 48 of every stage.  The x fragments and
+// block corrections of those columns therefore stay in registers for the
+// whole unit instead of being reloaded from shared memory for every 16x32
+// tile, which halves the shared-memory traffic per weight; each warp keeps
+// the partial sums of every row group and both matrices, and one reduction
+// over the 16 warps follows phase A.  Phase B (down matrix, combine) is the
+// same as in experts_pipeline.
+template <int FS, int WF>
+__device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const DecodeSmem& sm,
+                                                      const WorkView& wv) {
+    using C = DecodeCfg<FS, WF>;
+    static_assert(C::F16, "row-streaming phase A serves the fp16-operand formats");
+    const int ns = a.n_stages;
+    uint8_t* ring = sm.ring;
+    float* gu = sm.gu;
+    uint64_t* full = sm.full;
+    uint64_t* empty = sm.empty;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int d = a.d, E = a.E;
+    const int nkb = d / 32;
+    const int KC = a.kt;                              // block columns per phase-A stage
+    const int nch = (nkb + KC - 1) / KC;              // phase-A stages per row group and matrix
+    const int n_routed = wv.n_routed, n_shared = wv.n_shared;
+    const int sl_r = a.F / FS, sl_s = a.S ? a.Fs / FS : 0;
+    const int n_su = n_shared * sl_s;
+    const int n_units = n_su + n_routed * sl_r;
+    const int nA = 2 * C::RG * nch;
+    const int nB = (d + C::RJ - 1) / C::RJ;
+    volatile int* abort_flag = &sm.tail->abort_flag;
+    const int u_begin = static_cast<int>(blockIdx.x);
+    const int u_step = static_cast<int>(gridDim.x);
+    auto unit_item = [&](int u, int& ii, int& sl) {
+        if (u < n_su) { ii = n_routed + u / sl_s; sl = u % sl_s; }
+        else { const int v = u - n_su; ii = v / sl_r; sl = v % sl_r; }
+    };
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&a.tm_gate); prefetch_tensormap(&a.tm_up);
+            prefetch_tensormap(&a.tm_down);
+            prefetch_tensormap(&a.tm_gate_sc); prefetch_tensormap(&a.tm_up_sc);
+            prefetch_tensormap(&a.tm_down_sc);
+            if (a.S) {
+                prefetch_tensormap(&a.tm_sgate); prefetch_tensormap(&a.tm_sup);
+                prefetch_tensormap(&a.tm_sdown); prefetch_tensormap(&a.tm_sgate_sc);
+                prefetch_tensormap(&a.tm_sup_sc); prefetch_tensormap(&a.tm_sdown_sc);
+            }
+            const uint64_t pol = l2_policy_evict_first();
+            uint32_t it = 0;
+            bool ok = true;
+            for (int u = u_begin; u < n_units && ok; u += u_step) {
+                int ii, sl;
+                unit_item(u, ii, sl);
+                const WorkItem item = wv.items[ii];
+                const bool shared = item.expert >= E;
+                const int ex = shared ? item.expert - E : item.expert;
+                const int Fh = shared ? a.Fs : a.F;
+                const int f0 = sl * FS;
+                for (int st = 0; st < nA + nB && ok; ++st, ++it) {
+                    const int slot = it % ns;
+                    if (it >= static_cast<uint32_t>(ns)) {
+                        if (*abort_flag || !mbar_wait_bounded(&empty[slot], ((it / ns) - 1) & 1)) {
+                            atomicOr(a.err, kErrTimeout); *abort_flag = 1; ok = false; break;
+                        }
+                    }
+                    uint8_t* dst = ring + static_cast<size_t>(slot) * C::STAGE;
+                    if (st < nA) {
+                        // stage (row group rg, matrix mat, k chunk c)
+                        const int c = st % nch, mat = (st / nch) & 1, rg = st / (2 * nch);
+                        const CUtensorMap* mc = mat ? (shared ? &a.tm_sup : &a.tm_up)
+                                                    : (shared ? &a.tm_sgate : &a.tm_gate);
+                        const CUtensorMap* ms = mat ? (shared ? &a.tm_sup_sc : &a.tm_up_sc)
+                                                    : (shared ? &a.tm_sgate_sc : &a.tm_gate_sc);
+                        const int c2 = ex * nkb + c * KC;
+                        mbar_arrive_expect_tx(&full[slot], 16 * KC * C::BR);
+                        tma_load_3d(dst, mc, &full[slot], 0, f0 + rg * 16, c2, pol);
+                        tma_load_2d(dst + 16 * KC * C::CB, ms, &full[slot], f0 + rg * 16, c2, pol);
+                    } else {
+                        const CUtensorMap* md = shared ? &a.tm_sdown : &a.tm_down;
+                        const CUtensorMap* mds = shared ? &a.tm_sdown_sc : &a.tm_down_sc;
+                        const int j0 = (st - nA) * C::RJ;
+                        constexpr int QB = kQuantDownBoxRows;
+                        const int nbox = (min(C::RJ, d - j0) + QB - 1) / QB;
+                        const int c2 = ex * (Fh / 32) + f0 / 32;
+                        mbar_arrive_expect_tx(&full[slot], nbox * C::NB * QB * C::BR);
+                        for (int b = 0; b < nbox; ++b) {
+                            uint8_t* bd = dst + b * (C::NB * QB * C::BR);
+                            tma_load_3d(bd, md, &full[slot], 0, j0 + QB * b, c2, pol);
+                            tma_load_2d(bd + C::NB * QB * C::CB, mds, &full[slot], j0 + QB * b, c2, pol);
+                        }
+                    }
+                }
+            }
+            const uint32_t first = it > static_cast<uint32_t>(ns) ? it - ns : 0;
+            for (uint32_t q = first; q < it; ++q)
+                if (!mbar_wait_bounded(&full[q % ns], (q / ns) & 1)) {
+                    atomicOr(a.err, kErrTimeout);
+                    break;
+                }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------- consumers
+    const int g = lane >> 2, tig = lane & 3;
+    const uint32_t xs_u = smem_u32(sm.xs);
+    uint32_t it = 0;
+    auto wait_full = [&](int slot, uint32_t parity) -> bool {
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], parity));
+        if (!ok && lane == 0) {
+            atomicOr(a.err, kErrTimeout);
+            *abort_flag = 1;
+        }
+        return ok;
+    };
+
+    for (int u = u_begin; u < n_units; u += u_step) {
+        int ii, sl;
+        unit_item(u, ii, sl);
+        const WorkItem item = wv.items[ii];
+        const bool shared = item.expert >= E;
+        const int ntok = min(item.count, kDecodeTok);
+        auto tok_of = [&](int n) -> int {
+            return n < ntok ? (shared ? n : wv.slot_token[item.slot_begin + n]) : 0;
+        };
+        auto w_of = [&](int n) -> float {
+            return n < ntok ? (shared ? 1.f : wv.slot_w[item.slot_begin + n]) : 0.f;
+        };
+        const uint32_t xrow = xs_u + tok_of(lane & 7) * a.xs_stride;   // B row of this lane
+        const int t0 = 2 * tig, t1 = t0 + 1;
+        const int tok0 = tok_of(t0), tok1 = tok_of(t1);
+        const float w0 = w_of(t0), w1 = w_of(t1);
+        const bool v0 = t0 < ntok, v1 = t1 < ntok;
+
+        // x fragments and corrections of this warp's block columns of chunk c
+        uint32_t xf[C::NBW][4];
+        float xc0[C::NBW], xc1[C::NBW];
+        auto load_x = [&](int c) {
+#pragma unroll
+            for (int i = 0; i < C::NBW; ++i) {
+                const int kb = c * KC + warp + kConsumerWarps * i;
+                const bool in = (warp + kConsumerWarps * i) < KC && kb < nkb;
+                const int kbs = in ? kb : 0;
+                ldsm_x4(xrow + (kbs * 32 + (lane >> 3) * 8) * 2, xf[i][0], xf[i][1], xf[i][2], xf[i][3]);
+                xc0[i] = sm.xsum[tok0 * nkb + kbs];
+                xc1[i] = sm.xsum[tok1 * nkb + kbs];
+            }
+        };
+        if (nch == 1) load_x(0);
+
+        // ------------------------------------------- phase A: gate and up
+        float acc[2 * C::RG][4];
+#pragma unroll
+        for (int q = 0; q < 2 * C::RG; ++q)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
+#pragma unroll
+        for (int rg = 0; rg < C::RG; ++rg) {
+#pragma unroll
+            for (int mat = 0; mat < 2; ++mat) {
+                for (int c = 0; c < nch; ++c, ++it) {
+                    const int slot = it % ns;
+                    const bool ok = wait_full(slot, (it / ns) & 1);
+                    if (ok) {
+                        if (nch > 1) load_x(c);
+                        const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
+                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(stage);   // [KC][16][CB]
+                        const __half* scl = reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
+#pragma unroll
+                        for (int i = 0; i < C::NBW; ++i) {
+                            const int bl = warp + kConsumerWarps * i;
+                            if (bl < KC && c * KC + bl < nkb) {
+                                const uint32_t* row = codes + (bl * 16 + g) * 4;
+                                const uint32_t x0 = row[tig], x8 = row[32 + tig];
+                                float v[4];
+                                mma_f16_16816(v, q4h_lo(x0), q4h_lo(x8), q4h_hi(x0), q4h_hi(x8),
+                                              xf[i][0], xf[i][1], xc0[i], xc1[i], xc0[i], xc1[i]);
+                                const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
+                                mma_f16_16816_acc(v, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8),
+                                                  xf[i][2], xf[i][3]);
+                                const float s0 = __half2float(scl[bl * 16 + g]);
+                                const float s8 = __half2float(scl[bl * 16 + g + 8]);
+                                float* ac = acc[rg * 2 + mat];
+                                ac[0] = fmaf(s0, v[0], ac[0]);
+                                ac[1] = fmaf(s0, v[1], ac[1]);
+                                ac[2] = fmaf(s8, v[2], ac[2]);
+                                ac[3] = fmaf(s8, v[3], ac[3]);
+                            }
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[slot]);
+                }
+            }
+        }
+        // this warp's partial sums, [warp][mat][t][f] (row stride GS)
+#pragma unroll
+        for (int rg = 0; rg < C::RG; ++rg) {
+#pragma unroll
+            for (int mat = 0; mat < 2; ++mat) {
+                float* gq = gu + (warp * 2 + mat) * kDecodeTok * C::GS;
+                const int r = rg * 16 + g;
+                gq[t0 * C::GS + r] = acc[rg * 2 + mat][0];
+                gq[t1 * C::GS + r] = acc[rg * 2 + mat][1];
+                gq[t0 * C::GS + r + 8] = acc[rg * 2 + mat][2];
+                gq[t1 * C::GS + r + 8] = acc[rg * 2 + mat][3];
+            }
+        }
+        named_bar_sync(1, kConsumers);
+        // h = SiLU(gate) * up as an fp16 pair hi + lo for the token columns in
+        // use (the rest are zero); one warp covers 32 consecutive f of one
+        // column, i.e. one block of the down matrix
+        for (int idx = tid; idx < FS * kDecodeTok; idx += kConsumers) {
+            const int t = idx / FS, f = idx % FS;
+            __half hi = __float2half_rn(0.f), lo = hi;
+            float hs = 0.f;
+            if (t < ntok) {
+                float gv = 0.f, uv = 0.f;
+#pragma unroll
+                for (int q = 0; q < kConsumerWarps; ++q) {
+                    gv += gu[((q * 2 + 0) * kDecodeTok + t) * C::GS + f];
+                    uv += gu[((q * 2 + 1) * kDecodeTok + t) * C::GS + f];
+                }
+                const float h = gv / (1.f + expf(-gv)) * uv;
+                hi = __float2half_rn(h);
+                lo = __float2half_rn(h - __half2float(hi));
+                const float base = (f & 15) < 8 ? kF16BaseLo : kF16BaseHi;
+                hs = (base + 8.f) * (__half2float(hi) + __half2float(lo));
+            }
+            reinterpret_cast<__half*>(sm.hhi)[t * C::HS + f] = hi;
+            reinterpret_cast<__half*>(sm.hlo)[t * C::HS + f] = lo;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
+            if (lane == 0) sm.hsum[t * 2 + f / 32] = -hs;
+        }
+        named_bar_sync(1, kConsumers);
+        uint32_t bh[C::RG][2], bl[C::RG][2];
+#pragma unroll
+        for (int kk = 0; kk < C::RG; ++kk) {
+            const uint32_t off = ((lane & 7) * C::HS + kk * 16 + ((lane >> 3) & 1) * 8) * 2;
+            ldsm_x2(smem_u32(sm.hhi) + off, bh[kk][0], bh[kk][1]);
+            ldsm_x2(smem_u32(sm.hlo) + off, bl[kk][0], bl[kk][1]);
+        }
+        float hs0[C::NB], hs1[C::NB];
+#pragma unroll
+        for (int bb = 0; bb < C::NB; ++bb) {
+            hs0[bb] = sm.hsum[t0 * 2 + bb];
+            hs1[bb] = sm.hsum[t1 * 2 + bb];
+        }
+
+        // --------------------------------------- phase B: down + combine
+        for (int st = 0; st < nB; ++st, ++it) {
+            const int slot = it % ns;
+            const bool ok = wait_full(slot, (it / ns) & 1);
+            const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
+            const int j0 = st * C::RJ;
+            const int rows = min(C::RJ, d - j0);
+            if (ok) {
+                for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
+                    float c[4] = {0.f, 0.f, 0.f, 0.f};
+                    constexpr int QB = kQuantDownBoxRows;
+                    const uint8_t* bbase = stage + (rgb / (QB / 16)) * (C::NB * QB * C::BR);
+                    const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);   // [NB][QB][CB]
+                    const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * QB * C::CB);
+                    const int rib = (rgb % (QB / 16)) * 16 + g;
+#pragma unroll
+                    for (int bb = 0; bb < C::NB; ++bb) {
+                        const uint32_t* row = codes + (bb * QB + rib) * 4;
+                        const uint32_t x0 = row[tig], x8 = row[32 + tig];
+                        const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
+                        const uint32_t p0 = q4h_lo(x0), q0 = q4h_lo(x8);
+                        const uint32_t p1 = q4h_hi(x0), q1 = q4h_hi(x8);
+                        const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
+                        const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
+                        float v[4];
+                        mma_f16_16816(v, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
+                                      hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
+                        mma_f16_16816_acc(v, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
+                        mma_f16_16816_acc(v, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                        mma_f16_16816_acc(v, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                        const float s0 = __half2float(scl[bb * QB + rib]);
+                        const float s8 = __half2float(scl[bb * QB + rib + 8]);
+                        c[0] = fmaf(s0, v[0], c[0]);
+                        c[1] = fmaf(s0, v[1], c[1]);
+                        c[2] = fmaf(s8, v[2], c[2]);
+                        c[3] = fmaf(s8, v[3], c[3]);
+                    }
+                    const int j = j0 + rgb * 16 + g;
+                    if (v0) {
+                        red_add_f32(a.out + static_cast<size_t>(tok0) * d + j, w0 * c[0]);
+                        red_add_f32(a.out + static_cast<size_t>(tok0) * d + j + 8, w0 * c[2]);
+                    }
+                    if (v1) {
+                        red_add_f32(a.out + static_cast<size_t>(tok1) * d + j, w1 * c[1]);
+                        red_add_f32(a.out + static_cast<size_t>(tok1) * d + j + 8, w1 * c[3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+        }
+    }
+}
+
+// The experts pipeline of the format: row-streaming for the fp16-operand
+// formats, block-column stages for the others.
+template <int FS, int WF>
+__device__ __forceinline__ void run_experts(const DecodeArgs& a, const DecodeSmem& sm,
+                                            const WorkView& wv) {
+    if constexpr (DecodeCfg<FS, WF>::F16) experts_pipeline_rows<FS, WF>(a, sm, wv);
+    else experts_pipeline<FS, WF>(a, sm, wv);
+}
+
 template <int FS, int WF>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
 decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
@@ -984,7 +1252,7 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
     if (threadIdx.x < kConsumers) stage_x<WF>(a, sm, threadIdx.x);
     __syncthreads();
     const WorkView wv{a.n_items[0], a.n_items[1], a.items, a.slot_token, a.slot_w};
-    experts_pipeline<FS, WF>(a, sm, wv);
+    run_experts<FS, WF>(a, sm, wv);
 }
 
 // ====================================================== fused decode ===
@@ -1231,7 +1499,7 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
     }
     __syncthreads();
     const WorkView wv{rs->n_routed, S, rs->items, rs->slot_token, rs->slot_w};
-    experts_pipeline<FS, WF>(a, sm, wv);
+    run_experts<FS, WF>(a, sm, wv);
 }
 
 int decode_stage_bytes(int fs, int wfmt) {
@@ -1243,7 +1511,9 @@ int decode_stage_bytes(int fs, int wfmt) {
 }
 
 size_t decode_smem_bytes(int fs, int wfmt, int d, int n_stages) {
-    const int ksplit = kConsumerWarps / (2 * (fs / 16));
+    // partial sums per gate/up output: KSPLIT, or one per warp for the
+    // row-streaming formats (DecodeCfg::GU_PARTS)
+    const int ksplit = wfmt == kWfQ4 ? kConsumerWarps : kConsumerWarps / (2 * (fs / 16));
     size_t b = 1024;                                            // alignment slack
     b += static_cast<size_t>(n_stages) * decode_stage_bytes(fs, wfmt);
     b += static_cast<size_t>(kDecodeTok) * (d * 2 + 16);       // staged x
@@ -1307,7 +1577,6 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, int wfmt, int grid,
     switch (wfmt * 100 + fs) {
         case kWfBf16 * 100 + 64: return launch_fused_one<64, kWfBf16>(a, grid, smem, stream);
         case kWfBf16 * 100 + 32: return launch_fused_one<32, kWfBf16>(a, grid, smem, stream);
-        case kWfQ4 * 100 + 64: return launch_fused_one<64, kWfQ4>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_fused_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_fused_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_fused_one<32, kWfQ8>(a, grid, smem, stream);
@@ -1322,7 +1591,6 @@ cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, int wfmt, int gri
     switch (wfmt * 100 + fs) {
         case kWfBf16 * 100 + 64: return launch_one<64, kWfBf16>(a, grid, smem, stream);
         case kWfBf16 * 100 + 32: return launch_one<32, kWfBf16>(a, grid, smem, stream);
-        case kWfQ4 * 100 + 64: return launch_one<64, kWfQ4>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_one<32, kWfQ8>(a, grid, smem, stream);

@@ -8,11 +8,14 @@ Acceptance (the contract of the layer):
     still lie inside the tie band;
   * counts, offsets and the slot order bit-exact against the oracle's
     bucketing of the GPU's own ids (they are a pure function of the ids);
-  * routing weights within relative 5*sqrt(d)*2^-24: the GPU sums the d
+  * routing weights within relative c*sqrt(d)*2^-24: the GPU sums the d
     products of a logit in fp32, whose rounding error grows like sqrt(d)*2^-24
     times the partial sums (|partial sums| <~ 1 here), and a renormalised
-    weight's relative error is the difference of two such logit errors
-    (observed 1.6*sqrt(d)*2^-24 at d = 2048: a margin of about 3);
+    weight's relative error is the difference of two such logit errors.
+    c = 5 for the decode router (fp32 FMA; observed 1.6 at d = 2048) and
+    c = 24 for the prefill router, whose tensor-core accumulation of the
+    three exact bf16 parts rounds its fp32 sums less tightly (observed 10.3 on
+    the DeepSeek-shaped layer at d = 2048): a margin of 2 to 3 each;
   * out within relative L2 2e-3 (bf16 weights) or 5e-3 (Q4_0, Q8_0 and Q5_0
     weights) over every token: a token whose ids differ from the oracle's
     (a waived near tie) is compared with the oracle evaluated on the GPU's own
@@ -39,9 +42,9 @@ W_ABS = 1e-7
 DECODE_TRIPWIRE = 1e-4
 
 
-def w_rtol(d: int) -> float:
+def w_rtol(d: int, prefill: bool = False) -> float:
     """Relative tolerance of the renormalised routing weights (see above)."""
-    return 5.0 * np.sqrt(d) * 2.0 ** -24
+    return (24.0 if prefill else 5.0) * np.sqrt(d) * 2.0 ** -24
 
 
 def run_gpu(layer: D.DeviceLayer, x_bits: np.ndarray, T: int, regime=B.MOE_REGIME_AUTO,
@@ -113,7 +116,7 @@ def check_tie_choice(logits: np.ndarray, ids, k: int):
 
 
 def compare(inp: synth.MoEInputs, gpu_out, routing, oracle_res, tokens=None, tol=None,
-            tripwire=None):
+            tripwire=None, prefill=False):
     """Check one GPU call against the oracle; returns the relative L2 error
     over every token checked."""
     sh = inp.shape
@@ -128,7 +131,7 @@ def compare(inp: synth.MoEInputs, gpu_out, routing, oracle_res, tokens=None, tol
         f"expert ids differ on non-tied tokens {np.where(~ok_ids & ~waived)[0].tolist()}")
     for t in range(len(tok)):                     # ids valid and distinct everywhere
         assert len(set(g_ids[t].tolist())) == sh.k and g_ids[t].min() >= 0 and g_ids[t].max() < sh.E
-    np.testing.assert_allclose(g_w[ok_ids], o_w[ok_ids], rtol=w_rtol(sh.d), atol=W_ABS)
+    np.testing.assert_allclose(g_w[ok_ids], o_w[ok_ids], rtol=w_rtol(sh.d, prefill), atol=W_ABS)
     # buckets are a pure function of the ids: compare with the oracle's
     if tokens is None:
         c, o, sp = oracle.buckets(ids.astype(np.int32), sh.E)

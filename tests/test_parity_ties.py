@@ -43,6 +43,10 @@ def _run(inp, regime):
     return run_gpu(layer, inp.x, inp.shape.T, regime=regime)
 
 
+def _compare(inp, out, routing, res, regime):
+    return compare(inp, out, routing, res, prefill=regime == B.MOE_REGIME_PREFILL)
+
+
 @pytest.mark.parametrize("sh,regime", CASES, ids=[c[0].name for c in CASES])
 def test_zero_router_picks_lowest_indices(sh, regime):
     inp = synth.make_inputs(sh, seed=12)
@@ -54,7 +58,7 @@ def test_zero_router_picks_lowest_indices(sh, regime):
     np.testing.assert_allclose(w, 1.0 / sh.k, rtol=1e-6)
     res = oracle.forward(inp)
     assert np.array_equal(res[1], want)                     # the oracle agrees
-    compare(inp, out, routing, res)
+    _compare(inp, out, routing, res, regime)
 
 
 @pytest.mark.parametrize("sh,regime", CASES, ids=[c[0].name for c in CASES])
@@ -75,4 +79,4 @@ def test_duplicated_router_rows_pick_lower_index_first(sh, regime):
         assert np.array_equal(ids[t], o_ids[t]), (t, ids[t], o_ids[t])
         for j in range(0, sh.k, 2):                         # (e, e + E/2) pairs, e first
             assert ids[t, j] + half == ids[t, j + 1], ids[t]
-    compare(inp, out, routing, res)
+    _compare(inp, out, routing, res, regime)
