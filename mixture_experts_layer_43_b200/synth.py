@@ -45,6 +45,7 @@ WFMT_Q4_0 = 1
 WFMT_Q8_0 = 2
 WFMT_Q5_0 = 3
 WFMT_Q6_K = 4
+WFMT_BF16_F16DOWN = 5      # gate/up bf16; down matrices rounded once to fp16
 Q4_BLOCK = 32          # weights per Q4_0 block
 Q4_BLOCK_BYTES = 18    # 2-byte fp16 scale + 16 bytes of 4-bit codes
 Q8_BLOCK_BYTES = 34    # 2-byte fp16 scale + 32 signed 8-bit codes
@@ -124,6 +125,11 @@ WORKLOADS = {
     "deepseek_T4096_d2048_E64k6_F1408_S2": MoEShape(
         "deepseek_T4096_d2048_E64k6_F1408_S2", T=4096, d=2048, E=64, k=6,
         F=1408, S=2, Fs=1408, zipf_bias=1.1),
+    # the same prefill layer with its down matrices rounded once to fp16, so
+    # that h can be stored in fp16 between the two GEMMs (precision headroom)
+    "deepseek_f16down_T4096_d2048_E64k6_F1408_S2": MoEShape(
+        "deepseek_f16down_T4096_d2048_E64k6_F1408_S2", T=4096, d=2048, E=64, k=6,
+        F=1408, S=2, Fs=1408, zipf_bias=1.1, wfmt=WFMT_BF16_F16DOWN),
 }
 
 
@@ -133,6 +139,13 @@ def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     u = a.view(np.uint32).astype(np.uint64)
     u = u + 0x7FFF + ((u >> 16) & 1)
     return (u >> 16).astype(np.uint16)
+
+
+def bf16_bits_to_f16_bits(a: np.ndarray) -> np.ndarray:
+    """Round bf16 values to IEEE fp16 (nearest, ties to even; numpy's
+    conversion); return the fp16 bits.  Exact for 2^-17 <= |w| <= 65504."""
+    f = (np.ascontiguousarray(a, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+    return f.astype(np.float16).view(np.uint16)
 
 
 def _normal_bf16(rng: np.random.Generator, shape, std: float,
@@ -280,7 +293,7 @@ def make_inputs(shape: MoEShape, seed: int = 0,
     rb = zipf_log_bias(sh.E, sh.zipf_bias) if sh.zipf_bias > 0 else None
     if x_only:
         return MoEInputs(sh, x, wr, rb, None, None, None, None, None, None)
-    if sh.wfmt == WFMT_BF16:
+    if sh.wfmt in (WFMT_BF16, WFMT_BF16_F16DOWN):
         g = _normal_bf16(rng(3), (sh.E, sh.F, sh.d), sh.w_std)
         u = _normal_bf16(rng(4), (sh.E, sh.F, sh.d), sh.w_std)
         dn = _normal_bf16(rng(5), (sh.E, sh.d, sh.F), sh.w_std)
@@ -290,6 +303,9 @@ def make_inputs(shape: MoEShape, seed: int = 0,
             sd = _normal_bf16(rng(8), (sh.S, sh.d, sh.Fs), sh.w_std)
         else:
             sg = su = sd = None
+        if sh.wfmt == WFMT_BF16_F16DOWN:     # the same bf16 draws, down rounded to fp16
+            dn = bf16_bits_to_f16_bits(dn)
+            sd = None if sd is None else bf16_bits_to_f16_bits(sd)
     else:
         blocks, q, nbytes, per = {
             WFMT_Q4_0: (q4_0_blocks, sh.q4_scale_std, Q4_BLOCK_BYTES, Q4_BLOCK),
@@ -315,7 +331,7 @@ def weight_bytes_per_expert(shape: MoEShape, hidden: Optional[int] = None) -> in
     """Bytes one expert's three matrices occupy in HBM in the kernel format."""
     F = shape.F if hidden is None else hidden
     n = 3 * F * shape.d
-    if shape.wfmt == WFMT_BF16:
+    if shape.wfmt in (WFMT_BF16, WFMT_BF16_F16DOWN):
         return 2 * n
     if shape.wfmt == WFMT_Q4_0:
         return n // 32 * 18   # 16 code bytes + 2 scale bytes per 32 weights
@@ -333,7 +349,7 @@ def expert_flops(shape: MoEShape, n_tokens: int, hidden: Optional[int] = None) -
 
 def describe(shape: MoEShape) -> str:
     fmt = {WFMT_BF16: "bf16", WFMT_Q4_0: "q4_0", WFMT_Q8_0: "q8_0",
-           WFMT_Q5_0: "q5_0", WFMT_Q6_K: "q6_k"}[shape.wfmt]
+           WFMT_Q5_0: "q5_0", WFMT_Q6_K: "q6_k", WFMT_BF16_F16DOWN: "bf16/f16-down"}[shape.wfmt]
     s = (f"T={shape.T} d={shape.d} E={shape.E} k={shape.k} F={shape.F} "
          f"S={shape.S} Fs={shape.Fs} {fmt}")
     if shape.zipf_bias:

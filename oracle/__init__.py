@@ -26,6 +26,7 @@ WFMT_Q4_0 = 1
 WFMT_Q8_0 = 2
 WFMT_Q5_0 = 3
 WFMT_Q6_K = 4
+WFMT_BF16_F16DOWN = 5
 
 
 def build(force: bool = False) -> str:

@@ -49,6 +49,9 @@
  *   Q8_0: a row of K weights is K/32 blocks of 34 bytes.
  *   Q5_0: a row of K weights is K/32 blocks of 22 bytes.
  *   q6_K: a row of K weights is K/256 super-blocks of 210 bytes.
+ *   BF16_F16DOWN: gate/up as bf16 bits, every down matrix (routed and shared)
+ *   as IEEE fp16 bits [.][d][F] -- the bf16 weights rounded to fp16 once, so
+ *   that the prefill down GEMM can take h in fp16 (see the kernels).
  *
  * The pages print no worked example for the layer output, so the tests pin
  * every function here against what the mathematics fixes instead: brute-force
@@ -69,6 +72,8 @@
 #define ORACLE_WFMT_Q8_0 2
 #define ORACLE_WFMT_Q5_0 3
 #define ORACLE_WFMT_Q6_K 4
+#define ORACLE_WFMT_BF16_F16DOWN 5   /* gate/up bf16, down (routed and shared) fp16 */
+#define ORACLE_ROWS_F16 100          /* internal: rows of fp16 bit patterns */
 
 /* bfloat16 is the top half of an IEEE binary32. */
 double oracle_bf16_to_f64(uint16_t b) {
@@ -176,6 +181,9 @@ static void load_row(int wfmt, const void* base, int64_t m, int64_t rows,
     if (wfmt == ORACLE_WFMT_BF16) {
         const uint16_t* p = (const uint16_t*)base + row * K;
         for (int64_t i = 0; i < K; ++i) out[i] = oracle_bf16_to_f64(p[i]);
+    } else if (wfmt == ORACLE_ROWS_F16) {
+        const uint16_t* p = (const uint16_t*)base + row * K;
+        for (int64_t i = 0; i < K; ++i) out[i] = oracle_fp16_to_f64(p[i]);
     } else if (wfmt == ORACLE_WFMT_Q4_0) {
         const uint8_t* p = (const uint8_t*)base + row * (K / 32) * 18;
         q4_0_row(p, K, out);
@@ -279,6 +287,12 @@ int oracle_buckets(int T, int k, int E, const int32_t* ids, int32_t* counts,
     return 0;
 }
 
+/* Storage of the gate/up and of the down matrices for a weight format:
+ * every format stores all three alike, except BF16_F16DOWN (gate/up bf16,
+ * down fp16). */
+static int gate_up_fmt(int wfmt) { return wfmt == ORACLE_WFMT_BF16_F16DOWN ? ORACLE_WFMT_BF16 : wfmt; }
+static int down_fmt(int wfmt) { return wfmt == ORACLE_WFMT_BF16_F16DOWN ? ORACLE_ROWS_F16 : wfmt; }
+
 /* Step 6 for one token and one expert m of a stack: y = Wd (SiLU(Wg x) * Wu x). */
 static void expert_ffn(int wfmt, int d, int Fh, const void* wg, const void* wu,
                        const void* wd, int64_t m, const double* xt, double* y) {
@@ -289,16 +303,16 @@ static void expert_ffn(int wfmt, int d, int Fh, const void* wg, const void* wu,
 #pragma omp for schedule(static)
         for (int f = 0; f < Fh; ++f) {
             double g = 0.0, u = 0.0;
-            load_row(wfmt, wg, m, Fh, d, f, row);
+            load_row(gate_up_fmt(wfmt), wg, m, Fh, d, f, row);
             for (int i = 0; i < d; ++i) g += row[i] * xt[i];
-            load_row(wfmt, wu, m, Fh, d, f, row);
+            load_row(gate_up_fmt(wfmt), wu, m, Fh, d, f, row);
             for (int i = 0; i < d; ++i) u += row[i] * xt[i];
             h[f] = silu(g) * u;
         }
 #pragma omp for schedule(static)
         for (int j = 0; j < d; ++j) {
             double acc = 0.0;
-            load_row(wfmt, wd, m, d, Fh, j, row);
+            load_row(down_fmt(wfmt), wd, m, d, Fh, j, row);
             for (int f = 0; f < Fh; ++f) acc += row[f] * h[f];
             y[j] = acc;
         }
@@ -321,9 +335,11 @@ int oracle_forward(int d, int E, int k, int F, int S, int Fs, int wfmt,
         return 1;
     if (S > 0 && (Fs <= 0 || !sg || !su || !sd)) return 1;
     if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0 &&
-        wfmt != ORACLE_WFMT_Q5_0 && wfmt != ORACLE_WFMT_Q6_K)
+        wfmt != ORACLE_WFMT_Q5_0 && wfmt != ORACLE_WFMT_Q6_K && wfmt != ORACLE_WFMT_BF16_F16DOWN)
         return 1;
-    if (wfmt != ORACLE_WFMT_BF16 && (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
+    if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_BF16_F16DOWN &&
+        (d % 32 || F % 32 || (S > 0 && Fs % 32)))
+        return 1;
     if (wfmt == ORACLE_WFMT_Q6_K && (d % 256 || F % 256 || (S > 0 && Fs % 256))) return 1;
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);
@@ -373,9 +389,11 @@ int oracle_forward_routed(int d, int E, int k, int F, int S, int Fs, int wfmt,
         return 1;
     if (S > 0 && (Fs <= 0 || !sg || !su || !sd)) return 1;
     if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_Q4_0 && wfmt != ORACLE_WFMT_Q8_0 &&
-        wfmt != ORACLE_WFMT_Q5_0 && wfmt != ORACLE_WFMT_Q6_K)
+        wfmt != ORACLE_WFMT_Q5_0 && wfmt != ORACLE_WFMT_Q6_K && wfmt != ORACLE_WFMT_BF16_F16DOWN)
         return 1;
-    if (wfmt != ORACLE_WFMT_BF16 && (d % 32 || F % 32 || (S > 0 && Fs % 32))) return 1;
+    if (wfmt != ORACLE_WFMT_BF16 && wfmt != ORACLE_WFMT_BF16_F16DOWN &&
+        (d % 32 || F % 32 || (S > 0 && Fs % 32)))
+        return 1;
     if (wfmt == ORACLE_WFMT_Q6_K && (d % 256 || F % 256 || (S > 0 && Fs % 256))) return 1;
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);

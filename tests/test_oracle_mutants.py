@@ -13,10 +13,10 @@ MUTANTS = {
     "silu_sign": ("return z / (1.0 + exp(-z));", "return z / (1.0 + exp(z));"),
     "gate_up_swapped": ("h[f] = silu(g) * u;", "h[f] = silu(u) * g;"),
     "down_transposed": (
-        "load_row(wfmt, wd, m, d, Fh, j, row);\n"
+        "load_row(down_fmt(wfmt), wd, m, d, Fh, j, row);\n"
         "            for (int f = 0; f < Fh; ++f) acc += row[f] * h[f];",
         "for (int f = 0; f < Fh; ++f) {\n"
-        "                load_row(wfmt, wd, m, Fh, d, f, row);\n"
+        "                load_row(down_fmt(wfmt), wd, m, Fh, d, f, row);\n"
         "                acc += row[j] * h[f];\n            }"),
     "shared_dropped": ("for (int i = 0; i < d; ++i) o[i] += y[i];",
                        "for (int i = 0; i < d; ++i) o[i] += 0.0 * y[i];"),
@@ -52,6 +52,8 @@ MUTANTS = {
                                "int s8 = (int)sc[i / 16];"),
     "q6_sub_scale_index": ("int s8 = sc[i / 16] < 128", "int s8 = sc[i / 32] < 128"),
     "q6_odd_quarter_offset": ("ql[64 * h + ((c & 1) ? 32 : 0) + l]", "ql[64 * h + ((c & 1) ? 16 : 0) + l]"),
+    "f16_down_read_as_bf16": ("static int down_fmt(int wfmt) { return wfmt == ORACLE_WFMT_BF16_F16DOWN ? ORACLE_ROWS_F16 : wfmt; }",
+                              "static int down_fmt(int wfmt) { return wfmt == ORACLE_WFMT_BF16_F16DOWN ? ORACLE_WFMT_BF16 : wfmt; }"),
     "routed_weight_ignored": ("o[i] += w[(int64_t)n * k + j] * y[i];", "o[i] += y[i];"),
     "routed_shared_dropped": (
         "expert_ffn(wfmt, d, Fs, sg, su, sd, s2, xt, y);\n"
@@ -74,6 +76,7 @@ def _pins():
         yield (lambda sh=sh: pins.test_brute_force_tiny(sh))
     yield lambda: pins.test_buckets_match_sort(37, 6, 64, 2)
     yield lambda: pins.test_k_equals_E_is_dense_softmax_mixture(synth.WFMT_BF16)
+    yield lambda: pins.test_k_equals_E_is_dense_softmax_mixture(synth.WFMT_BF16_F16DOWN)
     yield lambda: pins.test_single_expert_is_plain_swiglu()
     yield lambda: pins.test_shared_only_when_routed_down_is_zero()
     yield lambda: pins.test_forward_routed_is_weighted_sum_of_ffns(synth.WFMT_BF16)

@@ -46,6 +46,23 @@ def test_fp16_decode_matches_numpy_all_patterns():
     assert np.array_equal(got[~nan], ref[~nan])
 
 
+def test_f16down_inputs_are_the_bf16_draws_rounded_to_fp16():
+    """The fp16 down matrices of the BF16_F16DOWN format are the bf16 draws
+    of the bf16 layer rounded to fp16 (torch's conversion), exactly equal
+    wherever 2^-17 <= |w| <= 65504 (every such bf16 value is an fp16 value)."""
+    sh = synth.MoEShape("conv", T=2, d=256, E=3, k=2, F=64, S=1, Fs=32)
+    a = synth.make_inputs(sh, seed=9)
+    b = synth.make_inputs(sh.replace(wfmt=synth.WFMT_BF16_F16DOWN), seed=9)
+    assert np.array_equal(a.gate, b.gate) and np.array_equal(a.up, b.up)
+    for bf, f16 in ((a.down, b.down), (a.shared_down, b.shared_down)):
+        t = torch.from_numpy(np.ascontiguousarray(bf).view(np.int16)).view(torch.bfloat16)
+        want = t.to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(f16, want)
+        v = t.double().numpy()
+        ok = (np.abs(v) >= 2.0 ** -17) | (v == 0)
+        assert np.array_equal(f16.view(np.float16).astype(np.float64)[ok], v[ok])
+
+
 def test_golden_fixtures_match_their_encoder():
     """The committed fixtures are exactly what make_golden.py (plain struct
     packing of the hand-chosen codes, no oracle code) writes."""
@@ -256,8 +273,15 @@ def _q6_rows(blocks):
     return out
 
 
+_F16_ROWS = "f16"      # down matrices of the BF16_F16DOWN format: IEEE fp16 bits
+
+
 def _mat(inp_arr, wfmt, m, rows, cols):
-    if wfmt == synth.WFMT_BF16:
+    if wfmt == _F16_ROWS:
+        a = inp_arr[m]
+        return [[struct.unpack("<e", struct.pack("<H", int(a[r, c])))[0] for c in range(cols)]
+                for r in range(rows)]
+    if wfmt in (synth.WFMT_BF16, synth.WFMT_BF16_F16DOWN):
         a = inp_arr[m]
         return [[_bf16(a[r, c]) for c in range(cols)] for r in range(rows)]
     if wfmt == synth.WFMT_Q6_K:
@@ -287,13 +311,14 @@ def _brute_layer(inp):
             h.append(g / (1.0 + math.exp(-g)) * u)
         return [sum(down[j][f] * h[f] for f in range(F)) for j in range(d)]
 
+    dfmt = _F16_ROWS if sh.wfmt == synth.WFMT_BF16_F16DOWN else sh.wfmt
     experts = [(_mat(inp.gate, sh.wfmt, e, sh.F, d), _mat(inp.up, sh.wfmt, e, sh.F, d),
-                _mat(inp.down, sh.wfmt, e, d, sh.F)) for e in range(sh.E)]
+                _mat(inp.down, dfmt, e, d, sh.F)) for e in range(sh.E)]
     shared = []
     if inp.shared_gate is not None:
         shared = [(_mat(inp.shared_gate, sh.wfmt, s, sh.Fs, d),
                    _mat(inp.shared_up, sh.wfmt, s, sh.Fs, d),
-                   _mat(inp.shared_down, sh.wfmt, s, d, sh.Fs)) for s in range(sh.S)]
+                   _mat(inp.shared_down, dfmt, s, d, sh.Fs)) for s in range(sh.S)]
     outs, sets, weights = [], [], []
     for t in range(T):
         xt = xs[t]
@@ -331,6 +356,8 @@ TINY = [
                    wfmt=synth.WFMT_Q5_0),
     synth.MoEShape("q6_shared", T=2, d=256, E=3, k=2, F=256, S=1, Fs=256,
                    wfmt=synth.WFMT_Q6_K),
+    synth.MoEShape("f16down_shared", T=2, d=12, E=5, k=2, F=6, S=1, Fs=4,
+                   wfmt=synth.WFMT_BF16_F16DOWN),
 ]
 
 
@@ -357,7 +384,9 @@ def test_brute_force_tiny(sh):
 
 def _f64_stack(arr, wfmt, rows, cols):
     """Dequantise a stack with torch/numpy (library decoders, not the oracle)."""
-    if wfmt == synth.WFMT_BF16:
+    if wfmt == _F16_ROWS:
+        return np.ascontiguousarray(arr).view(np.float16).astype(np.float64).reshape(-1, rows, cols)
+    if wfmt in (synth.WFMT_BF16, synth.WFMT_BF16_F16DOWN):
         t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
         return t.double().numpy().reshape(-1, rows, cols)
     if wfmt == synth.WFMT_Q8_0:
@@ -406,7 +435,7 @@ def _x64(inp):
 
 
 @pytest.mark.parametrize("wfmt", [synth.WFMT_BF16, synth.WFMT_Q4_0, synth.WFMT_Q8_0,
-                                  synth.WFMT_Q5_0, synth.WFMT_Q6_K])
+                                  synth.WFMT_Q5_0, synth.WFMT_Q6_K, synth.WFMT_BF16_F16DOWN])
 def test_k_equals_E_is_dense_softmax_mixture(wfmt):
     big = wfmt == synth.WFMT_Q6_K          # 256-weight super-blocks
     sh = synth.MoEShape("dense", T=5, d=256 if big else 64, E=4, k=4, F=256 if big else 32,
@@ -418,7 +447,7 @@ def test_k_equals_E_is_dense_softmax_mixture(wfmt):
     x = _x64(inp)
     G = _f64_stack(inp.gate, wfmt, sh.F, sh.d)
     U = _f64_stack(inp.up, wfmt, sh.F, sh.d)
-    D = _f64_stack(inp.down, wfmt, sh.d, sh.F)
+    D = _f64_stack(inp.down, _F16_ROWS if wfmt == synth.WFMT_BF16_F16DOWN else wfmt, sh.d, sh.F)
     lg = x @ inp.router_w.astype(np.float64).T
     p = np.exp(lg - lg.max(1, keepdims=True))
     p /= p.sum(1, keepdims=True)
