@@ -249,7 +249,12 @@ def run_reference(args, sh):
 # prefill layer.  The first is the headline line's workload.
 ALL_WORKLOADS = ("mixtral_T8_d4096_E8k2_F14336", "tiny_T4_d256_E8k2_F512",
                  "a3b_T1_d2048_E256k8_F512_S1", "a3b_q4_T1_d2048_E256k8_F512_S1",
-                 "a3b_q4_T8_d2048_E256k8_F512_S1", "deepseek_T4096_d2048_E64k6_F1408_S2")
+                 "a3b_q4_T8_d2048_E256k8_F512_S1", "deepseek_T4096_d2048_E64k6_F1408_S2",
+                 # the other weight formats of the 35B-A3B model's mix, and the
+                 # prefill layer with fp16 down matrices (h in fp16)
+                 "a3b_T8_d2048_E256k8_F512_S1", "a3b_q8_T8_d2048_E256k8_F512_S1",
+                 "a3b_q5_T8_d2048_E256k8_F512_S1",
+                 "deepseek_f16down_T4096_d2048_E64k6_F1408_S2")
 MIN_TIMED_MS = 150.0      # per-workload entries time at least this long (clock samples)
 
 
@@ -284,7 +289,8 @@ class _Setup:
         self.out = torch.empty((sh.T, sh.d), dtype=torch.float32, device=dev)
         self.plan = B.moe_plan_create(first.config(sh.T))
         self.routing = D.Routing(sh.T, sh.k, sh.E, dev)
-        self.prefill = sh.T > B.MOE_DECODE_MAX_T and sh.wfmt == synth.WFMT_BF16
+        self.prefill = sh.T > B.MOE_DECODE_MAX_T and sh.wfmt in (synth.WFMT_BF16,
+                                                                synth.WFMT_BF16_F16DOWN)
 
     def step(self, i, ev_a=None, ev_b=None):
         """One layer call.  Decode: moe_forward (the single fused launch),
@@ -496,7 +502,8 @@ def _entry(su: "_Setup", m: dict, ws: int, peaks):
 
 def _dtype(sh):
     return {synth.WFMT_BF16: "bf16", synth.WFMT_Q4_0: "q4_0/bf16",
-            synth.WFMT_Q8_0: "q8_0/bf16", synth.WFMT_Q5_0: "q5_0/bf16"}[sh.wfmt]
+            synth.WFMT_Q8_0: "q8_0/bf16", synth.WFMT_Q5_0: "q5_0/bf16",
+            synth.WFMT_Q6_K: "q6_k/bf16", synth.WFMT_BF16_F16DOWN: "bf16 (fp16 down)"}[sh.wfmt]
 
 
 def run_b200(args, sh):

@@ -75,12 +75,20 @@ typedef enum moe_status {
  *   5090 page lists q5_0 in the same list of formats; the canonical 22-byte
  *   block is the reading taken).  The kernels read the packed form written by
  *   moe_q5_0_pack.
+ * MOE_WFMT_BF16_F16DOWN: gate and up matrices bf16, every down matrix
+ *   (routed and shared) IEEE fp16 -- the bf16 weights rounded once to fp16
+ *   with moe_bf16_to_f16, exact for 2^-17 <= |w| <= 65504 (below 2^-17 the
+ *   rounding error is at most 2^-25).  The hidden activation h then travels
+ *   between the two prefill GEMMs as fp16 (11 significant bits) instead of
+ *   bf16 (8): the pages have no counterpart; it is the precision headroom of
+ *   the bf16 layer's 2e-3 bound.  Both regimes run it.
  * The quantised formats run in the decode regime only (T <= MOE_DECODE_MAX_T). */
 typedef enum moe_wfmt {
     MOE_WFMT_BF16 = 0,
     MOE_WFMT_Q4_0 = 1,
     MOE_WFMT_Q8_0 = 2,
-    MOE_WFMT_Q5_0 = 3
+    MOE_WFMT_Q5_0 = 3,
+    MOE_WFMT_BF16_F16DOWN = 5
 } moe_wfmt_t;
 
 /* Execution regime.  AUTO picks DECODE for T <= MOE_DECODE_MAX_T (and for
@@ -342,6 +350,14 @@ moe_status_t moe_q5_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
  * tensor-core fragments). */
 moe_status_t moe_q5_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
                            int64_t k, void* codes, void* scales, void* stream);
+
+/* Round n bf16 values (raw bits) to IEEE fp16 (nearest, ties to even) into
+ * dst: the down matrices of MOE_WFMT_BF16_F16DOWN.  Exact for 2^-17 <= |w|
+ * <= 65504 and for zeros; smaller values round to fp16 subnormals (error at
+ * most 2^-25), larger ones to +-inf.  Device pointers, 2-byte aligned, no
+ * overlap; enqueued on `stream`.  INVALID_ARG for n < 0 or NULL pointers
+ * with n > 0.  No counterpart on the pages (see MOE_WFMT_BF16_F16DOWN). */
+moe_status_t moe_bf16_to_f16(const void* src, int64_t n, void* dst, void* stream);
 
 /* Static description of a status code (never NULL).  No counterpart on the
  * pages. */

@@ -67,7 +67,7 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->n_shared > 0 && (c->d_ff_shared < 32 || c->d_ff_shared % 32 != 0))
         return MOE_ERR_INVALID_ARG;
     if (c->wfmt != MOE_WFMT_BF16 && c->wfmt != MOE_WFMT_Q4_0 && c->wfmt != MOE_WFMT_Q8_0 &&
-        c->wfmt != MOE_WFMT_Q5_0)
+        c->wfmt != MOE_WFMT_Q5_0 && c->wfmt != MOE_WFMT_BF16_F16DOWN)
         return MOE_ERR_INVALID_ARG;
     if (c->regime < MOE_REGIME_AUTO || c->regime > MOE_REGIME_PREFILL) return MOE_ERR_INVALID_ARG;
     if (c->device < 0) return MOE_ERR_INVALID_ARG;
@@ -77,14 +77,14 @@ moe_status_t check_config(const moe_config_t* c) {
     if (static_cast<int64_t>(c->n_experts) * c->d_ff >= (1ll << 31) ||
         static_cast<int64_t>(c->n_experts) * c->d_model >= (1ll << 31))
         return MOE_ERR_INVALID_ARG;
-    if (c->wfmt != MOE_WFMT_BF16 && c->regime == MOE_REGIME_PREFILL) return MOE_ERR_UNSUPPORTED;
+    if (wfmt_quantised(c->wfmt) && c->regime == MOE_REGIME_PREFILL) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
 
 bool use_decode(const moe_plan_s* p, int T) {
     if (p->cfg.regime == MOE_REGIME_DECODE) return true;
     if (p->cfg.regime == MOE_REGIME_PREFILL) return false;
-    return T <= MOE_DECODE_MAX_T || p->cfg.wfmt != MOE_WFMT_BF16;
+    return T <= MOE_DECODE_MAX_T || wfmt_quantised(p->cfg.wfmt);
 }
 
 moe_status_t check_matrix(const moe_matrix_t& m, bool quant) {
@@ -104,7 +104,7 @@ moe_status_t check_call(const moe_plan_s* p, const moe_weights_t* w, const void*
     if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
     if (!w->router_w || !aligned16(w->router_w)) return MOE_ERR_INVALID_ARG;
     if (w->router_b && (reinterpret_cast<uintptr_t>(w->router_b) & 3u)) return MOE_ERR_INVALID_ARG;
-    const bool quant = p->cfg.wfmt != MOE_WFMT_BF16;     // quantised: codes + scales
+    const bool quant = wfmt_quantised(p->cfg.wfmt);     // quantised: codes + scales
     moe_status_t s;
     if ((s = check_matrix(w->gate, quant)) || (s = check_matrix(w->up, quant)) ||
         (s = check_matrix(w->down, quant)))
@@ -223,7 +223,7 @@ DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
     memset(&a, 0, sizeof(a));
     const int64_t E = c.n_experts, d = c.d_model, F = c.d_ff, S = c.n_shared, Fs = c.d_ff_shared;
     bool ok = true;
-    if (c.wfmt == MOE_WFMT_BF16) {
+    if (!wfmt_quantised(c.wfmt)) {   // bf16 (fp16 down matrices: the same 2-byte maps)
         ok &= map_bf16(p, &a.tm_gate, w->gate.data, E, F, d, 64, fs);
         ok &= map_bf16(p, &a.tm_up, w->up.data, E, F, d, 64, fs);
         ok &= map_bf16(p, &a.tm_down, w->down.data, E, d, F, fs, 128);
@@ -426,7 +426,7 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     // workspace: one allocation, carved into 256-byte aligned pieces
     const int64_t T = cfg->t_max, E = cfg->n_experts, k = cfg->top_k, d = cfg->d_model;
     const int64_t S = cfg->n_shared, Fs = cfg->d_ff_shared, F = cfg->d_ff;
-    const bool prefill = cfg->wfmt == MOE_WFMT_BF16 &&
+    const bool prefill = !wfmt_quantised(cfg->wfmt) &&
                          (cfg->regime == MOE_REGIME_PREFILL ||
                           (cfg->regime == MOE_REGIME_AUTO && cfg->t_max > MOE_DECODE_MAX_T));
     size_t off = 0;
@@ -605,6 +605,16 @@ moe_status_t moe_debug_stall_barrier(moe_plan_t p, void* stream) {
     cudaError_t e = cudaMemsetAsync(p->ws.gbar, 0, 16, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = cudaMemsetAsync(p->ws.gbar, 0x01, 1, static_cast<cudaStream_t>(stream));
     return cuda_status(e);
+}
+
+moe_status_t moe_bf16_to_f16(const void* src, int64_t n, void* dst, void* stream) {
+    if (n < 0) return MOE_ERR_INVALID_ARG;
+    if (n == 0) return MOE_OK;
+    if (!src || !dst || (reinterpret_cast<uintptr_t>(src) & 1u) || (reinterpret_cast<uintptr_t>(dst) & 1u))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_bf16_to_f16(static_cast<const uint16_t*>(src), n,
+                                          static_cast<uint16_t*>(dst),
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_q4_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k, size_t* code_bytes,

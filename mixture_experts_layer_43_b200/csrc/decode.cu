@@ -223,6 +223,7 @@ constexpr int kDecodeThreads = kConsumers + 32;   // + one producer warp
 // Weight formats of the decode kernels (the values of moe_wfmt_t).
 constexpr int kWfBf16 = 0, kWfQ4 = 1, kWfQ8 = 2;
 constexpr int kWfQ5 = 3;
+constexpr int kWfF16d = 5;   // bf16 gate/up, fp16 down matrices (h travels in fp16)
 
 // The constant that turns the bf16 "128 + nibble" operands back into signed
 // codes (see q4_raw): Q4_0 subtracts 128 + 8; Q8_0, whose biased byte
@@ -237,7 +238,10 @@ struct DecodeCfg {
     static constexpr int ROLES = 2 * RG;          // (matrix, row group) pairs of phase A
     static constexpr int KSPLIT = kConsumerWarps / ROLES;
     static_assert(KSPLIT >= 1 && ROLES * KSPLIT == kConsumerWarps, "warp roles");
-    static constexpr bool QUANT = WF != kWfBf16;
+    static constexpr bool QUANT = WF == kWfQ4 || WF == kWfQ8 || WF == kWfQ5;
+    // bf16 phase A with fp16 down matrices: h is stored as an fp16 hi + lo
+    // pair and the down contraction runs on fp16 operands
+    static constexpr bool HALF_DOWN = WF == kWfF16d;
     static_assert(!QUANT || FS >= 32, "quantised slices hold whole blocks");
     // fp16 tensor-core operands (see q4h_lo): x staged as fp16, h as an fp16
     // hi + lo pair, per-block corrections with two code bases
@@ -523,14 +527,14 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
         for (int c = 0; c < 4; ++c) {
             const uint4 v = __ldg(src + c);
             dst[c] = v;
-            if constexpr (WF != kWfBf16) {
+            if constexpr (WF == kWfQ8 || WF == kWfQ5) {
                 const uint32_t q[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     s += __uint_as_float(q[j] << 16) + __uint_as_float(q[j] & 0xffff0000u);
             }
         }
-        if constexpr (WF != kWfBf16) sm.xsum[t * nkb + kb] = -quant_offset(WF) * s;
+        if constexpr (WF == kWfQ8 || WF == kWfQ5) sm.xsum[t * nkb + kb] = -quant_offset(WF) * s;
     }
 }
 
@@ -812,6 +816,12 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                 uv += gu[((q * 2 + 1) * kDecodeTok + t) * C::GS + f];
             }
             const float h = gv / (1.f + expf(-gv)) * uv;
+            if constexpr (C::HALF_DOWN) {
+                const __half hi = __float2half_rn(h);
+                reinterpret_cast<__half*>(hhi)[t * C::HS + f] = hi;
+                reinterpret_cast<__half*>(hlo)[t * C::HS + f] = __float2half_rn(h - __half2float(hi));
+                continue;
+            }
             const __nv_bfloat16 hi = __float2bfloat16_rn(h);
             const __nv_bfloat16 lo = __float2bfloat16_rn(h - __bfloat162float(hi));
             hhi[t * C::HS + f] = hi;
@@ -858,8 +868,13 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         for (int kk = 0; kk < C::RG; ++kk) {
                             uint32_t a0, a1, a2, a3;
                             ldsm_x4(tile + swz_offset(arow, kk * 2 + (m >> 1), FS * 2), a0, a1, a2, a3);
-                            mma_bf16_16816(c, a0, a1, a2, a3, bh[kk][0], bh[kk][1]);
-                            mma_bf16_16816(c, a0, a1, a2, a3, bl[kk][0], bl[kk][1]);
+                            if constexpr (C::HALF_DOWN) {
+                                mma_f16_16816_acc(c, a0, a1, a2, a3, bh[kk][0], bh[kk][1]);
+                                mma_f16_16816_acc(c, a0, a1, a2, a3, bl[kk][0], bl[kk][1]);
+                            } else {
+                                mma_bf16_16816(c, a0, a1, a2, a3, bh[kk][0], bh[kk][1]);
+                                mma_bf16_16816(c, a0, a1, a2, a3, bl[kk][0], bl[kk][1]);
+                            }
                         }
                     } else {
                         constexpr int QB = kQuantDownBoxRows;
@@ -1577,6 +1592,8 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, int wfmt, int grid,
     switch (wfmt * 100 + fs) {
         case kWfBf16 * 100 + 64: return launch_fused_one<64, kWfBf16>(a, grid, smem, stream);
         case kWfBf16 * 100 + 32: return launch_fused_one<32, kWfBf16>(a, grid, smem, stream);
+        case kWfF16d * 100 + 64: return launch_fused_one<64, kWfF16d>(a, grid, smem, stream);
+        case kWfF16d * 100 + 32: return launch_fused_one<32, kWfF16d>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_fused_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_fused_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_fused_one<32, kWfQ8>(a, grid, smem, stream);
@@ -1591,6 +1608,8 @@ cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, int wfmt, int gri
     switch (wfmt * 100 + fs) {
         case kWfBf16 * 100 + 64: return launch_one<64, kWfBf16>(a, grid, smem, stream);
         case kWfBf16 * 100 + 32: return launch_one<32, kWfBf16>(a, grid, smem, stream);
+        case kWfF16d * 100 + 64: return launch_one<64, kWfF16d>(a, grid, smem, stream);
+        case kWfF16d * 100 + 32: return launch_one<32, kWfF16d>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_one<32, kWfQ8>(a, grid, smem, stream);

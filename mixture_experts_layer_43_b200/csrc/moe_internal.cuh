@@ -123,6 +123,12 @@ cudaError_t launch_q8_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
                              uint8_t* codes, uint16_t* scales, cudaStream_t stream);
 cudaError_t launch_q5_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
                              uint8_t* codes, uint8_t* aux, cudaStream_t stream);
+cudaError_t launch_bf16_to_f16(const uint16_t* src, int64_t n, uint16_t* dst, cudaStream_t stream);
+
+// Formats whose matrices are quantised blocks (codes + scales).
+inline bool wfmt_quantised(int wfmt) {
+    return wfmt == MOE_WFMT_Q4_0 || wfmt == MOE_WFMT_Q8_0 || wfmt == MOE_WFMT_Q5_0;
+}
 
 // --------------------------------------------------------- device helpers
 #ifdef __CUDACC__
@@ -310,6 +316,13 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
 }
 
+// The same with fp16 A and B (format bits 0).
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
+    return (1u << 4)                                   // D format f32
+         | (static_cast<uint32_t>(N >> 3) << 17)       // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);      // M / 16
+}
+
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                           uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -430,6 +443,11 @@ __device__ __forceinline__ void warp_topk_any(const float* row, int E, int k, in
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 #endif  // __CUDACC__

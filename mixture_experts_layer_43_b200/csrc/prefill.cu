@@ -457,6 +457,7 @@ struct GemmArgs {
     float* out;                     // [T][d]
     uint32_t* err;
     int T, d, E, S, F, Fs;
+    int f16;                        // h and the down matrices fp16 (else bf16)
 };
 
 struct GemmTile {
@@ -639,7 +640,9 @@ prefill_gemm_kernel(const __grid_constant__ GemmArgs a) {
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA
         if (lane == 0 && rank == 0) {
-            constexpr uint32_t idesc = umma_idesc_bf16(C::BM, kBN);
+            // operand types: bf16, except fp16 h and down matrices in the down GEMM
+            const uint32_t idesc = (MODE == kDown && a.f16) ? umma_idesc_f16(C::BM, kBN)
+                                                            : umma_idesc_bf16(C::BM, kBN);
             uint32_t it = 0;
             int local = 0;
             for (int t = unit; t < n_tiles && !*abort_flag; t += n_units, ++local) {
@@ -715,8 +718,9 @@ prefill_gemm_kernel(const __grid_constant__ GemmArgs a) {
                         for (int i = 0; i < 16; ++i) {
                             const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
                             const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
-                            pk[i] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0,
-                                                g1 / (1.f + __expf(-g1)) * u1);
+                            const float h0 = g0 / (1.f + __expf(-g0)) * u0;
+                            const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+                            pk[i] = a.f16 ? pack_f16x2(h0, h1) : pack_bf16x2(h0, h1);
                         }
                         uint4* dst = reinterpret_cast<uint4*>(hrow + 32 * c);
 #pragma unroll
@@ -965,6 +969,7 @@ moe_status_t prefill_experts(PrefillState* st, const moe_config_t& c, const Work
         g->out = out;
         g->err = ws.err;
         g->T = T; g->d = d; g->E = E; g->S = S; g->F = F; g->Fs = Fs;
+        g->f16 = c.wfmt == MOE_WFMT_BF16_F16DOWN ? 1 : 0;
     }
     st->g1.tile_base = ws.tiles;
     st->g2.tile_base = ws.tiles + E + 1;

@@ -197,4 +197,24 @@ cudaError_t launch_q5_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
     return cudaGetLastError();
 }
 
+// ---- bf16 -> fp16 (the down matrices of MOE_WFMT_BF16_F16DOWN)
+__global__ void bf16_to_f16_kernel(const uint16_t* __restrict__ src, int64_t n,
+                                   uint16_t* __restrict__ dst) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float v = __uint_as_float(static_cast<uint32_t>(src[i]) << 16);
+        const __half h = __float2half_rn(v);
+        dst[i] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+}
+
+cudaError_t launch_bf16_to_f16(const uint16_t* src, int64_t n, uint16_t* dst, cudaStream_t stream) {
+    if (n == 0) return cudaSuccess;
+    const int threads = 256;
+    const int64_t want = (n + threads - 1) / threads;
+    const int grid = static_cast<int>(want < 65536 ? want : 65536);
+    bf16_to_f16_kernel<<<grid, threads, 0, stream>>>(src, n, dst);
+    return cudaGetLastError();
+}
+
 }  // namespace moe

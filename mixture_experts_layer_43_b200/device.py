@@ -29,9 +29,12 @@ class DeviceLayer:
         sh = inp.shape
         self.shape = sh
         self.device = torch.device(device)
-        self.q4 = sh.wfmt != synth.WFMT_BF16          # quantised: codes + scales
+        # quantised: codes + scales (bf16, and bf16 with fp16 down matrices,
+        # upload as they are)
+        self.q4 = sh.wfmt in (synth.WFMT_Q4_0, synth.WFMT_Q8_0, synth.WFMT_Q5_0)
         packed_bytes, pack = {
             synth.WFMT_BF16: (None, None),
+            synth.WFMT_BF16_F16DOWN: (None, None),
             synth.WFMT_Q4_0: (B.moe_q4_0_packed_bytes, B.moe_q4_0_pack),
             synth.WFMT_Q8_0: (B.moe_q8_0_packed_bytes, B.moe_q8_0_pack),
             synth.WFMT_Q5_0: (B.moe_q5_0_packed_bytes, B.moe_q5_0_pack)}[sh.wfmt]
@@ -108,22 +111,29 @@ def random_bf16_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") 
     make_inputs with this seed) and whose expert weights are drawn on the
     device from a seeded N(0, w_std) generator -- for timing sweeps where the
     weight values do not matter and host generation would dominate."""
-    assert shape.wfmt == synth.WFMT_BF16
+    assert shape.wfmt in (synth.WFMT_BF16, synth.WFMT_BF16_F16DOWN)
     inp = synth.make_inputs(shape, seed=seed, x_only=True)
     dev = torch.device(device)
     gen = torch.Generator(device=dev)
     gen.manual_seed(seed)
 
-    def mats(n, rows, cols):
+    def mats(n, rows, cols, down=False):
         t = torch.randn((n, rows, cols), generator=gen, device=dev, dtype=torch.float32)
-        return (t * shape.w_std).to(torch.bfloat16).view(torch.int16)
+        t = (t * shape.w_std).to(torch.bfloat16).view(torch.int16)
+        if down and shape.wfmt == synth.WFMT_BF16_F16DOWN:
+            # the library's own rounding of the bf16 draws to fp16
+            h = torch.empty_like(t)
+            B.moe_bf16_to_f16(t.data_ptr(), t.numel(), h.data_ptr(),
+                              torch.cuda.current_stream(dev).cuda_stream)
+            return h
+        return t
 
     L = DeviceLayer.__new__(DeviceLayer)
     L.shape, L.device, L.q4 = shape, dev, False
     L.router_w = _dev(inp.router_w.astype(np.float32), dev)
     L.router_b = None if inp.router_b is None else _dev(inp.router_b.astype(np.float32), dev)
     E, F, d, S, Fs = shape.E, shape.F, shape.d, shape.S, shape.Fs
-    L._keep = [mats(E, F, d), mats(E, F, d), mats(E, d, F)]
+    L._keep = [mats(E, F, d), mats(E, F, d), mats(E, d, F, down=True)]
     w = B.moe_weights_t()
     w.router_w = L.router_w.data_ptr()
     w.router_b = L.router_b.data_ptr() if L.router_b is not None else None
@@ -132,7 +142,7 @@ def random_bf16_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") 
     w.down = B.moe_matrix_t(L._keep[2].data_ptr(), None)
     L.n_shared = 0
     if S:
-        L._keep += [mats(S, Fs, d), mats(S, Fs, d), mats(S, d, Fs)]
+        L._keep += [mats(S, Fs, d), mats(S, Fs, d), mats(S, d, Fs, down=True)]
         w.shared_gate = B.moe_matrix_t(L._keep[3].data_ptr(), None)
         w.shared_up = B.moe_matrix_t(L._keep[4].data_ptr(), None)
         w.shared_down = B.moe_matrix_t(L._keep[5].data_ptr(), None)
@@ -149,7 +159,7 @@ def random_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") -> De
     with codes uniform on their range and scales |N(0, std)| as fp16, then
     repacked by the library's own packer.  For timing, where the weight
     values do not matter and host generation would dominate."""
-    if shape.wfmt == synth.WFMT_BF16:
+    if shape.wfmt in (synth.WFMT_BF16, synth.WFMT_BF16_F16DOWN):
         return random_bf16_layer(shape, seed, device)[0]
     inp = synth.make_inputs(shape, seed=seed, x_only=True)
     dev = torch.device(device)

@@ -63,6 +63,21 @@ def test_plan_create_q4_prefill_unsupported(L):
     assert s == B.MOE_ERR_UNSUPPORTED
     s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=3, regime=2)), ctypes.byref(plan))
     assert s == B.MOE_ERR_UNSUPPORTED
+    # bf16 with fp16 down matrices is a valid prefill format (without a GPU the
+    # call gets past the argument checks and fails at the device query)
+    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=5, regime=2)), ctypes.byref(plan))
+    assert s not in (B.MOE_ERR_UNSUPPORTED, B.MOE_ERR_INVALID_ARG)
+    # 4 is not a format of this ABI
+    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=4)), ctypes.byref(plan))
+    assert s == B.MOE_ERR_INVALID_ARG
+
+
+def test_bf16_to_f16_rejects_bad_args_without_gpu(L):
+    assert L.moe_bf16_to_f16(None, -1, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_bf16_to_f16(None, 4, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_bf16_to_f16(None, 0, None, None) == B.MOE_OK
+    assert L.moe_bf16_to_f16(ctypes.c_void_p(0x1001), 4, ctypes.c_void_p(0x2000), None) == \
+        B.MOE_ERR_INVALID_ARG
 
 
 def test_null_arguments(L):

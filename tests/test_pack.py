@@ -1,4 +1,5 @@
-"""GPU test of the repacking kernels (moe_q4_0_pack, moe_q8_0_pack, moe_q5_0_pack):
+"""GPU test of the repacking kernels (moe_q4_0_pack, moe_q8_0_pack, moe_q5_0_pack,
+moe_bf16_to_f16):
 byte work, so bit-exact.  The packed arrays are decoded here with numpy by
 inverting the layout include/moe.h documents, and the codes and scales must
 equal those of the canonical blocks exactly."""
@@ -100,4 +101,20 @@ def test_q5_0_pack_is_the_documented_records(n_mats, rows, k):
     assert np.array_equal(got, want)
     want_sc = canon[..., :2].copy().view(np.uint16)[..., 0]
     assert np.array_equal(sc.transpose(0, 2, 1), want_sc)
+
+
+def test_bf16_to_f16_every_pattern():
+    """The library's bf16 -> fp16 rounding equals torch's (round to nearest
+    even) bit for bit on all 65536 bf16 patterns (NaN stays NaN)."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    src = torch.from_numpy(bits.view(np.int16)).cuda()
+    dst = torch.zeros_like(src)
+    B.moe_bf16_to_f16(src.data_ptr(), src.numel(), dst.data_ptr(),
+                      torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    want = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float16)
+    got = dst.cpu().view(torch.float16)
+    nan = torch.isnan(want)
+    assert torch.equal(torch.isnan(got), nan)
+    assert torch.equal(got[~nan].view(torch.int16), want[~nan].view(torch.int16))
 

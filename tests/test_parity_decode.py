@@ -48,6 +48,11 @@ SMALL = [
                    wfmt=synth.WFMT_Q5_0),
     synth.MoEShape("max_limits_q5", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32,
                    wfmt=synth.WFMT_Q5_0),
+    # bf16 gate/up with fp16 down matrices (h in fp16): 32- and 64-row slices
+    synth.MoEShape("ragged_f16down", T=3, d=384, E=5, k=3, F=96, S=1, Fs=64,
+                   wfmt=synth.WFMT_BF16_F16DOWN),
+    synth.MoEShape("multi_unit_f16down", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512,
+                   wfmt=synth.WFMT_BF16_F16DOWN),
 ]
 
 

@@ -19,6 +19,8 @@ from mixture_experts_layer_43_b200 import synth
 from gpu_util import W_ABS, TOL, check_tie_choice, run_gpu, w_rtol, waived_tokens
 
 PREFILL_TRIPWIRE = 1.8e-3
+# with fp16 down matrices h travels in fp16 (11 significant bits, not 8)
+F16DOWN_TRIPWIRE = 5e-4
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +31,7 @@ def _gpu():
         pytest.skip("needs a CUDA device")
 
 
-def _check(sh, seed=0, regime=B.MOE_REGIME_PREFILL, sample=None):
+def _check(sh, seed=0, regime=B.MOE_REGIME_PREFILL, sample=None, tripwire=PREFILL_TRIPWIRE):
     inp = synth.make_inputs(sh, seed=seed)
     layer = D.DeviceLayer(inp)
     out, routing, launches = run_gpu(layer, inp.x, sh.T, regime=regime)
@@ -62,7 +64,7 @@ def _check(sh, seed=0, regime=B.MOE_REGIME_PREFILL, sample=None):
                                           tokens=tok[flip])
     err = float(np.linalg.norm(out[tok] - ref) / np.linalg.norm(ref))
     assert err <= TOL[sh.wfmt], f"relative L2 error {err:.3e}"
-    assert err <= PREFILL_TRIPWIRE, f"relative L2 error {err:.3e} above the regression tripwire"
+    assert err <= tripwire, f"relative L2 error {err:.3e} above the regression tripwire"
     assert np.all(np.isfinite(out))
     return err
 
@@ -100,3 +102,26 @@ def test_prefill_deepseek_full_size():
     sh = synth.WORKLOADS["deepseek_T4096_d2048_E64k6_F1408_S2"]
     err = _check(sh, seed=0, sample=256)
     print(f"deepseek T=4096: rel L2 {err:.3e} on 256 sampled tokens")
+
+
+F16DOWN = [
+    synth.MoEShape("f16down_ragged", T=37, d=256, E=8, k=2, F=128, S=1, Fs=192,
+                   wfmt=synth.WFMT_BF16_F16DOWN),
+    synth.MoEShape("f16down_cta_pairs", T=2300, d=512, E=4, k=2, F=384, S=1, Fs=256,
+                   wfmt=synth.WFMT_BF16_F16DOWN),
+]
+
+
+@pytest.mark.parametrize("sh", F16DOWN, ids=[s.name for s in F16DOWN])
+def test_prefill_f16down_small_shapes(sh):
+    err = _check(sh, seed=3, tripwire=F16DOWN_TRIPWIRE)
+    print(f"{sh.name}: rel L2 {err:.3e}")
+
+
+def test_prefill_deepseek_f16down_full_size():
+    """The DeepSeek-shaped prefill layer with fp16 down matrices: the same
+    bf16 draws, h in fp16 between the GEMMs."""
+    sh = synth.WORKLOADS["deepseek_f16down_T4096_d2048_E64k6_F1408_S2"]
+    err = _check(sh, seed=0, sample=256, tripwire=F16DOWN_TRIPWIRE)
+    print(f"deepseek f16down T=4096: rel L2 {err:.3e} on 256 sampled tokens")
+
