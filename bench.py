@@ -253,7 +253,7 @@ ALL_WORKLOADS = ("mixtral_T8_d4096_E8k2_F14336", "tiny_T4_d256_E8k2_F512",
                  # the other weight formats of the 35B-A3B model's mix, and the
                  # prefill layer with fp16 down matrices (h in fp16)
                  "a3b_T8_d2048_E256k8_F512_S1", "a3b_q8_T8_d2048_E256k8_F512_S1",
-                 "a3b_q5_T8_d2048_E256k8_F512_S1",
+                 "a3b_q5_T8_d2048_E256k8_F512_S1", "a3b_q6_T8_d2048_E256k8_F512_S1",
                  "deepseek_f16down_T4096_d2048_E64k6_F1408_S2")
 MIN_TIMED_MS = 150.0      # per-workload entries time at least this long (clock samples)
 

@@ -75,6 +75,13 @@ typedef enum moe_status {
  *   5090 page lists q5_0 in the same list of formats; the canonical 22-byte
  *   block is the reading taken).  The kernels read the packed form written by
  *   moe_q5_0_pack.
+ * MOE_WFMT_Q6_K: super-blocks of 256 consecutive weights along the reduction
+ *   dim, each an fp16 scale d, 16 signed 8-bit sub-block scales (one per 16
+ *   weights) and 256 6-bit codes q in 0..63, weight = d * sc * (q - 32) (the
+ *   5090 page lists q6_K among the formats of the 35B-A3B model; the
+ *   canonical 210-byte super-block is the reading taken).  The reduction dim
+ *   must be a multiple of 256 and every matrix's row count of 16.  The
+ *   kernels read the packed form written by moe_q6_k_pack.
  * MOE_WFMT_BF16_F16DOWN: gate and up matrices bf16, every down matrix
  *   (routed and shared) IEEE fp16 -- the bf16 weights rounded once to fp16
  *   with moe_bf16_to_f16, exact for 2^-17 <= |w| <= 65504 (below 2^-17 the
@@ -88,6 +95,7 @@ typedef enum moe_wfmt {
     MOE_WFMT_Q4_0 = 1,
     MOE_WFMT_Q8_0 = 2,
     MOE_WFMT_Q5_0 = 3,
+    MOE_WFMT_Q6_K = 4,
     MOE_WFMT_BF16_F16DOWN = 5
 } moe_wfmt_t;
 
@@ -350,6 +358,35 @@ moe_status_t moe_q5_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
  * tensor-core fragments). */
 moe_status_t moe_q5_0_pack(const void* blocks, int64_t n_mats, int64_t rows,
                            int64_t k, void* codes, void* scales, void* stream);
+
+/* Bytes of the packed q6_K form of n_mats matrices of [rows][k] weights:
+ * code_bytes = 16 per 32 weights (the low 4 bits), scale_bytes = 160 per 32
+ * weights and 16 rows (high bits and sub-block scales) followed by 2 per row
+ * and 256 weights (super-block scales).  k must be a multiple of 256 and rows
+ * of 16 (every matrix of a q6_K layer qualifies: d a multiple of 256, F and
+ * Fs multiples of 256).  Returns INVALID_ARG otherwise.  (q6_K is in the
+ * 5090 page's list of the model's formats.) */
+moe_status_t moe_q6_k_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
+                                   size_t* code_bytes, size_t* scale_bytes);
+
+/* Repack canonical q6_K super-blocks ([n_mats][rows][k/256] super-blocks of
+ * 210 bytes: ql[128], qh[64], 16 int8 sub-block scales, fp16 scale; element
+ * i = 128h + 32c + l takes its low 4 bits from the low (c < 2) or high
+ * nibble of ql[64h + 32(c%2) + l] and its high 2 bits from bits 2c, 2c+1 of
+ * qh[32h + l]) into the kernel layout:
+ *   codes  [n_mats][k/32][rows][16 bytes]: the low 4 bits, permuted exactly
+ *          like the Q4_0 codes;
+ *   scales [n_mats][k/32][rows/16][160 bytes]: per block and 16-row group,
+ *          32 words of high bits (word 4g+t: lane t's codes of rows g and
+ *          g+8, the code in nibble n of row g's code word at bit
+ *          {4,8,6,10,20,24,22,26}[n], row g+8's 8 bits higher, mod 32), then
+ *          per g the two int8 sub-block scales of row g and of row g+8;
+ *          followed by [n_mats][k/256][rows] fp16 super-block scales.
+ * Same 6.5625 bits per weight.  Device pointers; `codes`/`scales` 16-byte
+ * aligned.  Enqueued on `stream`.  The pages have no counterpart to this
+ * repacking (it serves the kernels' tensor-core fragments). */
+moe_status_t moe_q6_k_pack(const void* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                           void* codes, void* scales, void* stream);
 
 /* Round n bf16 values (raw bits) to IEEE fp16 (nearest, ties to even) into
  * dst: the down matrices of MOE_WFMT_BF16_F16DOWN.  Exact for 2^-17 <= |w|

@@ -28,6 +28,7 @@ MOE_WFMT_BF16 = 0
 MOE_WFMT_Q4_0 = 1
 MOE_WFMT_Q8_0 = 2
 MOE_WFMT_Q5_0 = 3
+MOE_WFMT_Q6_K = 4
 MOE_WFMT_BF16_F16DOWN = 5
 MOE_REGIME_AUTO = 0
 MOE_REGIME_DECODE = 1
@@ -118,6 +119,11 @@ def lib() -> ctypes.CDLL:
     L.moe_q5_0_packed_bytes.restype = S
     L.moe_q5_0_pack.argtypes = [P, I64, I64, I64, P, P, P]
     L.moe_q5_0_pack.restype = S
+    L.moe_q6_k_packed_bytes.argtypes = [I64, I64, I64, ctypes.POINTER(ctypes.c_size_t),
+                                        ctypes.POINTER(ctypes.c_size_t)]
+    L.moe_q6_k_packed_bytes.restype = S
+    L.moe_q6_k_pack.argtypes = [P, I64, I64, I64, P, P, P]
+    L.moe_q6_k_pack.restype = S
     L.moe_bf16_to_f16.argtypes = [P, I64, P, P]
     L.moe_bf16_to_f16.restype = S
     _lib = L
@@ -232,6 +238,18 @@ def moe_q5_0_packed_bytes(n_mats: int, rows: int, k: int):
 def moe_q5_0_pack(blocks: int, n_mats: int, rows: int, k: int, codes: int, scales: int,
                   stream: int = 0) -> None:
     _check(lib().moe_q5_0_pack(blocks, n_mats, rows, k, codes, scales, stream), "moe_q5_0_pack")
+
+
+def moe_q6_k_packed_bytes(n_mats: int, rows: int, k: int):
+    cb, sb = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().moe_q6_k_packed_bytes(n_mats, rows, k, ctypes.byref(cb), ctypes.byref(sb)),
+           "moe_q6_k_packed_bytes")
+    return cb.value, sb.value
+
+
+def moe_q6_k_pack(blocks: int, n_mats: int, rows: int, k: int, codes: int, scales: int,
+                  stream: int = 0) -> None:
+    _check(lib().moe_q6_k_pack(blocks, n_mats, rows, k, codes, scales, stream), "moe_q6_k_pack")
 
 
 def moe_bf16_to_f16(src: int, n: int, dst: int, stream: int = 0) -> None:

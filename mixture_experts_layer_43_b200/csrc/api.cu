@@ -67,7 +67,11 @@ moe_status_t check_config(const moe_config_t* c) {
     if (c->n_shared > 0 && (c->d_ff_shared < 32 || c->d_ff_shared % 32 != 0))
         return MOE_ERR_INVALID_ARG;
     if (c->wfmt != MOE_WFMT_BF16 && c->wfmt != MOE_WFMT_Q4_0 && c->wfmt != MOE_WFMT_Q8_0 &&
-        c->wfmt != MOE_WFMT_Q5_0 && c->wfmt != MOE_WFMT_BF16_F16DOWN)
+        c->wfmt != MOE_WFMT_Q5_0 && c->wfmt != MOE_WFMT_Q6_K && c->wfmt != MOE_WFMT_BF16_F16DOWN)
+        return MOE_ERR_INVALID_ARG;
+    // q6_K super-blocks run along the reduction dim of every matrix
+    if (c->wfmt == MOE_WFMT_Q6_K &&
+        (c->d_model % 256 || c->d_ff % 256 || (c->n_shared > 0 && c->d_ff_shared % 256)))
         return MOE_ERR_INVALID_ARG;
     if (c->regime < MOE_REGIME_AUTO || c->regime > MOE_REGIME_PREFILL) return MOE_ERR_INVALID_ARG;
     if (c->device < 0) return MOE_ERR_INVALID_ARG;
@@ -175,6 +179,29 @@ bool map_quant_scales(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t m
                       CU_TENSOR_MAP_SWIZZLE_NONE, 2 * box_rows);
 }
 
+// q6_K packed records [mats][K/32][N/16][160 bytes] seen as 3D {160, N/16,
+// mats*K/32}; a box of box_rows rows reads box_rows/16 records.
+bool map_q6_aux(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
+                int64_t K, uint32_t box_rows, uint32_t box_kb) {
+    uint64_t dims[3] = {160, static_cast<uint64_t>(N / 16), static_cast<uint64_t>(mats * (K / 32))};
+    uint64_t strides[2] = {160, static_cast<uint64_t>(N / 16) * 160};
+    uint32_t box[3] = {160, box_rows / 16, box_kb};
+    return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, 10 * box_rows);   // records are contiguous
+}
+
+// q6_K super-block scales [mats][K/256][N] fp16 seen as 2D {N, mats*K/256};
+// they follow the records in the packed scales array.
+bool map_q6_d(moe_plan_s* p, CUtensorMap* m, const void* scales, int64_t mats, int64_t N, int64_t K,
+              uint32_t box_rows, uint32_t box_sb) {
+    const uint8_t* base = static_cast<const uint8_t*>(scales) + mats * (N / 16) * (K / 32) * 160;
+    uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(mats * (K / 256))};
+    uint64_t strides[1] = {static_cast<uint64_t>(N) * 2};
+    uint32_t box[2] = {box_rows, box_sb};
+    return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, 2 * box_rows);
+}
+
 // Q5_0 packed scales and fifth bits [mats][K/32][N/8][48 bytes] seen as 3D
 // {48, N/8, mats*K/32}; a box of box_rows rows reads box_rows/8 records.
 bool map_q5_aux(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
@@ -200,7 +227,7 @@ int pick_fs(const moe_plan_s* p, int T) {
     double best_eff = -1.0;
     // Q4_0's row-streaming pipeline keeps every row group's partial sums in
     // registers, which fit for 32-row slices only
-    if (c.wfmt == MOE_WFMT_Q4_0) return 32;
+    if (c.wfmt == MOE_WFMT_Q4_0 || c.wfmt == MOE_WFMT_Q6_K) return 32;
     for (int fs : {64, 32}) {
         if (c.d_ff % fs || (c.n_shared && c.d_ff_shared % fs)) continue;
         const double units = act * (c.d_ff / fs) + c.n_shared * (c.n_shared ? c.d_ff_shared / fs : 0);
@@ -236,7 +263,7 @@ DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
         // phase-A boxes: Q4_0 streams 16-row groups over up to 64 block
         // columns (the row-streaming pipeline); the other formats stream
         // 512 / fs block columns of the whole slice
-        const bool rows16 = c.wfmt == MOE_WFMT_Q4_0;
+        const bool rows16 = c.wfmt == MOE_WFMT_Q4_0 || c.wfmt == MOE_WFMT_Q6_K;
         const uint32_t kb = rows16 ? static_cast<uint32_t>(d / 32 < 64 ? d / 32 : 64) : 512 / fs;
         const uint32_t ar = rows16 ? 16 : fs;
         const uint32_t nb = fs / 32;
@@ -245,9 +272,22 @@ DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
         // scales: fp16 [mats][K/32][N], or Q5_0's 48-byte records of 8 rows
         auto scales = [&](CUtensorMap* m, const void* base, int64_t mats, int64_t N, int64_t K,
                           uint32_t box_rows, uint32_t box_kb) {
+            if (c.wfmt == MOE_WFMT_Q6_K) return map_q6_aux(p, m, base, mats, N, K, box_rows, box_kb);
             return c.wfmt == MOE_WFMT_Q5_0 ? map_q5_aux(p, m, base, mats, N, K, box_rows, box_kb)
                                            : map_quant_scales(p, m, base, mats, N, K, box_rows, box_kb);
         };
+        if (c.wfmt == MOE_WFMT_Q6_K) {
+            // super-block scales: phase A 16 rows x kb/8 super-blocks, phase B
+            // 256 rows x the one super-block a slice lies in
+            ok &= map_q6_d(p, &a.tm_gate_d, w->gate.scales, E, F, d, 16, kb / 8);
+            ok &= map_q6_d(p, &a.tm_up_d, w->up.scales, E, F, d, 16, kb / 8);
+            ok &= map_q6_d(p, &a.tm_down_d, w->down.scales, E, d, F, kQuantDownBoxRows, 1);
+            if (S) {
+                ok &= map_q6_d(p, &a.tm_sgate_d, w->shared_gate.scales, S, Fs, d, 16, kb / 8);
+                ok &= map_q6_d(p, &a.tm_sup_d, w->shared_up.scales, S, Fs, d, 16, kb / 8);
+                ok &= map_q6_d(p, &a.tm_sdown_d, w->shared_down.scales, S, d, Fs, kQuantDownBoxRows, 1);
+            }
+        }
         ok &= map_quant_codes(p, &a.tm_gate, w->gate.data, E, F, d, ar, kb, cb);
         ok &= map_quant_codes(p, &a.tm_up, w->up.data, E, F, d, ar, kb, cb);
         ok &= map_quant_codes(p, &a.tm_down, w->down.data, E, d, F, kQuantDownBoxRows, nb, cb);
@@ -605,6 +645,27 @@ moe_status_t moe_debug_stall_barrier(moe_plan_t p, void* stream) {
     cudaError_t e = cudaMemsetAsync(p->ws.gbar, 0, 16, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = cudaMemsetAsync(p->ws.gbar, 0x01, 1, static_cast<cudaStream_t>(stream));
     return cuda_status(e);
+}
+
+moe_status_t moe_q6_k_packed_bytes(int64_t n_mats, int64_t rows, int64_t k, size_t* code_bytes,
+                                   size_t* scale_bytes) {
+    if (n_mats < 0 || rows < 0 || rows % 16 != 0 || k < 0 || k % 256 != 0) return MOE_ERR_INVALID_ARG;
+    const int64_t blocks = n_mats * rows * (k / 32);
+    if (code_bytes) *code_bytes = static_cast<size_t>(blocks) * 16;
+    if (scale_bytes)
+        *scale_bytes = static_cast<size_t>(blocks / 16) * 160 + static_cast<size_t>(blocks / 8) * 2;
+    return MOE_OK;
+}
+
+moe_status_t moe_q6_k_pack(const void* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                           void* codes, void* scales, void* stream) {
+    if (n_mats < 0 || rows < 0 || rows % 16 != 0 || k < 0 || k % 256 != 0) return MOE_ERR_INVALID_ARG;
+    if (n_mats * rows * k == 0) return MOE_OK;
+    if (!blocks || !codes || !scales || !aligned16(codes) || !aligned16(scales))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_q6_k_pack(static_cast<const uint8_t*>(blocks), n_mats, rows, k,
+                                        static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_bf16_to_f16(const void* src, int64_t n, void* dst, void* stream) {

@@ -223,6 +223,7 @@ constexpr int kDecodeThreads = kConsumers + 32;   // + one producer warp
 // Weight formats of the decode kernels (the values of moe_wfmt_t).
 constexpr int kWfBf16 = 0, kWfQ4 = 1, kWfQ8 = 2;
 constexpr int kWfQ5 = 3;
+constexpr int kWfQ6 = 4;     // q6_K super-blocks (row-streaming, fp16 operands)
 constexpr int kWfF16d = 5;   // bf16 gate/up, fp16 down matrices (h travels in fp16)
 
 // The constant that turns the bf16 "128 + nibble" operands back into signed
@@ -238,14 +239,17 @@ struct DecodeCfg {
     static constexpr int ROLES = 2 * RG;          // (matrix, row group) pairs of phase A
     static constexpr int KSPLIT = kConsumerWarps / ROLES;
     static_assert(KSPLIT >= 1 && ROLES * KSPLIT == kConsumerWarps, "warp roles");
-    static constexpr bool QUANT = WF == kWfQ4 || WF == kWfQ8 || WF == kWfQ5;
+    static constexpr bool QUANT = WF == kWfQ4 || WF == kWfQ8 || WF == kWfQ5 || WF == kWfQ6;
     // bf16 phase A with fp16 down matrices: h is stored as an fp16 hi + lo
     // pair and the down contraction runs on fp16 operands
     static constexpr bool HALF_DOWN = WF == kWfF16d;
     static_assert(!QUANT || FS >= 32, "quantised slices hold whole blocks");
     // fp16 tensor-core operands (see q4h_lo): x staged as fp16, h as an fp16
     // hi + lo pair, per-block corrections with two code bases
-    static constexpr bool F16 = WF == kWfQ4;
+    static constexpr bool F16 = WF == kWfQ4 || WF == kWfQ6;
+    // q6_K: per 32-wide block and 16-row group a 160-byte record (high bits,
+    // sub-block scales), per row and 256-wide super-block an fp16 scale
+    static constexpr bool Q6 = WF == kWfQ6;
     static constexpr int CB = WF == kWfQ8 ? 32 : 16;   // code bytes of one block row
     // + its fp16 scale (Q5_0: + its 32-bit word of fifth bits; scale and word
     // sit in 48-byte records of 8 rows, see q5_aux)
@@ -254,7 +258,9 @@ struct DecodeCfg {
     // Q4_0 / Q8_0 / Q5_0: phase A stage = gate+up [KB block cols][FS rows];
     //              phase B = [NB block cols][RJ rows]; codes, then the scales
     //              (Q5_0: the 48-byte records of scales and fifth bits)
-    static constexpr int STAGE = QUANT ? 2 * 512 * BR : 32768;
+    // q6_K: phase A 16 rows x 64 blocks (26880 B), phase B 4 boxes of 256
+    // rows (4 x 7168 B)
+    static constexpr int STAGE = Q6 ? 28672 : QUANT ? 2 * 512 * BR : 32768;
     static constexpr int KT = 8192 / FS;          // bf16 phase A k columns
     static constexpr int KB = 512 / FS;           // quantised phase A block columns
     static constexpr int NB = FS / 32;            // quantised block columns in a slice
@@ -456,7 +462,7 @@ struct DecodeSmem {
     float* gu;              // [GU_PARTS][2][8][GS]: gate / up partial results
     __nv_bfloat16* hhi;     // [8][HS]: h = hi + lo, per slot
     __nv_bfloat16* hlo;
-    float* hsum;            // [8][2]: -offset * block sums of hi + lo (quantised formats)
+    float* hsum;            // [8][4]: -offset * block (q6_K: sub-block) sums of hi + lo
     DecodeSmemTail* tail;
     uint64_t* full;
     uint64_t* empty;
@@ -471,11 +477,11 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
     sm.ring = smem;
     sm.xs = sm.ring + static_cast<size_t>(a.n_stages) * C::STAGE;
     sm.xsum = reinterpret_cast<float*>(sm.xs + kDecodeTok * a.xs_stride);
-    sm.gu = sm.xsum + kDecodeTok * (a.d / 32);
+    sm.gu = sm.xsum + kDecodeTok * (a.d / 16);
     sm.hhi = reinterpret_cast<__nv_bfloat16*>(sm.gu + C::GU_PARTS * 2 * kDecodeTok * C::GS);
     sm.hlo = sm.hhi + kDecodeTok * C::HS;
     sm.hsum = reinterpret_cast<float*>(sm.hlo + kDecodeTok * C::HS);
-    sm.tail = reinterpret_cast<DecodeSmemTail*>(sm.hsum + kDecodeTok * 2);
+    sm.tail = reinterpret_cast<DecodeSmemTail*>(sm.hsum + kDecodeTok * 4);
     sm.full = reinterpret_cast<uint64_t*>(sm.tail + 1);
     sm.empty = sm.full + a.n_stages;
     return sm;
@@ -489,7 +495,7 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
 template <int WF>
 __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& sm, int tid) {
     const int nkb = a.d / 32;
-    if constexpr (WF == kWfQ4) {
+    if constexpr (WF == kWfQ4 || WF == kWfQ6) {
         // fp16 copy of x (exact for |x| >= 2^-17; below, off by at most 2^-25)
         // and each block's accumulator start -sum((base_k + 8) x_k), base_k
         // 1024 for k % 16 < 8 and 64 otherwise (see q4h_lo)
@@ -497,7 +503,7 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
             const int t = idx / nkb, kb = idx % nkb;
             const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + kb * 32);
             uint4* dst = reinterpret_cast<uint4*>(sm.xs + t * a.xs_stride + kb * 64);
-            float s_lo = 0.f, s_hi = 0.f;
+            float s8[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const uint4 v = __ldg(src + c);
@@ -512,12 +518,19 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
                     h[j] = *reinterpret_cast<uint32_t*>(&hv);
                 }
                 dst[c] = make_uint4(h[0], h[1], h[2], h[3]);
-                if (c & 1) s_hi += s; else s_lo += s;      // elements 8c .. 8c+7
+                s8[c] = s;                                  // elements 8c .. 8c+7
             }
-            sm.xsum[t * nkb + kb] = -((kF16BaseLo + 8.f) * s_lo + (kF16BaseHi + 8.f) * s_hi);
+            if constexpr (WF == kWfQ4) {
+                sm.xsum[t * nkb + kb] =
+                    -((kF16BaseLo + 8.f) * (s8[0] + s8[2]) + (kF16BaseHi + 8.f) * (s8[1] + s8[3]));
+            } else {
+                // q6_K: one start per 16-wide sub-block, offset 32
+                sm.xsum[t * 2 * nkb + 2 * kb] = -((kF16BaseLo + 32.f) * s8[0] + (kF16BaseHi + 32.f) * s8[1]);
+                sm.xsum[t * 2 * nkb + 2 * kb + 1] =
+                    -((kF16BaseLo + 32.f) * s8[2] + (kF16BaseHi + 32.f) * s8[3]);
+            }
         }
-        return;
-    }
+    } else {
     for (int idx = tid; idx < a.T * nkb; idx += kConsumers) {
         const int t = idx / nkb, kb = idx % nkb;
         const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + kb * 32);
@@ -535,6 +548,7 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
             }
         }
         if constexpr (WF == kWfQ8 || WF == kWfQ5) sm.xsum[t * nkb + kb] = -quant_offset(WF) * s;
+    }
     }
 }
 
@@ -930,23 +944,61 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
 }
 
 
+// q6_K: the four fp16 operand registers of one row's 8 codes, from its code
+// word w (low 4 bits, packed like Q4_0) and its word e of high-bit pairs
+// (the pair of the code in nibble n at bit {4, 8, 6, 10, 20, 24, 22, 26}[n]):
+// each register is two values 1024 + q (k % 16 < 8) or 64 + q (k % 16 >= 8),
+// q = low + 16 * high in 0..63, exact in fp16 (see q4h_lo).  r0, r1 feed the
+// block's first 16-wide half (sub-block), r2, r3 the second.
+__device__ __forceinline__ void q6h_regs(uint32_t w, uint32_t e, uint32_t& r0, uint32_t& r1,
+                                         uint32_t& r2, uint32_t& r3) {
+    r0 = q4h_lo(w) | (e & 0x00300030u);
+    r1 = q4h_hi(w) | (e & 0x03000300u);
+    const uint32_t u = w >> 8, f = e >> 2;
+    r2 = q4h_lo(u) | (f & 0x00300030u);
+    r3 = q4h_hi(u) | (f & 0x03000300u);
+}
+
+// The four sub-block scales d * sc of rows r and r + 8 of one q6_K block:
+// sw holds the int8 sub-scales (row r: k 0-15, 16-31; row r + 8: the same).
+__device__ __forceinline__ void q6_scales(uint32_t sw, float dr, float dr8, float& s00, float& s01,
+                                          float& s80, float& s81) {
+    s00 = dr * static_cast<float>(static_cast<int8_t>(sw & 0xffu));
+    s01 = dr * static_cast<float>(static_cast<int8_t>((sw >> 8) & 0xffu));
+    s80 = dr8 * static_cast<float>(static_cast<int8_t>((sw >> 16) & 0xffu));
+    s81 = dr8 * static_cast<float>(static_cast<int8_t>(sw >> 24));
+}
+
 // The experts pipeline for the weight formats that feed fp16 operands to
-// the tensor cores (F16): phase A streams row groups instead of block
-// columns.  A phase-A stage is 16 consecutive rows of the gate or up slice
-// over the whole reduction dim (KC <= 64 block columns per stage, more
+// the tensor cores (F16: Q4_0, q6_K): phase A streams row groups instead of
+// block columns.  A phase-A stage is 16 consecutive rows of the gate or up
+// slice over the whole reduction dim (KC <= 64 block columns per stage, more
 // stages per row group when d > 2048), and consumer warp w owns block
 // columns w, w + 16, w + 32, w + 48 of every stage.  The x fragments and
 // block corrections of those columns therefore stay in registers for the
 // whole unit instead of being reloaded from shared memory for every 16x32
 // tile, which halves the shared-memory traffic per weight; each warp keeps
 // the partial sums of every row group and both matrices, and one reduction
-// over the 16 warps follows phase A.  Phase B (down matrix, combine) is the
-// same as in experts_pipeline.
+// over the 16 warps follows phase A.  Phase B (down matrix, combine) works
+// like experts_pipeline's.
+//
+// Stage layouts.  Q4_0 phase A: codes [KC][16 rows][16 B], scales [KC][16]
+// fp16; phase B per 256-row box: codes [NB][256][16 B], scales [NB][256].
+// q6_K phase A: codes [KC][16][16 B], records [KC][160 B], super-block scales
+// [KC/8][16] fp16; phase B per 256-row box: codes [NB][256][16 B], records
+// [NB][16][160 B], super-block scales [256] fp16 (a slice of FS <= 256
+// columns lies in one super-block).
 template <int FS, int WF>
 __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const DecodeSmem& sm,
                                                       const WorkView& wv) {
     using C = DecodeCfg<FS, WF>;
     static_assert(C::F16, "row-streaming phase A serves the fp16-operand formats");
+    static_assert(!C::Q6 || FS == 32, "q6_K slices are 32 rows");
+    constexpr int QB = kQuantDownBoxRows;
+    // phase-B bytes of one 256-row box
+    constexpr int BOXB = C::Q6 ? C::NB * QB * 16 + C::NB * (QB / 16) * 160 + QB * 2
+                               : C::NB * QB * C::BR;
+    static_assert((C::RJ / QB) * BOXB <= C::STAGE, "phase-B boxes fit a stage");
     const int ns = a.n_stages;
     uint8_t* ring = sm.ring;
     float* gu = sm.gu;
@@ -958,6 +1010,8 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
     const int nkb = d / 32;
     const int KC = a.kt;                              // block columns per phase-A stage
     const int nch = (nkb + KC - 1) / KC;              // phase-A stages per row group and matrix
+    // phase-A bytes of one stage
+    const int stage_a = C::Q6 ? KC * (16 * 16 + 160) + (KC / 8) * 32 : 16 * KC * C::BR;
     const int n_routed = wv.n_routed, n_shared = wv.n_shared;
     const int sl_r = a.F / FS, sl_s = a.S ? a.Fs / FS : 0;
     const int n_su = n_shared * sl_s;
@@ -979,10 +1033,18 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
             prefetch_tensormap(&a.tm_down);
             prefetch_tensormap(&a.tm_gate_sc); prefetch_tensormap(&a.tm_up_sc);
             prefetch_tensormap(&a.tm_down_sc);
+            if constexpr (C::Q6) {
+                prefetch_tensormap(&a.tm_gate_d); prefetch_tensormap(&a.tm_up_d);
+                prefetch_tensormap(&a.tm_down_d);
+            }
             if (a.S) {
                 prefetch_tensormap(&a.tm_sgate); prefetch_tensormap(&a.tm_sup);
                 prefetch_tensormap(&a.tm_sdown); prefetch_tensormap(&a.tm_sgate_sc);
                 prefetch_tensormap(&a.tm_sup_sc); prefetch_tensormap(&a.tm_sdown_sc);
+                if constexpr (C::Q6) {
+                    prefetch_tensormap(&a.tm_sgate_d); prefetch_tensormap(&a.tm_sup_d);
+                    prefetch_tensormap(&a.tm_sdown_d);
+                }
             }
             const uint64_t pol = l2_policy_evict_first();
             uint32_t it = 0;
@@ -1011,21 +1073,38 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                         const CUtensorMap* ms = mat ? (shared ? &a.tm_sup_sc : &a.tm_up_sc)
                                                     : (shared ? &a.tm_sgate_sc : &a.tm_gate_sc);
                         const int c2 = ex * nkb + c * KC;
-                        mbar_arrive_expect_tx(&full[slot], 16 * KC * C::BR);
-                        tma_load_3d(dst, mc, &full[slot], 0, f0 + rg * 16, c2, pol);
-                        tma_load_2d(dst + 16 * KC * C::CB, ms, &full[slot], f0 + rg * 16, c2, pol);
+                        const int r0 = f0 + rg * 16;
+                        mbar_arrive_expect_tx(&full[slot], stage_a);
+                        tma_load_3d(dst, mc, &full[slot], 0, r0, c2, pol);
+                        if constexpr (C::Q6) {
+                            const CUtensorMap* md = mat ? (shared ? &a.tm_sup_d : &a.tm_up_d)
+                                                        : (shared ? &a.tm_sgate_d : &a.tm_gate_d);
+                            tma_load_3d(dst + 16 * KC * 16, ms, &full[slot], 0, r0 / 16, c2, pol);
+                            tma_load_2d(dst + KC * (16 * 16 + 160), md, &full[slot], r0,
+                                        ex * (nkb / 8) + c * (KC / 8), pol);
+                        } else {
+                            tma_load_2d(dst + 16 * KC * C::CB, ms, &full[slot], r0, c2, pol);
+                        }
                     } else {
                         const CUtensorMap* md = shared ? &a.tm_sdown : &a.tm_down;
                         const CUtensorMap* mds = shared ? &a.tm_sdown_sc : &a.tm_down_sc;
                         const int j0 = (st - nA) * C::RJ;
-                        constexpr int QB = kQuantDownBoxRows;
                         const int nbox = (min(C::RJ, d - j0) + QB - 1) / QB;
                         const int c2 = ex * (Fh / 32) + f0 / 32;
-                        mbar_arrive_expect_tx(&full[slot], nbox * C::NB * QB * C::BR);
+                        mbar_arrive_expect_tx(&full[slot], nbox * BOXB);
                         for (int b = 0; b < nbox; ++b) {
-                            uint8_t* bd = dst + b * (C::NB * QB * C::BR);
+                            uint8_t* bd = dst + b * BOXB;
                             tma_load_3d(bd, md, &full[slot], 0, j0 + QB * b, c2, pol);
-                            tma_load_2d(bd + C::NB * QB * C::CB, mds, &full[slot], j0 + QB * b, c2, pol);
+                            if constexpr (C::Q6) {
+                                const CUtensorMap* mdd = shared ? &a.tm_sdown_d : &a.tm_down_d;
+                                tma_load_3d(bd + C::NB * QB * 16, mds, &full[slot], 0, (j0 + QB * b) / 16,
+                                            c2, pol);
+                                tma_load_2d(bd + C::NB * QB * 16 + C::NB * (QB / 16) * 160, mdd, &full[slot],
+                                            j0 + QB * b, ex * (Fh / 256) + f0 / 256, pol);
+                            } else {
+                                tma_load_2d(bd + C::NB * QB * C::CB, mds, &full[slot], j0 + QB * b, c2,
+                                            pol);
+                            }
                         }
                     }
                 }
@@ -1043,6 +1122,7 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
     // ---------------------------------------------------------- consumers
     const int g = lane >> 2, tig = lane & 3;
     const uint32_t xs_u = smem_u32(sm.xs);
+    constexpr int NC = C::Q6 ? 2 : 1;                 // corrections per block (per 16-k sub-block)
     uint32_t it = 0;
     auto wait_full = [&](int slot, uint32_t parity) -> bool {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
@@ -1074,7 +1154,7 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
 
         // x fragments and corrections of this warp's block columns of chunk c
         uint32_t xf[C::NBW][4];
-        float xc0[C::NBW], xc1[C::NBW];
+        float xc0[C::NBW][NC], xc1[C::NBW][NC];
         auto load_x = [&](int c) {
 #pragma unroll
             for (int i = 0; i < C::NBW; ++i) {
@@ -1082,8 +1162,11 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                 const bool in = (warp + kConsumerWarps * i) < KC && kb < nkb;
                 const int kbs = in ? kb : 0;
                 ldsm_x4(xrow + (kbs * 32 + (lane >> 3) * 8) * 2, xf[i][0], xf[i][1], xf[i][2], xf[i][3]);
-                xc0[i] = sm.xsum[tok0 * nkb + kbs];
-                xc1[i] = sm.xsum[tok1 * nkb + kbs];
+#pragma unroll
+                for (int j = 0; j < NC; ++j) {
+                    xc0[i][j] = sm.xsum[(tok0 * nkb + kbs) * NC + j];
+                    xc1[i][j] = sm.xsum[(tok1 * nkb + kbs) * NC + j];
+                }
             }
         };
         if (nch == 1) load_x(0);
@@ -1104,27 +1187,52 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                     if (ok) {
                         if (nch > 1) load_x(c);
                         const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
-                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(stage);   // [KC][16][CB]
-                        const __half* scl = reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
+                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(stage);   // [KC][16][16 B]
+                        float* ac = acc[rg * 2 + mat];
 #pragma unroll
                         for (int i = 0; i < C::NBW; ++i) {
                             const int bl = warp + kConsumerWarps * i;
                             if (bl < KC && c * KC + bl < nkb) {
                                 const uint32_t* row = codes + (bl * 16 + g) * 4;
                                 const uint32_t x0 = row[tig], x8 = row[32 + tig];
-                                float v[4];
-                                mma_f16_16816(v, q4h_lo(x0), q4h_lo(x8), q4h_hi(x0), q4h_hi(x8),
-                                              xf[i][0], xf[i][1], xc0[i], xc1[i], xc0[i], xc1[i]);
-                                const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
-                                mma_f16_16816_acc(v, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8),
-                                                  xf[i][2], xf[i][3]);
-                                const float s0 = __half2float(scl[bl * 16 + g]);
-                                const float s8 = __half2float(scl[bl * 16 + g + 8]);
-                                float* ac = acc[rg * 2 + mat];
-                                ac[0] = fmaf(s0, v[0], ac[0]);
-                                ac[1] = fmaf(s0, v[1], ac[1]);
-                                ac[2] = fmaf(s8, v[2], ac[2]);
-                                ac[3] = fmaf(s8, v[3], ac[3]);
+                                if constexpr (C::Q6) {
+                                    const uint32_t* rec =
+                                        reinterpret_cast<const uint32_t*>(stage + 16 * KC * 16 + bl * 160);
+                                    const __half* dsm =
+                                        reinterpret_cast<const __half*>(stage + KC * (16 * 16 + 160));
+                                    const uint32_t e = rec[4 * g + tig];
+                                    uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
+                                    q6h_regs(x0, e, p0, p1, p2, p3);
+                                    q6h_regs(x8, __funnelshift_r(e, e, 8), q0, q1, q2, q3);
+                                    float va[4], vb[4];
+                                    mma_f16_16816(va, p0, q0, p1, q1, xf[i][0], xf[i][1],
+                                                  xc0[i][0], xc1[i][0], xc0[i][0], xc1[i][0]);
+                                    mma_f16_16816(vb, p2, q2, p3, q3, xf[i][2], xf[i][3],
+                                                  xc0[i][NC - 1], xc1[i][NC - 1], xc0[i][NC - 1],
+                                                  xc1[i][NC - 1]);
+                                    float s00, s01, s80, s81;
+                                    q6_scales(rec[32 + g], __half2float(dsm[(bl >> 3) * 16 + g]),
+                                              __half2float(dsm[(bl >> 3) * 16 + g + 8]), s00, s01, s80, s81);
+                                    ac[0] = fmaf(s00, va[0], fmaf(s01, vb[0], ac[0]));
+                                    ac[1] = fmaf(s00, va[1], fmaf(s01, vb[1], ac[1]));
+                                    ac[2] = fmaf(s80, va[2], fmaf(s81, vb[2], ac[2]));
+                                    ac[3] = fmaf(s80, va[3], fmaf(s81, vb[3], ac[3]));
+                                } else {
+                                    const __half* scl = reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
+                                    float v[4];
+                                    mma_f16_16816(v, q4h_lo(x0), q4h_lo(x8), q4h_hi(x0), q4h_hi(x8),
+                                                  xf[i][0], xf[i][1], xc0[i][0], xc1[i][0], xc0[i][0],
+                                                  xc1[i][0]);
+                                    const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
+                                    mma_f16_16816_acc(v, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8),
+                                                      xf[i][2], xf[i][3]);
+                                    const float s0 = __half2float(scl[bl * 16 + g]);
+                                    const float s8 = __half2float(scl[bl * 16 + g + 8]);
+                                    ac[0] = fmaf(s0, v[0], ac[0]);
+                                    ac[1] = fmaf(s0, v[1], ac[1]);
+                                    ac[2] = fmaf(s8, v[2], ac[2]);
+                                    ac[3] = fmaf(s8, v[3], ac[3]);
+                                }
                             }
                         }
                     }
@@ -1149,7 +1257,8 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
         named_bar_sync(1, kConsumers);
         // h = SiLU(gate) * up as an fp16 pair hi + lo for the token columns in
         // use (the rest are zero); one warp covers 32 consecutive f of one
-        // column, i.e. one block of the down matrix
+        // column, i.e. one block of the down matrix.  The down block's (q6_K:
+        // sub-block's) accumulator starts at -sum((base_f + offset)(hi + lo)).
         for (int idx = tid; idx < FS * kDecodeTok; idx += kConsumers) {
             const int t = idx / FS, f = idx % FS;
             __half hi = __float2half_rn(0.f), lo = hi;
@@ -1165,13 +1274,19 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                 hi = __float2half_rn(h);
                 lo = __float2half_rn(h - __half2float(hi));
                 const float base = (f & 15) < 8 ? kF16BaseLo : kF16BaseHi;
-                hs = (base + 8.f) * (__half2float(hi) + __half2float(lo));
+                hs = (base + (C::Q6 ? 32.f : 8.f)) * (__half2float(hi) + __half2float(lo));
             }
             reinterpret_cast<__half*>(sm.hhi)[t * C::HS + f] = hi;
             reinterpret_cast<__half*>(sm.hlo)[t * C::HS + f] = lo;
+            if constexpr (C::Q6) {
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
-            if (lane == 0) sm.hsum[t * 2 + f / 32] = -hs;
+                for (int off = 8; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
+                if ((lane & 15) == 0) sm.hsum[t * 4 + f / 16] = -hs;
+            } else {
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
+                if (lane == 0) sm.hsum[t * 4 + f / 32] = -hs;
+            }
         }
         named_bar_sync(1, kConsumers);
         uint32_t bh[C::RG][2], bl[C::RG][2];
@@ -1181,11 +1296,13 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
             ldsm_x2(smem_u32(sm.hhi) + off, bh[kk][0], bh[kk][1]);
             ldsm_x2(smem_u32(sm.hlo) + off, bl[kk][0], bl[kk][1]);
         }
-        float hs0[C::NB], hs1[C::NB];
+        // corrections of the down blocks (Q4_0) or sub-blocks (q6_K), columns t0, t1
+        constexpr int NH = C::Q6 ? 2 * C::NB : C::NB;
+        float hs0[NH], hs1[NH];
 #pragma unroll
-        for (int bb = 0; bb < C::NB; ++bb) {
-            hs0[bb] = sm.hsum[t0 * 2 + bb];
-            hs1[bb] = sm.hsum[t1 * 2 + bb];
+        for (int j = 0; j < NH; ++j) {
+            hs0[j] = sm.hsum[t0 * 4 + j];
+            hs1[j] = sm.hsum[t1 * 4 + j];
         }
 
         // --------------------------------------- phase B: down + combine
@@ -1198,32 +1315,58 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
             if (ok) {
                 for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
                     float c[4] = {0.f, 0.f, 0.f, 0.f};
-                    constexpr int QB = kQuantDownBoxRows;
-                    const uint8_t* bbase = stage + (rgb / (QB / 16)) * (C::NB * QB * C::BR);
-                    const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);   // [NB][QB][CB]
-                    const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * QB * C::CB);
-                    const int rib = (rgb % (QB / 16)) * 16 + g;
+                    const uint8_t* bbase = stage + (rgb / (QB / 16)) * BOXB;
+                    const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);   // [NB][QB][16 B]
+                    const int grp = rgb % (QB / 16);
+                    const int rib = grp * 16 + g;
 #pragma unroll
                     for (int bb = 0; bb < C::NB; ++bb) {
                         const uint32_t* row = codes + (bb * QB + rib) * 4;
                         const uint32_t x0 = row[tig], x8 = row[32 + tig];
-                        const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
-                        const uint32_t p0 = q4h_lo(x0), q0 = q4h_lo(x8);
-                        const uint32_t p1 = q4h_hi(x0), q1 = q4h_hi(x8);
-                        const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
-                        const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
-                        float v[4];
-                        mma_f16_16816(v, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
-                                      hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
-                        mma_f16_16816_acc(v, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
-                        mma_f16_16816_acc(v, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
-                        mma_f16_16816_acc(v, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
-                        const float s0 = __half2float(scl[bb * QB + rib]);
-                        const float s8 = __half2float(scl[bb * QB + rib + 8]);
-                        c[0] = fmaf(s0, v[0], c[0]);
-                        c[1] = fmaf(s0, v[1], c[1]);
-                        c[2] = fmaf(s8, v[2], c[2]);
-                        c[3] = fmaf(s8, v[3], c[3]);
+                        if constexpr (C::Q6) {
+                            const uint32_t* rec = reinterpret_cast<const uint32_t*>(
+                                bbase + C::NB * QB * 16 + (bb * (QB / 16) + grp) * 160);
+                            const __half* dsm = reinterpret_cast<const __half*>(
+                                bbase + C::NB * QB * 16 + C::NB * (QB / 16) * 160);
+                            const uint32_t e = rec[4 * g + tig];
+                            uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
+                            q6h_regs(x0, e, p0, p1, p2, p3);
+                            q6h_regs(x8, __funnelshift_r(e, e, 8), q0, q1, q2, q3);
+                            float va[4], vb[4];
+                            mma_f16_16816(va, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
+                                          hs0[2 * bb], hs1[2 * bb], hs0[2 * bb], hs1[2 * bb]);
+                            mma_f16_16816_acc(va, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                            mma_f16_16816(vb, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1],
+                                          hs0[2 * bb + 1], hs1[2 * bb + 1], hs0[2 * bb + 1],
+                                          hs1[2 * bb + 1]);
+                            mma_f16_16816_acc(vb, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                            float s00, s01, s80, s81;
+                            q6_scales(rec[32 + g], __half2float(dsm[rib]), __half2float(dsm[rib + 8]),
+                                      s00, s01, s80, s81);
+                            c[0] = fmaf(s00, va[0], fmaf(s01, vb[0], c[0]));
+                            c[1] = fmaf(s00, va[1], fmaf(s01, vb[1], c[1]));
+                            c[2] = fmaf(s80, va[2], fmaf(s81, vb[2], c[2]));
+                            c[3] = fmaf(s80, va[3], fmaf(s81, vb[3], c[3]));
+                        } else {
+                            const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * QB * C::CB);
+                            const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
+                            const uint32_t p0 = q4h_lo(x0), q0 = q4h_lo(x8);
+                            const uint32_t p1 = q4h_hi(x0), q1 = q4h_hi(x8);
+                            const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
+                            const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
+                            float v[4];
+                            mma_f16_16816(v, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
+                                          hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
+                            mma_f16_16816_acc(v, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
+                            mma_f16_16816_acc(v, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                            mma_f16_16816_acc(v, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                            const float s0 = __half2float(scl[bb * QB + rib]);
+                            const float s8 = __half2float(scl[bb * QB + rib + 8]);
+                            c[0] = fmaf(s0, v[0], c[0]);
+                            c[1] = fmaf(s0, v[1], c[1]);
+                            c[2] = fmaf(s8, v[2], c[2]);
+                            c[3] = fmaf(s8, v[3], c[3]);
+                        }
                     }
                     const int j = j0 + rgb * 16 + g;
                     if (v0) {
@@ -1520,6 +1663,7 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
 int decode_stage_bytes(int fs, int wfmt) {
     (void)fs;
     if (wfmt == kWfQ4) return 2 * 512 * 18;
+    if (wfmt == kWfQ6) return 28672;
     if (wfmt == kWfQ8) return 2 * 512 * 34;
     if (wfmt == kWfQ5) return 2 * 512 * 22;
     return 32768;
@@ -1528,14 +1672,15 @@ int decode_stage_bytes(int fs, int wfmt) {
 size_t decode_smem_bytes(int fs, int wfmt, int d, int n_stages) {
     // partial sums per gate/up output: KSPLIT, or one per warp for the
     // row-streaming formats (DecodeCfg::GU_PARTS)
-    const int ksplit = wfmt == kWfQ4 ? kConsumerWarps : kConsumerWarps / (2 * (fs / 16));
+    const int ksplit = (wfmt == kWfQ4 || wfmt == kWfQ6) ? kConsumerWarps
+                                                         : kConsumerWarps / (2 * (fs / 16));
     size_t b = 1024;                                            // alignment slack
     b += static_cast<size_t>(n_stages) * decode_stage_bytes(fs, wfmt);
     b += static_cast<size_t>(kDecodeTok) * (d * 2 + 16);       // staged x
-    b += static_cast<size_t>(kDecodeTok) * (d / 32) * 4;       // block sums of x
+    b += static_cast<size_t>(kDecodeTok) * (d / 16) * 4;       // block (sub-block) sums of x
     b += static_cast<size_t>(ksplit) * 2 * kDecodeTok * (fs + 4) * 4;  // gate/up results
     b += 2ull * kDecodeTok * (fs + 8) * 2;                      // h hi/lo
-    b += static_cast<size_t>(kDecodeTok) * 2 * 4;              // block sums of h
+    b += static_cast<size_t>(kDecodeTok) * 4 * 4;              // block sums of h
     b += sizeof(DecodeSmemTail);
     b += 2ull * n_stages * 8;                                   // barriers
     return b;
@@ -1595,6 +1740,7 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, int wfmt, int grid,
         case kWfF16d * 100 + 64: return launch_fused_one<64, kWfF16d>(a, grid, smem, stream);
         case kWfF16d * 100 + 32: return launch_fused_one<32, kWfF16d>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_fused_one<32, kWfQ4>(a, grid, smem, stream);
+        case kWfQ6 * 100 + 32: return launch_fused_one<32, kWfQ6>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_fused_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_fused_one<32, kWfQ8>(a, grid, smem, stream);
         case kWfQ5 * 100 + 64: return launch_fused_one<64, kWfQ5>(a, grid, smem, stream);
@@ -1611,6 +1757,7 @@ cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, int wfmt, int gri
         case kWfF16d * 100 + 64: return launch_one<64, kWfF16d>(a, grid, smem, stream);
         case kWfF16d * 100 + 32: return launch_one<32, kWfF16d>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_one<32, kWfQ4>(a, grid, smem, stream);
+        case kWfQ6 * 100 + 32: return launch_one<32, kWfQ6>(a, grid, smem, stream);
         case kWfQ8 * 100 + 64: return launch_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_one<32, kWfQ8>(a, grid, smem, stream);
         case kWfQ5 * 100 + 64: return launch_one<64, kWfQ5>(a, grid, smem, stream);

@@ -88,6 +88,11 @@ struct DecodeArgs {
     // the 48-byte records of scales and fifth bits.
     CUtensorMap tm_gate_sc, tm_up_sc, tm_down_sc;
     CUtensorMap tm_sgate_sc, tm_sup_sc, tm_sdown_sc;
+    // q6_K only: 2D maps over the fp16 super-block scales [mats][K/256][rows]
+    // (the _sc maps above cover the 160-byte records of high bits and
+    // sub-block scales)
+    CUtensorMap tm_gate_d, tm_up_d, tm_down_d;
+    CUtensorMap tm_sgate_d, tm_sup_d, tm_sdown_d;
     const uint16_t* x;          // [T][d] bf16
     float* out;                 // [T][d] fp32, accumulated into
     const WorkItem* items;
@@ -123,11 +128,14 @@ cudaError_t launch_q8_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
                              uint8_t* codes, uint16_t* scales, cudaStream_t stream);
 cudaError_t launch_q5_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
                              uint8_t* codes, uint8_t* aux, cudaStream_t stream);
+cudaError_t launch_q6_k_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint8_t* scales, cudaStream_t stream);
 cudaError_t launch_bf16_to_f16(const uint16_t* src, int64_t n, uint16_t* dst, cudaStream_t stream);
 
 // Formats whose matrices are quantised blocks (codes + scales).
 inline bool wfmt_quantised(int wfmt) {
-    return wfmt == MOE_WFMT_Q4_0 || wfmt == MOE_WFMT_Q8_0 || wfmt == MOE_WFMT_Q5_0;
+    return wfmt == MOE_WFMT_Q4_0 || wfmt == MOE_WFMT_Q8_0 || wfmt == MOE_WFMT_Q5_0 ||
+           wfmt == MOE_WFMT_Q6_K;
 }
 
 // --------------------------------------------------------- device helpers

@@ -1,5 +1,5 @@
-// quant_pack.cu -- repack canonical Q4_0, Q8_0 and Q5_0 blocks into the
-// decode kernels' layout.
+// quant_pack.cu -- repack canonical Q4_0, Q8_0, Q5_0 blocks and q6_K
+// super-blocks into the decode kernels' layout.
 //
 // ---- Q4_0
 // Canonical block (32 weights along the reduction dim, 18 bytes): little-endian
@@ -194,6 +194,103 @@ cudaError_t launch_q5_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
     const int64_t want = (total + threads - 1) / threads;
     const int grid = static_cast<int>(want < 65536 ? want : 65536);
     q5_0_pack_kernel<<<grid, threads, 0, stream>>>(blocks, n_mats, rows, k / 32, codes, aux);
+    return cudaGetLastError();
+}
+
+// ---- q6_K
+// Canonical super-block (256 weights along the reduction dim, 210 bytes):
+// ql[128] low 4 bits, qh[64] high 2 bits, 16 signed 8-bit sub-block scales,
+// then a little-endian fp16 scale d.  Element i = 128 h + 32 c + l: low bits
+// in the low (c < 2) or high (c >= 2) nibble of ql[64 h + 32 (c % 2) + l],
+// high bits in bits 2c, 2c+1 of qh[32 h + l]; weight d * sc[i / 16] * (q - 32).
+// (The 5090 page lists q6_K among the formats of the model it measures; the
+// byte layout is the canonical llama.cpp one, a reading.)
+//
+// Kernel layout (same 6.5625 bits per weight):
+//   codes [mat][k/32][rows][16 B]        low 4 bits, packed exactly like Q4_0
+//   aux   [mat][k/32][rows/16][160 B]    per 32-wide block and 16-row group:
+//           bytes 0-127: 32 words, word 4 g + t (g = 0..7, t = 0..3) the high
+//             bits of lane t's 8 codes of rows g and g+8: the code in nibble n
+//             of row g's code word at bits P(n) = {4, 8, 6, 10, 20, 24, 22,
+//             26}[n], row g+8's at P(n) + 8 (mod 32) -- a rotation by 8 moves
+//             them onto row g's places (see q6h_regs);
+//           bytes 128-159: per g, the sub-block scales (int8) of row g for k
+//             0-15 and 16-31 of the block, then those of row g+8;
+//   d     [mat][k/256][rows] fp16        the super-block scales
+// scale_bytes covers aux followed by d (d starts at the aux size, a
+// multiple of 16 bytes).
+__device__ __forceinline__ int q6_code(const uint8_t* sb, int i) {
+    const int h = i >> 7, r = i & 127, c = r >> 5, l = r & 31;
+    const int byte = sb[64 * h + 32 * (c & 1) + l];
+    const int low = c >= 2 ? (byte >> 4) : (byte & 15);
+    const int high = (sb[128 + 32 * h + l] >> (2 * c)) & 3;
+    return low | (high << 4);
+}
+
+// one thread per (matrix, 16-row group, 32-wide block)
+__global__ void q6_k_pack_kernel(const uint8_t* __restrict__ blocks, int64_t n_mats, int64_t rows,
+                                 int64_t nkb, uint8_t* __restrict__ codes, uint8_t* __restrict__ aux,
+                                 uint16_t* __restrict__ dsc) {
+    const int64_t groups = rows / 16;
+    const int64_t total = n_mats * groups * nkb;
+    const int pos[8] = {4, 8, 6, 10, 20, 24, 22, 26};
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t kb = i % nkb;
+        const int64_t grp = (i / nkb) % groups;
+        const int64_t m = i / (nkb * groups);
+        const int64_t nsb = nkb / 8;
+        uint32_t hw[32];
+        uint8_t subs[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) hw[q] = 0u;
+        for (int rr = 0; rr < 16; ++rr) {
+            const int64_t r = grp * 16 + rr;
+            const uint8_t* sb = blocks + ((m * rows + r) * nsb + kb / 8) * 210;   // canonical [m][r][sb]
+            const int e0 = static_cast<int>(kb % 8) * 32;                         // first element of the block
+            uint8_t low[32], high[32];
+            for (int j = 0; j < 32; ++j) {
+                const int q = q6_code(sb, e0 + j);
+                low[j] = static_cast<uint8_t>(q & 15);
+                high[j] = static_cast<uint8_t>(q >> 4);
+            }
+            uint32_t w[4];
+            for (int t = 0; t < 4; ++t) {
+                const int e = 2 * t;
+                w[t] = static_cast<uint32_t>(low[e]) | (static_cast<uint32_t>(low[e + 8]) << 4) |
+                       (static_cast<uint32_t>(low[e + 16]) << 8) | (static_cast<uint32_t>(low[e + 24]) << 12) |
+                       (static_cast<uint32_t>(low[e + 1]) << 16) | (static_cast<uint32_t>(low[e + 9]) << 20) |
+                       (static_cast<uint32_t>(low[e + 17]) << 24) | (static_cast<uint32_t>(low[e + 25]) << 28);
+                // nibble n of word t holds element {0, 8, 16, 24, 1, 9, 17, 25}[n] + 2t
+                const int elem[8] = {e, e + 8, e + 16, e + 24, e + 1, e + 9, e + 17, e + 25};
+                const int g = rr & 7, shift = rr < 8 ? 0 : 8;
+                for (int n = 0; n < 8; ++n)
+                    hw[4 * g + t] |= static_cast<uint32_t>(high[elem[n]]) << ((pos[n] + shift) & 31);
+            }
+            const int64_t dst = (m * nkb + kb) * rows + r;                        // [m][kb][r]
+            *reinterpret_cast<uint4*>(codes + dst * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+            const int sub0 = static_cast<int>(kb % 8) * 2;
+            subs[(rr & 7) * 4 + (rr < 8 ? 0 : 2) + 0] = sb[192 + sub0];
+            subs[(rr & 7) * 4 + (rr < 8 ? 0 : 2) + 1] = sb[192 + sub0 + 1];
+            if (kb % 8 == 0)
+                dsc[(m * nsb + kb / 8) * rows + r] = static_cast<uint16_t>(sb[208] | (sb[209] << 8));
+        }
+        uint8_t* rec = aux + ((m * nkb + kb) * groups + grp) * 160;
+        for (int q = 0; q < 32; ++q) reinterpret_cast<uint32_t*>(rec)[q] = hw[q];
+        for (int q = 0; q < 32; ++q) rec[128 + q] = subs[q];
+    }
+}
+
+cudaError_t launch_q6_k_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows, int64_t k,
+                             uint8_t* codes, uint8_t* scales, cudaStream_t stream) {
+    const int64_t total = n_mats * (rows / 16) * (k / 32);
+    if (total == 0) return cudaSuccess;
+    const int64_t aux_bytes = total * 160;
+    const int threads = 128;
+    const int64_t want = (total + threads - 1) / threads;
+    const int grid = static_cast<int>(want < 65536 ? want : 65536);
+    q6_k_pack_kernel<<<grid, threads, 0, stream>>>(blocks, n_mats, rows, k / 32, codes, scales,
+                                                   reinterpret_cast<uint16_t*>(scales + aux_bytes));
     return cudaGetLastError();
 }
 

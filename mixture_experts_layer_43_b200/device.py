@@ -31,10 +31,11 @@ class DeviceLayer:
         self.device = torch.device(device)
         # quantised: codes + scales (bf16, and bf16 with fp16 down matrices,
         # upload as they are)
-        self.q4 = sh.wfmt in (synth.WFMT_Q4_0, synth.WFMT_Q8_0, synth.WFMT_Q5_0)
+        self.q4 = sh.wfmt in (synth.WFMT_Q4_0, synth.WFMT_Q8_0, synth.WFMT_Q5_0, synth.WFMT_Q6_K)
         packed_bytes, pack = {
             synth.WFMT_BF16: (None, None),
             synth.WFMT_BF16_F16DOWN: (None, None),
+            synth.WFMT_Q6_K: (B.moe_q6_k_packed_bytes, B.moe_q6_k_pack),
             synth.WFMT_Q4_0: (B.moe_q4_0_packed_bytes, B.moe_q4_0_pack),
             synth.WFMT_Q8_0: (B.moe_q8_0_packed_bytes, B.moe_q8_0_pack),
             synth.WFMT_Q5_0: (B.moe_q5_0_packed_bytes, B.moe_q5_0_pack)}[sh.wfmt]
@@ -168,10 +169,26 @@ def random_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") -> De
     packed_bytes, pack, std = {
         synth.WFMT_Q4_0: (B.moe_q4_0_packed_bytes, B.moe_q4_0_pack, shape.q4_scale_std),
         synth.WFMT_Q8_0: (B.moe_q8_0_packed_bytes, B.moe_q8_0_pack, shape.q8_scale_std),
-        synth.WFMT_Q5_0: (B.moe_q5_0_packed_bytes, B.moe_q5_0_pack, shape.q5_scale_std)}[shape.wfmt]
+        synth.WFMT_Q5_0: (B.moe_q5_0_packed_bytes, B.moe_q5_0_pack, shape.q5_scale_std),
+        synth.WFMT_Q6_K: (B.moe_q6_k_packed_bytes, B.moe_q6_k_pack, shape.q6_scale_std)}[shape.wfmt]
     st = torch.cuda.current_stream(dev)
 
     def blocks(n_rows: int, k: int) -> torch.Tensor:
+        if shape.wfmt == synth.WFMT_Q6_K:
+            nsb = k // 256
+            q = torch.randint(0, 64, (n_rows, nsb, 2, 4, 32), generator=gen, device=dev,
+                              dtype=torch.int32)                         # [h][c][l]
+            low, high = q & 15, q >> 4
+            ql = torch.stack([low[:, :, :, 0] | (low[:, :, :, 2] << 4),
+                              low[:, :, :, 1] | (low[:, :, :, 3] << 4)], dim=3)   # [h][c%2][l]
+            qh = high[:, :, :, 0] | (high[:, :, :, 1] << 2) | (high[:, :, :, 2] << 4) | \
+                (high[:, :, :, 3] << 6)
+            sc = torch.randint(-128, 128, (n_rows, nsb, 16), generator=gen, device=dev,
+                               dtype=torch.int32).to(torch.int8).view(torch.uint8)
+            dd = (torch.randn((n_rows, nsb), generator=gen, device=dev) * std).abs().half()
+            return torch.cat([ql.reshape(n_rows, nsb, 128).to(torch.uint8),
+                              qh.reshape(n_rows, nsb, 64).to(torch.uint8), sc,
+                              dd.view(torch.uint8).reshape(n_rows, nsb, 2)], dim=2)
         nb = k // 32
         sc = (torch.randn((n_rows, nb), generator=gen, device=dev) * std).abs().half()
         sc = sc.view(torch.uint8).reshape(n_rows, nb, 2)
@@ -203,6 +220,8 @@ def random_layer(shape: synth.MoEShape, seed: int, device: str = "cuda:0") -> De
         codes = torch.empty(cb, dtype=torch.uint8, device=dev)
         scales = torch.empty(sb // 2, dtype=torch.int16, device=dev)
         step = max(1, (1 << 26) // (rows * k))                  # bound the temporaries
+        if shape.wfmt == synth.WFMT_Q6_K:
+            step = n_mats          # the packed scales are two arrays (aux, then d): one call
         per_c, per_s = cb // n_mats, sb // n_mats
         for m0 in range(0, n_mats, step):
             m1 = min(n_mats, m0 + step)

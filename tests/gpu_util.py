@@ -16,8 +16,8 @@ Acceptance (the contract of the layer):
     c = 24 for the prefill router, whose tensor-core accumulation of the
     three exact bf16 parts rounds its fp32 sums less tightly (observed 10.3 on
     the DeepSeek-shaped layer at d = 2048): a margin of 2 to 3 each;
-  * out within relative L2 2e-3 (bf16 weights) or 5e-3 (Q4_0, Q8_0 and Q5_0
-    weights) over every token: a token whose ids differ from the oracle's
+  * out within relative L2 2e-3 (bf16 weights, also with fp16 down matrices)
+    or 5e-3 (Q4_0, Q8_0, Q5_0 and q6_K weights) over every token: a token whose ids differ from the oracle's
     (a waived near tie) is compared with the oracle evaluated on the GPU's own
     ids and weights.  Callers may add a tighter tripwire: the decode kernels
     measure about 5e-6 in every format, so a regression of 20x fails long
@@ -34,7 +34,7 @@ from mixture_experts_layer_43_b200 import device as D
 from mixture_experts_layer_43_b200 import synth
 
 TOL = {synth.WFMT_BF16: 2e-3, synth.WFMT_Q4_0: 5e-3, synth.WFMT_Q8_0: 5e-3,
-       synth.WFMT_Q5_0: 5e-3}
+       synth.WFMT_Q5_0: 5e-3, synth.WFMT_Q6_K: 5e-3, synth.WFMT_BF16_F16DOWN: 2e-3}
 GAP_REL = 1e-5
 W_ABS = 1e-7
 

@@ -46,7 +46,7 @@ def _cfg(**kw):
     dict(t_max=0), dict(d_model=100), dict(d_model=192), dict(d_ff=48), dict(n_experts=0),
     dict(n_experts=2000), dict(top_k=0), dict(top_k=9), dict(n_experts=32, top_k=17),
     dict(n_shared=-1), dict(n_shared=9), dict(n_shared=1, d_ff_shared=0),
-    dict(n_shared=1, d_ff_shared=40), dict(wfmt=4), dict(regime=3), dict(device=-1),
+    dict(n_shared=1, d_ff_shared=40), dict(wfmt=6), dict(regime=3), dict(device=-1),
 ])
 def test_plan_create_rejects_bad_config(L, kw):
     plan = ctypes.c_void_p(123)
@@ -67,9 +67,24 @@ def test_plan_create_q4_prefill_unsupported(L):
     # call gets past the argument checks and fails at the device query)
     s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=5, regime=2)), ctypes.byref(plan))
     assert s not in (B.MOE_ERR_UNSUPPORTED, B.MOE_ERR_INVALID_ARG)
-    # 4 is not a format of this ABI
-    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=4)), ctypes.byref(plan))
+    # 6 is not a format of this ABI
+    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=6)), ctypes.byref(plan))
     assert s == B.MOE_ERR_INVALID_ARG
+    # q6_K needs 256-multiples along every reduction dim, and runs in decode only
+    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=4, d_model=384)), ctypes.byref(plan))
+    assert s == B.MOE_ERR_INVALID_ARG
+    s = L.moe_plan_create(ctypes.byref(_cfg(wfmt=4, regime=2, d_model=256, d_ff=256)),
+                          ctypes.byref(plan))
+    assert s == B.MOE_ERR_UNSUPPORTED
+
+
+def test_q6_packed_bytes(L):
+    assert B.moe_q6_k_packed_bytes(2, 32, 512) == (2 * 32 * 16 * 16, 2 * 2 * 16 * 160 + 2 * 2 * 32 * 2)
+    for bad in ((1, 32, 288), (1, 24, 256), (-1, 16, 256)):
+        with pytest.raises(B.MoeError):
+            B.moe_q6_k_packed_bytes(*bad)
+    assert L.moe_q6_k_pack(None, 1, 16, 288, None, None, None) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_q6_k_pack(None, 1, 16, 256, None, None, None) == B.MOE_ERR_INVALID_ARG
 
 
 def test_bf16_to_f16_rejects_bad_args_without_gpu(L):

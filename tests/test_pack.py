@@ -118,3 +118,48 @@ def test_bf16_to_f16_every_pattern():
     assert torch.equal(torch.isnan(got), nan)
     assert torch.equal(got[~nan].view(torch.int16), want[~nan].view(torch.int16))
 
+
+_Q6_POS = [4, 8, 6, 10, 20, 24, 22, 26]     # bit of the high pair of nibble n, row g
+
+
+@pytest.mark.parametrize("n_mats,rows,k", [(1, 16, 256), (3, 48, 512), (2, 128, 1024)])
+def test_q6_k_pack_is_the_documented_records(n_mats, rows, k):
+    rng = np.random.default_rng(n_mats * 1000 + rows + 17)
+    canon = synth.q6_k_blocks(rng, n_mats * rows, k, 0.01).reshape(n_mats, rows, k // 256, 210)
+    codes, scales = _pack_on_gpu(B.moe_q6_k_packed_bytes, B.moe_q6_k_pack, canon, n_mats, rows, k)
+    nkb = k // 32
+    low = _unpack_nibble_words(codes.view(np.uint32).reshape(n_mats, nkb, rows, 4))   # [m][kb][r][32]
+    sb = scales.view(np.uint8)
+    aux_bytes = n_mats * nkb * (rows // 16) * 160
+    rec = sb[:aux_bytes].reshape(n_mats, nkb, rows // 16, 160)
+    hw = rec[..., :128].copy().view(np.uint32).reshape(n_mats, nkb, rows // 16, 8, 4)  # [g][t]
+    high = np.zeros((n_mats, nkb, rows, 32), np.int32)
+    for t in range(4):
+        slots = _word_slots(t)                     # (bit offset, element) of nibble n = offset // 4
+        for shift, idx in slots:
+            n = shift // 4
+            for half in (0, 1):                    # rows g and g + 8
+                p = (_Q6_POS[n] + 8 * half) % 32
+                v = (hw[..., t] >> p) & 3          # [m][kb][grp][g]
+                rr = (np.arange(rows // 16)[:, None] * 16 + np.arange(8)[None, :] + 8 * half)
+                high[:, :, rr.reshape(-1), idx] = v.reshape(n_mats, nkb, -1)
+    got = (low.astype(np.int32) + 16 * high).transpose(0, 2, 1, 3).reshape(n_mats, rows, k)
+    # canonical codes by the layout statement (element i = 128 h + 32 c + l)
+    ql = canon[..., :128].reshape(n_mats, rows, k // 256, 2, 2, 32).astype(np.int32)
+    qh = canon[..., 128:192].reshape(n_mats, rows, k // 256, 2, 32).astype(np.int32)
+    want = np.zeros((n_mats, rows, k // 256, 2, 4, 32), np.int32)
+    for c in range(4):
+        lo = (ql[..., :, c % 2, :] >> 4) if c >= 2 else (ql[..., :, c % 2, :] & 15)
+        want[..., c, :] = lo + 16 * ((qh >> (2 * c)) & 3)
+    assert np.array_equal(got, want.reshape(n_mats, rows, k))
+    subs = rec[..., 128:].reshape(n_mats, nkb, rows // 16, 8, 2, 2).view(np.int8)   # [g][row g/g+8][s]
+    got_sc = np.zeros((n_mats, rows, nkb, 2), np.int8)
+    for half in (0, 1):
+        rr = (np.arange(rows // 16)[:, None] * 16 + np.arange(8)[None, :] + 8 * half).reshape(-1)
+        got_sc[:, rr, :, :] = subs[:, :, :, :, half, :].reshape(n_mats, nkb, -1, 2).transpose(0, 2, 1, 3)
+    want_sc = canon[..., 192:208].copy().view(np.int8).reshape(n_mats, rows, k // 256, 8, 2)
+    assert np.array_equal(got_sc, want_sc.reshape(n_mats, rows, nkb, 2))
+    dd = sb[aux_bytes:].copy().view(np.uint16).reshape(n_mats, k // 256, rows)
+    want_d = canon[..., 208:210].copy().view(np.uint16)[..., 0]                        # [m][r][sb]
+    assert np.array_equal(dd.transpose(0, 2, 1), want_d)
+

@@ -48,6 +48,15 @@ SMALL = [
                    wfmt=synth.WFMT_Q5_0),
     synth.MoEShape("max_limits_q5", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32,
                    wfmt=synth.WFMT_Q5_0),
+    # q6_K (256-wide super-blocks): 24 block columns (a partial warp split), 72 block
+    # columns (two phase-A chunks, the second one partial), the interface limits
+    synth.MoEShape("ragged_q6", T=3, d=768, E=5, k=3, F=256, S=1, Fs=512, wfmt=synth.WFMT_Q6_K),
+    synth.MoEShape("chunked_q6", T=5, d=2304, E=8, k=2, F=512, S=1, Fs=256,
+                   wfmt=synth.WFMT_Q6_K),
+    synth.MoEShape("max_limits_q6", T=8, d=256, E=1024, k=16, F=256, S=8, Fs=256,
+                   wfmt=synth.WFMT_Q6_K),
+    # Q4_0 with 72 block columns: two phase-A chunks per row group
+    synth.MoEShape("chunked_q4", T=5, d=2304, E=8, k=2, F=96, S=1, Fs=64, wfmt=synth.WFMT_Q4_0),
     # bf16 gate/up with fp16 down matrices (h in fp16): 32- and 64-row slices
     synth.MoEShape("ragged_f16down", T=3, d=384, E=5, k=3, F=96, S=1, Fs=64,
                    wfmt=synth.WFMT_BF16_F16DOWN),
@@ -87,7 +96,9 @@ def _check(sh, seed=0, T=None, split=False):
                                   "a3b_q8_T1_d2048_E256k8_F512_S1",
                                   "a3b_q8_T8_d2048_E256k8_F512_S1",
                                   "a3b_q5_T1_d2048_E256k8_F512_S1",
-                                  "a3b_q5_T8_d2048_E256k8_F512_S1"])
+                                  "a3b_q5_T8_d2048_E256k8_F512_S1",
+                                  "a3b_q6_T1_d2048_E256k8_F512_S1",
+                                  "a3b_q6_T8_d2048_E256k8_F512_S1"])
 def test_decode_workloads_full_size(name):
     err = _check(W[name])
     print(f"{name}: rel L2 {err:.3e}")
@@ -103,7 +114,8 @@ def test_decode_small_shapes(sh):
     _check(sh, seed=1)
 
 
-SPLIT = SMALL[:6] + [SMALL[10], SMALL[-4], W["a3b_q4_T8_d2048_E256k8_F512_S1"]]
+SPLIT = SMALL[:6] + [SMALL[10], SMALL[-4], W["a3b_q4_T8_d2048_E256k8_F512_S1"],
+                     W["a3b_q6_T8_d2048_E256k8_F512_S1"]]
 
 
 @pytest.mark.parametrize("sh", SPLIT, ids=[s.name for s in SPLIT])
