@@ -158,14 +158,19 @@ bool map_bf16(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int
                       swizzle_for(static_cast<int>(box_k) * 2), box_k * 2);
 }
 
-// Q4_0 / Q8_0 / Q5_0 packed codes [mats][K/32][N][cb] (cb = 16 / 32 / 16
-// bytes per block row) seen as 3D {cb, N, mats*K/32}.
+// Q4_0 / Q8_0 / Q5_0 / q6_K packed codes [mats][K/32][N][cb] (cb = 16 / 32 /
+// 16 / 16 bytes per block row) seen as 3D {16 rows * cb, N/16, mats*K/32} in
+// 32-bit words: the innermost box dimension is a whole 16-row group, one
+// 256- or 512-byte line.  (Boxes of cb-byte lines move the same bytes in 16
+// times as many lines, and the TMA unit's line rate then caps the stream far
+// below HBM bandwidth.)  Coordinates: {0, first row / 16, block column}.
 bool map_quant_codes(moe_plan_s* p, CUtensorMap* m, const void* base, int64_t mats, int64_t N,
                      int64_t K, uint32_t box_rows, uint32_t box_kb, uint32_t cb) {
-    uint64_t dims[3] = {cb, static_cast<uint64_t>(N), static_cast<uint64_t>(mats * (K / 32))};
-    uint64_t strides[2] = {cb, static_cast<uint64_t>(N) * cb};
-    uint32_t box[3] = {cb, box_rows, box_kb};
-    return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+    uint64_t dims[3] = {16ull * cb / 4, static_cast<uint64_t>(N / 16),
+                        static_cast<uint64_t>(mats * (K / 32))};
+    uint64_t strides[2] = {16ull * cb, static_cast<uint64_t>(N) * cb};
+    uint32_t box[3] = {16 * cb / 4, box_rows / 16, box_kb};
+    return encode_map(p, m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, base, dims, strides, box,
                       CU_TENSOR_MAP_SWIZZLE_NONE, cb * box_rows);   // rows are contiguous
 }
 

@@ -472,8 +472,9 @@ template <int FS, int WF>
 __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const DecodeArgs& a) {
     using C = DecodeCfg<FS, WF>;
     DecodeSmem sm;
-    uint8_t* smem = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // align to 1 KB by pointer arithmetic on the shared array itself (a round
+    // trip through an integer would hide the address space from the compiler)
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     sm.ring = smem;
     sm.xs = sm.ring + static_cast<size_t>(a.n_stages) * C::STAGE;
     sm.xsum = reinterpret_cast<float*>(sm.xs + kDecodeTok * a.xs_stride);
@@ -628,7 +629,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                 for (int st = 0; st < nA + nB && ok; ++st, ++it) {
                     const int slot = it % ns;
                     if (it >= static_cast<uint32_t>(ns)) {
-                        if (*abort_flag || !mbar_wait_bounded(&empty[slot], ((it / ns) - 1) & 1)) {
+                        if (*abort_flag || !mbar_wait_bounded_sleep(&empty[slot], ((it / ns) - 1) & 1)) {
                             atomicOr(a.err, kErrTimeout); *abort_flag = 1; ok = false; break;
                         }
                     }
@@ -650,8 +651,9 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                             mbar_arrive_expect_tx(&full[slot], 2 * C::KB * FS * C::BR);
                             uint8_t* g = dst;
                             uint8_t* u2 = dst + C::KB * FS * C::BR;
-                            tma_load_3d(g, mg, &full[slot], 0, f0, c2, pol);
-                            tma_load_3d(u2, mu, &full[slot], 0, f0, c2, pol);
+                            // code maps address 16-row groups (one 256/512-byte line each)
+                            tma_load_3d(g, mg, &full[slot], 0, f0 / 16, c2, pol);
+                            tma_load_3d(u2, mu, &full[slot], 0, f0 / 16, c2, pol);
                             if constexpr (WF == kWfQ5) {
                                 // 48-byte records of 8 rows: {48 bytes, rows / 8, block columns}
                                 tma_load_3d(g + C::KB * FS * C::CB, mgs, &full[slot], 0, f0 / 8, c2, pol);
@@ -678,7 +680,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                             mbar_arrive_expect_tx(&full[slot], nbox * C::NB * QB * C::BR);
                             for (int b = 0; b < nbox; ++b) {
                                 uint8_t* bd = dst + b * (C::NB * QB * C::BR);
-                                tma_load_3d(bd, md, &full[slot], 0, j0 + QB * b, c2, pol);
+                                tma_load_3d(bd, md, &full[slot], 0, (j0 + QB * b) / 16, c2, pol);
                                 if constexpr (WF == kWfQ5)
                                     tma_load_3d(bd + C::NB * QB * C::CB, mds, &full[slot], 0,
                                                 (j0 + QB * b) / 8, c2, pol);
@@ -693,7 +695,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
             // drain: every issued stage must land before the CTA may exit
             const uint32_t first = it > static_cast<uint32_t>(ns) ? it - ns : 0;
             for (uint32_t q = first; q < it; ++q)
-                if (!mbar_wait_bounded(&full[q % ns], (q / ns) & 1)) {
+                if (!mbar_wait_bounded_sleep(&full[q % ns], (q / ns) & 1)) {
                     atomicOr(a.err, kErrTimeout);
                     break;
                 }
@@ -712,7 +714,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
     // warp-uniform: the ldmatrix / mma.sync that follow are warp-collective
     auto wait_full = [&](int slot, uint32_t parity) -> bool {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], parity));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded_sleep(&full[slot], parity));
         if (!ok && lane == 0) {
             atomicOr(a.err, kErrTimeout);
             *abort_flag = 1;
@@ -976,11 +978,16 @@ __device__ __forceinline__ void q6_scales(uint32_t sw, float dr, float dr8, floa
 // stages per row group when d > 2048), and consumer warp w owns block
 // columns w, w + 16, w + 32, w + 48 of every stage.  The x fragments and
 // block corrections of those columns therefore stay in registers for the
-// whole unit instead of being reloaded from shared memory for every 16x32
-// tile, which halves the shared-memory traffic per weight; each warp keeps
-// the partial sums of every row group and both matrices, and one reduction
-// over the 16 warps follows phase A.  Phase B (down matrix, combine) works
-// like experts_pipeline's.
+// whole unit; each warp keeps the partial sums of every row group and both
+// matrices, and one reduction over the 16 warps follows phase A.  Phase B
+// (down matrix, combine) works like experts_pipeline's.
+//
+// The hot loops are written for the instruction count: full stages (64
+// block columns, or RJ down rows) address shared memory through one 32-bit
+// per-lane base plus compile-time offsets, the ring slot and phase advance
+// incrementally (no division by the ring depth), and nothing branches per
+// block.  Partial stages (d not a multiple of 2048, the last down rows) take
+// a general path.
 //
 // Stage layouts.  Q4_0 phase A: codes [KC][16 rows][16 B], scales [KC][16]
 // fp16; phase B per 256-row box: codes [NB][256][16 B], scales [NB][256].
@@ -993,12 +1000,19 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                                                       const WorkView& wv) {
     using C = DecodeCfg<FS, WF>;
     static_assert(C::F16, "row-streaming phase A serves the fp16-operand formats");
-    static_assert(!C::Q6 || FS == 32, "q6_K slices are 32 rows");
+    static_assert(FS == 32, "row-streaming slices are 32 rows");
     constexpr int QB = kQuantDownBoxRows;
     // phase-B bytes of one 256-row box
     constexpr int BOXB = C::Q6 ? C::NB * QB * 16 + C::NB * (QB / 16) * 160 + QB * 2
                                : C::NB * QB * C::BR;
     static_assert((C::RJ / QB) * BOXB <= C::STAGE, "phase-B boxes fit a stage");
+    constexpr int RGW = C::RJ / 16 / kConsumerWarps;      // row groups per warp, full phase-B stage
+    static_assert(RGW * kConsumerWarps * 16 == C::RJ && C::RJ % QB == 0, "phase-B split");
+    constexpr int KCMAX = C::KCMAX;
+    // offsets inside a full phase-A stage (KC = 64)
+    constexpr uint32_t A_SCL = 16 * KCMAX * C::CB;                 // Q4_0 scales
+    constexpr uint32_t A_REC = 16 * KCMAX * 16;                    // q6_K records
+    constexpr uint32_t A_D = KCMAX * (16 * 16 + 160);              // q6_K super-block scales
     const int ns = a.n_stages;
     uint8_t* ring = sm.ring;
     float* gu = sm.gu;
@@ -1010,7 +1024,6 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
     const int nkb = d / 32;
     const int KC = a.kt;                              // block columns per phase-A stage
     const int nch = (nkb + KC - 1) / KC;              // phase-A stages per row group and matrix
-    // phase-A bytes of one stage
     const int stage_a = C::Q6 ? KC * (16 * 16 + 160) + (KC / 8) * 32 : 16 * KC * C::BR;
     const int n_routed = wv.n_routed, n_shared = wv.n_shared;
     const int sl_r = a.F / FS, sl_s = a.S ? a.Fs / FS : 0;
@@ -1047,7 +1060,9 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                 }
             }
             const uint64_t pol = l2_policy_evict_first();
-            uint32_t it = 0;
+            uint32_t it = 0;                  // stages issued
+            int slot = 0;
+            uint32_t ph = 0;                  // phase of the slot's current fill
             bool ok = true;
             for (int u = u_begin; u < n_units && ok; u += u_step) {
                 int ii, sl;
@@ -1058,9 +1073,8 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                 const int Fh = shared ? a.Fs : a.F;
                 const int f0 = sl * FS;
                 for (int st = 0; st < nA + nB && ok; ++st, ++it) {
-                    const int slot = it % ns;
                     if (it >= static_cast<uint32_t>(ns)) {
-                        if (*abort_flag || !mbar_wait_bounded(&empty[slot], ((it / ns) - 1) & 1)) {
+                        if (*abort_flag || !mbar_wait_bounded_sleep(&empty[slot], ph ^ 1u)) {
                             atomicOr(a.err, kErrTimeout); *abort_flag = 1; ok = false; break;
                         }
                     }
@@ -1075,7 +1089,7 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                         const int c2 = ex * nkb + c * KC;
                         const int r0 = f0 + rg * 16;
                         mbar_arrive_expect_tx(&full[slot], stage_a);
-                        tma_load_3d(dst, mc, &full[slot], 0, r0, c2, pol);
+                        tma_load_3d(dst, mc, &full[slot], 0, r0 / 16, c2, pol);   // 16-row groups
                         if constexpr (C::Q6) {
                             const CUtensorMap* md = mat ? (shared ? &a.tm_sup_d : &a.tm_up_d)
                                                         : (shared ? &a.tm_sgate_d : &a.tm_gate_d);
@@ -1094,7 +1108,7 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                         mbar_arrive_expect_tx(&full[slot], nbox * BOXB);
                         for (int b = 0; b < nbox; ++b) {
                             uint8_t* bd = dst + b * BOXB;
-                            tma_load_3d(bd, md, &full[slot], 0, j0 + QB * b, c2, pol);
+                            tma_load_3d(bd, md, &full[slot], 0, (j0 + QB * b) / 16, c2, pol);
                             if constexpr (C::Q6) {
                                 const CUtensorMap* mdd = shared ? &a.tm_sdown_d : &a.tm_down_d;
                                 tma_load_3d(bd + C::NB * QB * 16, mds, &full[slot], 0, (j0 + QB * b) / 16,
@@ -1107,11 +1121,13 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                             }
                         }
                     }
+                    if (++slot == ns) { slot = 0; ph ^= 1u; }
                 }
             }
+            // drain: every issued stage must land before the CTA may exit
             const uint32_t first = it > static_cast<uint32_t>(ns) ? it - ns : 0;
             for (uint32_t q = first; q < it; ++q)
-                if (!mbar_wait_bounded(&full[q % ns], (q / ns) & 1)) {
+                if (!mbar_wait_bounded_sleep(&full[q % ns], (q / ns) & 1)) {
                     atomicOr(a.err, kErrTimeout);
                     break;
                 }
@@ -1122,16 +1138,34 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
     // ---------------------------------------------------------- consumers
     const int g = lane >> 2, tig = lane & 3;
     const uint32_t xs_u = smem_u32(sm.xs);
+    const uint32_t ring_u = smem_u32(ring);
     constexpr int NC = C::Q6 ? 2 : 1;                 // corrections per block (per 16-k sub-block)
-    uint32_t it = 0;
-    auto wait_full = [&](int slot, uint32_t parity) -> bool {
+    // this lane's bases inside a stage: block column (phase A) or row group
+    // (phase B) `warp`, row g, code word tig
+    const uint32_t lane_code = warp * 256 + g * 16 + tig * 4;
+    const uint32_t lane_a_scl = A_SCL + warp * 32 + g * 2;
+    const uint32_t lane_a_rec = A_REC + warp * 160 + (4 * g + tig) * 4;
+    const uint32_t lane_a_sub = A_REC + warp * 160 + 128 + g * 4;
+    const uint32_t lane_a_d = A_D + (warp >> 3) * 32 + g * 2;
+    const uint32_t lane_b_scl = C::NB * QB * C::CB + warp * 32 + g * 2;
+    const uint32_t lane_b_rec = C::NB * QB * 16 + warp * 160 + (4 * g + tig) * 4;
+    const uint32_t lane_b_sub = C::NB * QB * 16 + warp * 160 + 128 + g * 4;
+    const uint32_t lane_b_d = C::NB * QB * 16 + C::NB * (QB / 16) * 160 + warp * 32 + g * 2;
+    int slot = 0;
+    uint32_t ph = 0;
+    auto wait_full = [&]() -> bool {
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], parity));
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded_sleep(&full[slot], ph));
         if (!ok && lane == 0) {
             atomicOr(a.err, kErrTimeout);
             *abort_flag = 1;
         }
         return ok;
+    };
+    auto release = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (++slot == ns) { slot = 0; ph ^= 1u; }
     };
 
     for (int u = u_begin; u < n_units; u += u_step) {
@@ -1171,73 +1205,102 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
         };
         if (nch == 1) load_x(0);
 
+        // one 16 x 32 block: x0 / x8 code words of rows g / g+8, e its q6_K
+        // high-bit word, sw the sub-scales, s0 / s8 (Q4_0) or dr / dr8 (q6_K)
+        // the scales; its two 16-wide halves are independent MMAs
+        auto block_q4 = [&](int i, uint32_t x0, uint32_t x8, float s0, float s8, float (&ac)[4]) {
+            const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
+            float va[4], vb[4];
+            mma_f16_16816(va, q4h_lo(x0), q4h_lo(x8), q4h_hi(x0), q4h_hi(x8), xf[i][0], xf[i][1],
+                          xc0[i][0], xc1[i][0], xc0[i][0], xc1[i][0]);
+            mma_f16_16816(vb, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8), xf[i][2], xf[i][3],
+                          0.f, 0.f, 0.f, 0.f);
+            ac[0] = fmaf(s0, va[0] + vb[0], ac[0]);
+            ac[1] = fmaf(s0, va[1] + vb[1], ac[1]);
+            ac[2] = fmaf(s8, va[2] + vb[2], ac[2]);
+            ac[3] = fmaf(s8, va[3] + vb[3], ac[3]);
+        };
+        auto block_q6 = [&](int i, uint32_t x0, uint32_t x8, uint32_t e, uint32_t sw, float dr, float dr8,
+                            float (&ac)[4]) {
+            uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
+            q6h_regs(x0, e, p0, p1, p2, p3);
+            q6h_regs(x8, __funnelshift_r(e, e, 8), q0, q1, q2, q3);
+            float va[4], vb[4];
+            mma_f16_16816(va, p0, q0, p1, q1, xf[i][0], xf[i][1], xc0[i][0], xc1[i][0], xc0[i][0],
+                          xc1[i][0]);
+            mma_f16_16816(vb, p2, q2, p3, q3, xf[i][2], xf[i][3], xc0[i][NC - 1], xc1[i][NC - 1],
+                          xc0[i][NC - 1], xc1[i][NC - 1]);
+            float s00, s01, s80, s81;
+            q6_scales(sw, dr, dr8, s00, s01, s80, s81);
+            ac[0] = fmaf(s00, va[0], fmaf(s01, vb[0], ac[0]));
+            ac[1] = fmaf(s00, va[1], fmaf(s01, vb[1], ac[1]));
+            ac[2] = fmaf(s80, va[2], fmaf(s81, vb[2], ac[2]));
+            ac[3] = fmaf(s80, va[3], fmaf(s81, vb[3], ac[3]));
+        };
+
         // ------------------------------------------- phase A: gate and up
         float acc[2 * C::RG][4];
 #pragma unroll
         for (int q = 0; q < 2 * C::RG; ++q)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
+        const bool fast_a = KC == KCMAX;
 #pragma unroll
         for (int rg = 0; rg < C::RG; ++rg) {
 #pragma unroll
             for (int mat = 0; mat < 2; ++mat) {
-                for (int c = 0; c < nch; ++c, ++it) {
-                    const int slot = it % ns;
-                    const bool ok = wait_full(slot, (it / ns) & 1);
+                for (int c = 0; c < nch; ++c) {
+                    const bool ok = wait_full();
                     if (ok) {
                         if (nch > 1) load_x(c);
-                        const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
-                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(stage);   // [KC][16][16 B]
-                        float* ac = acc[rg * 2 + mat];
+                        const uint32_t st_u = ring_u + slot * C::STAGE;
+                        float (&ac)[4] = acc[rg * 2 + mat];
+                        if (fast_a && (c + 1) * KCMAX <= nkb) {
+                            // all four block columns of this warp are in the stage
 #pragma unroll
-                        for (int i = 0; i < C::NBW; ++i) {
-                            const int bl = warp + kConsumerWarps * i;
-                            if (bl < KC && c * KC + bl < nkb) {
-                                const uint32_t* row = codes + (bl * 16 + g) * 4;
-                                const uint32_t x0 = row[tig], x8 = row[32 + tig];
+                            for (int i = 0; i < C::NBW; ++i) {
+                                const uint32_t cb = st_u + lane_code + i * (16 * 16 * 16);
+                                const uint32_t x0 = lds_u32(cb), x8 = lds_u32(cb + 128);
                                 if constexpr (C::Q6) {
-                                    const uint32_t* rec =
-                                        reinterpret_cast<const uint32_t*>(stage + 16 * KC * 16 + bl * 160);
-                                    const __half* dsm =
-                                        reinterpret_cast<const __half*>(stage + KC * (16 * 16 + 160));
-                                    const uint32_t e = rec[4 * g + tig];
-                                    uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
-                                    q6h_regs(x0, e, p0, p1, p2, p3);
-                                    q6h_regs(x8, __funnelshift_r(e, e, 8), q0, q1, q2, q3);
-                                    float va[4], vb[4];
-                                    mma_f16_16816(va, p0, q0, p1, q1, xf[i][0], xf[i][1],
-                                                  xc0[i][0], xc1[i][0], xc0[i][0], xc1[i][0]);
-                                    mma_f16_16816(vb, p2, q2, p3, q3, xf[i][2], xf[i][3],
-                                                  xc0[i][NC - 1], xc1[i][NC - 1], xc0[i][NC - 1],
-                                                  xc1[i][NC - 1]);
-                                    float s00, s01, s80, s81;
-                                    q6_scales(rec[32 + g], __half2float(dsm[(bl >> 3) * 16 + g]),
-                                              __half2float(dsm[(bl >> 3) * 16 + g + 8]), s00, s01, s80, s81);
-                                    ac[0] = fmaf(s00, va[0], fmaf(s01, vb[0], ac[0]));
-                                    ac[1] = fmaf(s00, va[1], fmaf(s01, vb[1], ac[1]));
-                                    ac[2] = fmaf(s80, va[2], fmaf(s81, vb[2], ac[2]));
-                                    ac[3] = fmaf(s80, va[3], fmaf(s81, vb[3], ac[3]));
+                                    const uint32_t e = lds_u32(st_u + lane_a_rec + i * (16 * 160));
+                                    const uint32_t sw = lds_u32(st_u + lane_a_sub + i * (16 * 160));
+                                    const float dr = lds_f16_as_f32(st_u + lane_a_d + i * 64);
+                                    const float dr8 = lds_f16_as_f32(st_u + lane_a_d + i * 64 + 16);
+                                    block_q6(i, x0, x8, e, sw, dr, dr8, ac);
                                 } else {
-                                    const __half* scl = reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
-                                    float v[4];
-                                    mma_f16_16816(v, q4h_lo(x0), q4h_lo(x8), q4h_hi(x0), q4h_hi(x8),
-                                                  xf[i][0], xf[i][1], xc0[i][0], xc1[i][0], xc0[i][0],
-                                                  xc1[i][0]);
-                                    const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
-                                    mma_f16_16816_acc(v, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8),
-                                                      xf[i][2], xf[i][3]);
-                                    const float s0 = __half2float(scl[bl * 16 + g]);
-                                    const float s8 = __half2float(scl[bl * 16 + g + 8]);
-                                    ac[0] = fmaf(s0, v[0], ac[0]);
-                                    ac[1] = fmaf(s0, v[1], ac[1]);
-                                    ac[2] = fmaf(s8, v[2], ac[2]);
-                                    ac[3] = fmaf(s8, v[3], ac[3]);
+                                    const float s0 = lds_f16_as_f32(st_u + lane_a_scl + i * 512);
+                                    const float s8 = lds_f16_as_f32(st_u + lane_a_scl + i * 512 + 16);
+                                    block_q4(i, x0, x8, s0, s8, ac);
+                                }
+                            }
+                        } else {
+                            const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
+                            const uint32_t* codes = reinterpret_cast<const uint32_t*>(stage);
+#pragma unroll
+                            for (int i = 0; i < C::NBW; ++i) {
+                                const int bl = warp + kConsumerWarps * i;
+                                if (bl < KC && c * KC + bl < nkb) {
+                                    const uint32_t* row = codes + (bl * 16 + g) * 4;
+                                    const uint32_t x0 = row[tig], x8 = row[32 + tig];
+                                    if constexpr (C::Q6) {
+                                        const uint32_t* rec =
+                                            reinterpret_cast<const uint32_t*>(stage + 16 * KC * 16 + bl * 160);
+                                        const __half* dsm =
+                                            reinterpret_cast<const __half*>(stage + KC * (16 * 16 + 160));
+                                        block_q6(i, x0, x8, rec[4 * g + tig], rec[32 + g],
+                                                 __half2float(dsm[(bl >> 3) * 16 + g]),
+                                                 __half2float(dsm[(bl >> 3) * 16 + g + 8]), ac);
+                                    } else {
+                                        const __half* scl =
+                                            reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
+                                        block_q4(i, x0, x8, __half2float(scl[bl * 16 + g]),
+                                                 __half2float(scl[bl * 16 + g + 8]), ac);
+                                    }
                                 }
                             }
                         }
                     }
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[slot]);
+                    release();
                 }
             }
         }
@@ -1306,81 +1369,101 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
         }
 
         // --------------------------------------- phase B: down + combine
-        for (int st = 0; st < nB; ++st, ++it) {
-            const int slot = it % ns;
-            const bool ok = wait_full(slot, (it / ns) & 1);
-            const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
+        // one 16-row group, given its 32-bit stage addresses: the block's
+        // halves (q6_K: sub-blocks) are independent MMA chains (hi part, then
+        // lo part of h)
+        auto rowgroup = [&](uint32_t code_u, uint32_t scl_u, uint32_t rec_u, uint32_t sub_u,
+                            uint32_t d_u, float (&c)[4]) {
+            c[0] = c[1] = c[2] = c[3] = 0.f;
+#pragma unroll
+            for (int bb = 0; bb < C::NB; ++bb) {
+                const uint32_t x0 = lds_u32(code_u + bb * (QB * 16));
+                const uint32_t x8 = lds_u32(code_u + bb * (QB * 16) + 128);
+                if constexpr (C::Q6) {
+                    const uint32_t e = lds_u32(rec_u + bb * (16 * 160));
+                    uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
+                    q6h_regs(x0, e, p0, p1, p2, p3);
+                    q6h_regs(x8, __funnelshift_r(e, e, 8), q0, q1, q2, q3);
+                    float va[4], vb[4];
+                    mma_f16_16816(va, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
+                                  hs0[2 * bb], hs1[2 * bb], hs0[2 * bb], hs1[2 * bb]);
+                    mma_f16_16816(vb, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1],
+                                  hs0[2 * bb + 1], hs1[2 * bb + 1], hs0[2 * bb + 1], hs1[2 * bb + 1]);
+                    mma_f16_16816_acc(va, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                    mma_f16_16816_acc(vb, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                    float s00, s01, s80, s81;
+                    q6_scales(lds_u32(sub_u + bb * (16 * 160)), lds_f16_as_f32(d_u),
+                              lds_f16_as_f32(d_u + 16), s00, s01, s80, s81);
+                    c[0] = fmaf(s00, va[0], fmaf(s01, vb[0], c[0]));
+                    c[1] = fmaf(s00, va[1], fmaf(s01, vb[1], c[1]));
+                    c[2] = fmaf(s80, va[2], fmaf(s81, vb[2], c[2]));
+                    c[3] = fmaf(s80, va[3], fmaf(s81, vb[3], c[3]));
+                } else {
+                    const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
+                    const uint32_t p0 = q4h_lo(x0), q0 = q4h_lo(x8);
+                    const uint32_t p1 = q4h_hi(x0), q1 = q4h_hi(x8);
+                    const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
+                    const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
+                    float va[4], vb[4];
+                    mma_f16_16816(va, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
+                                  hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
+                    mma_f16_16816(vb, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1],
+                                  0.f, 0.f, 0.f, 0.f);
+                    mma_f16_16816_acc(va, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                    mma_f16_16816_acc(vb, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                    const float s0 = lds_f16_as_f32(scl_u + bb * (QB * 2));
+                    const float s8 = lds_f16_as_f32(scl_u + bb * (QB * 2) + 16);
+                    c[0] = fmaf(s0, va[0] + vb[0], c[0]);
+                    c[1] = fmaf(s0, va[1] + vb[1], c[1]);
+                    c[2] = fmaf(s8, va[2] + vb[2], c[2]);
+                    c[3] = fmaf(s8, va[3] + vb[3], c[3]);
+                }
+            }
+        };
+        auto combine = [&](int j, const float (&c)[4]) {      // j: first row of the group + g
+            if (v0) {
+                red_add_f32(a.out + static_cast<size_t>(tok0) * d + j, w0 * c[0]);
+                red_add_f32(a.out + static_cast<size_t>(tok0) * d + j + 8, w0 * c[2]);
+            }
+            if (v1) {
+                red_add_f32(a.out + static_cast<size_t>(tok1) * d + j, w1 * c[1]);
+                red_add_f32(a.out + static_cast<size_t>(tok1) * d + j + 8, w1 * c[3]);
+            }
+        };
+        for (int st = 0; st < nB; ++st) {
+            const bool ok = wait_full();
             const int j0 = st * C::RJ;
             const int rows = min(C::RJ, d - j0);
             if (ok) {
-                for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
-                    float c[4] = {0.f, 0.f, 0.f, 0.f};
-                    const uint8_t* bbase = stage + (rgb / (QB / 16)) * BOXB;
-                    const uint32_t* codes = reinterpret_cast<const uint32_t*>(bbase);   // [NB][QB][16 B]
-                    const int grp = rgb % (QB / 16);
-                    const int rib = grp * 16 + g;
+                const uint32_t st_u = ring_u + slot * C::STAGE;
+                if (rows == C::RJ) {
+                    // row groups warp + 16 q (q < RGW) sit in box q at group `warp`:
+                    // all of them first, then all their reductions into out
+                    float c[RGW][4];
 #pragma unroll
-                    for (int bb = 0; bb < C::NB; ++bb) {
-                        const uint32_t* row = codes + (bb * QB + rib) * 4;
-                        const uint32_t x0 = row[tig], x8 = row[32 + tig];
-                        if constexpr (C::Q6) {
-                            const uint32_t* rec = reinterpret_cast<const uint32_t*>(
-                                bbase + C::NB * QB * 16 + (bb * (QB / 16) + grp) * 160);
-                            const __half* dsm = reinterpret_cast<const __half*>(
-                                bbase + C::NB * QB * 16 + C::NB * (QB / 16) * 160);
-                            const uint32_t e = rec[4 * g + tig];
-                            uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
-                            q6h_regs(x0, e, p0, p1, p2, p3);
-                            q6h_regs(x8, __funnelshift_r(e, e, 8), q0, q1, q2, q3);
-                            float va[4], vb[4];
-                            mma_f16_16816(va, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
-                                          hs0[2 * bb], hs1[2 * bb], hs0[2 * bb], hs1[2 * bb]);
-                            mma_f16_16816_acc(va, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
-                            mma_f16_16816(vb, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1],
-                                          hs0[2 * bb + 1], hs1[2 * bb + 1], hs0[2 * bb + 1],
-                                          hs1[2 * bb + 1]);
-                            mma_f16_16816_acc(vb, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
-                            float s00, s01, s80, s81;
-                            q6_scales(rec[32 + g], __half2float(dsm[rib]), __half2float(dsm[rib + 8]),
-                                      s00, s01, s80, s81);
-                            c[0] = fmaf(s00, va[0], fmaf(s01, vb[0], c[0]));
-                            c[1] = fmaf(s00, va[1], fmaf(s01, vb[1], c[1]));
-                            c[2] = fmaf(s80, va[2], fmaf(s81, vb[2], c[2]));
-                            c[3] = fmaf(s80, va[3], fmaf(s81, vb[3], c[3]));
-                        } else {
-                            const __half* scl = reinterpret_cast<const __half*>(bbase + C::NB * QB * C::CB);
-                            const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
-                            const uint32_t p0 = q4h_lo(x0), q0 = q4h_lo(x8);
-                            const uint32_t p1 = q4h_hi(x0), q1 = q4h_hi(x8);
-                            const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
-                            const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
-                            float v[4];
-                            mma_f16_16816(v, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
-                                          hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
-                            mma_f16_16816_acc(v, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
-                            mma_f16_16816_acc(v, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
-                            mma_f16_16816_acc(v, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
-                            const float s0 = __half2float(scl[bb * QB + rib]);
-                            const float s8 = __half2float(scl[bb * QB + rib + 8]);
-                            c[0] = fmaf(s0, v[0], c[0]);
-                            c[1] = fmaf(s0, v[1], c[1]);
-                            c[2] = fmaf(s8, v[2], c[2]);
-                            c[3] = fmaf(s8, v[3], c[3]);
-                        }
+                    for (int q = 0; q < RGW; ++q) {
+                        const uint32_t bq = st_u + q * BOXB;
+                        rowgroup(bq + lane_code, bq + lane_b_scl, bq + lane_b_rec, bq + lane_b_sub,
+                                 bq + lane_b_d, c[q]);
                     }
-                    const int j = j0 + rgb * 16 + g;
-                    if (v0) {
-                        red_add_f32(a.out + static_cast<size_t>(tok0) * d + j, w0 * c[0]);
-                        red_add_f32(a.out + static_cast<size_t>(tok0) * d + j + 8, w0 * c[2]);
-                    }
-                    if (v1) {
-                        red_add_f32(a.out + static_cast<size_t>(tok1) * d + j, w1 * c[1]);
-                        red_add_f32(a.out + static_cast<size_t>(tok1) * d + j + 8, w1 * c[3]);
+#pragma unroll
+                    for (int q = 0; q < RGW; ++q)
+                        combine(j0 + (warp + kConsumerWarps * q) * 16 + g, c[q]);
+                } else {
+                    for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
+                        const int grp = rgb % (QB / 16);
+                        const uint32_t bq = st_u + (rgb / (QB / 16)) * BOXB;
+                        const uint32_t lc = grp * 256 + g * 16 + tig * 4;
+                        float c[4];
+                        rowgroup(bq + lc, bq + C::NB * QB * C::CB + grp * 32 + g * 2,
+                                 bq + C::NB * QB * 16 + grp * 160 + (4 * g + tig) * 4,
+                                 bq + C::NB * QB * 16 + grp * 160 + 128 + g * 4,
+                                 bq + C::NB * QB * 16 + C::NB * (QB / 16) * 160 + grp * 32 + g * 2, c);
+                        combine(j0 + rgb * 16 + g, c);
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
+            release();
         }
     }
 }
