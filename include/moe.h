@@ -190,8 +190,9 @@ void moe_plan_destroy(moe_plan_t plan);
  * `routing` may be NULL; when given, the routing tables are copied to it
  * (device-to-device, on `stream`).  T = 0 enqueues nothing.
  * Launches: decode regime -- 1 cooperative kernel (router, top-k, buckets,
- * every routed and shared expert, weighted combine; a grid barrier separates
- * routing from the experts); if the device cannot co-schedule that grid, the
+ * every routed and shared expert, weighted combine; each CTA waits for the
+ * router logits of all others, tagged with the launch, before it routes);
+ * if the device cannot co-schedule that grid, the
  * two-launch path of moe_route + moe_experts.  Prefill regime -- 4 kernels
  * (router, bucket scatter + row gather, gate/up GEMM, down GEMM with the
  * weighted combine).  Work enqueued with one plan must not overlap on the
@@ -271,24 +272,26 @@ int32_t moe_last_launch_count(moe_plan_t plan);
 /* Read and clear the sticky device error word (synchronises `plan`'s device).
  * The pages have no counterpart (they describe no failure handling).
  * OK, DEVICE_FLAG (a kernel saw an out-of-range id or count) or TIMEOUT (a
- * bounded wait -- of a pipeline stage or the fused kernel's grid barrier --
- * gave up, after at most 2 s; the kernel then skipped its remaining work, so
- * that call's `out` is incomplete).  A fused decode launch that starts while
- * such a timeout is still unread does no work at all: it writes NaN to its
- * `out` and the next read of this word also returns TIMEOUT (a timed-out
- * grid barrier may have been left mid-round, and computing on it could
- * route on stale logits).  Reading the word resets the plan's barrier. */
+ * bounded wait -- of a pipeline stage, or of the fused kernel's wait for
+ * the other CTAs' router logits -- gave up, after at most 2 s; the kernel
+ * then skipped its remaining work, so that call's `out` is incomplete).  A
+ * fused decode launch that starts while such a timeout is still unread does
+ * no work at all: it writes NaN to its `out` and the next read of this word
+ * also returns TIMEOUT (the launch ticket count a timeout leaves behind may
+ * be mid-round, and computing on it could route on stale logits).  Reading
+ * a TIMEOUT resets the plan's ticket count and logit words. */
 moe_status_t moe_get_device_status(moe_plan_t plan);
 
 /* Failure-path check (the pages have no counterpart): make the next fused
- * decode launch of `plan` unable to pass its grid barrier, by setting the
- * plan's barrier count to 1 (async memsets on `stream`), a value the
- * launch's arrivals cannot bring to the last CTA's target.  That CTA waits
- * the bounded 2 s, skips its expert work, and exits, so the call's `out` is
- * incomplete; moe_get_device_status then returns MOE_ERR_TIMEOUT and resets
- * the barrier, after which the plan works normally again.  Nothing hangs and
- * nothing faults.  UNSUPPORTED if the device cannot run the fused
- * (cooperative) launch. */
+ * decode launch of `plan` unable to finish routing, by setting the plan's
+ * launch ticket count to 1 (async memsets on `stream`), a value from which
+ * the launch's CTAs derive two different tags, so that no CTA ever sees
+ * every router logit carry its own tag.  Each waits the bounded 2 s, skips
+ * its expert work, and exits, so the call's `out` is incomplete;
+ * moe_get_device_status then returns MOE_ERR_TIMEOUT and resets the count,
+ * after which the plan works normally again.  Nothing hangs and nothing
+ * faults.  UNSUPPORTED if the device cannot run the fused (cooperative)
+ * launch. */
 moe_status_t moe_debug_stall_barrier(moe_plan_t plan, void* stream);
 
 /* Bytes of the packed Q4_0 form of n_mats matrices of [rows][k] weights.

@@ -365,8 +365,10 @@ moe_status_t decode_args(moe_plan_s* p, const moe_weights_t* w, const void* x, i
     int ns = static_cast<int>((p->smem_optin - fixed) / (stage + 16));
     if (ns > 8) ns = 8;
     if (ns < 2) return MOE_ERR_UNSUPPORTED;
-    // the fused kernel keeps the T x E logits in the ring during routing
-    if (fused && static_cast<size_t>(ns) * stage < static_cast<size_t>(T) * c.n_experts * 4)
+    // the fused kernel keeps its router partial sums ([experts per CTA][16][8]
+    // fp32) in the ring during routing
+    const size_t n_loc = (static_cast<size_t>(c.n_experts) + p->num_sms - 1) / p->num_sms;
+    if (fused && static_cast<size_t>(ns) * stage < n_loc * kDecodeConsumerWarps * kDecodeTok * 4)
         return MOE_ERR_UNSUPPORTED;
     a.n_stages = ns;
     *out_args = ap;
@@ -481,6 +483,7 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     const size_t o_sp = take(T * k * 4), o_st = take(T * k * 4), o_sw = take(T * k * 4);
     const size_t o_items = take((E + S) * sizeof(WorkItem)), o_nitems = take(16);
     const size_t o_ticket = take(16), o_err = take(16), o_gbar = take(16);
+    const size_t o_tl = take(static_cast<size_t>(kDecodeTok) * E * 8);
     size_t o_xp = 0, o_hr = 0, o_hs = 0, o_tiles = 0, o_nt = 0;
     if (prefill) {
         o_xp = take(T * k * d * 2);
@@ -510,6 +513,7 @@ moe_status_t moe_plan_create(const moe_config_t* cfg, moe_plan_t* out) {
     w.ticket = reinterpret_cast<uint32_t*>(b + o_ticket);
     w.err = reinterpret_cast<uint32_t*>(b + o_err);
     w.gbar = reinterpret_cast<uint32_t*>(b + o_gbar);
+    w.tlogits = reinterpret_cast<unsigned long long*>(b + o_tl);
     if (prefill) {
         w.x_perm = reinterpret_cast<uint16_t*>(b + o_xp);
         w.h_routed = reinterpret_cast<uint16_t*>(b + o_hr);
@@ -632,8 +636,12 @@ moe_status_t moe_get_device_status(moe_plan_t p) {
     if (v && cudaMemset(p->ws.err, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
     if (v & (kErrTimeout | kErrSkipped)) {
         // a launch gave up waiting (or skipped its work because of an earlier
-        // timeout): leave the grid barrier words clean for the next one
-        if (cudaMemset(p->ws.gbar, 0, 16) != cudaSuccess) return MOE_ERR_CUDA;
+        // timeout): leave the launch ticket count and the tagged logit words
+        // clean for the next one
+        if (cudaMemset(p->ws.gbar, 0, 16) != cudaSuccess ||
+            cudaMemset(p->ws.tlogits, 0, static_cast<size_t>(kDecodeTok) * p->cfg.n_experts * 8) !=
+                cudaSuccess)
+            return MOE_ERR_CUDA;
         return MOE_ERR_TIMEOUT;
     }
     if (v) return MOE_ERR_DEVICE_FLAG;
@@ -644,10 +652,14 @@ moe_status_t moe_debug_stall_barrier(moe_plan_t p, void* stream) {
     if (!p) return MOE_ERR_INVALID_ARG;
     if (!p->coop) return MOE_ERR_UNSUPPORTED;
     DeviceGuard dg(p->cfg.device);
-    // an arrival count of 1 (not a multiple of the grid): after the next
-    // launch's G arrivals the count is G + 1, short of the target 2G of the
-    // CTA that arrives last, whose bounded wait runs out
+    // a ticket count of 1 (not a multiple of the grid): the next launch's
+    // CTAs draw tickets 1..G, from which the one holding ticket G derives the
+    // tag 2G and the others G; its wait for logits tagged 2G (and, when it
+    // publishes logits, the others' wait for logits tagged G) runs out
     cudaError_t e = cudaMemsetAsync(p->ws.gbar, 0, 16, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(p->ws.tlogits, 0, static_cast<size_t>(kDecodeTok) * p->cfg.n_experts * 8,
+                            static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = cudaMemsetAsync(p->ws.gbar, 0x01, 1, static_cast<cudaStream_t>(stream));
     return cuda_status(e);
 }

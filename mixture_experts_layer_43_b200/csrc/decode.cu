@@ -27,6 +27,7 @@
 // written back ("MMVQ" page: read quantised weights once, never expand them).
 #include <float.h>
 #include <math.h>
+#include <stddef.h>
 
 #include "moe_internal.cuh"
 
@@ -216,7 +217,7 @@ cudaError_t launch_decode_route(const RouteArgs& a, cudaStream_t stream) {
 }
 
 // ============================================================ experts ===
-constexpr int kConsumerWarps = 16;
+constexpr int kConsumerWarps = kDecodeConsumerWarps;
 constexpr int kConsumers = kConsumerWarps * 32;
 constexpr int kDecodeThreads = kConsumers + 32;   // + one producer warp
 
@@ -1499,13 +1500,17 @@ decode_experts_kernel(const __grid_constant__ DecodeArgs a) {
 // ====================================================== fused decode ===
 // One cooperative launch for the whole layer (T <= 8):
 //   R  every CTA computes the router logits of experts b, b+G, ... (fp32 FMA,
-//      each dot product split over 8 warps and summed in a fixed order) and
-//      zero-fills its share of `out`;
-//   -  grid barrier (a 64-bit arrival count that only grows, bounded wait);
-//   T  every CTA reads all T x E logits and computes the same top-k,
-//      renormalised weights, stable slots and work list in its own shared
-//      memory (no second barrier); CTA 0 also writes the routing tables;
+//      each dot product split over the 16 consumer warps and summed in a
+//      fixed order) and publishes them, each as one 64-bit word that also
+//      holds this launch's tag; the producer warp zero-fills the CTA's share
+//      of `out` meanwhile;
+//   T  every CTA reads all T x E logit words, waiting (bounded) until each
+//      carries this launch's tag, and computes the same top-k, renormalised
+//      weights, stable slots and work list in its own shared memory; CTA 0
+//      also writes the routing tables;
 //   X  the experts pipeline, reading the work list from shared memory.
+// There is no separate grid barrier: the tag on every logit is the only
+// signal a CTA waits for (see the notes above decode_fused_kernel).
 // Compared with the two-launch path this removes the launch gap between
 // router and experts and the router kernel's last-CTA tail.
 constexpr int kFusedMaxPairs = kDecodeTok * kMaxTopK;   // 128
@@ -1517,32 +1522,123 @@ struct alignas(16) FusedRouteSmem {
     float w[kFusedMaxPairs];
     int slot_token[kFusedMaxPairs];
     float slot_w[kFusedMaxPairs];
-    float sel[kDecodeTok][kMaxTopK];
     uint32_t emask[kMaxExperts / 32];   // bit e: expert e was selected by some token
     int n_routed;
     int skip;                           // this launch does no work (see decode_fused_kernel)
-    int pad[2];
+    unsigned long long tag;             // this launch's logit tag (in the high 32 bits)
 };
+
+static_assert(kFusedMaxPairs % 4 == 0 && offsetof(FusedRouteSmem, ids) % 16 == 0,
+              "pair ids read as whole int4s");
+static_assert(kFusedMaxPairs <= kConsumers / 2, "pair threads and table threads are disjoint");
 
 size_t decode_fused_extra_smem() { return sizeof(FusedRouteSmem); }
 
-// Grid-wide barrier of a cooperative launch; thread 0 of each CTA calls it.
-// gbar[0..1] is a 64-bit arrival counter that only grows: the G CTAs of one
-// launch raise it from n*G to (n+1)*G.  Each CTA takes its launch's target
-// from the value its own arrival returned and polls until the counter
-// reaches it (one atomic per CTA, no reset, no second word to publish).
-// The count starts at a multiple of G as long as every earlier launch
-// arrived completely; after a timed-out wait the host resets it to 0.
-__device__ __forceinline__ bool grid_barrier(uint32_t* gbar, uint32_t nblocks) {
-    unsigned long long* ctr = reinterpret_cast<unsigned long long*>(gbar);
-    __threadfence();                       // this CTA's logits before its arrival
-    const unsigned long long old = atomicAdd(ctr, 1ull);
-    const unsigned long long target = old - old % nblocks + nblocks;
+// How the CTAs of one fused launch agree that routing may start, without a
+// grid barrier:
+//  - Launch tag.  At its start each CTA takes a ticket: one relaxed atomic
+//    increment of a 64-bit count that only grows.  The G CTAs of a launch
+//    raise it from n*G to (n+1)*G, so each CTA derives the same tag
+//    (n+1)*G from its own ticket, as long as every earlier launch took all
+//    its tickets (after a timeout the host resets the count to 0).  The
+//    ticket's latency hides behind the router loads.
+//  - Logit words.  Logit (t, e) is stored as one 64-bit word, fp32 bits low
+//    and the low 32 bits of the tag high (one single-copy-atomic word: a
+//    reader that sees the tag sees the value).  The producer warp stores
+//    them, relaxed, after a release fence that follows its zero-fill of
+//    `out`.  Every launch writes all kDecodeTok token rows of its experts
+//    (rows t >= T with a zero value), so before a launch writes, each word
+//    holds the previous launch's tag, never the current one.
+//  - `out` zero-fill.  Done by the CTAs that own experts (b < E), each of
+//    which publishes logits that every CTA's warp 0 reads.
+// Reader side: warp t of each CTA loads the E words of token t with relaxed
+// loads until every one carries the tag (bounded by kWaitLimitNs; on
+// timeout it records kErrTimeout and the CTA skips phase X) and routes on
+// the values.  Its acquire fence comes after routing, at the start of phase
+// X: the fence pairs with the writers' release fences, and a named barrier
+// of the consumers separates it from the first add into `out`.  So every
+// add follows every zero-fill, and the fence's wait overlaps the first
+// weight loads instead of delaying the routing.
+
+// Token t's routing in the fused kernel (one warp): wait until all E logit
+// words of the token carry `tag`, then the top-k of the values (the caller
+// issues the acquire fence later, before phase X).
+// Returns false when the bounded wait ran out (the selection is then made
+// from whatever the words hold; the caller aborts phase X).
+template <int PER>
+__device__ __forceinline__ bool fused_token_topk(const unsigned long long* row, int E, int k,
+                                                 uint32_t tag, uint32_t* err, float& sel, int& id) {
+    const int lane = threadIdx.x & 31;
+    unsigned long long wv[PER];
     const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_u64(ctr) < target) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    bool ok = true;
+    while (true) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int x = lane + 32 * i;
+            wv[i] = ld_relaxed_u64(row + (x < E ? x : E - 1));
+        }
+        bool mine = true;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) mine &= static_cast<uint32_t>(wv[i] >> 32) == tag;
+        if (__all_sync(0xffffffffu, mine)) break;
+        if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {
+            ok = false;
+            break;
+        }
     }
-    return true;
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        v[i] = __uint_as_float(static_cast<uint32_t>(wv[i]));
+        if (lane + 32 * i >= E || isnan(v[i])) v[i] = -INFINITY;
+    }
+    warp_topk_select<PER>(v, E, k, err, sel, id);
+    return ok;
+}
+
+// The same for E > 256: the wait checks the tags only, the values are read
+// again after it (64 words per lane would not fit in registers next to the
+// values).
+__device__ __forceinline__ bool fused_token_topk_wide(const unsigned long long* row, int E, int k,
+                                                      uint32_t tag, uint32_t* err, float& sel,
+                                                      int& id) {
+    constexpr int PER = 32;
+    const int lane = threadIdx.x & 31;
+    const uint64_t t0 = globaltimer_ns();
+    bool ok = true;
+    while (true) {
+        bool mine = true;
+#pragma unroll 8
+        for (int i = 0; i < PER; ++i) {
+            const int x = lane + 32 * i;
+            mine &= static_cast<uint32_t>(ld_relaxed_u64(row + (x < E ? x : E - 1)) >> 32) == tag;
+        }
+        if (__all_sync(0xffffffffu, mine)) break;
+        if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > kWaitLimitNs)) {
+            ok = false;
+            break;
+        }
+    }
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int x = lane + 32 * i;
+        v[i] = __uint_as_float(static_cast<uint32_t>(ld_relaxed_u64(row + (x < E ? x : E - 1))));
+        if (x >= E || isnan(v[i])) v[i] = -INFINITY;
+    }
+    warp_topk_select<PER>(v, E, k, err, sel, id);
+    return ok;
+}
+
+__device__ __forceinline__ bool fused_token_topk_any(const unsigned long long* row, int E, int k,
+                                                     uint32_t tag, uint32_t* err, float& sel,
+                                                     int& id) {
+    if (E <= 32) return fused_token_topk<1>(row, E, k, tag, err, sel, id);
+    if (E <= 64) return fused_token_topk<2>(row, E, k, tag, err, sel, id);
+    if (E <= 128) return fused_token_topk<4>(row, E, k, tag, err, sel, id);
+    if (E <= 256) return fused_token_topk<8>(row, E, k, tag, err, sel, id);
+    return fused_token_topk_wide(row, E, k, tag, err, sel, id);
 }
 
 template <int FS, int WF>
@@ -1556,182 +1652,234 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
     const int T = a.T, d = a.d, E = a.E, k = a.k, S = a.S;
     const int G = gridDim.x, b = blockIdx.x;
 
-    // A timeout of an earlier launch that the host has not yet read (and
-    // cleared, resetting the barrier) may have left the grid barrier's count
-    // short of a whole round, so that some CTAs of this launch would pass it
-    // before every CTA has written its logits.  Every CTA reads the sticky
-    // error word first; if a timeout is pending, the whole launch skips its
-    // work, writes NaN to `out` (so a caller that ignores the status cannot
-    // take the result for a valid one) and records kErrSkipped.
-    // (The flag lives in the dynamic shared memory: a static __shared__
-    // variable would add a 1 KB block, the dynamic block's alignment, on top
-    // of a launch sized to the opt-in limit.)
-    if (tid == 0)
-        rs->skip = (*reinterpret_cast<volatile uint32_t*>(a.err) & (kErrTimeout | kErrSkipped)) != 0;
-    __syncthreads();
-    if (rs->skip) {
+    // The producer warp, idle until phase X, sets up the ring barriers, takes
+    // the launch ticket (see the notes above), reads the sticky error word
+    // and fills the CTA's share of `out`, while the consumers' router loads
+    // are in flight.  A timeout of an earlier launch that the host has not
+    // yet read (and cleared, resetting the ticket count and the logit words)
+    // may have left the count short of a whole round, so that the CTAs of
+    // this launch could derive different tags.  If a timeout is pending, the
+    // whole launch skips its work, writes NaN to `out` (so a caller that
+    // ignores the status cannot take the result for a valid one) and records
+    // kErrSkipped.  (The flag lives in the dynamic shared memory: a static
+    // __shared__ variable would add a 1 KB block, the dynamic block's
+    // alignment, on top of a launch sized to the opt-in limit.)
+    if (warp == kConsumerWarps) {
+        int skip = 0;
+        if (lane == 0) {
+            const uint32_t ev = *reinterpret_cast<volatile uint32_t*>(a.err);
+            const unsigned long long old = atomicAdd(reinterpret_cast<unsigned long long*>(a.gbar), 1ull);
+            for (int s = 0; s < a.n_stages; ++s) {
+                mbar_init(&sm.full[s], 1);
+                mbar_init(&sm.empty[s], kConsumerWarps);
+            }
+            sm.tail->abort_flag = 0;
+            fence_mbar_init();
+            // fetch the tensor maps now, so the first TMA of phase X does not
+            // wait for them
+            prefetch_tensormap(&a.tm_gate); prefetch_tensormap(&a.tm_up); prefetch_tensormap(&a.tm_down);
+            if (S) { prefetch_tensormap(&a.tm_sgate); prefetch_tensormap(&a.tm_sup);
+                     prefetch_tensormap(&a.tm_sdown); }
+            if constexpr (C::QUANT) {
+                prefetch_tensormap(&a.tm_gate_sc); prefetch_tensormap(&a.tm_up_sc);
+                prefetch_tensormap(&a.tm_down_sc);
+                if (S) { prefetch_tensormap(&a.tm_sgate_sc); prefetch_tensormap(&a.tm_sup_sc);
+                         prefetch_tensormap(&a.tm_sdown_sc); }
+            }
+            const unsigned long long gl = static_cast<unsigned long long>(G);
+            rs->tag = (old - old % gl + gl) << 32;
+            skip = (ev & (kErrTimeout | kErrSkipped)) != 0;
+            rs->skip = skip;
+        }
+        skip = __shfl_sync(0xffffffffu, skip, 0);
         float4* o = reinterpret_cast<float4*>(a.out);
-        const float qnan = __uint_as_float(0x7fc00000u);
         const int n4 = (T * d) >> 2;
-        for (int i = b * kDecodeThreads + tid; i < n4; i += G * kDecodeThreads)
-            o[i] = make_float4(qnan, qnan, qnan, qnan);
-        if (b == 0 && tid == 0) atomicOr(a.err, kErrSkipped);
-        return;
-    }
-
-    if (tid == 0) {
-        for (int s = 0; s < a.n_stages; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], kConsumerWarps);
-        }
-        sm.tail->abort_flag = 0;
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    // the producer warp idles through R and T: fetch the tensor maps now, so
-    // the first TMA of phase X does not wait for them
-    if (warp == kConsumerWarps && lane == 0) {
-        prefetch_tensormap(&a.tm_gate); prefetch_tensormap(&a.tm_up); prefetch_tensormap(&a.tm_down);
-        if (S) { prefetch_tensormap(&a.tm_sgate); prefetch_tensormap(&a.tm_sup);
-                 prefetch_tensormap(&a.tm_sdown); }
-        if constexpr (C::QUANT) {
-            prefetch_tensormap(&a.tm_gate_sc); prefetch_tensormap(&a.tm_up_sc);
-            prefetch_tensormap(&a.tm_down_sc);
-            if (S) { prefetch_tensormap(&a.tm_sgate_sc); prefetch_tensormap(&a.tm_sup_sc);
-                     prefetch_tensormap(&a.tm_sdown_sc); }
+        if (skip) {
+            const float qnan = __uint_as_float(0x7fc00000u);
+            for (int i = b * 32 + lane; i < n4; i += G * 32) o[i] = make_float4(qnan, qnan, qnan, qnan);
+        } else if (b < E) {
+            const int gz = G < E ? G : E;   // the CTAs that publish logits
+            for (int i = b * 32 + lane; i < n4; i += gz * 32) o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            // release fence: this lane's logit words (stored after it in
+            // program order) publish the zero-fill with them
+            __threadfence();
         }
     }
 
-    // ---- R: logits of this CTA's experts; zero-fill of out; x staged for X
+    // ---- R: logits of this CTA's experts b, b + G, ...  Warp w sums slice w
+    // of d; it takes two experts per pass, so that both weight rows and the
+    // shared x slice are requested before the first use.
+    float* part = reinterpret_cast<float*>(sm.ring);          // [n_loc][16 slices][8 tok]
+    const int n_loc = (E - b + G - 1) / G;
+    // The producer warp also publishes the logit words (after its release
+    // fence); lane l takes words l and l + 32 first, whose biases it loads now.
+    float bias0 = 0.f, bias1 = 0.f;
+    if (warp == kConsumerWarps && a.br) {
+        if (lane < n_loc * kDecodeTok) bias0 = __ldg(a.br + b + (lane / kDecodeTok) * G);
+        if (lane + 32 < n_loc * kDecodeTok) bias1 = __ldg(a.br + b + ((lane + 32) / kDecodeTok) * G);
+    }
     if (warp < kConsumerWarps) {
-        stage_x<WF>(a, sm, tid);
-        if (tid < kMaxExperts / 32) rs->emask[tid] = 0u;
-        {
-            float4* o = reinterpret_cast<float4*>(a.out);
-            const int n4 = (T * d) >> 2;
-            for (int i = b * kConsumers + tid; i < n4; i += G * kConsumers)
-                o[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        float* part = reinterpret_cast<float*>(sm.ring);          // [n_loc][8 chunks][8 tok]
-        const int n_loc = (E - b + G - 1) / G;
         const int chunk = d / kConsumerWarps;
-        for (int item = warp; item < n_loc * kConsumerWarps; item += kConsumerWarps) {
-            const int loc = item / kConsumerWarps, ch = item % kConsumerWarps;
-            const int e = b + loc * G;
-            float acc[kDecodeTok];
+        for (int loc = 0; loc < n_loc; loc += 2) {
+            const bool two = loc + 1 < n_loc;
+            const float* w0 = a.wr + static_cast<size_t>(b + loc * G) * d;
+            const float* w1 = two ? w0 + static_cast<size_t>(G) * d : w0;
+            float acc0[kDecodeTok], acc1[kDecodeTok];
 #pragma unroll
-            for (int t = 0; t < kDecodeTok; ++t) acc[t] = 0.f;
-            const float* wrow = a.wr + static_cast<size_t>(e) * d;
-#pragma unroll 4
-            for (int i = ch * chunk + lane * 4; i < (ch + 1) * chunk; i += 128) {
-                const float4 wv = __ldg(reinterpret_cast<const float4*>(wrow + i));
+            for (int t = 0; t < kDecodeTok; ++t) acc0[t] = acc1[t] = 0.f;
+#pragma unroll 2
+            for (int i = warp * chunk + lane * 4; i < (warp + 1) * chunk; i += 128) {
+                const float4 wa = __ldg(reinterpret_cast<const float4*>(w0 + i));
+                const float4 wb = __ldg(reinterpret_cast<const float4*>(w1 + i));
 #pragma unroll
                 for (int t = 0; t < kDecodeTok; ++t) {
                     if (t < T) {
                         const uint2 xv = __ldg(reinterpret_cast<const uint2*>(
                             a.x + static_cast<size_t>(t) * d + i));
-                        acc[t] = fmaf(__uint_as_float(xv.x << 16), wv.x, acc[t]);
-                        acc[t] = fmaf(__uint_as_float(xv.x & 0xffff0000u), wv.y, acc[t]);
-                        acc[t] = fmaf(__uint_as_float(xv.y << 16), wv.z, acc[t]);
-                        acc[t] = fmaf(__uint_as_float(xv.y & 0xffff0000u), wv.w, acc[t]);
+                        const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+                        const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
+                        acc0[t] = fmaf(x0, wa.x, acc0[t]);
+                        acc0[t] = fmaf(x1, wa.y, acc0[t]);
+                        acc0[t] = fmaf(x2, wa.z, acc0[t]);
+                        acc0[t] = fmaf(x3, wa.w, acc0[t]);
+                        acc1[t] = fmaf(x0, wb.x, acc1[t]);
+                        acc1[t] = fmaf(x1, wb.y, acc1[t]);
+                        acc1[t] = fmaf(x2, wb.z, acc1[t]);
+                        acc1[t] = fmaf(x3, wb.w, acc1[t]);
                     }
                 }
             }
 #pragma unroll
             for (int t = 0; t < kDecodeTok; ++t) {
+                if (t < T) {
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1)
-                    acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], off);
+                    for (int off = 16; off > 0; off >>= 1) {
+                        acc0[t] += __shfl_xor_sync(0xffffffffu, acc0[t], off);
+                        acc1[t] += __shfl_xor_sync(0xffffffffu, acc1[t], off);
+                    }
+                }
             }
             if (lane == 0) {
 #pragma unroll
-                for (int t = 0; t < kDecodeTok; ++t) part[(loc * kConsumerWarps + ch) * kDecodeTok + t] = acc[t];
+                for (int t = 0; t < kDecodeTok; ++t) {
+                    part[(loc * kConsumerWarps + warp) * kDecodeTok + t] = acc0[t];
+                    if (two) part[((loc + 1) * kConsumerWarps + warp) * kDecodeTok + t] = acc1[t];
+                }
             }
         }
-        named_bar_sync(1, kConsumers);
-        for (int i = tid; i < n_loc * T; i += kConsumers) {
-            const int loc = i / T, t = i % T;
+    }
+    __syncthreads();
+    if (rs->skip) {
+        if (b == 0 && tid == 0) atomicOr(a.err, kErrSkipped);
+        return;
+    }
+    const unsigned long long tag = rs->tag;
+    if (warp == kConsumerWarps) {
+        // publish every token row of this CTA's experts (rows t >= T with 0):
+        // relaxed stores, ordered after the zero-fill by the fence above
+        for (int i = lane; i < n_loc * kDecodeTok; i += 32) {
+            const int loc = i / kDecodeTok, t = i % kDecodeTok;
             const int e = b + loc * G;
             float v = 0.f;
-            for (int ch = 0; ch < kConsumerWarps; ++ch) v += part[(loc * kConsumerWarps + ch) * kDecodeTok + t];
-            if (a.br) v += a.br[e];
-            a.ws.logits[t * E + e] = v;
+            if (t < T) {
+                for (int ch = 0; ch < kConsumerWarps; ++ch) v += part[(loc * kConsumerWarps + ch) * kDecodeTok + t];
+                if (a.br) v += (i == lane) ? bias0 : (i == lane + 32) ? bias1 : a.br[e];
+            }
+            st_relaxed_u64(a.ws.tlogits + static_cast<size_t>(t) * E + e, tag | __float_as_uint(v));
         }
+    } else {
+        // x for phase X, while the logits travel
+        stage_x<WF>(a, sm, tid);
+        if (tid < kMaxExperts / 32) rs->emask[tid] = 0u;
+        named_bar_sync(1, kConsumers);
     }
-    __syncthreads();
-    if (tid == 0 && !grid_barrier(a.gbar, G)) {
-        atomicOr(a.err, kErrTimeout);
-        sm.tail->abort_flag = 1;
-    }
-    __syncthreads();
 
     // ---- T: routing, computed redundantly by every CTA
     const int P = T * k;
     if (warp < kConsumerWarps) {
-        float* lg = reinterpret_cast<float*>(sm.ring);            // [T][E]
-        for (int i = tid; i < T * E; i += kConsumers) {
-            float v = __ldcg(a.ws.logits + i);
-            if (isnan(v)) v = -INFINITY;
-            lg[i] = v;
-        }
-        named_bar_sync(1, kConsumers);
         if (warp < T) {
+            // warp t: wait for token t's logits, top-k, then the softmax over
+            // the k selected logits (the same sum order as the other routing
+            // paths: j = 0, 1, ...)
             const int t = warp;
-            warp_topk_any(lg + t * E, E, k, &rs->ids[t * k], rs->sel[t], a.err);
-            __syncwarp();
+            float sv;
+            int sid;
+            const bool ok = fused_token_topk_any(a.ws.tlogits + static_cast<size_t>(t) * E, E, k,
+                                                 static_cast<uint32_t>(tag >> 32), a.err, sv, sid);
+            if (!ok && lane == 0) {
+                atomicOr(a.err, kErrTimeout);
+                sm.tail->abort_flag = 1;
+            }
+            const float m = __shfl_sync(0xffffffffu, sv, 0);
+            const float ej = (lane < k) ? expf(sv - m) : 0.f;
+            // lanes j >= k hold 0, so the unrolled sum over kMaxTopK lanes
+            // equals the sum over the k selections, in the same order
+            float den = 0.f;
+#pragma unroll
+            for (int j = 0; j < kMaxTopK; ++j) den += __shfl_sync(0xffffffffu, ej, j);
             if (lane < k) {
-                const float m = rs->sel[t][0];
-                float den = 0.f;
-                for (int j = 0; j < k; ++j) den += expf(rs->sel[t][j] - m);
-                float wj = expf(rs->sel[t][lane] - m) / den;
+                float wj = ej / den;
                 if (!(m > -INFINITY)) wj = 1.f / k;
+                rs->ids[t * k + lane] = sid;
                 rs->w[t * k + lane] = wj;
-                const int e = rs->ids[t * k + lane];
-                atomicOr(&rs->emask[e >> 5], 1u << (e & 31));
+                atomicOr(&rs->emask[sid >> 5], 1u << (sid & 31));
             }
         }
+        if (tid == kConsumers - 1)      // pad the pair ids to whole int4s (never below an id)
+            for (int q = P; q < ((P + 3) & ~3); ++q) rs->ids[q] = 0x7fffffff;
         named_bar_sync(1, kConsumers);
         // stable slots: pairs with a smaller expert id come first, ties by pair
         // index; the first pair of each expert writes its work item, whose
-        // index is the number of selected experts below it (mask popcount)
-        for (int p = tid; p < P; p += kConsumers) {
+        // index is the number of selected experts below it (mask popcount).
+        // The routing tables in global memory (identical in every CTA) are
+        // written in shares: pair p by CTA p mod G, offsets/counts of expert x
+        // by CTA x mod G.
+        const int4* ids4 = reinterpret_cast<const int4*>(rs->ids);
+        const int nq4 = (P + 3) >> 2;
+        if (tid < P) {
+            const int p = tid;
             const int e = rs->ids[p];
             int lt = 0, before = 0, cnt = 0;
-            for (int q = 0; q < P; ++q) {
-                const int eq = rs->ids[q];
-                lt += eq < e;
-                cnt += eq == e;
-                before += (eq == e) & (q < p);
+            for (int q4 = 0; q4 < nq4; ++q4) {
+                const int4 v = ids4[q4];
+                const int q = 4 * q4;
+                lt += (v.x < e) + (v.y < e) + (v.z < e) + (v.w < e);
+                cnt += (v.x == e) + (v.y == e) + (v.z == e) + (v.w == e);
+                before += ((v.x == e) & (q < p)) + ((v.y == e) & (q + 1 < p)) +
+                          ((v.z == e) & (q + 2 < p)) + ((v.w == e) & (q + 3 < p));
             }
             const int slot = lt + before;
             rs->slot_token[slot] = p / k;
             rs->slot_w[slot] = rs->w[p];
             if (before == 0) {
                 int idx = __popc(rs->emask[e >> 5] & ((1u << (e & 31)) - 1u));
-                for (int wd = 0; wd < (e >> 5); ++wd) idx += __popc(rs->emask[wd]);
+                const int nw = e >> 5;
+#pragma unroll 8
+                for (int wd = 0; wd < nw; ++wd) idx += __popc(rs->emask[wd]);
                 rs->items[idx] = WorkItem{e, lt, cnt, 0};
             }
-            if (b == 0) {
+            if (p % G == b) {
                 a.ws.slot_pair[slot] = p;
                 a.ws.slot_token[slot] = p / k;
                 a.ws.slot_w[slot] = rs->w[p];
                 a.ws.ids[p] = e;
                 a.ws.wts[p] = rs->w[p];
             }
-        }
-        if (tid == kConsumers - 1) {     // a thread the pair loop above rarely uses
+        } else if (tid == kConsumers - 1) {
             int n = 0;
-            for (int wd = 0; wd < (E + 31) / 32; ++wd) n += __popc(rs->emask[wd]);
+            const int nw = (E + 31) / 32;
+#pragma unroll 8
+            for (int wd = 0; wd < nw; ++wd) n += __popc(rs->emask[wd]);
             rs->n_routed = n;
             for (int s2 = 0; s2 < S; ++s2) rs->items[n + s2] = WorkItem{E + s2, -1, T, 0};
-        }
-        if (b == 0) {
-            for (int x = tid; x <= E; x += kConsumers) {
+        } else if (tid >= kConsumers / 2) {
+            constexpr int kTab = kConsumers / 2 - 1;    // threads kConsumers/2 .. kConsumers-2
+            for (int x = b + G * (tid - kConsumers / 2); x <= E; x += G * kTab) {
                 int lt = 0, cnt = 0;
-                for (int q = 0; q < P; ++q) {
-                    lt += rs->ids[q] < x;
-                    cnt += rs->ids[q] == x;
+                for (int q4 = 0; q4 < nq4; ++q4) {
+                    const int4 v = ids4[q4];
+                    lt += (v.x < x) + (v.y < x) + (v.z < x) + (v.w < x);
+                    cnt += (v.x == x) + (v.y == x) + (v.z == x) + (v.w == x);
                 }
                 a.ws.offsets[x] = lt;
                 if (x < E) a.ws.counts[x] = cnt;
@@ -1739,6 +1887,11 @@ decode_fused_kernel(const __grid_constant__ DecodeArgs a) {
         }
     }
     __syncthreads();
+    // acquire: the warps that read the logit words order the other CTAs'
+    // zero-fill of `out` before every add of phase X (which follows a named
+    // barrier of the consumers); done here, not before routing, so that it
+    // overlaps the first weight loads
+    if (warp < T) fence_acq_rel_gpu();
     const WorkView wv{rs->n_routed, S, rs->items, rs->slot_token, rs->slot_w};
     run_experts<FS, WF>(a, sm, wv);
 }

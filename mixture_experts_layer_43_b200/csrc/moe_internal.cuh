@@ -18,6 +18,7 @@ constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxShared = 8;
 constexpr int kDecodeTok = 8;        // mma N: tokens per expert pass (>= MOE_DECODE_MAX_T)
+constexpr int kDecodeConsumerWarps = 16;   // consumer warps of a decode CTA (+ 1 producer)
 static_assert(MOE_DECODE_MAX_T <= kDecodeTok, "decode pass holds every token");
 
 // Device error word bits (sticky until moe_get_device_status reads them).
@@ -56,7 +57,8 @@ struct Workspace {
     int32_t* n_items;      // [2]: routed items, shared items
     uint32_t* ticket;      // last-CTA ticket of the decode router
     uint32_t* err;         // sticky device error word
-    uint32_t* gbar;        // grid barrier of the fused decode kernel: 64-bit arrival count (8-aligned)
+    uint32_t* gbar;        // fused decode kernel: [0..1] 64-bit launch ticket count (8-aligned)
+    unsigned long long* tlogits;  // fused decode kernel: [kDecodeTok][E] logit bits | launch tag << 32
     // prefill
     uint16_t* x_perm;      // [t_max*k][d] bf16 rows gathered per slot
     uint16_t* h_routed;    // [t_max*k][F] bf16
@@ -110,7 +112,7 @@ struct DecodeArgs {
     const float* br;            // [E] or nullptr
     int k;
     Workspace ws;
-    uint32_t* gbar;             // [0..1] 64-bit arrival count of the grid barrier
+    uint32_t* gbar;             // [0..1] 64-bit launch ticket count
 };
 
 // Host launchers (decode.cu, quant_pack.cu).
@@ -162,6 +164,20 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
     unsigned long long v;
     asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -419,65 +435,185 @@ __device__ __forceinline__ void red_add_v4_f32(float* p, float a, float b, float
 }
 
 // --------------------------------------------------------- warp top-k
-// Warp-wide float maximum (sm_100a: one redux.sync instead of five shuffle
-// rounds).
-__device__ __forceinline__ float warp_max_f32(float v) {
-    float r;
-    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-    return r;
+// Order-preserving 32-bit key of a logit (NaN excluded): larger logit,
+// larger key; -0 maps like +0, so that equal logits have equal keys.
+__device__ __forceinline__ uint32_t logit_key(float f) {
+    const uint32_t u = f == 0.f ? 0u : __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float logit_of_key(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
-// Top-k of one token's E logits (shared memory, E <= 32 * PER) by one warp.
-// Each lane keeps logits lane, lane+32, ... in registers; a bitmask marks the
-// ones already taken.  A round is a register scan, a warp max of the lanes'
-// best values and a warp min over the indices holding that max.
-// Order: descending logit, equal logits -> lower expert index; NaN counts as
-// -inf.  Lane 0 writes ids[j] and the selected logits sel[j].
-template <int PER>
-__device__ __forceinline__ void warp_topk(const float* row, int E, int k, int* ids, float* sel,
-                                          uint32_t* err) {
+// Top-k of one token's E logits (E <= 32 * PER) by one warp, from
+// registers: lane l holds the logits of experts l, l + 32, ... in v[0..PER)
+// (entries past E and NaN already set to -inf).  Each value becomes its
+// order-preserving key, and the lane sorts its PER keys with a bitonic
+// network into selection order: descending logit, equal logits by
+// ascending expert index.  Round j takes the warp maximum m of the lanes'
+// first keys and the lowest expert index among the first keys equal to m
+// (two integer warp reductions); the lane holding that entry drops it (its
+// list moves up by one).  KMAX >= k rounds run unrolled and without
+// branches (a lone warp's chain of dependent steps is what this costs, and
+// a branch per round about doubled it); rounds past k change nothing that
+// is returned.  Lane j < k returns selection j in (sel, id); the other
+// lanes return (-inf, 0).  For PER <= 8 (E <= 256); larger E takes
+// warp_topk_scan_select.
+template <int PER, int KMAX>
+__device__ __forceinline__ void warp_topk_sorted_select(float (&v)[PER], int E, int k,
+                                                        uint32_t* err, float& sel, int& id) {
     const int lane = threadIdx.x & 31;
-    float v[PER];
+    uint32_t key[PER];
+    int ix[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        key[i] = logit_key(v[i]);
+        ix[i] = lane + 32 * i;
+    }
+#pragma unroll
+    for (int size = 2; size <= PER; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+#pragma unroll
+            for (int i = 0; i < PER; ++i) {
+                const int l = i ^ stride;
+                if (l > i) {
+                    // entry p goes first in this run's order
+                    const int p = ((i & size) == 0) ? i : l;
+                    const int q = (p == i) ? l : i;
+                    const bool sw = key[q] > key[p] || (key[q] == key[p] && ix[q] < ix[p]);
+                    const uint32_t tk = key[p];
+                    const int ti = ix[p];
+                    key[p] = sw ? key[q] : tk;
+                    ix[p] = sw ? ix[q] : ti;
+                    key[q] = sw ? tk : key[q];
+                    ix[q] = sw ? ti : ix[q];
+                }
+            }
+        }
+    }
+    uint32_t selk = 0u;
+    int sid = 0;
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+        const uint32_t m = __reduce_max_sync(0xffffffffu, key[0]);
+        const int w = static_cast<int>(
+            __reduce_min_sync(0xffffffffu, key[0] == m ? static_cast<uint32_t>(ix[0]) : 0xffffffffu));
+        const bool mine = ix[0] == w;
+#pragma unroll
+        for (int i = 0; i + 1 < PER; ++i) {
+            key[i] = mine ? key[i + 1] : key[i];
+            ix[i] = mine ? ix[i + 1] : ix[i];
+        }
+        key[PER - 1] = mine ? 0u : key[PER - 1];     // below every logit key (-inf: 0x007fffff)
+        ix[PER - 1] = mine ? 0x7fffffff : ix[PER - 1];
+        selk = (lane == j) ? m : selk;
+        sid = (lane == j) ? w : sid;
+    }
+    if (lane < k && (sid < 0 || sid >= E)) {   // cannot happen for k <= E; keep ids in range
+        atomicOr(err, kErrBadId);
+        sid = 0;
+    }
+    sel = lane < k ? logit_of_key(selk) : -INFINITY;
+    id = lane < k ? sid : 0;
+}
+
+// The same selection for E up to 1024 (PER = 32), where a sorted copy would
+// not fit in registers: a bitmask marks the entries already taken and round
+// j scans the lane's PER keys for its best one before the same two warp
+// reductions.  Same order and outputs as warp_topk_sorted_select.
+template <int PER>
+__device__ __forceinline__ void warp_topk_scan_select(const float (&v)[PER], int E, int k,
+                                                      uint32_t* err, float& sel, int& id) {
+    const int lane = threadIdx.x & 31;
+    uint32_t key[PER];
     uint32_t taken = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-        const int x = lane + 32 * i;
-        float t = -INFINITY;
-        if (x < E) {
-            t = row[x];
-            if (isnan(t)) t = -INFINITY;
-        } else {
-            taken |= 1u << i;
-        }
-        v[i] = t;
+        key[i] = logit_key(v[i]);
+        if (lane + 32 * i >= E) taken |= 1u << i;
     }
+    sel = -INFINITY;
+    id = 0;
     for (int j = 0; j < k; ++j) {
-        float bv = -INFINITY;
+        uint32_t bk = 0u;
         int bi = 0x7fffffff;
 #pragma unroll
         for (int i = 0; i < PER; ++i)   // strict '>': the lowest index wins inside a lane
-            if (!((taken >> i) & 1u) && (v[i] > bv || bi == 0x7fffffff)) { bv = v[i]; bi = lane + 32 * i; }
-        const float m = warp_max_f32(bv);
-        const uint32_t cand = (bv == m) ? static_cast<uint32_t>(bi) : 0xffffffffu;
+            if (!((taken >> i) & 1u) && (key[i] > bk || bi == 0x7fffffff)) { bk = key[i]; bi = lane + 32 * i; }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t cand = (bk == m && bi != 0x7fffffff) ? static_cast<uint32_t>(bi) : 0xffffffffu;
         int w = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
-        if (w < 0 || w >= E) {         // cannot happen for k <= E; keep ids in range
+        if (w < 0 || w >= E) {
             if (lane == 0) atomicOr(err, kErrBadId);
             w = 0;
         } else if ((w & 31) == lane) {
             taken |= 1u << (w >> 5);
         }
-        if (lane == 0) { ids[j] = w; sel[j] = m; }
+        if (lane == j) {
+            sel = logit_of_key(m);
+            id = w;
+        }
     }
 }
 
-// warp_topk with PER chosen from E at run time.
+template <int PER>
+__device__ __forceinline__ void warp_topk_select(float (&v)[PER], int E, int k, uint32_t* err,
+                                                 float& sel, int& id) {
+    if constexpr (PER <= 8) {
+        if (k <= 2) warp_topk_sorted_select<PER, 2>(v, E, k, err, sel, id);
+        else if (k <= 4) warp_topk_sorted_select<PER, 4>(v, E, k, err, sel, id);
+        else if (k <= 8) warp_topk_sorted_select<PER, 8>(v, E, k, err, sel, id);
+        else warp_topk_sorted_select<PER, kMaxTopK>(v, E, k, err, sel, id);
+    } else {
+        warp_topk_scan_select<PER>(v, E, k, err, sel, id);
+    }
+}
+
+// Top-k of a logit row in memory (shared, or global through L2 when CG: for
+// logits that other CTAs of the same launch wrote).  Every load is issued
+// (index clamped into the row) before the first use, so that the PER reads
+// overlap; NaN reads as -inf.
+template <int PER, bool CG>
+__device__ __forceinline__ void warp_topk_reg(const float* row, int E, int k, uint32_t* err,
+                                              float& sel, int& id) {
+    const int lane = threadIdx.x & 31;
+    float v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int x = lane + 32 * i;
+        const int xc = x < E ? x : E - 1;
+        v[i] = CG ? __ldcg(row + xc) : row[xc];
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        if (lane + 32 * i >= E || isnan(v[i])) v[i] = -INFINITY;
+    warp_topk_select<PER>(v, E, k, err, sel, id);
+}
+
+// warp_topk_reg with PER chosen from E at run time.
+template <bool CG>
+__device__ __forceinline__ void warp_topk_reg_any(const float* row, int E, int k, uint32_t* err,
+                                                  float& sel, int& id) {
+    if (E <= 32) warp_topk_reg<1, CG>(row, E, k, err, sel, id);
+    else if (E <= 64) warp_topk_reg<2, CG>(row, E, k, err, sel, id);
+    else if (E <= 128) warp_topk_reg<4, CG>(row, E, k, err, sel, id);
+    else if (E <= 256) warp_topk_reg<8, CG>(row, E, k, err, sel, id);
+    else warp_topk_reg<32, CG>(row, E, k, err, sel, id);
+}
+
+// The same selection written to shared memory: ids[j] and the selected
+// logits sel[j] for j < k.
 __device__ __forceinline__ void warp_topk_any(const float* row, int E, int k, int* ids, float* sel,
                                               uint32_t* err) {
-    if (E <= 32) warp_topk<1>(row, E, k, ids, sel, err);
-    else if (E <= 64) warp_topk<2>(row, E, k, ids, sel, err);
-    else if (E <= 128) warp_topk<4>(row, E, k, ids, sel, err);
-    else if (E <= 256) warp_topk<8>(row, E, k, ids, sel, err);
-    else warp_topk<32>(row, E, k, ids, sel, err);
+    float s;
+    int i;
+    warp_topk_reg_any<false>(row, E, k, err, s, i);
+    const int lane = threadIdx.x & 31;
+    if (lane < k) {
+        ids[lane] = i;
+        sel[lane] = s;
+    }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

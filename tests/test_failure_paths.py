@@ -1,7 +1,8 @@
 """Failure detection without a GPU fault: a bounded device wait that runs out
 reports MOE_ERR_TIMEOUT through the host, the context stays usable and the
-plan recovers.  The wait is made to run out by a barrier count that no launch
-can complete (a flag nothing sets); nothing traps, faults or hangs."""
+plan recovers.  The fused decode kernel's wait for the other CTAs' router
+logits is made to run out by a launch ticket count from which the CTAs derive
+different tags (a flag nothing sets); nothing traps, faults or hangs."""
 import numpy as np
 import pytest
 import torch
@@ -22,7 +23,7 @@ def _gpu():
         pytest.skip("needs a CUDA device")
 
 
-def test_grid_barrier_timeout_is_reported_and_recovered():
+def test_routing_wait_timeout_is_reported_and_recovered():
     sh = synth.MoEShape("stall", T=4, d=256, E=8, k=2, F=128, S=1, Fs=64)
     inp = synth.make_inputs(sh, seed=31)
     layer = D.DeviceLayer(inp)
@@ -36,7 +37,7 @@ def test_grid_barrier_timeout_is_reported_and_recovered():
         assert B.moe_last_launch_count(plan) == 1
         torch.cuda.synchronize()                       # the launch ends by itself
         # a second call before the status is read must not compute on the
-        # barrier the timeout left mid-round: it skips its work and its out
+        # ticket count the timeout left mid-round: it skips its work and its out
         # is NaN, never a plausible wrong value
         out2 = torch.zeros((sh.T, sh.d), device="cuda")
         B.moe_forward(plan, layer.weights, x.data_ptr(), sh.T, sh.k, sh.wfmt, out2.data_ptr(),

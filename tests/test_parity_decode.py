@@ -2,6 +2,8 @@
 oracle on seeded inputs, at the full sizes of the decode workloads and at
 small shapes that cover ragged tails, k = E, E = 1, several shared experts
 and T = 0."""
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -189,5 +191,25 @@ def test_decode_invalid_call_enqueues_nothing():
         torch.cuda.synchronize()
         assert torch.all(out == 0.0)                                      # nothing ran
         assert B.moe_get_device_status(plan) == B.MOE_OK
+    finally:
+        B.moe_plan_destroy(plan)
+
+
+def test_plan_reused_across_token_counts():
+    """One plan, consecutive fused launches with T = 8, 1, 5, 8, 2, 8 and a
+    fresh x each time: every call matches the oracle.  (A launch publishes
+    router logits for all 8 token rows, tagged with the launch; rows beyond
+    its own T must never pass for a later launch's.)"""
+    sh8 = synth.MoEShape("reuse", T=8, d=512, E=64, k=6, F=128, S=1, Fs=128)
+    base = synth.make_inputs(sh8, seed=41)
+    layer = D.DeviceLayer(base)
+    plan = B.moe_plan_create(layer.config(8))
+    try:
+        for j, T in enumerate((8, 1, 5, 8, 2, 8)):
+            xb = synth.make_inputs(sh8, seed=200 + j, x_only=True).x[:T]
+            inp = dataclasses.replace(base, shape=dataclasses.replace(sh8, T=T), x=xb)
+            got, routing, launches = run_gpu(layer, xb, T, plan=plan)
+            assert launches == 1
+            compare(inp, got, routing, oracle.forward(inp))
     finally:
         B.moe_plan_destroy(plan)
