@@ -1155,6 +1155,9 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
     int slot = 0;
     uint32_t ph = 0;
     auto wait_full = [&]() -> bool {
+        // fast path: the stage has landed (the abort flag matters only to a
+        // wait that would otherwise run into the limit)
+        if (__all_sync(0xffffffffu, mbar_try_wait(&full[slot], ph))) return true;
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded_sleep(&full[slot], ph));
         if (!ok && lane == 0) {
@@ -1240,83 +1243,74 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
         };
 
         // ------------------------------------------- phase A: gate and up
-        float acc[2 * C::RG][4];
-#pragma unroll
-        for (int q = 0; q < 2 * C::RG; ++q)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[q][i] = 0.f;
+        // stage group sq = (row group rg, matrix mat); one loop body for all
+        // of them (not unrolled: the unit loop stays small enough for the
+        // instruction cache), each group's sums stored once it is complete
         const bool fast_a = KC == KCMAX;
+#pragma unroll 1
+        for (int sq = 0; sq < 2 * C::RG; ++sq) {
+            const int rg = sq >> 1, mat = sq & 1;
+            float ac[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int c = 0; c < nch; ++c) {
+                const bool ok = wait_full();
+                if (ok) {
+                    if (nch > 1) load_x(c);
+                    const uint32_t st_u = ring_u + slot * C::STAGE;
+                    if (__builtin_expect(fast_a && (c + 1) * KCMAX <= nkb, 1)) {
+                        // all four block columns of this warp are in the stage
 #pragma unroll
-        for (int rg = 0; rg < C::RG; ++rg) {
-#pragma unroll
-            for (int mat = 0; mat < 2; ++mat) {
-                for (int c = 0; c < nch; ++c) {
-                    const bool ok = wait_full();
-                    if (ok) {
-                        if (nch > 1) load_x(c);
-                        const uint32_t st_u = ring_u + slot * C::STAGE;
-                        float (&ac)[4] = acc[rg * 2 + mat];
-                        if (fast_a && (c + 1) * KCMAX <= nkb) {
-                            // all four block columns of this warp are in the stage
-#pragma unroll
-                            for (int i = 0; i < C::NBW; ++i) {
-                                const uint32_t cb = st_u + lane_code + i * (16 * 16 * 16);
-                                const uint32_t x0 = lds_u32(cb), x8 = lds_u32(cb + 128);
-                                if constexpr (C::Q6) {
-                                    const uint32_t e = lds_u32(st_u + lane_a_rec + i * (16 * 160));
-                                    const uint32_t sw = lds_u32(st_u + lane_a_sub + i * (16 * 160));
-                                    const float dr = lds_f16_as_f32(st_u + lane_a_d + i * 64);
-                                    const float dr8 = lds_f16_as_f32(st_u + lane_a_d + i * 64 + 16);
-                                    block_q6(i, x0, x8, e, sw, dr, dr8, ac);
-                                } else {
-                                    const float s0 = lds_f16_as_f32(st_u + lane_a_scl + i * 512);
-                                    const float s8 = lds_f16_as_f32(st_u + lane_a_scl + i * 512 + 16);
-                                    block_q4(i, x0, x8, s0, s8, ac);
-                                }
+                        for (int i = 0; i < C::NBW; ++i) {
+                            const uint32_t cb = st_u + lane_code + i * (16 * 16 * 16);
+                            const uint32_t x0 = lds_u32(cb), x8 = lds_u32(cb + 128);
+                            if constexpr (C::Q6) {
+                                const uint32_t e = lds_u32(st_u + lane_a_rec + i * (16 * 160));
+                                const uint32_t sw = lds_u32(st_u + lane_a_sub + i * (16 * 160));
+                                const float dr = lds_f16_as_f32(st_u + lane_a_d + i * 64);
+                                const float dr8 = lds_f16_as_f32(st_u + lane_a_d + i * 64 + 16);
+                                block_q6(i, x0, x8, e, sw, dr, dr8, ac);
+                            } else {
+                                const float s0 = lds_f16_as_f32(st_u + lane_a_scl + i * 512);
+                                const float s8 = lds_f16_as_f32(st_u + lane_a_scl + i * 512 + 16);
+                                block_q4(i, x0, x8, s0, s8, ac);
                             }
-                        } else {
-                            const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
-                            const uint32_t* codes = reinterpret_cast<const uint32_t*>(stage);
+                        }
+                    } else {
+                        const uint8_t* stage = ring + static_cast<size_t>(slot) * C::STAGE;
+                        const uint32_t* codes = reinterpret_cast<const uint32_t*>(stage);
 #pragma unroll
-                            for (int i = 0; i < C::NBW; ++i) {
-                                const int bl = warp + kConsumerWarps * i;
-                                if (bl < KC && c * KC + bl < nkb) {
-                                    const uint32_t* row = codes + (bl * 16 + g) * 4;
-                                    const uint32_t x0 = row[tig], x8 = row[32 + tig];
-                                    if constexpr (C::Q6) {
-                                        const uint32_t* rec =
-                                            reinterpret_cast<const uint32_t*>(stage + 16 * KC * 16 + bl * 160);
-                                        const __half* dsm =
-                                            reinterpret_cast<const __half*>(stage + KC * (16 * 16 + 160));
-                                        block_q6(i, x0, x8, rec[4 * g + tig], rec[32 + g],
-                                                 __half2float(dsm[(bl >> 3) * 16 + g]),
-                                                 __half2float(dsm[(bl >> 3) * 16 + g + 8]), ac);
-                                    } else {
-                                        const __half* scl =
-                                            reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
-                                        block_q4(i, x0, x8, __half2float(scl[bl * 16 + g]),
-                                                 __half2float(scl[bl * 16 + g + 8]), ac);
-                                    }
+                        for (int i = 0; i < C::NBW; ++i) {
+                            const int bl = warp + kConsumerWarps * i;
+                            if (bl < KC && c * KC + bl < nkb) {
+                                const uint32_t* row = codes + (bl * 16 + g) * 4;
+                                const uint32_t x0 = row[tig], x8 = row[32 + tig];
+                                if constexpr (C::Q6) {
+                                    const uint32_t* rec =
+                                        reinterpret_cast<const uint32_t*>(stage + 16 * KC * 16 + bl * 160);
+                                    const __half* dsm =
+                                        reinterpret_cast<const __half*>(stage + KC * (16 * 16 + 160));
+                                    block_q6(i, x0, x8, rec[4 * g + tig], rec[32 + g],
+                                             __half2float(dsm[(bl >> 3) * 16 + g]),
+                                             __half2float(dsm[(bl >> 3) * 16 + g + 8]), ac);
+                                } else {
+                                    const __half* scl =
+                                        reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
+                                    block_q4(i, x0, x8, __half2float(scl[bl * 16 + g]),
+                                             __half2float(scl[bl * 16 + g + 8]), ac);
                                 }
                             }
                         }
                     }
-                    release();
                 }
+                release();
             }
-        }
-        // this warp's partial sums, [warp][mat][t][f] (row stride GS)
-#pragma unroll
-        for (int rg = 0; rg < C::RG; ++rg) {
-#pragma unroll
-            for (int mat = 0; mat < 2; ++mat) {
-                float* gq = gu + (warp * 2 + mat) * kDecodeTok * C::GS;
-                const int r = rg * 16 + g;
-                gq[t0 * C::GS + r] = acc[rg * 2 + mat][0];
-                gq[t1 * C::GS + r] = acc[rg * 2 + mat][1];
-                gq[t0 * C::GS + r + 8] = acc[rg * 2 + mat][2];
-                gq[t1 * C::GS + r + 8] = acc[rg * 2 + mat][3];
-            }
+            // this warp's partial sums of the group, [warp][mat][t][f] (row
+            // stride GS)
+            float* gq = gu + (warp * 2 + mat) * kDecodeTok * C::GS;
+            const int r = rg * 16 + g;
+            gq[t0 * C::GS + r] = ac[0];
+            gq[t1 * C::GS + r] = ac[1];
+            gq[t0 * C::GS + r + 8] = ac[2];
+            gq[t1 * C::GS + r + 8] = ac[3];
         }
         named_bar_sync(1, kConsumers);
         // h = SiLU(gate) * up as an fp16 pair hi + lo for the token columns in
@@ -1421,15 +1415,11 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                 }
             }
         };
+        float* const out0 = a.out + static_cast<size_t>(tok0) * d;   // this lane's two token rows
+        float* const out1 = a.out + static_cast<size_t>(tok1) * d;
         auto combine = [&](int j, const float (&c)[4]) {      // j: first row of the group + g
-            if (v0) {
-                red_add_f32(a.out + static_cast<size_t>(tok0) * d + j, w0 * c[0]);
-                red_add_f32(a.out + static_cast<size_t>(tok0) * d + j + 8, w0 * c[2]);
-            }
-            if (v1) {
-                red_add_f32(a.out + static_cast<size_t>(tok1) * d + j, w1 * c[1]);
-                red_add_f32(a.out + static_cast<size_t>(tok1) * d + j + 8, w1 * c[3]);
-            }
+            if (v0) red_add_f32_rows8(out0 + j, w0 * c[0], w0 * c[2]);
+            if (v1) red_add_f32_rows8(out1 + j, w1 * c[1], w1 * c[3]);
         };
         for (int st = 0; st < nB; ++st) {
             const bool ok = wait_full();
@@ -1437,19 +1427,17 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
             const int rows = min(C::RJ, d - j0);
             if (ok) {
                 const uint32_t st_u = ring_u + slot * C::STAGE;
-                if (rows == C::RJ) {
-                    // row groups warp + 16 q (q < RGW) sit in box q at group `warp`:
-                    // all of them first, then all their reductions into out
-                    float c[RGW][4];
-#pragma unroll
+                if (__builtin_expect(rows == C::RJ, 1)) {
+                    // row group warp + 16 q (q < RGW) sits in box q at group
+                    // `warp` (one loop body, for the instruction cache)
+#pragma unroll 1
                     for (int q = 0; q < RGW; ++q) {
                         const uint32_t bq = st_u + q * BOXB;
+                        float c[4];
                         rowgroup(bq + lane_code, bq + lane_b_scl, bq + lane_b_rec, bq + lane_b_sub,
-                                 bq + lane_b_d, c[q]);
+                                 bq + lane_b_d, c);
+                        combine(j0 + (warp + kConsumerWarps * q) * 16 + g, c);
                     }
-#pragma unroll
-                    for (int q = 0; q < RGW; ++q)
-                        combine(j0 + (warp + kConsumerWarps * q) * 16 + g, c[q]);
                 } else {
                     for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
                         const int grp = rgb % (QB / 16);

@@ -327,6 +327,13 @@ __device__ __forceinline__ void red_add_f32(float* p, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
+// p[0] += a and p[8] += b (two rows of one mma fragment column), one address
+// register with an immediate offset.
+__device__ __forceinline__ void red_add_f32_rows8(float* p, float a, float b) {
+    asm volatile("red.global.add.f32 [%0], %1;\n\tred.global.add.f32 [%0+32], %2;"
+                 ::"l"(p), "f"(a), "f"(b) : "memory");
+}
+
 // Named barrier among `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
