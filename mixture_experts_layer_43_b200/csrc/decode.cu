@@ -1429,8 +1429,9 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                 const uint32_t st_u = ring_u + slot * C::STAGE;
                 if (__builtin_expect(rows == C::RJ, 1)) {
                     // row group warp + 16 q (q < RGW) sits in box q at group
-                    // `warp` (one loop body, for the instruction cache)
-#pragma unroll 1
+                    // `warp` (two row groups per loop body: independent MMA
+                    // chains to overlap, and still a small loop)
+#pragma unroll 2
                     for (int q = 0; q < RGW; ++q) {
                         const uint32_t bq = st_u + q * BOXB;
                         float c[4];
