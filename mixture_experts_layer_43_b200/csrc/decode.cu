@@ -712,8 +712,11 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
     const int nkb = d / 32;
     uint32_t it = 0;
 
-    // warp-uniform: the ldmatrix / mma.sync that follow are warp-collective
+    // warp-uniform: the ldmatrix / mma.sync that follow are warp-collective;
+    // fast path when the stage has landed (the abort flag matters only to a
+    // wait that would otherwise run into the limit)
     auto wait_full = [&](int slot, uint32_t parity) -> bool {
+        if (__all_sync(0xffffffffu, mbar_try_wait(&full[slot], parity))) return true;
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return false;
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded_sleep(&full[slot], parity));
         if (!ok && lane == 0) {
