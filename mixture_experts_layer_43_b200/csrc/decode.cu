@@ -1215,17 +1215,18 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
         // one 16 x 32 block: x0 / x8 code words of rows g / g+8, e its q6_K
         // high-bit word, sw the sub-scales, s0 / s8 (Q4_0) or dr / dr8 (q6_K)
         // the scales; its two 16-wide halves are independent MMAs
+        // (Q4_0: the second half's MMA accumulates onto the first's, which
+        // saves the adds and operand moves of a second accumulator)
         auto block_q4 = [&](int i, uint32_t x0, uint32_t x8, float s0, float s8, float (&ac)[4]) {
             const uint32_t u0 = x0 >> 8, u8 = x8 >> 8;
-            float va[4], vb[4];
+            float va[4];
             mma_f16_16816(va, q4h_lo(x0), q4h_lo(x8), q4h_hi(x0), q4h_hi(x8), xf[i][0], xf[i][1],
                           xc0[i][0], xc1[i][0], xc0[i][0], xc1[i][0]);
-            mma_f16_16816(vb, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8), xf[i][2], xf[i][3],
-                          0.f, 0.f, 0.f, 0.f);
-            ac[0] = fmaf(s0, va[0] + vb[0], ac[0]);
-            ac[1] = fmaf(s0, va[1] + vb[1], ac[1]);
-            ac[2] = fmaf(s8, va[2] + vb[2], ac[2]);
-            ac[3] = fmaf(s8, va[3] + vb[3], ac[3]);
+            mma_f16_16816_acc(va, q4h_lo(u0), q4h_lo(u8), q4h_hi(u0), q4h_hi(u8), xf[i][2], xf[i][3]);
+            ac[0] = fmaf(s0, va[0], ac[0]);
+            ac[1] = fmaf(s0, va[1], ac[1]);
+            ac[2] = fmaf(s8, va[2], ac[2]);
+            ac[3] = fmaf(s8, va[3], ac[3]);
         };
         auto block_q6 = [&](int i, uint32_t x0, uint32_t x8, uint32_t e, uint32_t sw, float dr, float dr8,
                             float (&ac)[4]) {
@@ -1402,19 +1403,19 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                     const uint32_t p1 = q4h_hi(x0), q1 = q4h_hi(x8);
                     const uint32_t p2 = q4h_lo(u0), q2 = q4h_lo(u8);
                     const uint32_t p3 = q4h_hi(u0), q3 = q4h_hi(u8);
-                    float va[4], vb[4];
+                    // one accumulator chain: both halves of h hi, then of h lo
+                    float va[4];
                     mma_f16_16816(va, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
                                   hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
-                    mma_f16_16816(vb, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1],
-                                  0.f, 0.f, 0.f, 0.f);
+                    mma_f16_16816_acc(va, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
                     mma_f16_16816_acc(va, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
-                    mma_f16_16816_acc(vb, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                    mma_f16_16816_acc(va, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
                     const float s0 = lds_f16_as_f32(scl_u + bb * (QB * 2));
                     const float s8 = lds_f16_as_f32(scl_u + bb * (QB * 2) + 16);
-                    c[0] = fmaf(s0, va[0] + vb[0], c[0]);
-                    c[1] = fmaf(s0, va[1] + vb[1], c[1]);
-                    c[2] = fmaf(s8, va[2] + vb[2], c[2]);
-                    c[3] = fmaf(s8, va[3] + vb[3], c[3]);
+                    c[0] = fmaf(s0, va[0], c[0]);
+                    c[1] = fmaf(s0, va[1], c[1]);
+                    c[2] = fmaf(s8, va[2], c[2]);
+                    c[3] = fmaf(s8, va[3], c[3]);
                 }
             }
         };

@@ -90,3 +90,36 @@ def test_reference_arm_prints_one_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_profile_traffic_is_null_unless_the_capture_matches_the_sources(tmp_path, monkeypatch):
+    """`roofline.traffic` comes from a committed ncu summary only while that
+    summary's source hash equals the current kernel sources' hash."""
+    sys.path.insert(0, ROOT)
+    import bench
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p = tmp_path / "profiles" / "k__w.txt"
+    p.write_text("# command: ...\nkernel_source_sha256: abc\ndram_bytes_per_launch: 1234\n")
+    assert bench._profile_traffic("k", "w", "abc") == 1234.0
+    assert bench._profile_traffic("k", "w", "abd") is None          # sources changed since
+    assert bench._profile_traffic("k", "other", "abc") is None      # no capture for it
+    p.write_text("kernel_source_sha256: abc\n")
+    assert bench._profile_traffic("k", "w", "abc") is None          # capture without the figure
+
+
+def test_committed_profiles_name_the_hash_of_their_sources():
+    """Every committed decode / prefill DRAM summary records the hash of the
+    sources of its kernel (so the bench can tell whether it still applies),
+    and none carries a hand-written note about a recomputed hash."""
+    import glob
+    sys.path.insert(0, ROOT)
+    files = glob.glob(os.path.join(ROOT, "profiles", "*.txt"))
+    assert files
+    for f in files:
+        txt = open(f).read()
+        assert "kernel_source_sha256:" in txt, f
+        assert "recomputed" not in txt, f
+        sha = [ln.split(":", 1)[1].strip() for ln in txt.splitlines()
+               if ln.startswith("kernel_source_sha256:")][0]
+        assert len(sha) == 64 and all(c in "0123456789abcdef" for c in sha), f
