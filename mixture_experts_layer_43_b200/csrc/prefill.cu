@@ -468,7 +468,18 @@ struct GemmTile {
     bool shared;
     int group;
     int nk;             // k blocks
+    int nsw;            // > 0: a swapped tail tile with this many token columns (see below)
 };
+
+// An expert's last row tile holds `valid` < 128 rows; as a 128-row MMA tile
+// the rest would be padding.  Such a tail tile (single-CTA GEMMs, routed
+// experts) swaps the operands instead: the weight rows already in the stage
+// become the 128-row A side and the tile's X_perm / h rows the N side,
+// rounded up to 16 -- two MMAs per k step (gate and up rows, or the two
+// 128-row halves of the down tile) into TMEM columns [0, N) and [128, 128 +
+// N).  The loads are the same as for a normal tile.  Tails that round up to
+// more than kSwapMaxN columns stay normal tiles.
+constexpr int kSwapMaxN = 112;
 
 // Tile t of the expert-major tile table (BM rows of the whole tile).
 template <int MODE, int BM>
@@ -489,6 +500,10 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmArgs& a, const int* s_tb
         g.shared = false;
         g.row0 = a.offsets[e] + mt * BM;
         g.valid = min(BM, a.counts[e] - mt * BM);
+        if constexpr (BM == kBM) {
+            const int n16 = (g.valid + 15) & ~15;
+            if (n16 <= kSwapMaxN) g.nsw = n16;
+        }
         if (MODE == kGateUp) {
             g.n0 = nt * 128;
             g.brow = e * a.F + nt * 128;
@@ -665,6 +680,24 @@ prefill_gemm_kernel(const __grid_constant__ GemmArgs a) {
                     tc_fence_after();
                     const uint32_t A = smem_u32(ring + s * C::STAGE);
                     const uint32_t Bt = A + kStageA;
+                    if constexpr (CG == 1) {
+                        if (g.nsw > 0) {
+                            // swapped tail tile: weight rows x token rows
+                            const uint32_t idesc_sw = (MODE == kDown && a.f16)
+                                                          ? umma_idesc_f16(kBM, g.nsw)
+                                                          : umma_idesc_bf16(kBM, g.nsw);
+#pragma unroll
+                            for (int kk = 0; kk < kBK / 16; ++kk) {
+                                const uint32_t acc = (kb | kk) ? 1u : 0u;
+                                umma_bf16(d_tmem, umma_desc_sw128(Bt + kk * 32),
+                                          umma_desc_sw128(A + kk * 32), idesc_sw, acc);
+                                umma_bf16(d_tmem + 128, umma_desc_sw128(Bt + C::STAGE_B / 2 + kk * 32),
+                                          umma_desc_sw128(A + kk * 32), idesc_sw, acc);
+                            }
+                            umma_commit(&empty[s]);
+                            continue;
+                        }
+                    }
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk) {
                         if constexpr (CG == 2)
@@ -701,7 +734,51 @@ prefill_gemm_kernel(const __grid_constant__ GemmArgs a) {
             const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kBN;
             const int row0 = g.row0 + kBM * static_cast<int>(rank);     // this CTA's rows
             const bool row_ok = r < g.valid - kBM * static_cast<int>(rank);
-            if (MODE == kGateUp) {
+            if (CG == 1 && g.nsw > 0) {
+                // swapped tail tile: this thread holds weight row r of the
+                // tile (TMEM lane r) for every token column
+#pragma unroll 1
+                for (int c = 0; c < g.nsw; c += 32) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld32(taddr + c, v0);
+                    tmem_ld32(taddr + 128 + c, v1);
+                    tmem_ld_wait();
+                    if (MODE == kGateUp) {
+                        const int f = g.n0 + r;                      // gate row f, up row f
+                        if (f < a.F) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                if (c + i < g.valid) {
+                                    const float gg = __uint_as_float(v0[i]), uu = __uint_as_float(v1[i]);
+                                    const float h = gg / (1.f + __expf(-gg)) * uu;
+                                    a.h_r[static_cast<size_t>(row0 + c + i) * a.F + f] =
+                                        a.f16 ? __half_as_ushort(__float2half_rn(h))
+                                              : __bfloat16_as_ushort(__float2bfloat16_rn(h));
+                                }
+                            }
+                        }
+                    } else {
+                        // rows n0 + r and n0 + 128 + r of out, one token per column
+                        int tk = 0;
+                        float wv = 0.f;
+                        if (c + lane < g.valid) {
+                            tk = a.slot_token[row0 + c + lane];
+                            wv = a.slot_w[row0 + c + lane];
+                        }
+                        const int j0 = g.n0 + r;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int tok_i = __shfl_sync(0xffffffffu, tk, i);
+                            const float w_i = __shfl_sync(0xffffffffu, wv, i);
+                            if (c + i < g.valid) {
+                                float* orow = a.out + static_cast<size_t>(tok_i) * a.d;
+                                if (j0 < a.d) red_add_f32(orow + j0, w_i * __uint_as_float(v0[i]));
+                                if (j0 + 128 < a.d) red_add_f32(orow + j0 + 128, w_i * __uint_as_float(v1[i]));
+                            }
+                        }
+                    }
+                }
+            } else if (MODE == kGateUp) {
                 const int Fh = g.shared ? a.Fs : a.F;
                 uint16_t* hrow = g.shared
                     ? a.h_s + static_cast<size_t>(row0 + r) * (a.S * a.Fs) + g.shared_s * a.Fs + g.n0
