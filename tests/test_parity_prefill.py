@@ -125,3 +125,36 @@ def test_prefill_deepseek_f16down_full_size():
     err = _check(sh, seed=0, sample=256, tripwire=F16DOWN_TRIPWIRE)
     print(f"deepseek f16down T=4096: rel L2 {err:.3e} on 256 sampled tokens")
 
+
+
+# Every token is sent to experts 0 and 1 (a +100 router bias on them), so each
+# of the two gets exactly T rows and its last row tile holds T mod 128 rows:
+# tails on both sides of the swapped-tile limit (N = tail rounded up to 16,
+# swapped up to 112; 113..127 stay 128-row tiles), in both weight formats.
+TAILS = [(1, synth.WFMT_BF16), (16, synth.WFMT_BF16), (17, synth.WFMT_BF16),
+         (100, synth.WFMT_BF16), (112, synth.WFMT_BF16), (113, synth.WFMT_BF16),
+         (127, synth.WFMT_BF16), (17, synth.WFMT_BF16_F16DOWN), (112, synth.WFMT_BF16_F16DOWN)]
+
+
+@pytest.mark.parametrize("tail,wfmt", TAILS, ids=[f"tail{t}_{'f16down' if w else 'bf16'}"
+                                                  for t, w in TAILS])
+def test_prefill_expert_tail_tiles(tail, wfmt):
+    import dataclasses
+    T = 128 + tail
+    sh = synth.MoEShape(f"tail{tail}", T=T, d=256, E=4, k=2, F=256, S=1, Fs=128, wfmt=wfmt)
+    inp = synth.make_inputs(sh, seed=11)
+    bias = np.zeros(sh.E, dtype=np.float32)
+    bias[:2] = 100.0
+    inp = dataclasses.replace(inp, router_b=bias)
+    layer = D.DeviceLayer(inp)
+    out, routing, launches = run_gpu(layer, inp.x, sh.T, regime=B.MOE_REGIME_PREFILL)
+    assert launches == 4
+    ids, w, counts, offsets, slot_pair = routing
+    assert list(counts) == [T, T, 0, 0]
+    ref, r_ids, r_w, _ = oracle.forward(inp)
+    assert np.array_equal(ids, r_ids)
+    np.testing.assert_allclose(w, r_w, rtol=w_rtol(sh.d, prefill=True), atol=W_ABS)
+    err = float(np.linalg.norm(out - ref) / np.linalg.norm(ref))
+    trip = F16DOWN_TRIPWIRE if wfmt == synth.WFMT_BF16_F16DOWN else PREFILL_TRIPWIRE
+    assert err <= trip, f"relative L2 error {err:.3e}"
+    assert np.all(np.isfinite(out))
