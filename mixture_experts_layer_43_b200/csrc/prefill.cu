@@ -349,19 +349,36 @@ __global__ void __launch_bounds__(kScatterThreads) prefill_scatter_kernel(const 
         a.ws.slot_w[slot] = a.ws.wts[p0 + i];
     }
     __syncthreads();
-    // gather x rows into X_perm (one warp per pair, 16 bytes per lane)
+    // gather x rows into X_perm: a warp copies kGatherRows pairs' rows at a
+    // time, 16 bytes per lane, every load of the group issued before its
+    // stores (one round trip per group of rows, not per row)
+    constexpr int kGatherRows = 4;
+    constexpr int kWarps = kScatterThreads / 32;
     const int cpr = a.d / 8;
-    for (int i = warp; i < np; i += kScatterThreads / 32) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + i / k) * a.d);
-        uint4* dst = reinterpret_cast<uint4*>(a.ws.x_perm + static_cast<size_t>(s_slot[i]) * a.d);
-        for (int cb = lane; cb < cpr; cb += 32 * 8) {     // 8 independent loads in flight
-            uint4 v[8];
+    for (int i0 = warp; i0 < np; i0 += kWarps * kGatherRows) {
+        for (int cb = lane; cb < cpr; cb += 32 * 8) {
+            uint4 v[kGatherRows][8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (cb + 32 * u < cpr) v[u] = __ldg(src + cb + 32 * u);
+            for (int p = 0; p < kGatherRows; ++p) {
+                const int i = i0 + kWarps * p;
+                if (i < np) {
+                    const uint4* src =
+                        reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t0 + i / k) * a.d);
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                if (cb + 32 * u < cpr) dst[cb + 32 * u] = v[u];
+                    for (int u = 0; u < 8; ++u)
+                        if (cb + 32 * u < cpr) v[p][u] = __ldg(src + cb + 32 * u);
+                }
+            }
+#pragma unroll
+            for (int p = 0; p < kGatherRows; ++p) {
+                const int i = i0 + kWarps * p;
+                if (i < np) {
+                    uint4* dst = reinterpret_cast<uint4*>(a.ws.x_perm + static_cast<size_t>(s_slot[i]) * a.d);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (cb + 32 * u < cpr) dst[cb + 32 * u] = v[p][u];
+                }
+            }
         }
     }
 }
