@@ -506,6 +506,32 @@ def _dtype(sh):
             synth.WFMT_Q6_K: "q6_k/bf16", synth.WFMT_BF16_F16DOWN: "bf16 (fp16 down)"}[sh.wfmt]
 
 
+def _read_stream_gbs(dev, stream) -> float:
+    """A read-only streaming reference measured on this GPU: torch.sum over
+    4 GiB of float32 resident on the device (each byte read once), best of
+    five timed with CUDA events on the launching stream.  The copy peak reads
+    and writes every byte; a read-only stream could run faster, and the
+    decode kernel only reads weights, so both are reported."""
+    import torch
+    n = (4 << 30) // 4
+    buf = torch.ones(n, dtype=torch.float32, device=dev)
+    best = float("inf")
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            buf.sum()
+        for _ in range(5):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            buf.sum()
+            b.record(stream)
+            stream.synchronize()
+            best = min(best, a.elapsed_time(b))
+    del buf
+    torch.cuda.empty_cache()
+    return (4 << 30) / (best / 1e3) / 1e9
+
+
 def run_b200(args, sh):
     import torch
 
@@ -561,6 +587,13 @@ def run_b200(args, sh):
         "gpu_launches": head["gpu_launches"],
         "clocks": head["clocks"],
     }
+    if not head["roofline"]["unit"] == "TFLOP/s":
+        rs = _read_stream_gbs(dev, stream)
+        line["roofline"] = dict(line["roofline"], read_stream_gbs=rs,
+                                frac_of_read_stream=line["roofline"]["achieved"] / rs,
+                                read_stream_note=("reference: torch.sum over 4 GiB of float32 on "
+                                                  "this GPU, read-only; frac stays against the "
+                                                  "copy peak"))
     if configs:
         configs[sh.name] = {k: head[k] for k in head}
         line["configs"] = configs
