@@ -2,8 +2,9 @@
 //
 // moe_forward runs the whole layer as ONE cooperative launch,
 // decode_fused_kernel (its phases are described above the kernel): router
-// logits, a grid barrier, top-k / buckets / work list computed by every CTA,
-// then the experts pipeline.  moe_route + moe_experts (and moe_forward when a
+// logits published with a launch tag, top-k / buckets / work list computed by
+// every CTA once every logit of its tokens carries that tag, then the experts
+// pipeline.  moe_route + moe_experts (and moe_forward when a
 // cooperative launch cannot place one CTA per SM) use two launches instead:
 //  1. decode_route_kernel: router logits (fp32 FMA), softmax + top-k with
 //     renormalised weights, per-expert buckets (counts, exclusive offsets,
@@ -1947,7 +1948,8 @@ static cudaError_t launch_fused_one(const DecodeArgs& a, int grid, size_t smem, 
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) set_bytes[dev] = static_cast<int>(smem);
     }
-    // cooperative: every CTA is resident at once, which the grid barrier needs
+    // cooperative: every CTA is resident at once, which the wait for every
+    // CTA's tagged logits needs
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kDecodeThreads);

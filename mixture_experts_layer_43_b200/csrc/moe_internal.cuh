@@ -26,10 +26,10 @@ constexpr uint32_t kErrBadId = 1u;        // an expert id or count out of range
 constexpr uint32_t kErrTimeout = 2u;      // a bounded wait ran out
 constexpr uint32_t kErrTooManyTok = 4u;   // an expert got more tokens than a pass holds
 // A fused decode launch found kErrTimeout (or this bit) already set when it
-// started: an earlier launch's grid barrier may have been left short of a
+// started: an earlier launch may have left the launch ticket count short of a
 // whole round, so the launch did no routing or expert work and wrote NaN to
 // `out`.  Cleared with the timeout by moe_get_device_status, which also
-// resets the barrier.
+// resets the ticket count and the tagged logit words.
 constexpr uint32_t kErrSkipped = 8u;
 
 // Bounded waits give up after this long (a healthy wait lasts microseconds).
@@ -107,7 +107,7 @@ struct DecodeArgs {
     int xs_stride;              // bytes per token row of the staged x
     int kt;                     // phase A: k columns (bf16) / block columns (quantised) per stage
     int rj;                     // phase B: output rows per stage
-    // fused single-launch path only: router inputs, routing tables, grid barrier
+    // fused single-launch path only: router inputs, routing tables, launch tickets
     const float* wr;            // [E][d]
     const float* br;            // [E] or nullptr
     int k;
