@@ -116,6 +116,23 @@ def test_decode_small_shapes(sh):
     _check(sh, seed=1)
 
 
+# Router widths and top-k sizes that select every variant of the warp top-k:
+# logits per lane 2, 4 and 8 (E = 40, 100, 200; 1024 is max_limits above)
+# with 2, 4 and 16 unrolled selection rounds (k = 2, 3, 12)
+TOPK_SHAPES = [
+    synth.MoEShape("topk_E40_k2", T=6, d=256, E=40, k=2, F=64, S=1, Fs=64),
+    synth.MoEShape("topk_E100_k3", T=4, d=256, E=100, k=3, F=64, S=1, Fs=64),
+    synth.MoEShape("topk_E200_k12", T=8, d=256, E=200, k=12, F=64, S=1, Fs=64),
+    synth.MoEShape("topk_E200_k12_q4", T=3, d=256, E=200, k=12, F=64, S=1, Fs=64,
+                   wfmt=synth.WFMT_Q4_0),
+]
+
+
+@pytest.mark.parametrize("sh", TOPK_SHAPES, ids=[s.name for s in TOPK_SHAPES])
+def test_decode_topk_variants(sh):
+    _check(sh, seed=5)
+
+
 SPLIT = SMALL[:6] + [SMALL[10], SMALL[-4], W["a3b_q4_T8_d2048_E256k8_F512_S1"],
                      W["a3b_q6_T8_d2048_E256k8_F512_S1"]]
 

@@ -84,6 +84,8 @@ SMALL = [
     synth.MoEShape("cta_pairs", T=2300, d=512, E=4, k=2, F=384, S=1, Fs=256),
     # the prefill limit E = 256: four 64-expert router passes, k = 8
     synth.MoEShape("E256", T=300, d=256, E=256, k=8, F=128, S=1, Fs=128, zipf_bias=1.1),
+    # k > 8: the 16-round selection of the warp top-k
+    synth.MoEShape("E200_k12", T=160, d=256, E=200, k=12, F=128, S=1, Fs=128),
 ]
 
 
