@@ -323,9 +323,11 @@ moe_status_t moe_q8_0_packed_bytes(int64_t n_mats, int64_t rows, int64_t k,
 /* Repack canonical Q8_0 blocks ([n_mats][rows][k/32] blocks of 34 bytes: a
  * little-endian fp16 scale, then 32 signed bytes, element j in byte j) into
  * the kernel layout:
- *   codes  [n_mats][k/32][rows][32 bytes]: each code biased to q + 128 and
- *          split into two 4-bit planes, each permuted like the Q4_0 codes,
- *          the planes' 32-bit words interleaved (low, high, low, high, ...);
+ *   codes  [n_mats][k/32][rows][32 bytes]: one byte per code, biased to
+ *          u = q + 128; byte 8t + n of a block row (t = 0..3, n = 0..7)
+ *          holds element 2t + (n & 1) + 8 ((n >> 1) & 1) + 16 (n >> 2), so
+ *          that t's first 4 bytes are elements 2t, 2t+1, 2t+8, 2t+9 and its
+ *          last 4 the same plus 16;
  *   scales [n_mats][k/32][rows] fp16.
  * Same 8.5 bits per weight.  All pointers are device pointers; `blocks`
  * needs no alignment, `codes`/`scales` 16 bytes.  Enqueued on `stream`.

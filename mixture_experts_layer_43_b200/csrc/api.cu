@@ -230,9 +230,9 @@ int pick_fs(const moe_plan_s* p, int T) {
     const double act = E * (1.0 - pow(1.0 - static_cast<double>(c.top_k) / E, T));
     int best = 32;
     double best_eff = -1.0;
-    // Q4_0's row-streaming pipeline keeps every row group's partial sums in
-    // registers, which fit for 32-row slices only
-    if (c.wfmt == MOE_WFMT_Q4_0 || c.wfmt == MOE_WFMT_Q6_K) return 32;
+    // the row-streaming pipeline (Q4_0, Q8_0, q6_K) keeps every row group's
+    // partial sums in registers, which fit for 32-row slices only
+    if (c.wfmt == MOE_WFMT_Q4_0 || c.wfmt == MOE_WFMT_Q8_0 || c.wfmt == MOE_WFMT_Q6_K) return 32;
     for (int fs : {64, 32}) {
         if (c.d_ff % fs || (c.n_shared && c.d_ff_shared % fs)) continue;
         const double units = act * (c.d_ff / fs) + c.n_shared * (c.n_shared ? c.d_ff_shared / fs : 0);
@@ -265,10 +265,11 @@ DecodeArgs* build_decode_maps(moe_plan_s* p, const moe_weights_t* w, int fs) {
             ok &= map_bf16(p, &a.tm_sdown, w->shared_down.data, S, d, Fs, fs, 128);
         }
     } else {
-        // phase-A boxes: Q4_0 streams 16-row groups over up to 64 block
-        // columns (the row-streaming pipeline); the other formats stream
+        // phase-A boxes: Q4_0, Q8_0 and q6_K stream 16-row groups over up to
+        // 64 block columns (the row-streaming pipeline); Q5_0 streams
         // 512 / fs block columns of the whole slice
-        const bool rows16 = c.wfmt == MOE_WFMT_Q4_0 || c.wfmt == MOE_WFMT_Q6_K;
+        const bool rows16 = c.wfmt == MOE_WFMT_Q4_0 || c.wfmt == MOE_WFMT_Q8_0 ||
+                            c.wfmt == MOE_WFMT_Q6_K;
         const uint32_t kb = rows16 ? static_cast<uint32_t>(d / 32 < 64 ? d / 32 : 64) : 512 / fs;
         const uint32_t ar = rows16 ? 16 : fs;
         const uint32_t nb = fs / 32;

@@ -228,12 +228,9 @@ constexpr int kWfQ5 = 3;
 constexpr int kWfQ6 = 4;     // q6_K super-blocks (row-streaming, fp16 operands)
 constexpr int kWfF16d = 5;   // bf16 gate/up, fp16 down matrices (h travels in fp16)
 
-// The constant that turns the bf16 "128 + nibble" operands back into signed
-// codes (see q4_raw): Q4_0 subtracts 128 + 8; Q8_0, whose biased byte
-// u = q + 128 = 16 hi + lo enters as two nibble planes weighted 1 and 16,
-// subtracts 128 + 16 * 128 + 128; Q5_0 (operands 128 + q, q < 32, see
-// q5_raw) subtracts 128 + 16.
-constexpr float quant_offset(int wf) { return wf == kWfQ8 ? 2304.f : wf == kWfQ5 ? 144.f : 136.f; }
+// The constant that turns Q5_0's bf16 operands 128 + q (q < 32, see q5_raw)
+// back into its signed codes q - 16: 128 + 16.
+constexpr float kQ5Offset = 144.f;
 
 template <int FS, int WF>
 struct DecodeCfg {
@@ -246,9 +243,10 @@ struct DecodeCfg {
     // pair and the down contraction runs on fp16 operands
     static constexpr bool HALF_DOWN = WF == kWfF16d;
     static_assert(!QUANT || FS >= 32, "quantised slices hold whole blocks");
-    // fp16 tensor-core operands (see q4h_lo): x staged as fp16, h as an fp16
-    // hi + lo pair, per-block corrections with two code bases
-    static constexpr bool F16 = WF == kWfQ4 || WF == kWfQ6;
+    // fp16 tensor-core operands (see q4h_lo, q8h_lo): x staged as fp16, h as
+    // an fp16 hi + lo pair, per-block corrections of the code bases
+    static constexpr bool F16 = WF == kWfQ4 || WF == kWfQ6 || WF == kWfQ8;
+    static constexpr bool Q8 = WF == kWfQ8;
     // q6_K: per 32-wide block and 16-row group a 160-byte record (high bits,
     // sub-block scales), per row and 256-wide super-block an fp16 scale
     static constexpr bool Q6 = WF == kWfQ6;
@@ -257,9 +255,11 @@ struct DecodeCfg {
     // sit in 48-byte records of 8 rows, see q5_aux)
     static constexpr int BR = CB + (WF == kWfQ5 ? 6 : 2);
     // bf16: phase A stage = gate+up [FS rows][KT cols]; phase B = down [RJ rows][FS cols]
-    // Q4_0 / Q8_0 / Q5_0: phase A stage = gate+up [KB block cols][FS rows];
-    //              phase B = [NB block cols][RJ rows]; codes, then the scales
-    //              (Q5_0: the 48-byte records of scales and fifth bits)
+    // Q5_0: phase A stage = gate+up [KB block cols][FS rows]; phase B =
+    //       [NB block cols][RJ rows]; codes, then the 48-byte records of
+    //       scales and fifth bits
+    // Q4_0 / Q8_0: phase A 16 rows x 64 blocks (codes, then scales), phase B
+    //       4 boxes of 256 rows (18 or 34 KB per stage)
     // q6_K: phase A 16 rows x 64 blocks (26880 B), phase B 4 boxes of 256
     // rows (4 x 7168 B)
     static constexpr int STAGE = Q6 ? 28672 : QUANT ? 2 * 512 * BR : 32768;
@@ -306,82 +306,17 @@ __device__ __forceinline__ uint32_t q4h_lo(uint32_t w) { return (w & 0x000F000Fu
 __device__ __forceinline__ uint32_t q4h_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x54005400u; }
 constexpr float kF16BaseLo = 1024.f, kF16BaseHi = 64.f;
 
-// One quantised block (32 weights along k) of rows r and r+8 of an mma A
-// tile, times the B fragment of the same 32 k (b0 b1: k 0-15, b2 b3: k
-// 16-31).  row_r / row_r8 point at the rows' packed code words; c0, c1 are
-// the accumulator start values of the lane's two token columns.  v gets the
-// block's four dot products before the block scale.
-//   Q4_0: one word per lane holds 8 codes, both 16-wide halves;
-//   Q8_0: the biased byte u = q + 128 is two Q4_0-packed nibble planes
-//         (words 2 tig = low nibbles, 2 tig + 1 = high nibbles), weighted 1
-//         and 16.
-template <int WF>
-__device__ __forceinline__ void quant_block_a(const uint32_t* row_r, const uint32_t* row_r8,
-                                              int tig, float c0, float c1, uint32_t b0,
-                                              uint32_t b1, uint32_t b2, uint32_t b3, float v[4]) {
-    if constexpr (WF == kWfQ4) {
-        const uint32_t w0 = row_r[tig], w8 = row_r8[tig];
-        // the two halves go to independent accumulators; the first starts at c
-        float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_bf16_16816(cb0, q4_raw(w0, 0), q4_raw(w8, 0), q4_raw(w0, 4), q4_raw(w8, 4), b0, b1);
-        mma_bf16_16816(cb1, q4_raw(w0, 8), q4_raw(w8, 8), q4_raw(w0, 12), q4_raw(w8, 12), b2, b3);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = cb0[i] + cb1[i];
-    } else {
-        const uint2 p = reinterpret_cast<const uint2*>(row_r)[tig];
-        const uint2 q = reinterpret_cast<const uint2*>(row_r8)[tig];
-        float cl[4] = {c0, c1, c0, c1}, ch[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_bf16_16816(cl, q4_raw(p.x, 0), q4_raw(q.x, 0), q4_raw(p.x, 4), q4_raw(q.x, 4), b0, b1);
-        mma_bf16_16816(ch, q4_raw(p.y, 0), q4_raw(q.y, 0), q4_raw(p.y, 4), q4_raw(q.y, 4), b0, b1);
-        mma_bf16_16816(cl, q4_raw(p.x, 8), q4_raw(q.x, 8), q4_raw(p.x, 12), q4_raw(q.x, 12), b2, b3);
-        mma_bf16_16816(ch, q4_raw(p.y, 8), q4_raw(q.y, 8), q4_raw(p.y, 12), q4_raw(q.y, 12), b2, b3);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = fmaf(16.f, ch[i], cl[i]);
-    }
-}
-
-// The same for the down contraction, whose B operand is h as a bf16 pair:
-// bh / bl hold the hi and lo fragments of the block's two 16-wide halves.
-template <int WF>
-__device__ __forceinline__ void quant_block_b(const uint32_t* row_r, const uint32_t* row_r8,
-                                              int tig, float c0, float c1, const uint32_t* bh0,
-                                              const uint32_t* bh1, const uint32_t* bl0,
-                                              const uint32_t* bl1, float v[4]) {
-    if constexpr (WF == kWfQ4) {
-        const uint32_t w0 = row_r[tig], w8 = row_r8[tig];
-        const uint32_t p0 = q4_raw(w0, 0), q0 = q4_raw(w8, 0), p1 = q4_raw(w0, 4), q1 = q4_raw(w8, 4);
-        const uint32_t p2 = q4_raw(w0, 8), q2 = q4_raw(w8, 8), p3 = q4_raw(w0, 12), q3 = q4_raw(w8, 12);
-        float cb0[4] = {c0, c1, c0, c1}, cb1[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_bf16_16816(cb0, p0, q0, p1, q1, bh0[0], bh0[1]);
-        mma_bf16_16816(cb1, p2, q2, p3, q3, bh1[0], bh1[1]);
-        mma_bf16_16816(cb0, p0, q0, p1, q1, bl0[0], bl0[1]);
-        mma_bf16_16816(cb1, p2, q2, p3, q3, bl1[0], bl1[1]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = cb0[i] + cb1[i];
-    } else {
-        const uint2 p = reinterpret_cast<const uint2*>(row_r)[tig];
-        const uint2 q = reinterpret_cast<const uint2*>(row_r8)[tig];
-        float cl[4] = {c0, c1, c0, c1}, ch[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-            const uint32_t p0 = q4_raw(p.x, 0), q0 = q4_raw(q.x, 0), p1 = q4_raw(p.x, 4), q1 = q4_raw(q.x, 4);
-            const uint32_t p2 = q4_raw(p.x, 8), q2 = q4_raw(q.x, 8), p3 = q4_raw(p.x, 12), q3 = q4_raw(q.x, 12);
-            mma_bf16_16816(cl, p0, q0, p1, q1, bh0[0], bh0[1]);
-            mma_bf16_16816(cl, p2, q2, p3, q3, bh1[0], bh1[1]);
-            mma_bf16_16816(cl, p0, q0, p1, q1, bl0[0], bl0[1]);
-            mma_bf16_16816(cl, p2, q2, p3, q3, bl1[0], bl1[1]);
-        }
-        {
-            const uint32_t p0 = q4_raw(p.y, 0), q0 = q4_raw(q.y, 0), p1 = q4_raw(p.y, 4), q1 = q4_raw(q.y, 4);
-            const uint32_t p2 = q4_raw(p.y, 8), q2 = q4_raw(q.y, 8), p3 = q4_raw(p.y, 12), q3 = q4_raw(q.y, 12);
-            mma_bf16_16816(ch, p0, q0, p1, q1, bh0[0], bh0[1]);
-            mma_bf16_16816(ch, p2, q2, p3, q3, bh1[0], bh1[1]);
-            mma_bf16_16816(ch, p0, q0, p1, q1, bl0[0], bl0[1]);
-            mma_bf16_16816(ch, p2, q2, p3, q3, bl1[0], bl1[1]);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) v[i] = fmaf(16.f, ch[i], cl[i]);
-    }
-}
+// Q8_0 on fp16 operands, one byte permute per register.  A packed byte is
+// the biased code u = q + 128; with the byte 0x64 above it, it reads as the
+// fp16 value 1024 + u (exact: the unit in the last place of [1024, 2048) is
+// 1).  Lane tig's 32-bit word of a block half holds u of k = 2tig, 2tig+1,
+// 2tig+8, 2tig+9 in its four bytes (see the Q8_0 packer), so q8h_lo gives
+// the A-fragment register of the pair (2tig, 2tig+1) and q8h_hi that of
+// (2tig+8, 2tig+9).  The weight is d q = d ((1024 + u) - 1152): the block's
+// accumulator starts at -1152 * (sum of the block's 32 activations).
+__device__ __forceinline__ uint32_t q8h_lo(uint32_t w) { return __byte_perm(w, 0x64646464u, 0x4140u); }
+__device__ __forceinline__ uint32_t q8h_hi(uint32_t w) { return __byte_perm(w, 0x64646464u, 0x4342u); }
+constexpr float kQ8Offset = 1024.f + 128.f;
 
 // ---- Q5_0.  The low 4 bits of each code are packed exactly like Q4_0
 // codes.  The fifth bits of a block row form one 32-bit word in which lane
@@ -390,7 +325,7 @@ __device__ __forceinline__ void quant_block_b(const uint32_t* row_r, const uint3
 // eight bits to bits 4-7 and 20-23, so that (e >> n) & 0x00100010 is the
 // fifth bit, worth 16, of the two codes q4_raw(w, 4n) extracts: q5_raw is
 // then two bf16 values 128 + q, q in 0..31 (exact; Q5_0's weight is
-// d * (q - 16), the 16 folded into quant_offset like Q4_0's 8).
+// d * (q - 16), the 128 + 16 folded into kQ5Offset).
 __device__ __forceinline__ uint32_t q5_lane_bits(uint32_t word, int tig) {
     return ((word >> (4 * tig)) & 0x000F000Fu) << 4;
 }
@@ -492,16 +427,17 @@ __device__ __forceinline__ DecodeSmem decode_smem(uint8_t* smem_raw, const Decod
 
 // Consumer threads copy the T token rows of x into shared memory once per
 // launch; every work unit then addresses its tokens' rows directly.  For
-// the quantised formats the same pass stores -offset * (sum of each 32-wide
-// block of a row), the starting value of that block's accumulator (see
-// q4_raw and quant_offset).
+// the quantised formats the same pass stores each 32-wide block's (q6_K:
+// 16-wide sub-block's) accumulator start, minus the code bases times the
+// block's activations (see q4h_lo, q8h_lo, q6h_regs and q5_raw).
 template <int WF>
 __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& sm, int tid) {
     const int nkb = a.d / 32;
-    if constexpr (WF == kWfQ4 || WF == kWfQ6) {
+    if constexpr (WF == kWfQ4 || WF == kWfQ6 || WF == kWfQ8) {
         // fp16 copy of x (exact for |x| >= 2^-17; below, off by at most 2^-25)
-        // and each block's accumulator start -sum((base_k + 8) x_k), base_k
-        // 1024 for k % 16 < 8 and 64 otherwise (see q4h_lo)
+        // and each block's accumulator start: Q4_0 -sum((base_k + 8) x_k),
+        // base_k 1024 for k % 16 < 8 and 64 otherwise (see q4h_lo); Q8_0
+        // -1152 sum(x_k) (see q8h_lo)
         for (int idx = tid; idx < a.T * nkb; idx += kConsumers) {
             const int t = idx / nkb, kb = idx % nkb;
             const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<size_t>(t) * a.d + kb * 32);
@@ -526,6 +462,8 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
             if constexpr (WF == kWfQ4) {
                 sm.xsum[t * nkb + kb] =
                     -((kF16BaseLo + 8.f) * (s8[0] + s8[2]) + (kF16BaseHi + 8.f) * (s8[1] + s8[3]));
+            } else if constexpr (WF == kWfQ8) {
+                sm.xsum[t * nkb + kb] = -kQ8Offset * ((s8[0] + s8[1]) + (s8[2] + s8[3]));
             } else {
                 // q6_K: one start per 16-wide sub-block, offset 32
                 sm.xsum[t * 2 * nkb + 2 * kb] = -((kF16BaseLo + 32.f) * s8[0] + (kF16BaseHi + 32.f) * s8[1]);
@@ -543,14 +481,14 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
         for (int c = 0; c < 4; ++c) {
             const uint4 v = __ldg(src + c);
             dst[c] = v;
-            if constexpr (WF == kWfQ8 || WF == kWfQ5) {
+            if constexpr (WF == kWfQ5) {
                 const uint32_t q[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
                     s += __uint_as_float(q[j] << 16) + __uint_as_float(q[j] & 0xffff0000u);
             }
         }
-        if constexpr (WF == kWfQ8 || WF == kWfQ5) sm.xsum[t * nkb + kb] = -quant_offset(WF) * s;
+        if constexpr (WF == kWfQ5) sm.xsum[t * nkb + kb] = -kQ5Offset * s;
     }
     }
 }
@@ -784,29 +722,17 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                         const uint32_t* row = codes + (bb * FS + r0) * (C::CB / 4);
                         uint32_t b0, b1, b2, b3;
                         ldsm_x4(xrow + ((kb0 + bb) * 32 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
-                        float v[4];
-                        if constexpr (WF == kWfQ5) {
-                            float s0, s8;
-                            uint32_t h0, h8;
-                            q5_aux(reinterpret_cast<const uint8_t*>(scl), bb, FS, r0, s0, s8, h0, h8);
-                            q5_block_a(row, row + 8 * (C::CB / 4), q5_lane_bits(h0, tig),
-                                       q5_lane_bits(h8, tig), tig, xsum0[bb], xsum1[bb], b0, b1, b2,
-                                       b3, v);
-                            cacc[0] = fmaf(s0, v[0], cacc[0]);
-                            cacc[1] = fmaf(s0, v[1], cacc[1]);
-                            cacc[2] = fmaf(s8, v[2], cacc[2]);
-                            cacc[3] = fmaf(s8, v[3], cacc[3]);
-                        } else {
-                            // the accumulator starts at -offset * sum(x) of the block
-                            quant_block_a<WF>(row, row + 8 * (C::CB / 4), tig, xsum0[bb], xsum1[bb],
-                                              b0, b1, b2, b3, v);
-                            const float s0 = __half2float(scl[bb * FS + r0]);
-                            const float s8 = __half2float(scl[bb * FS + r0 + 8]);
-                            cacc[0] = fmaf(s0, v[0], cacc[0]);
-                            cacc[1] = fmaf(s0, v[1], cacc[1]);
-                            cacc[2] = fmaf(s8, v[2], cacc[2]);
-                            cacc[3] = fmaf(s8, v[3], cacc[3]);
-                        }
+                        // Q5_0; the accumulator starts at -144 * sum(x) of the block
+                        float v[4], s0, s8;
+                        uint32_t h0, h8;
+                        q5_aux(reinterpret_cast<const uint8_t*>(scl), bb, FS, r0, s0, s8, h0, h8);
+                        q5_block_a(row, row + 8 * (C::CB / 4), q5_lane_bits(h0, tig),
+                                   q5_lane_bits(h8, tig), tig, xsum0[bb], xsum1[bb], b0, b1, b2,
+                                   b3, v);
+                        cacc[0] = fmaf(s0, v[0], cacc[0]);
+                        cacc[1] = fmaf(s0, v[1], cacc[1]);
+                        cacc[2] = fmaf(s8, v[2], cacc[2]);
+                        cacc[3] = fmaf(s8, v[3], cacc[3]);
                     }
                     }
                 }
@@ -851,7 +777,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
                 float hs = __bfloat162float(hi) + __bfloat162float(lo);
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) hs += __shfl_xor_sync(0xffffffffu, hs, off);
-                if (lane == 0) sm.hsum[t * 2 + f / 32] = -quant_offset(WF) * hs;
+                if (lane == 0) sm.hsum[t * 2 + f / 32] = -kQ5Offset * hs;
             }
         }
         named_bar_sync(1, kConsumers);
@@ -907,29 +833,17 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
 #pragma unroll
                         for (int bb = 0; bb < C::NB; ++bb) {
                             const uint32_t* row = codes + (bb * QB + rib) * (C::CB / 4);
-                            float v[4];
-                            if constexpr (WF == kWfQ5) {
-                                float s0, s8;
-                                uint32_t h0, h8;
-                                q5_aux(reinterpret_cast<const uint8_t*>(scl), bb, QB, rib, s0, s8, h0, h8);
-                                q5_block_b(row, row + 8 * (C::CB / 4), q5_lane_bits(h0, tig),
-                                           q5_lane_bits(h8, tig), tig, hs0[bb], hs1[bb], bh[2 * bb],
-                                           bh[2 * bb + 1], bl[2 * bb], bl[2 * bb + 1], v);
-                                c[0] = fmaf(s0, v[0], c[0]);
-                                c[1] = fmaf(s0, v[1], c[1]);
-                                c[2] = fmaf(s8, v[2], c[2]);
-                                c[3] = fmaf(s8, v[3], c[3]);
-                            } else {
-                                // the accumulator starts at -offset * sum(hi + lo) of the block
-                                quant_block_b<WF>(row, row + 8 * (C::CB / 4), tig, hs0[bb], hs1[bb],
-                                                  bh[2 * bb], bh[2 * bb + 1], bl[2 * bb], bl[2 * bb + 1], v);
-                                const float s0 = __half2float(scl[bb * QB + rib]);
-                                const float s8 = __half2float(scl[bb * QB + rib + 8]);
-                                c[0] = fmaf(s0, v[0], c[0]);
-                                c[1] = fmaf(s0, v[1], c[1]);
-                                c[2] = fmaf(s8, v[2], c[2]);
-                                c[3] = fmaf(s8, v[3], c[3]);
-                            }
+                            // Q5_0; the accumulator starts at -144 * sum(hi + lo) of the block
+                            float v[4], s0, s8;
+                            uint32_t h0, h8;
+                            q5_aux(reinterpret_cast<const uint8_t*>(scl), bb, QB, rib, s0, s8, h0, h8);
+                            q5_block_b(row, row + 8 * (C::CB / 4), q5_lane_bits(h0, tig),
+                                       q5_lane_bits(h8, tig), tig, hs0[bb], hs1[bb], bh[2 * bb],
+                                       bh[2 * bb + 1], bl[2 * bb], bl[2 * bb + 1], v);
+                            c[0] = fmaf(s0, v[0], c[0]);
+                            c[1] = fmaf(s0, v[1], c[1]);
+                            c[2] = fmaf(s8, v[2], c[2]);
+                            c[3] = fmaf(s8, v[3], c[3]);
                         }
                         }
                     }
@@ -977,7 +891,7 @@ __device__ __forceinline__ void q6_scales(uint32_t sw, float dr, float dr8, floa
 }
 
 // The experts pipeline for the weight formats that feed fp16 operands to
-// the tensor cores (F16: Q4_0, q6_K): phase A streams row groups instead of
+// the tensor cores (F16: Q4_0, Q8_0, q6_K): phase A streams row groups instead of
 // block columns.  A phase-A stage is 16 consecutive rows of the gate or up
 // slice over the whole reduction dim (KC <= 64 block columns per stage, more
 // stages per row group when d > 2048), and consumer warp w owns block
@@ -994,8 +908,9 @@ __device__ __forceinline__ void q6_scales(uint32_t sw, float dr, float dr8, floa
 // block.  Partial stages (d not a multiple of 2048, the last down rows) take
 // a general path.
 //
-// Stage layouts.  Q4_0 phase A: codes [KC][16 rows][16 B], scales [KC][16]
-// fp16; phase B per 256-row box: codes [NB][256][16 B], scales [NB][256].
+// Stage layouts.  Q4_0 / Q8_0 phase A: codes [KC][16 rows][CB = 16 / 32 B],
+// scales [KC][16] fp16; phase B per 256-row box: codes [NB][256][CB],
+// scales [NB][256].
 // q6_K phase A: codes [KC][16][16 B], records [KC][160 B], super-block scales
 // [KC/8][16] fp16; phase B per 256-row box: codes [NB][256][16 B], records
 // [NB][16][160 B], super-block scales [256] fp16 (a slice of FS <= 256
@@ -1015,7 +930,8 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
     static_assert(RGW * kConsumerWarps * 16 == C::RJ && C::RJ % QB == 0, "phase-B split");
     constexpr int KCMAX = C::KCMAX;
     // offsets inside a full phase-A stage (KC = 64)
-    constexpr uint32_t A_SCL = 16 * KCMAX * C::CB;                 // Q4_0 scales
+    constexpr uint32_t A_SCL = 16 * KCMAX * C::CB;                 // Q4_0 / Q8_0 scales
+    constexpr uint32_t RGB = 16 * C::CB;                           // codes of a 16-row group
     constexpr uint32_t A_REC = 16 * KCMAX * 16;                    // q6_K records
     constexpr uint32_t A_D = KCMAX * (16 * 16 + 160);              // q6_K super-block scales
     const int ns = a.n_stages;
@@ -1147,7 +1063,7 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
     constexpr int NC = C::Q6 ? 2 : 1;                 // corrections per block (per 16-k sub-block)
     // this lane's bases inside a stage: block column (phase A) or row group
     // (phase B) `warp`, row g, code word tig
-    const uint32_t lane_code = warp * 256 + g * 16 + tig * 4;
+    const uint32_t lane_code = warp * RGB + g * C::CB + tig * (C::CB / 4);
     const uint32_t lane_a_scl = A_SCL + warp * 32 + g * 2;
     const uint32_t lane_a_rec = A_REC + warp * 160 + (4 * g + tig) * 4;
     const uint32_t lane_a_sub = A_REC + warp * 160 + 128 + g * 4;
@@ -1229,6 +1145,18 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
             ac[2] = fmaf(s8, va[2], ac[2]);
             ac[3] = fmaf(s8, va[3], ac[3]);
         };
+        // Q8_0: x0 / x8 the lane's two words (block halves) of rows g / g+8
+        auto block_q8 = [&](int i, uint2 x0, uint2 x8, float s0, float s8, float (&ac)[4]) {
+            float va[4];
+            mma_f16_16816(va, q8h_lo(x0.x), q8h_lo(x8.x), q8h_hi(x0.x), q8h_hi(x8.x), xf[i][0], xf[i][1],
+                          xc0[i][0], xc1[i][0], xc0[i][0], xc1[i][0]);
+            mma_f16_16816_acc(va, q8h_lo(x0.y), q8h_lo(x8.y), q8h_hi(x0.y), q8h_hi(x8.y), xf[i][2],
+                              xf[i][3]);
+            ac[0] = fmaf(s0, va[0], ac[0]);
+            ac[1] = fmaf(s0, va[1], ac[1]);
+            ac[2] = fmaf(s8, va[2], ac[2]);
+            ac[3] = fmaf(s8, va[3], ac[3]);
+        };
         auto block_q6 = [&](int i, uint32_t x0, uint32_t x8, uint32_t e, uint32_t sw, float dr, float dr8,
                             float (&ac)[4]) {
             uint32_t p0, p1, p2, p3, q0, q1, q2, q3;
@@ -1265,7 +1193,14 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                         // all four block columns of this warp are in the stage
 #pragma unroll
                         for (int i = 0; i < C::NBW; ++i) {
-                            const uint32_t cb = st_u + lane_code + i * (16 * 16 * 16);
+                            const uint32_t cb = st_u + lane_code + i * (16 * RGB);
+                            if constexpr (C::Q8) {
+                                const uint2 x0 = lds_u32x2(cb), x8 = lds_u32x2(cb + 8 * C::CB);
+                                const float s0 = lds_f16_as_f32(st_u + lane_a_scl + i * 512);
+                                const float s8 = lds_f16_as_f32(st_u + lane_a_scl + i * 512 + 16);
+                                block_q8(i, x0, x8, s0, s8, ac);
+                                continue;
+                            }
                             const uint32_t x0 = lds_u32(cb), x8 = lds_u32(cb + 128);
                             if constexpr (C::Q6) {
                                 const uint32_t e = lds_u32(st_u + lane_a_rec + i * (16 * 160));
@@ -1286,6 +1221,14 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                         for (int i = 0; i < C::NBW; ++i) {
                             const int bl = warp + kConsumerWarps * i;
                             if (bl < KC && c * KC + bl < nkb) {
+                                if constexpr (C::Q8) {
+                                    const uint2* row = reinterpret_cast<const uint2*>(codes) + (bl * 16 + g) * 4;
+                                    const __half* scl =
+                                        reinterpret_cast<const __half*>(stage + 16 * KC * C::CB);
+                                    block_q8(i, row[tig], row[32 + tig], __half2float(scl[bl * 16 + g]),
+                                             __half2float(scl[bl * 16 + g + 8]), ac);
+                                    continue;
+                                }
                                 const uint32_t* row = codes + (bl * 16 + g) * 4;
                                 const uint32_t x0 = row[tig], x8 = row[32 + tig];
                                 if constexpr (C::Q6) {
@@ -1321,7 +1264,8 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
         // h = SiLU(gate) * up as an fp16 pair hi + lo for the token columns in
         // use (the rest are zero); one warp covers 32 consecutive f of one
         // column, i.e. one block of the down matrix.  The down block's (q6_K:
-        // sub-block's) accumulator starts at -sum((base_f + offset)(hi + lo)).
+        // sub-block's) accumulator starts at -sum((base_f + offset)(hi + lo))
+        // (Q8_0: -1152 sum(hi + lo)).
         for (int idx = tid; idx < FS * kDecodeTok; idx += kConsumers) {
             const int t = idx / FS, f = idx % FS;
             __half hi = __float2half_rn(0.f), lo = hi;
@@ -1337,7 +1281,8 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                 hi = __float2half_rn(h);
                 lo = __float2half_rn(h - __half2float(hi));
                 const float base = (f & 15) < 8 ? kF16BaseLo : kF16BaseHi;
-                hs = (base + (C::Q6 ? 32.f : 8.f)) * (__half2float(hi) + __half2float(lo));
+                hs = (C::Q8 ? kQ8Offset : base + (C::Q6 ? 32.f : 8.f)) *
+                     (__half2float(hi) + __half2float(lo));
             }
             reinterpret_cast<__half*>(sm.hhi)[t * C::HS + f] = hi;
             reinterpret_cast<__half*>(sm.hlo)[t * C::HS + f] = lo;
@@ -1359,7 +1304,7 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
             ldsm_x2(smem_u32(sm.hhi) + off, bh[kk][0], bh[kk][1]);
             ldsm_x2(smem_u32(sm.hlo) + off, bl[kk][0], bl[kk][1]);
         }
-        // corrections of the down blocks (Q4_0) or sub-blocks (q6_K), columns t0, t1
+        // corrections of the down blocks (Q4_0, Q8_0) or sub-blocks (q6_K), columns t0, t1
         constexpr int NH = C::Q6 ? 2 * C::NB : C::NB;
         float hs0[NH], hs1[NH];
 #pragma unroll
@@ -1377,6 +1322,27 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
             c[0] = c[1] = c[2] = c[3] = 0.f;
 #pragma unroll
             for (int bb = 0; bb < C::NB; ++bb) {
+                if constexpr (C::Q8) {
+                    const uint2 x0 = lds_u32x2(code_u + bb * (QB * C::CB));
+                    const uint2 x8 = lds_u32x2(code_u + bb * (QB * C::CB) + 8 * C::CB);
+                    const uint32_t p0 = q8h_lo(x0.x), q0 = q8h_lo(x8.x);
+                    const uint32_t p1 = q8h_hi(x0.x), q1 = q8h_hi(x8.x);
+                    const uint32_t p2 = q8h_lo(x0.y), q2 = q8h_lo(x8.y);
+                    const uint32_t p3 = q8h_hi(x0.y), q3 = q8h_hi(x8.y);
+                    float va[4];
+                    mma_f16_16816(va, p0, q0, p1, q1, bh[2 * bb][0], bh[2 * bb][1],
+                                  hs0[bb], hs1[bb], hs0[bb], hs1[bb]);
+                    mma_f16_16816_acc(va, p2, q2, p3, q3, bh[2 * bb + 1][0], bh[2 * bb + 1][1]);
+                    mma_f16_16816_acc(va, p0, q0, p1, q1, bl[2 * bb][0], bl[2 * bb][1]);
+                    mma_f16_16816_acc(va, p2, q2, p3, q3, bl[2 * bb + 1][0], bl[2 * bb + 1][1]);
+                    const float s0 = lds_f16_as_f32(scl_u + bb * (QB * 2));
+                    const float s8 = lds_f16_as_f32(scl_u + bb * (QB * 2) + 16);
+                    c[0] = fmaf(s0, va[0], c[0]);
+                    c[1] = fmaf(s0, va[1], c[1]);
+                    c[2] = fmaf(s8, va[2], c[2]);
+                    c[3] = fmaf(s8, va[3], c[3]);
+                    continue;
+                }
                 const uint32_t x0 = lds_u32(code_u + bb * (QB * 16));
                 const uint32_t x8 = lds_u32(code_u + bb * (QB * 16) + 128);
                 if constexpr (C::Q6) {
@@ -1448,7 +1414,7 @@ __device__ __forceinline__ void experts_pipeline_rows(const DecodeArgs& a, const
                     for (int rgb = warp; rgb < rows / 16; rgb += kConsumerWarps) {
                         const int grp = rgb % (QB / 16);
                         const uint32_t bq = st_u + (rgb / (QB / 16)) * BOXB;
-                        const uint32_t lc = grp * 256 + g * 16 + tig * 4;
+                        const uint32_t lc = grp * RGB + g * C::CB + tig * (C::CB / 4);
                         float c[4];
                         rowgroup(bq + lc, bq + C::NB * QB * C::CB + grp * 32 + g * 2,
                                  bq + C::NB * QB * 16 + grp * 160 + (4 * g + tig) * 4,
@@ -1902,7 +1868,7 @@ int decode_stage_bytes(int fs, int wfmt) {
 size_t decode_smem_bytes(int fs, int wfmt, int d, int n_stages) {
     // partial sums per gate/up output: KSPLIT, or one per warp for the
     // row-streaming formats (DecodeCfg::GU_PARTS)
-    const int ksplit = (wfmt == kWfQ4 || wfmt == kWfQ6) ? kConsumerWarps
+    const int ksplit = (wfmt == kWfQ4 || wfmt == kWfQ6 || wfmt == kWfQ8) ? kConsumerWarps
                                                          : kConsumerWarps / (2 * (fs / 16));
     size_t b = 1024;                                            // alignment slack
     b += static_cast<size_t>(n_stages) * decode_stage_bytes(fs, wfmt);
@@ -1972,7 +1938,6 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, int fs, int wfmt, int grid,
         case kWfF16d * 100 + 32: return launch_fused_one<32, kWfF16d>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_fused_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ6 * 100 + 32: return launch_fused_one<32, kWfQ6>(a, grid, smem, stream);
-        case kWfQ8 * 100 + 64: return launch_fused_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_fused_one<32, kWfQ8>(a, grid, smem, stream);
         case kWfQ5 * 100 + 64: return launch_fused_one<64, kWfQ5>(a, grid, smem, stream);
         case kWfQ5 * 100 + 32: return launch_fused_one<32, kWfQ5>(a, grid, smem, stream);
@@ -1989,7 +1954,6 @@ cudaError_t launch_decode_experts(const DecodeArgs& a, int fs, int wfmt, int gri
         case kWfF16d * 100 + 32: return launch_one<32, kWfF16d>(a, grid, smem, stream);
         case kWfQ4 * 100 + 32: return launch_one<32, kWfQ4>(a, grid, smem, stream);
         case kWfQ6 * 100 + 32: return launch_one<32, kWfQ6>(a, grid, smem, stream);
-        case kWfQ8 * 100 + 64: return launch_one<64, kWfQ8>(a, grid, smem, stream);
         case kWfQ8 * 100 + 32: return launch_one<32, kWfQ8>(a, grid, smem, stream);
         case kWfQ5 * 100 + 64: return launch_one<64, kWfQ5>(a, grid, smem, stream);
         case kWfQ5 * 100 + 32: return launch_one<32, kWfQ5>(a, grid, smem, stream);

@@ -77,18 +77,15 @@ cudaError_t launch_q4_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
 // Kernel layout (same 8.5 bits per weight):
 //   codes  [mat][k/32][rows][32 B]
 //   scales [mat][k/32][rows] fp16
-// Each code is biased to u = q + 128 (0..255) and split into its nibbles
-// u = 16 hi + lo.  Both nibble planes are packed exactly like Q4_0 codes
-// above (one 32-bit word per lane holds the 8 values of the lane's A
-// fragment for both halves of the block); the 8 words of a block row are
-// interleaved as lo0 hi0 lo1 hi1 lo2 hi2 lo3 hi3, so lane tig fetches both
-// of its words with one 64-bit load.
-__device__ __forceinline__ uint32_t pack_q4_lane(const uint8_t* q, int t) {
-    const int e = 2 * t;
-    return static_cast<uint32_t>(q[e]) | (static_cast<uint32_t>(q[e + 8]) << 4) |
-           (static_cast<uint32_t>(q[e + 16]) << 8) | (static_cast<uint32_t>(q[e + 24]) << 12) |
-           (static_cast<uint32_t>(q[e + 1]) << 16) | (static_cast<uint32_t>(q[e + 9]) << 20) |
-           (static_cast<uint32_t>(q[e + 17]) << 24) | (static_cast<uint32_t>(q[e + 25]) << 28);
+// Each code is stored biased, u = q + 128 (0..255), one byte per code.  A
+// block row is four 8-byte lane shares; lane tig's share holds, in this
+// order, the codes of elements
+//   2tig, 2tig+1, 2tig+8, 2tig+9, 16+2tig, 17+2tig, 24+2tig, 25+2tig,
+// i.e. its first 32-bit word covers the lane's A-fragment elements of the
+// block's first 16-wide half and its second word those of the second half,
+// in fragment order (pair 2tig/2tig+1, then pair 2tig+8/2tig+9).
+__device__ __forceinline__ int q8_lane_elem(int t, int n) {   // n-th byte of lane t's share
+    return 2 * t + (n & 1) + 8 * ((n >> 1) & 1) + 16 * (n >> 2);
 }
 
 __global__ void q8_0_pack_kernel(const uint8_t* __restrict__ blocks, int64_t n_mats, int64_t rows,
@@ -101,18 +98,19 @@ __global__ void q8_0_pack_kernel(const uint8_t* __restrict__ blocks, int64_t n_m
         const int64_t r = (i / nkb) % rows;
         const int64_t m = i / (nkb * rows);
         const uint8_t* src = blocks + i * 34;            // [m][r][kb] canonical
-        uint8_t lo[32], hi[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const uint8_t u = static_cast<uint8_t>(src[2 + j] ^ 0x80u);   // q + 128
-            lo[j] = u & 0x0f;
-            hi[j] = u >> 4;
-        }
         uint32_t w[8];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-            w[2 * t] = pack_q4_lane(lo, t);
-            w[2 * t + 1] = pack_q4_lane(hi, t);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t v = 0;
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    const uint32_t u = static_cast<uint32_t>(src[2 + q8_lane_elem(t, 4 * h + n)] ^ 0x80u);
+                    v |= u << (8 * n);
+                }
+                w[2 * t + h] = v;
+            }
         }
         const int64_t dst = (m * nkb + kb) * rows + r;   // [m][kb][r]
         uint4* o = reinterpret_cast<uint4*>(codes + dst * 32);
@@ -151,6 +149,15 @@ cudaError_t launch_q8_0_pack(const uint8_t* blocks, int64_t n_mats, int64_t rows
 // In a row's word of fifth bits, lane t (0..3) owns bits 4t+n and 16+4t+n
 // (n = 0..3): the fifth bits of the codes in nibbles n and n+4 of its code
 // word (elements 2t+8n and 2t+1+8n).
+// lane t's 32-bit word of 4-bit values q[0..31], in the Q4_0 permutation
+__device__ __forceinline__ uint32_t pack_q4_lane(const uint8_t* q, int t) {
+    const int e = 2 * t;
+    return static_cast<uint32_t>(q[e]) | (static_cast<uint32_t>(q[e + 8]) << 4) |
+           (static_cast<uint32_t>(q[e + 16]) << 8) | (static_cast<uint32_t>(q[e + 24]) << 12) |
+           (static_cast<uint32_t>(q[e + 1]) << 16) | (static_cast<uint32_t>(q[e + 9]) << 20) |
+           (static_cast<uint32_t>(q[e + 17]) << 24) | (static_cast<uint32_t>(q[e + 25]) << 28);
+}
+
 __global__ void q5_0_pack_kernel(const uint8_t* __restrict__ blocks, int64_t n_mats, int64_t rows,
                                  int64_t nkb, uint8_t* __restrict__ codes, uint8_t* __restrict__ aux) {
     const int64_t total = n_mats * rows * nkb;

@@ -71,14 +71,16 @@ def test_q4_0_pack_is_the_documented_permutation(n_mats, rows, k):
 
 
 @pytest.mark.parametrize("n_mats,rows,k", [(1, 1, 32), (3, 40, 96), (2, 128, 512)])
-def test_q8_0_pack_is_the_documented_planes(n_mats, rows, k):
+def test_q8_0_pack_is_the_documented_byte_order(n_mats, rows, k):
     rng = np.random.default_rng(n_mats * 1000 + rows + 7)
     canon = synth.q8_0_blocks(rng, n_mats * rows, k, 0.01).reshape(n_mats, rows, k // 32, 34)
     codes, scales = _pack_on_gpu(B.moe_q8_0_packed_bytes, B.moe_q8_0_pack, canon, n_mats, rows, k)
-    words = codes.view(np.uint32).reshape(n_mats, k // 32, rows, 8)
-    lo = _unpack_nibble_words(words[..., 0::2]).astype(np.int32)
-    hi = _unpack_nibble_words(words[..., 1::2]).astype(np.int32)
-    got = (16 * hi + lo - 128).transpose(0, 2, 1, 3)                # signed codes [m][r][kb][32]
+    packed = codes.reshape(n_mats, k // 32, rows, 32).astype(np.int32) - 128   # q = u - 128
+    got = np.zeros_like(packed)
+    for t in range(4):
+        for n in range(8):
+            got[..., 2 * t + (n & 1) + 8 * ((n >> 1) & 1) + 16 * (n >> 2)] = packed[..., 8 * t + n]
+    got = got.transpose(0, 2, 1, 3)                                   # signed codes [m][r][kb][32]
     want = canon[..., 2:].copy().view(np.int8).astype(np.int32)
     assert np.array_equal(got, want)
     want_sc = canon[..., :2].copy().view(np.uint16)[..., 0]
