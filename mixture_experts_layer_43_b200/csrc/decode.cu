@@ -306,6 +306,12 @@ __device__ __forceinline__ uint32_t q4h_lo(uint32_t w) { return (w & 0x000F000Fu
 __device__ __forceinline__ uint32_t q4h_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x54005400u; }
 constexpr float kF16BaseLo = 1024.f, kF16BaseHi = 64.f;
 
+__device__ __forceinline__ uint2 lds_u32x2(uint32_t addr) {   // addr 8-byte aligned
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
 // Q8_0 on fp16 operands, one byte permute per register.  A packed byte is
 // the biased code u = q + 128; with the byte 0x64 above it, it reads as the
 // fp16 value 1024 + u (exact: the unit in the last place of [1024, 2048) is
