@@ -36,6 +36,11 @@ SMALL = [
                    wfmt=synth.WFMT_Q8_0),
     synth.MoEShape("multi_unit_q8", T=8, d=1024, E=8, k=2, F=2048, S=1, Fs=512,
                    wfmt=synth.WFMT_Q8_0),
+    # Q8_0 with 72 block columns (two phase-A chunks per row group, the second
+    # partial) and at the interface's limits
+    synth.MoEShape("chunked_q8", T=5, d=2304, E=8, k=2, F=96, S=1, Fs=64, wfmt=synth.WFMT_Q8_0),
+    synth.MoEShape("max_limits_q8", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32,
+                   wfmt=synth.WFMT_Q8_0),
     # the interface's limits: E = 1024 experts, k = 16, 8 shared experts, T = 8
     # (128 token-expert pairs, a 32-word expert mask, the widest register top-k)
     synth.MoEShape("max_limits", T=8, d=256, E=1024, k=16, F=64, S=8, Fs=32),
@@ -134,7 +139,7 @@ def test_decode_topk_variants(sh):
 
 
 SPLIT = SMALL[:6] + [SMALL[10], SMALL[-4], W["a3b_q4_T8_d2048_E256k8_F512_S1"],
-                     W["a3b_q6_T8_d2048_E256k8_F512_S1"]]
+                     W["a3b_q6_T8_d2048_E256k8_F512_S1"], W["a3b_q8_T8_d2048_E256k8_F512_S1"]]
 
 
 @pytest.mark.parametrize("sh", SPLIT, ids=[s.name for s in SPLIT])
