@@ -23,9 +23,10 @@
 // ring of stages fed by one producer warp, so every SM keeps tens of KB in
 // flight ("MoE on RTX 5090 reaches 41% of bandwidth" page: small reads per
 // kernel cap bandwidth; the fix it predicts is more bytes per launch).  The
-// contraction over the <= 8 tokens of an expert runs on mma.sync (bf16 in,
-// fp32 accumulate); Q4_0 codes are dequantised in registers and never
-// written back ("MMVQ" page: read quantised weights once, never expand them).
+// contraction over the <= 8 tokens of an expert runs on mma.sync (bf16 or
+// fp16 in, fp32 accumulate); quantised codes (Q4_0, Q8_0, Q5_0, q6_K) become
+// operand fragments in registers and are never written back ("MMVQ" page:
+// read quantised weights once, never expand them).
 #include <float.h>
 #include <math.h>
 #include <stddef.h>
@@ -284,10 +285,8 @@ struct alignas(16) DecodeSmemTail {
 };
 
 // ((w >> s) & 0x000F000F) | 0x43004300 puts two 4-bit codes q in the low
-// mantissa bits of two bf16 values 128 + q (exact).  Q4_0's weight is
-// d * (q - 8) = d * ((128 + q) - 136): instead of subtracting 136 from every
-// weight, the block's accumulator starts at -136 * (sum of the block's 32
-// activations), so one block contributes d * sum((128 + q) x) - 136 d sum(x).
+// mantissa bits of two bf16 values 128 + q (exact): the bf16 operands of
+// the Q5_0 kernels, which add the fifth bit on top (see q5_raw).
 __device__ __forceinline__ uint32_t q4_raw(uint32_t w, int s) {
     return ((w >> s) & 0x000F000Fu) | 0x43004300u;
 }
@@ -353,8 +352,14 @@ __device__ __forceinline__ void q5_aux(const uint8_t* aux, int bb, int nrows, in
     h8 = *reinterpret_cast<const uint32_t*>(rec + 48 + 16 + 4 * i);
 }
 
-// quant_block_a / quant_block_b for Q5_0: e0, e8 are q5_lane_bits of rows r
-// and r + 8.
+// One Q5_0 block (32 weights along k) of rows r and r+8 of an mma A tile,
+// times the B fragment of the same 32 k (b0 b1: k 0-15, b2 b3: k 16-31).
+// row_r / row_r8 point at the rows' code words, e0 / e8 are q5_lane_bits of
+// their fifth-bit words, c0 / c1 the accumulator starts of the lane's two
+// token columns (-144 * the block's activation sums); v gets the block's
+// four dot products before the block scale.  q5_block_b is the same for the
+// down contraction, whose B operand is h as a bf16 pair: bh / bl hold the hi
+// and lo fragments of the block's two 16-wide halves.
 __device__ __forceinline__ void q5_block_a(const uint32_t* row_r, const uint32_t* row_r8,
                                            uint32_t e0, uint32_t e8, int tig, float c0, float c1,
                                            uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3,
@@ -401,11 +406,11 @@ struct WorkView {
 struct DecodeSmem {
     uint8_t* ring;
     uint8_t* xs;            // [8][xs_stride]: the T token rows of x, staged once
-    float* xsum;            // [8][d/32]: -offset * block sums of x (quantised formats)
+    float* xsum;            // [8][d/16]: block (q6_K: sub-block) accumulator starts (quantised formats)
     float* gu;              // [GU_PARTS][2][8][GS]: gate / up partial results
     __nv_bfloat16* hhi;     // [8][HS]: h = hi + lo, per slot
     __nv_bfloat16* hlo;
-    float* hsum;            // [8][4]: -offset * block (q6_K: sub-block) sums of hi + lo
+    float* hsum;            // [8][4]: down block (q6_K: sub-block) accumulator starts from hi + lo
     DecodeSmemTail* tail;
     uint64_t* full;
     uint64_t* empty;
@@ -499,11 +504,11 @@ __device__ __forceinline__ void stage_x(const DecodeArgs& a, const DecodeSmem& s
     }
 }
 
-// The expert stage: work units are (expert, slice of FS hidden rows), shared
+// The expert stage with block-column stages (bf16, bf16 with fp16 down
+// matrices, Q5_0): work units are (expert, slice of FS hidden rows), shared
 // experts' units first, then the routed experts' in ascending expert order
-// (assignment to CTAs: see experts_pipeline).  The last warp (lane 0) is the
-// TMA producer, the others consume.  Barriers must be initialised by the
-// caller.
+// (assignment to CTAs: see below).  The last warp (lane 0) is the TMA
+// producer, the others consume.  Barriers must be initialised by the caller.
 template <int FS, int WF>
 __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const DecodeSmem& sm,
                                                  const WorkView& wv) {
@@ -758,7 +763,7 @@ __device__ __forceinline__ void experts_pipeline(const DecodeArgs& a, const Deco
         }
         named_bar_sync(1, kConsumers);
         // h = SiLU(gate) * up, kept as a bf16 pair hi + lo (|h - hi - lo| <= 2^-16 |h|).
-        // One warp covers 32 consecutive f of one slot, i.e. one Q4_0 block of
+        // One warp covers 32 consecutive f of one slot, i.e. one Q5_0 block of
         // the down matrix (FS * 8 is a multiple of 32: the loop is warp-uniform).
         for (int idx = tid; idx < FS * kDecodeTok; idx += kConsumers) {
             const int t = idx / FS, f = idx % FS;
